@@ -1,0 +1,186 @@
+/*
+ * fp4.h -- C ABI of the B200 (sm_100a) microscaling FP4 library (libfp4.so).
+ *
+ * What the operations are (sources, by page and section):
+ *  - "FP4 All the Way: Fully Quantized Training of LLMs", Abstract: FP4 (E2M1)
+ *    for weights, activations and gradients; NVFP4 = blocks of 16 E2M1 values
+ *    sharing an E4M3 scale; round-to-nearest forward, stochastic rounding for
+ *    the backward and update passes; block size, scale format and rounding are
+ *    the design choices.
+ *  - "Bridging the Gap Between Promise and Performance for Microscaling FP4
+ *    Quantization", Abstract: MXFP4 (power-of-two scales) and NVFP4;
+ *    block-wise Hadamard rotations fused into the weights and computed online
+ *    for the activations; FP4 GEMM kernels on B200.
+ *  - "Oscillation-Reduced MXFP4 Training for Vision Transformers", Abstract:
+ *    MX fine-grained per-group scaling, supported by Blackwell.
+ *
+ * Encodings (the pages fix none; OCP MX v1.0 conventions are used):
+ *  - E2M1 code: bit 3 sign, magnitudes 0,0.5,1,1.5,2,3,4,6 for codes 0..7.
+ *    Two codes per byte: element 2j in the low nibble, 2j+1 in the high one.
+ *  - MXFP4: 32-element blocks, E8M0 scale byte b (2^(b-127)),
+ *    E = clamp(floor(log2 amax_b) - 2, -127, 127); byte 0 for all-zero blocks.
+ *  - NVFP4: 16-element blocks, E4M3 scale sb = RNE_sat((amax_b/6)/s_t) under a
+ *    per-tensor fp32 scale s_t = amax/(6*448) (1.0 for an all-zero tensor).
+ *  - RTN = round to nearest, ties to even code, saturating at +-6, sign kept.
+ *    SR = Philox4x32-10 (Salmon et al., SC'11), key = seed, counter =
+ *    (idx>>2 as 64-bit, 0, 0), the element with row-major input index idx
+ *    takes output word idx&3; round up iff word < ceil(p * 2^32).
+ *  - Blocks whose scale is zero (amax_b == 0, NV sb == 0) get codes +0.
+ *
+ * Scale-factor layouts:
+ *  - FP4_SF_ROWMAJOR: [out_rows, L/block] bytes, row-major.
+ *  - FP4_SF_MMA: the layout the block-scaled tensor-core MMA consumes: rows
+ *    padded to 128 and k-groups to 4 (pads written as 0), 128x4 tiles stored
+ *    with the k-tile index fastest, tile (rb,kb) at byte ((rb*G4)+kb)*512 and
+ *    row r / k-group g inside it at (r%32)*16 + (r/32)*4 + g.  fp4_gemm reads
+ *    only this layout.
+ *
+ * Conventions for every entry point:
+ *  - All data pointers are DEVICE pointers (cudaMalloc'd or torch-owned) on
+ *    the current device; the caller allocates and owns every buffer.  The
+ *    library holds one small per-device scratch buffer (tensor-amax partials
+ *    and a device error word), allocated on first use and kept until exit.
+ *  - `stream` is a cudaStream_t owned by the caller (NULL = legacy default
+ *    stream).  Every call is asynchronous on it; none synchronizes, except
+ *    fp4_check_device_errors.
+ *  - Argument, shape and alignment errors return a negative fp4_status before
+ *    anything is launched.  A failed launch returns FP4_ERR_CUDA.  Nothing
+ *    aborts, prints or throws across the ABI.  Calls that compute a tensor
+ *    scale share the per-device scratch: two such calls that overlap in time
+ *    on different streams of one device race.
+ *  - Quantized tensors: axis = 1 quantizes along columns of x[rows, cols]
+ *    (codes [rows, cols/2], scales per row); axis = 0 quantizes along rows
+ *    and writes the transpose (codes [cols, rows/2]), so that the packed axis
+ *    is always the contraction axis of fp4_gemm.  "out_rows" and "L" below
+ *    are (rows, cols) for axis 1 and (cols, rows) for axis 0.
+ *
+ * Supported (format, block): (FP4_MXFP4, 32), (FP4_NVFP4, 16).
+ */
+#ifndef FP4_H_
+#define FP4_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef int fp4_status;
+enum {
+  FP4_OK = 0,
+  FP4_ERR_ARG = -1,          /* null pointer, bad enum value, negative size       */
+  FP4_ERR_SHAPE = -2,        /* size not a multiple of what the format needs     */
+  FP4_ERR_ALIGN = -3,        /* pointer or leading dimension misaligned          */
+  FP4_ERR_UNSUPPORTED = -4,  /* (format, block) or option combination not built  */
+  FP4_ERR_CUDA = -5,         /* CUDA runtime error at launch or set-up           */
+  FP4_ERR_TIMEOUT = -6       /* a bounded device wait expired (reported later by
+                                fp4_check_device_errors)                           */
+};
+
+enum { FP4_MXFP4 = 0, FP4_NVFP4 = 1 };              /* fp4_format    */
+enum { FP4_RTN = 0, FP4_SR = 1 };                   /* fp4_round     */
+enum { FP4_SF_ROWMAJOR = 0, FP4_SF_MMA = 1 };       /* fp4_sf_layout */
+enum { FP4_OUT_F32 = 0, FP4_OUT_BF16 = 1 };         /* fp4_dtype     */
+
+/*
+ * fp4_quantize -- block-scaled FP4 quantization of a bf16 matrix
+ * ("FP4 All the Way", Abstract: NVFP4 blocks of 16 E2M1 with an E4M3 scale,
+ * RTN forward / SR backward; "Bridging the Gap", Abstract: MXFP4
+ * power-of-two scales).
+ *
+ *   x          bf16 [rows, cols], row stride `ld` elements (ld >= cols).
+ *              16-byte aligned; cols and ld multiples of 8.
+ *   fmt,block  (FP4_MXFP4, 32) or (FP4_NVFP4, 16).
+ *   axis       1: blocks along cols (cols % block == 0);
+ *              0: blocks along rows (rows % block == 0), output transposed.
+ *   rnd, seed  FP4_RTN, or FP4_SR with the 64-bit Philox key `seed`.
+ *   tensor_scale_in   NV only, nullable, device fp32: use this s_t.
+ *   tensor_scale_out  NV only, device fp32: receives the s_t used (may equal
+ *              tensor_scale_in).  Required for NV, ignored for MX.
+ *   codes      uint8 [out_rows, L/2], 16-byte aligned.
+ *   scales     uint8, fp4_scales_bytes(...) bytes in layout `sf_layout`.
+ * NV without tensor_scale_in launches an amax pass over x first.
+ */
+fp4_status fp4_quantize(const void* x, int64_t rows, int64_t cols, int64_t ld,
+                        int fmt, int block, int axis, int rnd, uint64_t seed,
+                        const float* tensor_scale_in, float* tensor_scale_out,
+                        uint8_t* codes, uint8_t* scales, int sf_layout, void* stream);
+
+/*
+ * fp4_hadamard_quantize -- fp4_quantize with a block-diagonal Hadamard
+ * rotation applied along the quantization axis first ("Bridging the Gap",
+ * Abstract: block-wise Hadamard computed online for the activations; its
+ * summary post, item 3: block-diagonal rotations).  Rotation: contiguous
+ * blocks of `had_block` in {16, 32, 64, 128}, Sylvester order, scaled by
+ * 1/sqrt(had_block), in fp32 in registers.  axis = 1 only; cols must be a
+ * multiple of had_block.  rotated_out (nullable) receives the fp32 rotated
+ * values [rows, cols] (row stride cols) for testing.
+ */
+fp4_status fp4_hadamard_quantize(const void* x, int64_t rows, int64_t cols, int64_t ld,
+                                 int fmt, int block, int axis, int rnd, uint64_t seed,
+                                 const float* tensor_scale_in, float* tensor_scale_out,
+                                 uint8_t* codes, uint8_t* scales, int sf_layout,
+                                 int had_block, float* rotated_out, void* stream);
+
+/*
+ * fp4_dequantize -- codes + scales (+ s_t) back to floating point
+ * ("FP4 All the Way", Abstract: the E2M1 values times their block scale).
+ * MX: G[c] * 2^(b-127), exact in fp32.  NV: fp32(fp32(G[c] * sb) * s_t).
+ *   codes  uint8 [rows, cols/2] (rows, cols = out_rows, L of the quantizer)
+ *   scales in `sf_layout`; tensor_scale device fp32 (NV), ignored for MX.
+ *   out    fp32 or bf16 (RNE of the fp32 value) [rows, cols], row stride cols.
+ */
+fp4_status fp4_dequantize(const uint8_t* codes, const uint8_t* scales, const float* tensor_scale,
+                          int64_t rows, int64_t cols, int fmt, int block, int sf_layout,
+                          void* out, int out_dtype, void* stream);
+
+/*
+ * fp4_gemm -- block-scaled FP4 x FP4 GEMM with fp32 accumulation on the
+ * tcgen05 tensor cores ("Bridging the Gap", Abstract: FP4 GEMM on B200;
+ * "Oscillation-Reduced MXFP4 Training", Abstract: MX matmuls on Blackwell).
+ *   Y[M,N] = alpha * sum_k a[m,k] * b[n,k],  alpha = 1 (MX) or *a_ts * *b_ts (NV)
+ *   a     uint8 codes [M, K/2] (K-major), a_sf scales in FP4_SF_MMA layout
+ *   b     uint8 codes [N, K/2] (K-major), b_sf scales in FP4_SF_MMA layout
+ *   a_ts, b_ts  device fp32 tensor scales (NV), ignored for MX
+ *   y     fp32 or bf16 [M, N] with row stride ldy elements (ldy >= N)
+ * K must be a multiple of 64 (K/2 bytes a multiple of 32); a, b, a_sf, b_sf
+ * 16-byte aligned; y aligned to its element size (rows whose byte pitch and
+ * base are 16-byte aligned get 128-bit stores); M, N >= 1 arbitrary.  Uses cudaGetDriverEntryPoint once to find
+ * cuTensorMapEncodeTiled.
+ */
+fp4_status fp4_gemm(const uint8_t* a, const uint8_t* a_sf, const float* a_ts,
+                    const uint8_t* b, const uint8_t* b_sf, const float* b_ts,
+                    int64_t M, int64_t N, int64_t K, int fmt, int block,
+                    void* y, int64_t ldy, int y_dtype, void* stream);
+
+/*
+ * fp4_amax -- max |x| over a bf16 matrix into one device fp32 (the first
+ * pass of NVFP4's per-tensor scale, "FP4 All the Way", Abstract).  Used when
+ * a tensor is sharded and the maxima are combined across ranks before
+ * fp4_nv_tensor_scale.  Same x requirements as fp4_quantize.
+ */
+fp4_status fp4_amax(const void* x, int64_t rows, int64_t cols, int64_t ld,
+                    float* amax_out, void* stream);
+
+/* fp4_nv_tensor_scale -- s_t = fp32(amax / 2688), 1.0 for amax == 0, on the
+ * device (one thread).  amax and tensor_scale_out are device fp32 pointers. */
+fp4_status fp4_nv_tensor_scale(const float* amax, float* tensor_scale_out, void* stream);
+
+/* Bytes of packed codes for a [rows, cols] input (either axis). */
+size_t fp4_codes_bytes(int64_t rows, int64_t cols);
+/* Bytes of scales for a [rows, cols] input quantized along `axis`; 0 on bad arguments. */
+size_t fp4_scales_bytes(int64_t rows, int64_t cols, int block, int axis, int sf_layout);
+
+/* Synchronizes `stream`, then reads and clears the device error word that
+ * bounded waits set; returns FP4_ERR_TIMEOUT if any wait expired since the
+ * last check, FP4_ERR_CUDA on a runtime error, else FP4_OK. */
+fp4_status fp4_check_device_errors(void* stream);
+
+/* Static string for a status code. */
+const char* fp4_status_string(fp4_status status);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* FP4_H_ */

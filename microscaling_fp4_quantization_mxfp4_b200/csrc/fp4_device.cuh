@@ -1,0 +1,195 @@
+// Device-side building blocks shared by the quantize, dequantize and GEMM
+// kernels of libfp4 (sm_100a only).
+//
+// Formats follow the OCP MX v1.0 conventions (the pages name E2M1, E8M0-style
+// power-of-two scales for MXFP4 and E4M3 scales for NVFP4 -- "FP4 All the
+// Way", Abstract; "Bridging the Gap ...", Abstract -- but print no encodings).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace fp4dev {
+
+// ---------------------------------------------------------------- bf16 -----
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+__device__ __forceinline__ void unpack8(const uint4& v, float (&x)[8]) {
+  x[0] = bf16_lo(v.x); x[1] = bf16_hi(v.x);
+  x[2] = bf16_lo(v.y); x[3] = bf16_hi(v.y);
+  x[4] = bf16_lo(v.z); x[5] = bf16_hi(v.z);
+  x[6] = bf16_lo(v.w); x[7] = bf16_hi(v.w);
+}
+
+// ------------------------------------------------------------ E2M1 codes ---
+// Hardware conversion: round to nearest even, saturating to +-6, sign kept.
+// Element `a` lands in the low nibble, `b` in the high nibble.
+__device__ __forceinline__ uint32_t e2m1x4_rn(float a0, float b0, float a1, float b1,
+                                              float a2, float b2, float a3, float b3) {
+  uint32_t out;
+  asm("{\n\t.reg .b8 q0, q1, q2, q3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 q0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 q1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 q2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 q3, %8, %7;\n\t"
+      "mov.b32 %0, {q0, q1, q2, q3};\n\t}"
+      : "=r"(out)
+      : "f"(a0), "f"(b0), "f"(a1), "f"(b1), "f"(a2), "f"(b2), "f"(a3), "f"(b3));
+  return out;
+}
+
+// 8 scaled values -> 8 packed RTN nibbles (element 2j low, 2j+1 high).
+__device__ __forceinline__ uint32_t pack8_rtn(const float (&v)[8]) {
+  return e2m1x4_rn(v[0], v[1], v[2], v[3], v[4], v[5], v[6], v[7]);
+}
+
+// Stochastic rounding of one scaled value with a 32-bit random word:
+// lo <= |v| < hi adjacent grid points, p = (|v| - lo) / (hi - lo) (exact in
+// fp32), round up iff r < ceil(p * 2^32); |v| >= 6 gives 6; sign kept.
+__device__ __forceinline__ uint32_t e2m1_sr(float v, uint32_t r) {
+  const float a = fabsf(v);
+  uint32_t code;
+  if (!(a < 6.0f)) {
+    code = 7u;
+  } else {
+    uint32_t lo_code;
+    float lo, inv_w;
+    if (a < 2.0f) {                       // grid 0, .5, 1, 1.5: width 0.5
+      lo_code = (uint32_t)(a * 2.0f);     // exact product, truncation = floor
+      lo = (float)lo_code * 0.5f;
+      inv_w = 2.0f;
+    } else if (a < 4.0f) {                // grid 2, 3: width 1
+      const uint32_t f = (uint32_t)a;     // 2 or 3
+      lo_code = f + 2u;
+      lo = (float)f;
+      inv_w = 1.0f;
+    } else {                              // grid 4 -> 6: width 2
+      lo_code = 6u;
+      lo = 4.0f;
+      inv_w = 0.5f;
+    }
+    const float p = __fmul_rn(__fsub_rn(a, lo), inv_w);            // both steps exact
+    const unsigned long long thr = __float2ull_ru(__fmul_rn(p, 4294967296.0f));
+    code = lo_code + (((unsigned long long)r < thr) ? 1u : 0u);
+  }
+  return code | ((__float_as_uint(v) >> 31) << 3);
+}
+
+// ---------------------------------------------------------------- Philox ----
+// Philox4x32 with 10 rounds (Salmon, Moraes, Dror, Shaw, SC'11): two 32x32
+// multiplies per round with the published multipliers, Weyl key schedule.
+struct u32x4 { uint32_t x, y, z, w; };
+
+__device__ __forceinline__ u32x4 philox4x32_10(uint32_t c0, uint32_t c1, uint32_t k0, uint32_t k1) {
+  uint32_t c2 = 0u, c3 = 0u;
+#pragma unroll
+  for (int i = 0; i < 10; ++i) {
+    const uint32_t p0_lo = 0xD2511F53u * c0, p0_hi = __umulhi(0xD2511F53u, c0);
+    const uint32_t p1_lo = 0xCD9E8D57u * c2, p1_hi = __umulhi(0xCD9E8D57u, c2);
+    const uint32_t n0 = p1_hi ^ c1 ^ k0;
+    const uint32_t n2 = p0_hi ^ c3 ^ k1;
+    c0 = n0; c1 = p1_lo; c2 = n2; c3 = p0_lo;
+    k0 += 0x9E3779B9u;
+    k1 += 0xBB67AE85u;
+  }
+  return {c0, c1, c2, c3};
+}
+
+// Random words for 8 consecutive elements starting at linear index idx0
+// (idx0 % 8 == 0): two counters, words in index order.
+__device__ __forceinline__ void philox_words8(unsigned long long idx0, unsigned long long seed,
+                                              uint32_t (&r)[8]) {
+  const unsigned long long j = idx0 >> 2;
+  const uint32_t k0 = (uint32_t)seed, k1 = (uint32_t)(seed >> 32);
+  const u32x4 a = philox4x32_10((uint32_t)j, (uint32_t)(j >> 32), k0, k1);
+  const u32x4 b = philox4x32_10((uint32_t)(j + 1), (uint32_t)((j + 1) >> 32), k0, k1);
+  r[0] = a.x; r[1] = a.y; r[2] = a.z; r[3] = a.w;
+  r[4] = b.x; r[5] = b.y; r[6] = b.z; r[7] = b.w;
+}
+
+// Random word of one element.
+__device__ __forceinline__ uint32_t philox_word(unsigned long long idx, unsigned long long seed) {
+  const unsigned long long j = idx >> 2;
+  const u32x4 a = philox4x32_10((uint32_t)j, (uint32_t)(j >> 32), (uint32_t)seed, (uint32_t)(seed >> 32));
+  const uint32_t s = (uint32_t)(idx & 3u);
+  return s == 0 ? a.x : (s == 1 ? a.y : (s == 2 ? a.z : a.w));
+}
+
+// ------------------------------------------------------------ MX scales -----
+// E = clamp(floor(log2 amax) - 2, -127, 127); byte = E + 127.  For a finite
+// amax with biased exponent field f, floor(log2 amax) = f - 127 when f > 0,
+// and E clamps to -127 for zero or subnormal amax: byte = max(f - 2, 0).
+__device__ __forceinline__ uint32_t mx_scale_byte(float amax) {
+  const int f = (int)((__float_as_uint(amax) >> 23) & 0xFFu);
+  return (uint32_t)max(f - 2, 0);
+}
+// 2^(127 - byte) = 1 / 2^E as an exact fp32 (byte <= 252 for finite bf16 input).
+__device__ __forceinline__ float mx_inv_scale(uint32_t byte) {
+  return __uint_as_float((254u - byte) << 23);
+}
+// 2^(byte - 127) exactly (byte 0 is the subnormal 2^-127).
+__device__ __forceinline__ float mx_scale_value(uint32_t byte) {
+  return byte == 0u ? __uint_as_float(0x00400000u) : __uint_as_float(byte << 23);
+}
+
+// ------------------------------------------------------------ NV scales -----
+// E4M3 byte of min(t, 448) with round-to-nearest-even and saturation.
+__device__ __forceinline__ uint32_t e4m3_rn_sat(float t) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.0f), "f"(fminf(t, 448.0f)));
+  return (uint32_t)(r & 0xFFu);
+}
+// Value of an E4M3 byte (non-negative; bias 7, subnormals m * 2^-9).
+__device__ __forceinline__ float e4m3_value(uint32_t b) {
+  const uint32_t e = (b >> 3) & 0xFu, m = b & 7u;
+  if (e == 0u) return __fmul_rn((float)m, 0.001953125f);                 // m * 2^-9, exact
+  return __uint_as_float(((e + 120u) << 23) | (m << 20));                // (1 + m/8) * 2^(e-7)
+}
+
+// -------------------------------------------------------- E2M1 decoding -----
+__device__ __forceinline__ float e2m1_value(uint32_t c) {
+  const uint32_t e = (c >> 1) & 3u, m = c & 1u;
+  float mag = (e == 0u) ? (m ? 0.5f : 0.0f) : __uint_as_float(((e + 126u) << 23) | (m << 22));
+  return (c & 8u) ? -mag : mag;
+}
+
+// -------------------------------------------------- scale-factor offsets ----
+// Byte offset of the scale of (row, k-group g) in the tensor-core layout:
+// 128x4 tiles, k-tile index fastest, (r%32)*16 + (r/32)*4 + g inside a tile.
+__device__ __forceinline__ long long sf_mma_offset(long long row, long long g, long long g4) {
+  return (((row >> 7) * g4 + (g >> 2)) << 9) + ((row & 31) << 4) + (((row >> 5) & 3) << 2) + (g & 3);
+}
+
+// ------------------------------------------------------ Hadamard (fp32) -----
+// In-register fast Walsh-Hadamard transform of a contiguous block of HB
+// elements held 8 per lane by HB/8 consecutive lanes (Sylvester order:
+// pairs (i, i + 2^s) -> (a + b, a - b)), then scaled by 1/sqrt(HB).
+template <int HB>
+__device__ __forceinline__ void hadamard_rotate(float (&x)[8], int lane) {
+#pragma unroll
+  for (int d = 1; d < 8; d <<= 1) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      if ((i & d) == 0) {
+        const float a = x[i], b = x[i + d];
+        x[i] = __fadd_rn(a, b);
+        x[i + d] = __fsub_rn(a, b);
+      }
+    }
+  }
+#pragma unroll
+  for (int ld = 1; ld < HB / 8; ld <<= 1) {
+    const bool upper = (lane & ld) != 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float p = __shfl_xor_sync(0xFFFFFFFFu, x[i], ld);
+      x[i] = upper ? __fsub_rn(p, x[i]) : __fadd_rn(x[i], p);
+    }
+  }
+  const float s = HB == 16 ? 0.25f : HB == 32 ? 0.17677669529663687f : HB == 64 ? 0.125f : 0.08838834764831845f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) x[i] = __fmul_rn(x[i], s);
+}
+
+}  // namespace fp4dev

@@ -1,0 +1,69 @@
+// Host-side internal interface between the C-ABI layer (api.cu) and the
+// kernel launchers (quantize.cu, gemm.cu).  Not part of the public ABI.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace fp4lib {
+
+enum { FMT_MX = 0, FMT_NV = 1 };
+enum { RND_RTN = 0, RND_SR = 1 };
+
+// Per-device scratch owned by the library (allocated once per device).
+struct Scratch {
+  float* partials;      // per-CTA maxima of the tensor-amax pass
+  unsigned* counter;    // CTA ticket counter of the amax pass (self-resetting)
+  unsigned* error;      // device error word set by bounded waits
+};
+constexpr int kMaxAmaxBlocks = 2048;
+
+// Unsigned 32-bit division by a runtime constant (round-up multiplier method,
+// Hacker's Delight ch. 10): q = (umulhi(n, mul) + n) >> shift for n < 2^32.
+struct FastDiv {
+  uint32_t d, mul, shift;
+};
+FastDiv make_fastdiv(uint32_t d);
+
+struct QuantizeParams {
+  const void* x;
+  int64_t rows, cols, ld;
+  int fmt, axis, rnd;
+  uint64_t seed;
+  const float* ts;        // s_t the kernel reads (NV): caller's or the amax pass output
+  float* ts_copy_out;     // if non-null and != ts, block 0 writes s_t here
+  uint8_t* codes;
+  uint8_t* scales;
+  int sf_mma;
+  int had;                // 0 or Hadamard block size
+  float* rotated;         // optional fp32 dump of the rotated input
+};
+
+// amax pass: mode 0 writes max|x| (after rotation when had > 0) to `out`,
+// mode 1 writes s_t = amax / 2688 (1.0 for amax == 0).
+cudaError_t launch_amax(const void* x, int64_t rows, int64_t cols, int64_t ld, int had, int mode,
+                        float* out, const Scratch& s, int num_sms, cudaStream_t st);
+cudaError_t launch_nv_tensor_scale(const float* amax, float* out, cudaStream_t st);
+cudaError_t launch_quantize(const QuantizeParams& p, int num_sms, cudaStream_t st);
+cudaError_t launch_dequantize(const uint8_t* codes, const uint8_t* scales, const float* ts, int64_t rows,
+                              int64_t cols, int fmt, int sf_mma, void* out, int out_bf16, int num_sms,
+                              cudaStream_t st);
+
+struct GemmParams {
+  const uint8_t* a;
+  const uint8_t* a_sf;
+  const float* a_ts;
+  const uint8_t* b;
+  const uint8_t* b_sf;
+  const float* b_ts;
+  int64_t M, N, K;
+  int fmt;
+  void* y;
+  int64_t ldy;
+  int y_bf16;
+  unsigned* error;
+};
+// Returns cudaErrorNotSupported if the driver entry point for tensor maps is missing.
+cudaError_t launch_gemm(const GemmParams& p, int num_sms, cudaStream_t st);
+
+}  // namespace fp4lib

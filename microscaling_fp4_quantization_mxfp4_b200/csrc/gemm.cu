@@ -1,0 +1,531 @@
+// Block-scaled FP4 x FP4 GEMM with fp32 accumulation on the sm_100a tensor
+// cores (tcgen05), fed by TMA.
+//
+// Method: "Bridging the Gap Between Promise and Performance for Microscaling
+// FP4 Quantization", Abstract (FP4 GEMM kernels on B200 for MXFP4/NVFP4);
+// "Oscillation-Reduced MXFP4 Training for Vision Transformers", Abstract (MX
+// matmuls on Blackwell).  Y[M,N] = alpha * sum_k (cA*sA)(cB*sB), both operands
+// K-major ("TN"); the quantizer writes its scale bytes straight into the
+// tensor-core scale layout, so nothing is reshuffled here.
+//
+// Design (one CTA per SM, persistent over 128 x BN output tiles):
+//   warp 0      TMA producer: A/B code tiles (128-byte rows, 128B swizzle) and
+//               the scale-factor atoms (plain bulk copies) into a STAGES-deep
+//               shared-memory ring guarded by full/empty mbarriers.
+//   warp 1      allocates tensor memory; one thread copies each stage's scale
+//               factors to tensor memory (tcgen05.cp 32x128b.warpx4) and
+//               issues 4 block-scaled MMAs (K = 64 each) per 256-wide k-tile,
+//               committing to the stage's empty barrier.
+//   warps 2..5  epilogue: tcgen05.ld the fp32 accumulator (two accumulator
+//               buffers in tensor memory so the next tile's MMAs overlap the
+//               stores), multiply by alpha, store fp32 or bf16.
+// Every mbarrier wait is bounded; on expiry the CTA raises a shared abort
+// flag and a device error word, drains its own copies and MMAs, frees tensor
+// memory and returns.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+#include <stdint.h>
+
+#include <mutex>
+
+#include "fp4_internal.h"
+
+namespace fp4lib {
+namespace {
+
+constexpr int BM = 128;
+constexpr int BK = 256;               // fp4 elements per k-tile (128 bytes per row)
+constexpr int BK_BYTES = BK / 2;
+constexpr int kThreads = 192;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kSfaCol = 256;
+constexpr uint32_t kSfbCol = 288;
+constexpr unsigned long long kWaitLimitNs = 4000000000ull;   // 4 s per wait
+
+template <int FMT>
+struct FmtTraits {
+  static constexpr int kBlock = FMT == FMT_MX ? 32 : 16;
+  static constexpr int kAtomsPerKTile = BK / kBlock / 4;     // 128x4 scale atoms per 128 rows per k-tile
+};
+
+template <int BN, int FMT>
+struct Cfg {
+  static constexpr int kAccStages = BN == 128 ? 2 : 1;
+  static constexpr int kApk = FmtTraits<FMT>::kAtomsPerKTile;
+  static constexpr int kABytes = BM * BK_BYTES;
+  static constexpr int kBBytes = BN * BK_BYTES;
+  static constexpr int kSfaBytes = kApk * 512;
+  static constexpr int kSfbBytes = (BN / 128) * kApk * 512;
+  static constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;
+  static constexpr int kStages = (220 * 1024) / kStageBytes > 8 ? 8 : (220 * 1024) / kStageBytes;
+  static constexpr int kBarrierBytes = 1024;
+  static constexpr int kSmemBytes = 1024 /*alignment slack*/ + kStages * kStageBytes + kBarrierBytes;
+};
+
+// ------------------------------------------------------------ PTX wrappers --
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0u;
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ uint64_t global_timer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+// Bounded wait: false when the time limit passes or another role raised abort.
+__device__ __noinline__ bool wait_bounded(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 255u) == 0u) {
+      if (*abort_flag != 0) return false;
+      if (global_timer() - t0 > kWaitLimitNs) return false;
+    }
+  }
+}
+__device__ __forceinline__ void raise_abort(volatile int* abort_flag, unsigned* error) {
+  *abort_flag = 1;
+  atomicOr(error, 1u);
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::
+          "r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(src), "r"(bytes), "r"(bar)
+               : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void tc_cp_sf(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+template <int FMT>
+__device__ __forceinline__ void tc_mma(uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t sfa,
+                                       uint32_t sfb, uint32_t accumulate) {
+  if (FMT == FMT_MX) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.scale_vec::2X [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+        : "memory");
+  } else {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.scale_vec::4X [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
+            d),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+        : "memory");
+  }
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]),
+        "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor: K-major operand, 128-byte rows, 128B
+// swizzle, 8-row groups 1024 bytes apart (Blackwell descriptor version 1).
+__device__ __forceinline__ uint64_t desc_sw128(uint32_t addr) {
+  return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)1u << 16) | ((uint64_t)(1024u >> 4) << 32) |
+         ((uint64_t)1u << 46) | ((uint64_t)2u << 61);
+}
+// Descriptor of one 512-byte scale atom: 32 rows of 16 bytes, no swizzle,
+// 8-row core matrices 128 bytes apart.
+__device__ __forceinline__ uint64_t desc_sf(uint32_t addr) {
+  return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)1u << 16) | ((uint64_t)(128u >> 4) << 32) |
+         ((uint64_t)1u << 46);
+}
+
+// Instruction descriptor of the block-scaled MMA: E2M1 x E2M1, K-major
+// operands, M = 128, N = BN, scale format UE8M0 (MX) or UE4M3 (NV).
+template <int BN, int FMT>
+__device__ __forceinline__ uint32_t idesc_base() {
+  return (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | ((FMT == FMT_MX ? 1u : 0u) << 23) |
+         ((uint32_t)(BM >> 4) << 24);
+}
+
+struct KernelArgs {
+  const uint8_t* a_sf;
+  const uint8_t* b_sf;
+  const float* a_ts;
+  const float* b_ts;
+  void* y;
+  int64_t ldy;
+  int M, N, K;
+  int num_m, num_n;
+  int g4;                 // padded k-groups / 4 of both scale tensors
+  int vec_store;          // output rows 16-byte aligned: 128-bit stores
+  unsigned* error;
+};
+
+__device__ __forceinline__ void tile_coords(int t, int num_m, int num_n, int& mt, int& nt) {
+  constexpr int kGroup = 8;
+  const int band = t / (kGroup * num_n);
+  const int first = band * kGroup;
+  const int gsize = min(kGroup, num_m - first);
+  const int local = t - band * kGroup * num_n;
+  mt = first + local % gsize;
+  nt = local / gsize;
+}
+
+template <int BN, int FMT, bool BF16>
+__global__ void __launch_bounds__(kThreads, 1)
+    fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
+                    KernelArgs p) {
+  using C = Cfg<BN, FMT>;
+  constexpr int S = C::kStages;
+  constexpr int APK = C::kApk;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = sA + S * C::kABytes;
+  uint8_t* sSFA = sB + S * C::kBBytes;
+  uint8_t* sSFB = sSFA + S * C::kSfaBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sSFB + S * C::kSfbBytes);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + S;
+  uint64_t* tfull = bars + 2 * S;
+  uint64_t* tempty = bars + 2 * S + 2;
+  uint64_t* drain = bars + 2 * S + 4;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 5);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(smem_u32(&full[s]), 1);
+      mbar_init(smem_u32(&empty[s]), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(smem_u32(&tfull[a]), 1);
+      mbar_init(smem_u32(&tempty[a]), 4);
+    }
+    mbar_init(smem_u32(drain), 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  const int num_tiles = p.num_m * p.num_n;
+  const int nkb = (p.K + BK - 1) / BK;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer --
+    if (lane == 0) {
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_a)) : "memory");
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_b)) : "memory");
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued = 0, issued_parity = 0;   // per-stage bits: ever issued / parity of the last issue
+      const int rb_total = (p.N + 127) / 128;
+      bool ok = true;
+      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+        int mt, nt;
+        tile_coords(t, p.num_m, p.num_n, mt, nt);
+        const int rb_here = min(BN / 128, rb_total - nt * (BN / 128));
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!wait_bounded(smem_u32(&empty[stage]), phase ^ 1u, abort_flag)) {
+            raise_abort(abort_flag, p.error);
+            ok = false;
+            break;
+          }
+          const int kvalid = min(BK, p.K - kb * BK);
+          const int atoms = (kvalid / FmtTraits<FMT>::kBlock + 3) / 4;
+          const uint32_t fb = smem_u32(&full[stage]);
+          mbar_expect_tx(fb, (uint32_t)(C::kABytes + C::kBBytes + atoms * 512 * (1 + rb_here)));
+          tma_load_2d(smem_u32(sA + stage * C::kABytes), &tmap_a, kb * BK_BYTES, mt * BM, fb);
+          tma_load_2d(smem_u32(sB + stage * C::kBBytes), &tmap_b, kb * BK_BYTES, nt * BN, fb);
+          bulk_load(smem_u32(sSFA + stage * C::kSfaBytes),
+                    p.a_sf + ((size_t)mt * p.g4 + (size_t)kb * APK) * 512, (uint32_t)atoms * 512u, fb);
+          for (int rb = 0; rb < rb_here; ++rb)
+            bulk_load(smem_u32(sSFB + stage * C::kSfbBytes + rb * APK * 512),
+                      p.b_sf + ((size_t)(nt * (BN / 128) + rb) * p.g4 + (size_t)kb * APK) * 512,
+                      (uint32_t)atoms * 512u, fb);
+          issued |= 1u << stage;
+          issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok) {
+        // let every copy already issued land before the CTA can exit
+        for (int s = 0; s < S; ++s)
+          if (issued & (1u << s)) {
+            volatile int never = 0;
+            wait_bounded(smem_u32(&full[s]), (issued_parity >> s) & 1u, &never);
+          }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer --
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int local = 0;
+      bool ok = true;
+      bool any_mma = false;
+      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x, ++local) {
+        int mt, nt;
+        tile_coords(t, p.num_m, p.num_n, mt, nt);
+        (void)mt;
+        const int acc = local % C::kAccStages;
+        const uint32_t use = (uint32_t)(local / C::kAccStages);
+        if (!wait_bounded(smem_u32(&tempty[acc]), (use & 1u) ^ 1u, abort_flag)) {
+          raise_abort(abort_flag, p.error);
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem + (uint32_t)(acc * BN);
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!wait_bounded(smem_u32(&full[stage]), phase, abort_flag)) {
+            raise_abort(abort_flag, p.error);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const int kvalid = min(BK, p.K - kb * BK);
+          const int atoms = (kvalid / FmtTraits<FMT>::kBlock + 3) / 4;
+          for (int i = 0; i < atoms; ++i) {
+            tc_cp_sf(tmem + kSfaCol + 4u * i, desc_sf(smem_u32(sSFA + stage * C::kSfaBytes + i * 512)));
+            for (int rb = 0; rb < BN / 128; ++rb)
+              tc_cp_sf(tmem + kSfbCol + 4u * (i * (BN / 128) + rb),
+                       desc_sf(smem_u32(sSFB + stage * C::kSfbBytes + (rb * APK + i) * 512)));
+          }
+          const uint64_t adesc = desc_sw128(smem_u32(sA + stage * C::kABytes));
+          const uint64_t bdesc = desc_sw128(smem_u32(sB + stage * C::kBBytes));
+          const int nmma = kvalid / 64;
+          for (int j = 0; j < nmma; ++j) {
+            uint32_t chunk, sf_id;
+            if (FMT == FMT_MX) {      // 2 scales per row per MMA: k-groups 2j, 2j+1
+              chunk = (uint32_t)(j >> 1);
+              sf_id = (uint32_t)((j & 1) * 2);
+            } else {                  // 4 scales per row per MMA
+              chunk = (uint32_t)j;
+              sf_id = 0u;
+            }
+            const uint32_t idesc = idesc_base<BN, FMT>() | (sf_id << 29) | (sf_id << 4);
+            tc_mma<FMT>(d_tmem, adesc + (uint64_t)(2 * j), bdesc + (uint64_t)(2 * j), idesc,
+                        tmem + kSfaCol + 4u * chunk, tmem + kSfbCol + 4u * chunk * (BN / 128),
+                        (kb > 0 || j > 0) ? 1u : 0u);
+            any_mma = true;
+          }
+          tc_commit(smem_u32(&empty[stage]));
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        tc_commit(smem_u32(&tfull[acc]));
+      }
+      if (!ok && any_mma) {
+        // wait for the MMAs already issued before tensor memory is released
+        tc_commit(smem_u32(drain));
+        volatile int never = 0;
+        wait_bounded(smem_u32(drain), 0u, &never);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue --
+    const int q = warp & 3;                  // tensor-memory lane quadrant of this warp
+    const int row_in_tile = q * 32 + lane;
+    const float alpha = FMT == FMT_NV ? __fmul_rn(*p.a_ts, *p.b_ts) : 1.0f;
+    int local = 0;
+    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++local) {
+      int mt, nt;
+      tile_coords(t, p.num_m, p.num_n, mt, nt);
+      const int acc = local % C::kAccStages;
+      const uint32_t use = (uint32_t)(local / C::kAccStages);
+      int ok = 1;
+      if (lane == 0) ok = wait_bounded(smem_u32(&tfull[acc]), use & 1u, abort_flag) ? 1 : 0;
+      ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+      if (!ok) {
+        if (lane == 0) raise_abort(abort_flag, p.error);
+        break;
+      }
+      tc_fence_after();
+      const int m = mt * BM + row_in_tile;
+      const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
+#pragma unroll 1
+      for (int c0 = 0; c0 < BN; c0 += 32) {
+        uint32_t r[32];
+        tmem_ld32(tbase + (uint32_t)c0, r);
+        if (c0 + 32 == BN) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(smem_u32(&tempty[acc]));
+        }
+        const int n0 = nt * BN + c0;
+        if (m < p.M && n0 < p.N) {
+          if (BF16) {
+            __nv_bfloat16* yr = reinterpret_cast<__nv_bfloat16*>(p.y) + (size_t)m * p.ldy + n0;
+            if (p.vec_store && n0 + 32 <= p.N) {
+#pragma unroll
+              for (int v = 0; v < 4; ++v) {
+                uint32_t w[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                  const float lo = __fmul_rn(__uint_as_float(r[8 * v + 2 * i]), alpha);
+                  const float hi = __fmul_rn(__uint_as_float(r[8 * v + 2 * i + 1]), alpha);
+                  w[i] = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(lo)) |
+                         ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(hi)) << 16);
+                }
+                reinterpret_cast<uint4*>(yr)[v] = make_uint4(w[0], w[1], w[2], w[3]);
+              }
+            } else {
+#pragma unroll
+              for (int i = 0; i < 32; ++i)
+                if (n0 + i < p.N) yr[i] = __float2bfloat16_rn(__fmul_rn(__uint_as_float(r[i]), alpha));
+            }
+          } else {
+            float* yr = reinterpret_cast<float*>(p.y) + (size_t)m * p.ldy + n0;
+            if (p.vec_store && n0 + 32 <= p.N) {
+#pragma unroll
+              for (int v = 0; v < 8; ++v)
+                reinterpret_cast<float4*>(yr)[v] =
+                    make_float4(__fmul_rn(__uint_as_float(r[4 * v]), alpha), __fmul_rn(__uint_as_float(r[4 * v + 1]), alpha),
+                                __fmul_rn(__uint_as_float(r[4 * v + 2]), alpha), __fmul_rn(__uint_as_float(r[4 * v + 3]), alpha));
+            } else {
+#pragma unroll
+              for (int i = 0; i < 32; ++i)
+                if (n0 + i < p.N) yr[i] = __fmul_rn(__uint_as_float(r[i]), alpha);
+            }
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
+  }
+}
+
+// ------------------------------------------------------------------ host ---
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  return g_encode;
+}
+
+// 2-D uint8 view [rows, K/2] of packed codes, box 128 bytes x box_rows, 128B swizzle.
+bool make_code_map(CUtensorMap* map, const uint8_t* base, int64_t rows, int64_t kbytes, int box_rows) {
+  auto enc = encode_fn();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)kbytes, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)kbytes};
+  cuuint32_t box[2] = {(cuuint32_t)BK_BYTES, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int BN, int FMT, bool BF16>
+cudaError_t run(const GemmParams& gp, int num_sms, cudaStream_t st) {
+  using C = Cfg<BN, FMT>;
+  static_assert(C::kStages >= 2, "shared memory too small for two stages");
+  static const cudaError_t attr = cudaFuncSetAttribute(fp4_gemm_kernel<BN, FMT, BF16>,
+                                                       cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+  if (attr != cudaSuccess) return attr;
+  CUtensorMap ta, tb;
+  if (!make_code_map(&ta, gp.a, gp.M, gp.K / 2, BM)) return cudaErrorNotSupported;
+  if (!make_code_map(&tb, gp.b, gp.N, gp.K / 2, BN)) return cudaErrorNotSupported;
+  KernelArgs ka;
+  ka.a_sf = gp.a_sf;
+  ka.b_sf = gp.b_sf;
+  ka.a_ts = gp.a_ts;
+  ka.b_ts = gp.b_ts;
+  ka.y = gp.y;
+  ka.ldy = gp.ldy;
+  ka.M = (int)gp.M;
+  ka.N = (int)gp.N;
+  ka.K = (int)gp.K;
+  ka.num_m = (int)((gp.M + BM - 1) / BM);
+  ka.num_n = (int)((gp.N + BN - 1) / BN);
+  ka.g4 = (int)((gp.K / FmtTraits<FMT>::kBlock + 3) / 4);
+  ka.error = gp.error;
+  {
+    const int64_t esz = gp.y_bf16 ? 2 : 4;
+    ka.vec_store = ((gp.ldy * esz) % 16 == 0 && (reinterpret_cast<uintptr_t>(gp.y) & 15u) == 0) ? 1 : 0;
+  }
+  const int tiles = ka.num_m * ka.num_n;
+  const int grid = tiles < num_sms ? tiles : num_sms;
+  fp4_gemm_kernel<BN, FMT, BF16><<<grid, kThreads, C::kSmemBytes, st>>>(ta, tb, ka);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_gemm(const GemmParams& p, int num_sms, cudaStream_t st) {
+  if (p.fmt == FMT_MX) return p.y_bf16 ? run<128, FMT_MX, true>(p, num_sms, st) : run<128, FMT_MX, false>(p, num_sms, st);
+  return p.y_bf16 ? run<128, FMT_NV, true>(p, num_sms, st) : run<128, FMT_NV, false>(p, num_sms, st);
+}
+
+}  // namespace fp4lib

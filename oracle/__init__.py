@@ -36,14 +36,14 @@ from .formats import (E2M1_GRID, e2m1_decode, e2m1_rtn, e2m1_sr, e4m3_decode, e4
                       mx_scale_exponent)
 from .philox import philox4x32_10, philox_words
 from .hadamard import sylvester, block_hadamard
-from .quantize import quantize, dequantize, pack_nibbles, unpack_nibbles, nv_tensor_scale
+from .quantize import quantize, quantize_values, dequantize, pack_nibbles, unpack_nibbles, nv_tensor_scale
 from .layout import sf_to_mma, sf_from_mma, sf_mma_bytes
 from .gemm import gemm_ref, gemm_ref_rows, gemm_ref_cols, deq_for_gemm
 
 __all__ = [
     "E2M1_GRID", "e2m1_decode", "e2m1_rtn", "e2m1_sr", "e4m3_decode", "e4m3_rne_sat",
     "mx_scale_exponent", "philox4x32_10", "philox_words", "sylvester", "block_hadamard",
-    "quantize", "dequantize", "pack_nibbles", "unpack_nibbles", "nv_tensor_scale",
+    "quantize", "quantize_values", "dequantize", "pack_nibbles", "unpack_nibbles", "nv_tensor_scale",
     "sf_to_mma", "sf_from_mma", "sf_mma_bytes", "gemm_ref", "gemm_ref_rows", "gemm_ref_cols",
     "deq_for_gemm",
 ]

@@ -82,7 +82,9 @@ def e2m1_sr(v, r) -> np.ndarray:
     lo = E2M1_GRID[lo_i].astype(np.float32)
     hi = E2M1_GRID[hi_i].astype(np.float32)
     width = np.where(sat, np.float32(1.0), hi - lo).astype(np.float32)
-    p = ((a - lo) / width).astype(np.float32)                       # fp32, exact
+    with np.errstate(invalid="ignore"):
+        p = ((a - lo) / width).astype(np.float32)                   # fp32, exact
+        p = np.where(np.isfinite(p), p, np.float32(0))              # non-finite v: saturated above
     thr = np.ceil(p.astype(np.float64) * 2.0 ** 32).astype(np.uint64)  # p*2^32 exact in fp64
     up = (r < thr) & ~sat
     mag_code = np.where(sat, 7, np.where(up, hi_i, lo_i)).astype(np.uint8)

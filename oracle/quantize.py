@@ -97,8 +97,36 @@ def _quantize_rows(xw: np.ndarray, idxw: np.ndarray, fmt: str, bs: int, rnd: str
     return codes.reshape(n, L), scale_bytes
 
 
+def quantize_values(x32, fmt: str = "mxfp4", block: int | None = None, axis: int = 1, rnd: str = "rtn",
+                    seed: int = 0, tensor_scale=None, idx_base: int = 0, idx_cols: int | None = None):
+    """Steps 2-7 on fp32 values x32 [rows, cols] (already widened/rotated).
+
+    The Philox index of element (r, c) is idx_base + r * idx_cols + c (idx_cols
+    defaults to cols), so a row slice of a larger tensor can be quantized with
+    its global indices.  For NVFP4 without `tensor_scale`, s_t comes from x32.
+    """
+    bs = block or FMT_BLOCK[fmt]
+    if (fmt, bs) not in (("mxfp4", 32), ("nvfp4", 16)):
+        raise ValueError("supported: (mxfp4, 32), (nvfp4, 16)")
+    x = np.asarray(x32, dtype=np.float32)
+    R, C = x.shape
+    ic = C if idx_cols is None else idx_cols
+    idx = (np.int64(idx_base) + np.arange(R, dtype=np.int64)[:, None] * ic
+           + np.arange(C, dtype=np.int64)[None, :])
+    xw, idxw = (x, idx) if axis == 1 else (x.T, idx.T)
+    if xw.shape[1] % bs:
+        raise ValueError("quantization axis length must be a multiple of the block size")
+    s_t = None
+    if fmt == "nvfp4":
+        s_t = np.float32(tensor_scale) if tensor_scale is not None else nv_tensor_scale(x)
+    codes, scales = _quantize_rows(np.ascontiguousarray(xw), np.ascontiguousarray(idxw),
+                                   fmt, bs, rnd, seed, s_t)
+    return {"codes": pack_nibbles(codes), "scales": scales, "tensor_scale": s_t}
+
+
 def quantize(x_bits, fmt: str = "mxfp4", block: int | None = None, axis: int = 1,
-             rnd: str = "rtn", seed: int = 0, tensor_scale=None, had_block: int | None = None):
+             rnd: str = "rtn", seed: int = 0, tensor_scale=None, had_block: int | None = None,
+             idx_base: int = 0, idx_cols: int | None = None):
     """Quantize a bf16 tensor (given as uint16 bit patterns, [rows, cols]).
 
     Returns a dict with
@@ -108,26 +136,14 @@ def quantize(x_bits, fmt: str = "mxfp4", block: int | None = None, axis: int = 1
       tensor_scale np.float32 s_t (NV) or None (MX),
       rotated      fp32 [rows, cols] rotated input (only when had_block is given).
     """
-    bs = block or FMT_BLOCK[fmt]
-    if (fmt, bs) not in (("mxfp4", 32), ("nvfp4", 16)):
-        raise ValueError("supported: (mxfp4, 32), (nvfp4, 16)")
     x = _bf16_to_f32(x_bits)
-    R, C = x.shape
-    idx = np.arange(R * C, dtype=np.int64).reshape(R, C)
     rotated = None
     if had_block:
         x = block_hadamard(x.astype(np.float64), had_block, axis=axis).astype(np.float32)
         rotated = x
-    xw, idxw = (x, idx) if axis == 1 else (x.T, idx.T)
-    if xw.shape[1] % bs:
-        raise ValueError("quantization axis length must be a multiple of the block size")
-    s_t = None
-    if fmt == "nvfp4":
-        s_t = np.float32(tensor_scale) if tensor_scale is not None else nv_tensor_scale(x)
-    codes, scales = _quantize_rows(np.ascontiguousarray(xw), np.ascontiguousarray(idxw),
-                                   fmt, bs, rnd, seed, s_t)
-    return {"codes": pack_nibbles(codes), "scales": scales, "tensor_scale": s_t,
-            "rotated": rotated}
+    out = quantize_values(x, fmt, block, axis, rnd, seed, tensor_scale, idx_base, idx_cols)
+    out["rotated"] = rotated
+    return out
 
 
 def dequantize(codes_packed, scales, fmt: str = "mxfp4", block: int | None = None,

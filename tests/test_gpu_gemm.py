@@ -1,0 +1,154 @@
+"""GPU parity: the tcgen05 block-scaled FP4 GEMM through the C ABI against the
+oracle's fp64 reference: |dY| <= 1e-5 * sum_k |alpha a b| per element (fp32
+output); bf16 output = RNE_bf16 of the fp32 output within one bf16 ulp."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import microscaling_fp4_quantization_mxfp4_b200 as F
+from gpu_utils import dev_bf16, host_f32, host_u8
+from workloads import (bf16_to_f32, hadamard_acts, hadamard_weights, mx_linear_128x512, vit_layer,
+                       normal_bf16)
+
+pytestmark = pytest.mark.gpu
+
+TOL = 1e-5
+
+
+def _gpu_quant(x_dev, fmt, axis=1, rnd="rtn", seed=0):
+    return F.fp4_quantize(x_dev, fmt=fmt, axis=axis, rnd=rnd, seed=seed, sf_layout="mma")
+
+
+def _as_oracle(q, fmt, rows, k):
+    """GPU quantizer output -> oracle operand dict (scales read back from the tensor-core layout)."""
+    bs = 32 if fmt == "mxfp4" else 16
+    d = {"codes": host_u8(q.codes), "scales": O.sf_from_mma(host_u8(q.scales), rows, k // bs)}
+    d["tensor_scale"] = None if q.tensor_scale is None else host_f32(q.tensor_scale)[0]
+    return d
+
+
+def _check(y_gpu, y_ref, bound):
+    err = np.abs(y_gpu.astype(np.float64) - y_ref)
+    bad = err > TOL * bound
+    assert not bad.any(), f"{bad.sum()} elements out of tolerance; worst ratio {np.max(err / np.maximum(bound, 1e-300))}"
+
+
+def _bf16_ulp_check(y_bf16, y_f32):
+    want = y_f32.astype(np.float32)
+    got = y_bf16.float().cpu().numpy().astype(np.float64)
+    ref = torch.from_numpy(want).to(torch.bfloat16).float().numpy().astype(np.float64)
+    ulp = np.abs(np.spacing(ref.astype(np.float32)).astype(np.float64)) * 2 ** 16   # bf16 ulp at ref
+    assert np.all(np.abs(got - ref) <= ulp + 1e-45)
+
+
+def test_mx_linear_128x512():
+    """X[128,512] ~ N(0,1), W[512,512] ~ N(0,0.02), MXFP4 RTN along K, Y = deq(X) deq(W)^T in fp32."""
+    xb, wb = mx_linear_128x512(0)
+    qx, qw = _gpu_quant(dev_bf16(xb), "mxfp4"), _gpu_quant(dev_bf16(wb), "mxfp4")
+    y = F.fp4_gemm(qx.codes, qx.scales, qw.codes, qw.scales, fmt="mxfp4", out_dtype="f32")
+    ox = O.quantize(xb, fmt="mxfp4")
+    ow = O.quantize(wb, fmt="mxfp4")
+    # the GPU operands equal the oracle's (quantize parity), so the reference uses the oracle's
+    np.testing.assert_array_equal(_as_oracle(qx, "mxfp4", 128, 512)["codes"], ox["codes"])
+    yr, bd = O.gemm_ref(ox, ow, "mxfp4")
+    _check(host_f32(y), yr, bd)
+
+
+SHAPES = [(128, 128, 256), (200, 300, 512), (1, 256, 4096), (16, 512, 320), (257, 129, 576), (384, 1024, 1024)]
+
+
+@pytest.mark.parametrize("fmt", ["mxfp4", "nvfp4"])
+@pytest.mark.parametrize("mnk", SHAPES)
+def test_gemm_shapes(mnk, fmt):
+    M, N, K = mnk
+    g = np.random.default_rng(M * 31 + N * 7 + K)
+    from workloads import bf16_bits
+    a = bf16_bits(g.standard_normal((M, K)).astype(np.float32))
+    b = bf16_bits((g.standard_normal((N, K)) * 0.02).astype(np.float32))
+    qa, qb = _gpu_quant(dev_bf16(a), fmt), _gpu_quant(dev_bf16(b), fmt)
+    y32 = F.fp4_gemm(qa.codes, qa.scales, qb.codes, qb.scales, fmt=fmt, a_tensor_scale=qa.tensor_scale,
+                     b_tensor_scale=qb.tensor_scale, out_dtype="f32")
+    y16 = F.fp4_gemm(qa.codes, qa.scales, qb.codes, qb.scales, fmt=fmt, a_tensor_scale=qa.tensor_scale,
+                     b_tensor_scale=qb.tensor_scale, out_dtype="bf16")
+    yr, bd = O.gemm_ref(_as_oracle(qa, fmt, M, K), _as_oracle(qb, fmt, N, K), fmt)
+    got = host_f32(y32)
+    _check(got, yr, bd)
+    _bf16_ulp_check(y16, got)
+    F.fp4_check_device_errors()
+
+
+def test_gemm_strided_output():
+    M, N, K = 64, 96, 256
+    g = np.random.default_rng(1)
+    from workloads import bf16_bits
+    a = bf16_bits(g.standard_normal((M, K)).astype(np.float32))
+    b = bf16_bits(g.standard_normal((N, K)).astype(np.float32))
+    qa, qb = _gpu_quant(dev_bf16(a), "mxfp4"), _gpu_quant(dev_bf16(b), "mxfp4")
+    big = torch.full((M, 128), 7.0, dtype=torch.float32, device="cuda")
+    F.fp4_gemm(qa.codes, qa.scales, qb.codes, qb.scales, fmt="mxfp4", out_dtype="f32", out=big[:, :N])
+    yr, bd = O.gemm_ref(_as_oracle(qa, "mxfp4", M, K), _as_oracle(qb, "mxfp4", N, K), "mxfp4")
+    out = host_f32(big)
+    _check(out[:, :N], yr, bd)
+    assert np.all(out[:, N:] == 7.0)          # nothing written past N
+
+
+@pytest.mark.parametrize("had", [16, 128])
+def test_full_size_hadamard_mxfp4_8192x11008x4096(had):
+    """X[8192,4096] N(0,1) with 41 channels x50, rotated online; W[11008,4096] N(0,0.02) rotated
+    and quantized offline; 64 sampled rows and 64 sampled columns of Y checked (fp32 run), bf16 run
+    against the fp32 run."""
+    xb = hadamard_acts(8192, 4096, seed=2)
+    wb = hadamard_weights(11008, 4096, seed=2)
+    qw = F.fp4_hadamard_quantize(dev_bf16(wb), had, fmt="mxfp4", sf_layout="mma")   # offline weights
+    qx = F.fp4_hadamard_quantize(dev_bf16(xb), had, fmt="mxfp4", sf_layout="mma")
+    y16 = F.fp4_gemm(qx.codes, qx.scales, qw.codes, qw.scales, fmt="mxfp4", out_dtype="bf16")
+    y32 = F.fp4_gemm(qx.codes, qx.scales, qw.codes, qw.scales, fmt="mxfp4", out_dtype="f32")
+    oa, ob = _as_oracle(qx, "mxfp4", 8192, 4096), _as_oracle(qw, "mxfp4", 11008, 4096)
+    g = np.random.default_rng(had)
+    rows = np.sort(g.choice(8192, 64, replace=False))
+    cols = np.sort(g.choice(11008, 64, replace=False))
+    yr, bd = O.gemm_ref_rows(oa, ob, "mxfp4", rows)
+    full32 = y32[torch.from_numpy(rows).cuda()].float().cpu().numpy()
+    _check(full32, yr, bd)
+    yc, bc = O.gemm_ref_cols(oa, ob, "mxfp4", cols)
+    _check(y32[:, torch.from_numpy(cols).cuda()].float().cpu().numpy(), yc, bc)
+    _bf16_ulp_check(y16[torch.from_numpy(rows).cuda()], full32)
+    F.fp4_check_device_errors()
+
+
+def test_vit_qkv_fwd_dgrad_wgrad_full_size():
+    """ViT-B/16 qkv linear, M = 50432: forward (RTN), dgrad and wgrad with SR-quantized dY,
+    each operand quantized along its own contraction axis (axis 0 = transposed blocks)."""
+    xb, wb, dyb = vit_layer("qkv")
+    M, K = xb.shape
+    N = wb.shape[0]
+    x, w, dy = dev_bf16(xb), dev_bf16(wb), dev_bf16(dyb)
+    g = np.random.default_rng(3)
+    # forward Y = X W^T, contraction K
+    qx, qw = _gpu_quant(x, "mxfp4"), _gpu_quant(w, "mxfp4")
+    y = F.fp4_gemm(qx.codes, qx.scales, qw.codes, qw.scales, fmt="mxfp4", out_dtype="f32")
+    rows = np.sort(g.choice(M, 64, replace=False))
+    yr, bd = O.gemm_ref_rows(_as_oracle(qx, "mxfp4", M, K), _as_oracle(qw, "mxfp4", N, K), "mxfp4", rows)
+    _check(y[torch.from_numpy(rows).cuda()].cpu().numpy(), yr, bd)
+    # dgrad dX = dY W, contraction N: dY along N (SR, seed 3), W along N (axis 0, RTN)
+    qdy = _gpu_quant(dy, "mxfp4", axis=1, rnd="sr", seed=3)
+    qwt = _gpu_quant(w, "mxfp4", axis=0)
+    dx = F.fp4_gemm(qdy.codes, qdy.scales, qwt.codes, qwt.scales, fmt="mxfp4", out_dtype="f32")
+    yr, bd = O.gemm_ref_rows(_as_oracle(qdy, "mxfp4", M, N), _as_oracle(qwt, "mxfp4", K, N), "mxfp4", rows)
+    _check(dx[torch.from_numpy(rows).cuda()].cpu().numpy(), yr, bd)
+    # wgrad dW = dY^T X, contraction M: dY along M (axis 0, SR, seed 4), X along M (axis 0, RTN)
+    qdyt = _gpu_quant(dy, "mxfp4", axis=0, rnd="sr", seed=4)
+    qxt = _gpu_quant(x, "mxfp4", axis=0)
+    dw = F.fp4_gemm(qdyt.codes, qdyt.scales, qxt.codes, qxt.scales, fmt="mxfp4", out_dtype="f32")
+    wrows = np.sort(g.choice(N, 32, replace=False))
+    yr, bd = O.gemm_ref_rows(_as_oracle(qdyt, "mxfp4", N, M), _as_oracle(qxt, "mxfp4", K, M), "mxfp4", wrows)
+    _check(dw[torch.from_numpy(wrows).cuda()].cpu().numpy(), yr, bd)
+    # the SR operands themselves: sampled output rows against the oracle with global Philox indices
+    dy32 = bf16_to_f32(dyb)
+    for c in np.sort(g.choice(N, 8, replace=False)):
+        ref = O.quantize_values(dy32[:, c:c + 1], fmt="mxfp4", axis=0, rnd="sr", seed=4, idx_base=int(c), idx_cols=N)
+        np.testing.assert_array_equal(host_u8(qdyt.codes[c:c + 1]), ref["codes"])
+        np.testing.assert_array_equal(
+            O.sf_from_mma(host_u8(qdyt.scales), N, M // 32)[c:c + 1], ref["scales"])
+    F.fp4_check_device_errors()

@@ -1,0 +1,196 @@
+"""GPU parity: quantize / Hadamard-quantize / dequantize / amax through the C ABI
+against the CPU oracle.  Codes, scales and tensor scales must be bit-exact;
+rotated values within 1e-6 of the block RMS."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import microscaling_fp4_quantization_mxfp4_b200 as F
+from gpu_utils import dev_bf16, host_f32, host_u8, host_bf16_bits, mixed_input
+from workloads import bf16_to_f32, nvfp4_student_t
+
+pytestmark = pytest.mark.gpu
+
+SHAPES_AX1 = [(1, 32), (7, 64), (200, 384), (129, 4096), (33, 1056)]
+SHAPES_AX0 = [(32, 8), (96, 200), (384, 136), (160, 72)]
+
+
+def _check_against_oracle(q, ref, fmt, axis, rows, cols, sf):
+    np.testing.assert_array_equal(host_u8(q.codes), ref["codes"])
+    if sf == "rowmajor":
+        np.testing.assert_array_equal(host_u8(q.scales), ref["scales"])
+    else:
+        np.testing.assert_array_equal(host_u8(q.scales), O.sf_to_mma(ref["scales"]))
+    if fmt == "nvfp4":
+        assert host_f32(q.tensor_scale)[0] == ref["tensor_scale"]
+
+
+@pytest.mark.parametrize("sf", ["rowmajor", "mma"])
+@pytest.mark.parametrize("rnd", ["rtn", "sr"])
+@pytest.mark.parametrize("fmt", ["mxfp4", "nvfp4"])
+@pytest.mark.parametrize("shape", SHAPES_AX1)
+def test_quantize_axis1(shape, fmt, rnd, sf):
+    rows, cols = shape
+    xb = mixed_input(rows, cols, rows * 7 + cols, fmt)
+    q = F.fp4_quantize(dev_bf16(xb), fmt=fmt, axis=1, rnd=rnd, seed=1234567890123, sf_layout=sf)
+    ref = O.quantize(xb, fmt=fmt, axis=1, rnd=rnd, seed=1234567890123)
+    _check_against_oracle(q, ref, fmt, 1, rows, cols, sf)
+
+
+@pytest.mark.parametrize("sf", ["rowmajor", "mma"])
+@pytest.mark.parametrize("rnd", ["rtn", "sr"])
+@pytest.mark.parametrize("fmt", ["mxfp4", "nvfp4"])
+@pytest.mark.parametrize("shape", SHAPES_AX0 + [(48, 24)])
+def test_quantize_axis0(shape, fmt, rnd, sf):
+    rows, cols = shape
+    if rows % (32 if fmt == "mxfp4" else 16):
+        pytest.skip("rows not a multiple of the block")
+    xb = mixed_input(rows, cols, rows * 5 + cols, fmt)
+    q = F.fp4_quantize(dev_bf16(xb), fmt=fmt, axis=0, rnd=rnd, seed=42, sf_layout=sf)
+    ref = O.quantize(xb, fmt=fmt, axis=0, rnd=rnd, seed=42)
+    _check_against_oracle(q, ref, fmt, 0, rows, cols, sf)
+
+
+@pytest.mark.parametrize("axis", [0, 1])
+@pytest.mark.parametrize("fmt", ["mxfp4", "nvfp4"])
+def test_quantize_strided_input(fmt, axis):
+    xb_full = mixed_input(128, 320, 3, fmt)
+    xt = dev_bf16(xb_full)[:, :256]                      # ld = 320 > cols = 256
+    xb = np.ascontiguousarray(xb_full[:, :256])
+    q = F.fp4_quantize(xt, fmt=fmt, axis=axis, rnd="sr", seed=5)
+    ref = O.quantize(xb, fmt=fmt, axis=axis, rnd="sr", seed=5)
+    _check_against_oracle(q, ref, fmt, axis, 128, 256, "rowmajor")
+
+
+def test_nv_tensor_scale_in_and_copy_out():
+    xb = mixed_input(64, 128, 9, "nvfp4")
+    ts = torch.tensor([0.0123], dtype=torch.float32, device="cuda")
+    out = torch.zeros(1, dtype=torch.float32, device="cuda")
+    q = F.fp4_quantize(dev_bf16(xb), fmt="nvfp4", tensor_scale_in=ts, tensor_scale_out=out)
+    ref = O.quantize(xb, fmt="nvfp4", tensor_scale=np.float32(0.0123))
+    np.testing.assert_array_equal(host_u8(q.codes), ref["codes"])
+    np.testing.assert_array_equal(host_u8(q.scales), ref["scales"])
+    assert host_f32(out)[0] == np.float32(0.0123)
+
+
+def test_sr_deterministic_and_seeded():
+    xb = mixed_input(64, 512, 11, "mxfp4")
+    x = dev_bf16(xb)
+    a = F.fp4_quantize(x, fmt="mxfp4", rnd="sr", seed=7)
+    b = F.fp4_quantize(x, fmt="mxfp4", rnd="sr", seed=7)
+    c = F.fp4_quantize(x, fmt="mxfp4", rnd="sr", seed=8)
+    assert torch.equal(a.codes, b.codes)
+    assert not torch.equal(a.codes, c.codes)
+
+
+def test_zero_tensor_nv():
+    x = torch.zeros((16, 64), dtype=torch.bfloat16, device="cuda")
+    q = F.fp4_quantize(x, fmt="nvfp4")
+    assert host_f32(q.tensor_scale)[0] == 1.0
+    assert int(q.codes.sum()) == 0 and int(q.scales.sum()) == 0
+
+
+@pytest.mark.parametrize("out", ["f32", "bf16"])
+@pytest.mark.parametrize("sf", ["rowmajor", "mma"])
+@pytest.mark.parametrize("fmt", ["mxfp4", "nvfp4"])
+def test_dequantize(fmt, sf, out):
+    xb = mixed_input(200, 384, 21, fmt)
+    q = F.fp4_quantize(dev_bf16(xb), fmt=fmt, sf_layout=sf)
+    y = F.fp4_dequantize(q.codes, q.scales, q.tensor_scale, fmt=fmt, sf_layout=sf, out_dtype=out)
+    ref = O.quantize(xb, fmt=fmt)
+    want = O.dequantize(ref["codes"], ref["scales"], fmt=fmt, tensor_scale=ref["tensor_scale"], out=out)
+    if out == "f32":
+        got = host_f32(y)
+        np.testing.assert_array_equal(got.view(np.uint32), want.view(np.uint32))
+    else:
+        np.testing.assert_array_equal(host_bf16_bits(y), want)
+
+
+def test_dequantize_mx_extreme_scales():
+    # every scale byte the quantizer can emit for finite bf16 input, including 2^-127
+    codes = torch.arange(256, dtype=torch.int64).remainder(256).to(torch.uint8).reshape(8, 32).cuda()
+    sc = torch.tensor([[0, 1], [2, 60], [100, 127], [128, 150], [200, 240], [250, 251], [252, 0], [3, 4]],
+                      dtype=torch.uint8, device="cuda")
+    y = F.fp4_dequantize(codes, sc, fmt="mxfp4")
+    want = O.dequantize(host_u8(codes), host_u8(sc), fmt="mxfp4")
+    np.testing.assert_array_equal(host_f32(y).view(np.uint32), want.view(np.uint32))
+
+
+@pytest.mark.parametrize("had", [16, 32, 64, 128])
+@pytest.mark.parametrize("fmt", ["mxfp4", "nvfp4"])
+def test_hadamard_quantize(fmt, had):
+    rows, cols = 96, 1024
+    g = np.random.default_rng(had)
+    x = g.standard_normal((rows, cols)).astype(np.float32)
+    x[:, g.choice(cols, 10, replace=False)] *= 50.0         # outlier channels
+    from workloads import bf16_bits
+    xb = bf16_bits(x)
+    rot = torch.empty((rows, cols), dtype=torch.float32, device="cuda")
+    q = F.fp4_hadamard_quantize(dev_bf16(xb), had, fmt=fmt, rotated_out=rot)
+    ref = O.quantize(xb, fmt=fmt, had_block=had)
+    got_rot = host_f32(rot)
+    # rotated values within 1e-6 of the block RMS
+    rms = np.sqrt(np.mean(ref["rotated"].astype(np.float64).reshape(rows, -1, had) ** 2, axis=2))
+    err = np.abs(got_rot.astype(np.float64) - ref["rotated"]).reshape(rows, -1, had)
+    assert np.all(err <= 1e-6 * rms[..., None] + 1e-30)
+    # the quantizer applied to the GPU's own rotated values is bit-exact
+    ts = None if fmt == "mxfp4" else O.nv_tensor_scale(got_rot)
+    ref_gpu_rot = O.quantize_values(got_rot, fmt=fmt, tensor_scale=ts)
+    np.testing.assert_array_equal(host_u8(q.codes), ref_gpu_rot["codes"])
+    np.testing.assert_array_equal(host_u8(q.scales), ref_gpu_rot["scales"])
+    if fmt == "nvfp4":
+        assert host_f32(q.tensor_scale)[0] == ts
+    # against the oracle's own rotation: at most 1e-4 of codes differ, each by one grid step
+    # (positions on the signed grid -6 .. -0.5, 0, 0.5 .. 6, where +0 and -0 are one point)
+    gc = O.unpack_nibbles(host_u8(q.codes)).astype(np.int64)
+    rc = O.unpack_nibbles(ref["codes"]).astype(np.int64)
+    gpos = np.where(gc & 8, -(gc & 7), gc & 7)
+    rpos = np.where(rc & 8, -(rc & 7), rc & 7)
+    diff = gpos != rpos
+    assert diff.mean() <= 1e-4
+    assert np.all(np.abs(gpos - rpos) <= 1)
+
+
+def test_amax_and_tensor_scale():
+    xb = mixed_input(300, 264, 17, "nvfp4")
+    x = dev_bf16(xb)
+    a = F.fp4_amax(x)
+    want = np.float32(np.max(np.abs(bf16_to_f32(xb))))
+    assert host_f32(a)[0] == want
+    ts = F.fp4_nv_tensor_scale(a)
+    assert host_f32(ts)[0] == O.nv_tensor_scale(bf16_to_f32(xb))
+    z = F.fp4_nv_tensor_scale(torch.zeros(1, device="cuda"))
+    assert host_f32(z)[0] == 1.0
+
+
+@pytest.mark.parametrize("rnd", ["rtn", "sr"])
+def test_full_size_nvfp4_student_t_4096(rnd):
+    """4096 x 4096 0.1*Student-t(3), seed 1: the full quantize+dequantize case, all outputs
+    for RTN; 256 sampled rows (with their global Philox indices) for SR."""
+    xb = nvfp4_student_t(4096, 4096, seed=1)
+    x = dev_bf16(xb)
+    q = F.fp4_quantize(x, fmt="nvfp4", rnd=rnd, seed=1, sf_layout="rowmajor")
+    y = F.fp4_dequantize(q.codes, q.scales, q.tensor_scale, fmt="nvfp4")
+    x32 = bf16_to_f32(xb)
+    s_t = O.nv_tensor_scale(x32)
+    assert host_f32(q.tensor_scale)[0] == s_t
+    if rnd == "rtn":
+        rows = np.arange(4096)
+    else:
+        rows = np.sort(np.random.default_rng(0).choice(4096, 256, replace=False))
+    codes, scales, deq = host_u8(q.codes), host_u8(q.scales), host_f32(y)
+    for r0 in range(0, len(rows), 512):
+        blk = rows[r0:r0 + 512]
+        if rnd == "rtn":
+            ref = O.quantize_values(x32[blk], fmt="nvfp4", rnd=rnd, seed=1, tensor_scale=s_t)
+            np.testing.assert_array_equal(codes[blk], ref["codes"])
+            np.testing.assert_array_equal(scales[blk], ref["scales"])
+        else:
+            for r in blk:
+                ref = O.quantize_values(x32[r:r + 1], fmt="nvfp4", rnd=rnd, seed=1, tensor_scale=s_t,
+                                        idx_base=int(r) * 4096)
+                np.testing.assert_array_equal(codes[r:r + 1], ref["codes"])
+                np.testing.assert_array_equal(scales[r:r + 1], ref["scales"])
+        want = O.dequantize(codes[blk], scales[blk], fmt="nvfp4", tensor_scale=s_t)
+        np.testing.assert_array_equal(deq[blk].view(np.uint32), want.view(np.uint32))
