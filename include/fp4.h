@@ -163,6 +163,29 @@ fp4_status fp4_gemm(const uint8_t* a, const uint8_t* a_sf, const float* a_ts,
 fp4_status fp4_amax(const void* x, int64_t rows, int64_t cols, int64_t ld,
                     float* amax_out, void* stream);
 
+/*
+ * fp4_amax_noalloc -- the same max |x| as fp4_amax, for callers that must not
+ * allocate device memory.  (The pages describe nothing like it; it exists for
+ * deployment.)  Callers that cannot call cudaMalloc include a process whose
+ * caching allocator already owns all free device memory, a latency-critical
+ * path that cannot absorb the synchronization an allocation may cause, and
+ * code running inside an allocator callback, which must not re-enter the CUDA
+ * allocator.  fp4_amax allocates its scratch on first use; this entry point
+ * never calls cudaMalloc, cudaFree or any allocating routine.
+ *   Scratch: a fixed 33,024-byte array inside libfp4 (partial maxima of up to
+ *   8192 CTAs plus a counter), held by every GPU that loads the library until
+ *   the process exits.  One CTA covers 8192 elements, so inputs are limited to
+ *   rows * cols <= 2^26 (67,108,864) elements; larger inputs return
+ *   FP4_ERR_SHAPE.  Other requirements and errors as fp4_amax.
+ *   The first call on each device looks up the array's device address
+ *   (cudaGetSymbolAddress) with that device current; make that first call
+ *   before any stream capture.  Every call resets the counter, and all calls
+ *   share the one array: calls that overlap on the GPU (e.g. on two streams)
+ *   race, so the caller must serialize them.
+ */
+fp4_status fp4_amax_noalloc(const void* x, int64_t rows, int64_t cols, int64_t ld,
+                            float* amax_out, void* stream);
+
 /* fp4_nv_tensor_scale -- s_t = fp32(amax / 2688), 1.0 for amax == 0, on the
  * device (one thread).  amax and tensor_scale_out are device fp32 pointers. */
 fp4_status fp4_nv_tensor_scale(const float* amax, float* tensor_scale_out, void* stream);

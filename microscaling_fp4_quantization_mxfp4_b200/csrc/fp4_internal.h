@@ -43,6 +43,9 @@ struct QuantizeParams {
 // mode 1 writes s_t = amax / 2688 (1.0 for amax == 0).
 cudaError_t launch_amax(const void* x, int64_t rows, int64_t cols, int64_t ld, int had, int mode,
                         float* out, const Scratch& s, int num_sms, cudaStream_t st);
+// amax pass (mode 0) with a caller-chosen grid; scratch must hold `grid` partials.
+cudaError_t launch_amax_fixed_grid(const void* x, int64_t rows, int64_t cols, int64_t ld, float* out,
+                                   const Scratch& s, uint32_t grid, cudaStream_t st);
 cudaError_t launch_nv_tensor_scale(const float* amax, float* out, cudaStream_t st);
 cudaError_t launch_quantize(const QuantizeParams& p, int num_sms, cudaStream_t st);
 cudaError_t launch_dequantize(const uint8_t* codes, const uint8_t* scales, const float* ts, int64_t rows,

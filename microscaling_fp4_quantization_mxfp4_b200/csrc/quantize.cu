@@ -433,6 +433,21 @@ cudaError_t launch_amax(const void* x, int64_t rows, int64_t cols, int64_t ld, i
   }
 }
 
+cudaError_t launch_amax_fixed_grid(const void* x, int64_t rows, int64_t cols, int64_t ld, float* out,
+                                   const Scratch& s, uint32_t grid, cudaStream_t st) {
+  AmaxParams ap;
+  ap.x = static_cast<const uint16_t*>(x);
+  ap.rows_x_cpr = (uint32_t)(rows * (cols / 8));
+  ap.cpr = make_fastdiv((uint32_t)(cols / 8));
+  ap.ld = ld;
+  ap.partials = s.partials;
+  ap.counter = s.counter;
+  ap.out = out;
+  ap.mode = 0;
+  amax_kernel<0><<<grid, 256, 0, st>>>(ap);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_nv_tensor_scale(const float* amax, float* out, cudaStream_t st) {
   nv_tensor_scale_kernel<<<1, 1, 0, st>>>(amax, out);
   return cudaGetLastError();
