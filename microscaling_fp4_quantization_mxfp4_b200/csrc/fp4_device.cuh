@@ -47,34 +47,42 @@ __device__ __forceinline__ uint32_t pack8_rtn(const float (&v)[8]) {
 // Stochastic rounding of one scaled value with a 32-bit random word:
 // lo <= |v| < hi adjacent grid points, p = (|v| - lo) / (hi - lo) (exact in
 // fp32), round up iff r < ceil(p * 2^32); |v| >= 6 gives 6; sign kept.
+// Branch-free: on [0,2), [2,4), [4,6) the grid step is 0.5, 1, 2, so with
+// s = |v| / step (exact) the lower grid point is floor(s) steps in and p is
+// the fractional part of s.
 __device__ __forceinline__ uint32_t e2m1_sr(float v, uint32_t r) {
   const float a = fabsf(v);
-  uint32_t code;
-  if (!(a < 6.0f)) {
-    code = 7u;
-  } else {
-    uint32_t lo_code;
-    float lo, inv_w;
-    if (a < 2.0f) {                       // grid 0, .5, 1, 1.5: width 0.5
-      lo_code = (uint32_t)(a * 2.0f);     // exact product, truncation = floor
-      lo = (float)lo_code * 0.5f;
-      inv_w = 2.0f;
-    } else if (a < 4.0f) {                // grid 2, 3: width 1
-      const uint32_t f = (uint32_t)a;     // 2 or 3
-      lo_code = f + 2u;
-      lo = (float)f;
-      inv_w = 1.0f;
-    } else {                              // grid 4 -> 6: width 2
-      lo_code = 6u;
-      lo = 4.0f;
-      inv_w = 0.5f;
-    }
-    const float p = __fmul_rn(__fsub_rn(a, lo), inv_w);            // both steps exact
-    const unsigned long long thr = __float2ull_ru(__fmul_rn(p, 4294967296.0f));
-    code = lo_code + (((unsigned long long)r < thr) ? 1u : 0u);
-  }
+  const float inv_step = a < 2.0f ? 2.0f : (a < 4.0f ? 1.0f : 0.5f);
+  const uint32_t base = a < 2.0f ? 0u : (a < 4.0f ? 2u : 4u);
+  const float s = __fmul_rn(a, inv_step);
+  const float fl = floorf(s);
+  const float p = __fsub_rn(s, fl);
+  const uint32_t thr = __float2uint_ru(__fmul_rn(p, 4294967296.0f));   // < 2^32 since p < 1
+  uint32_t code = (uint32_t)fl + base + (r < thr ? 1u : 0u);
+  code = a < 6.0f ? code : 7u;
   return code | ((__float_as_uint(v) >> 31) << 3);
 }
+
+// ------------------------------------------------------- scale division -----
+// x / S rounded to nearest-even, bit-identical to IEEE division, from the
+// correctly rounded reciprocal y = RN(1/S) shared by a whole block:
+// q0 = RN(x*y) is within 1.5 ulp of x/S; one FMA correction
+// q1 = RN(q0 + (x - S*q0)*y) is faithful, and a second correction with a
+// faithful quotient and y = RN(1/S) is correctly rounded (Markstein's
+// theorem).  The residuals x - S*q are exact while x, S and the quotient stay
+// well inside the normal range; `ok` is false otherwise and the caller then
+// uses the IEEE division.  copysign keeps the sign of a zero dividend.
+__device__ __forceinline__ float div_by_recip(float x, float S, float y, bool& ok) {
+  float q = __fmul_rn(x, y);
+  float r = __fmaf_rn(-q, S, x);
+  q = __fmaf_rn(r, y, q);
+  r = __fmaf_rn(-q, S, x);
+  q = __fmaf_rn(r, y, q);
+  const float ax = fabsf(x);
+  ok = (ax == 0.0f) || (ax >= 0x1p-100f && fabsf(q) >= 0x1p-120f);
+  return copysignf(q, x);
+}
+__device__ __forceinline__ bool recip_usable(float S) { return S >= 0x1p-125f && S <= 0x1p+124f; }
 
 // ---------------------------------------------------------------- Philox ----
 // Philox4x32 with 10 rounds (Salmon, Moraes, Dror, Shaw, SC'11): two 32x32
@@ -85,11 +93,11 @@ __device__ __forceinline__ u32x4 philox4x32_10(uint32_t c0, uint32_t c1, uint32_
   uint32_t c2 = 0u, c3 = 0u;
 #pragma unroll
   for (int i = 0; i < 10; ++i) {
-    const uint32_t p0_lo = 0xD2511F53u * c0, p0_hi = __umulhi(0xD2511F53u, c0);
-    const uint32_t p1_lo = 0xCD9E8D57u * c2, p1_hi = __umulhi(0xCD9E8D57u, c2);
-    const uint32_t n0 = p1_hi ^ c1 ^ k0;
-    const uint32_t n2 = p0_hi ^ c3 ^ k1;
-    c0 = n0; c1 = p1_lo; c2 = n2; c3 = p0_lo;
+    const unsigned long long p0 = (unsigned long long)0xD2511F53u * c0;   // one wide multiply each
+    const unsigned long long p1 = (unsigned long long)0xCD9E8D57u * c2;
+    const uint32_t n0 = (uint32_t)(p1 >> 32) ^ c1 ^ k0;
+    const uint32_t n2 = (uint32_t)(p0 >> 32) ^ c3 ^ k1;
+    c0 = n0; c1 = (uint32_t)p1; c2 = n2; c3 = (uint32_t)p0;
     k0 += 0x9E3779B9u;
     k1 += 0xBB67AE85u;
   }

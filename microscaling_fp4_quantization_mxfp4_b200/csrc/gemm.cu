@@ -27,6 +27,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 #include <stdint.h>
+#include <stdlib.h>
 
 #include <mutex>
 
@@ -38,10 +39,8 @@ namespace {
 constexpr int BM = 128;
 constexpr int BK = 256;               // fp4 elements per k-tile (128 bytes per row)
 constexpr int BK_BYTES = BK / 2;
-constexpr int kThreads = 192;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kSfaCol = 256;
-constexpr uint32_t kSfbCol = 288;
+constexpr uint32_t kSfCols = 48;      // one scale-factor buffer: SFA (<= 16 cols) then SFB (<= 32 cols)
 constexpr unsigned long long kWaitLimitNs = 4000000000ull;   // 4 s per wait
 
 template <int FMT>
@@ -53,6 +52,9 @@ struct FmtTraits {
 template <int BN, int FMT>
 struct Cfg {
   static constexpr int kAccStages = BN == 128 ? 2 : 1;
+  static constexpr int kEpiWarps = BN == 256 ? 8 : 4;          // each epilogue warp drains 128 columns
+  static constexpr int kThreads = 64 + 32 * kEpiWarps;
+  static constexpr uint32_t kSfBase = (uint32_t)(kAccStages * BN);   // two scale buffers after the accumulators
   static constexpr int kApk = FmtTraits<FMT>::kAtomsPerKTile;
   static constexpr int kABytes = BM * BK_BYTES;
   static constexpr int kBBytes = BN * BK_BYTES;
@@ -94,15 +96,26 @@ __device__ __forceinline__ uint64_t global_timer() {
   return t;
 }
 // Bounded wait: false when the time limit passes or another role raised abort.
+// try_wait with a suspend-time hint: the warp sleeps in hardware until the
+// phase completes or ~20 us pass, instead of spinning on issue slots.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(20000u)
+      : "memory");
+  return ok != 0u;
+}
 __device__ __noinline__ bool wait_bounded(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer();
-  for (uint32_t i = 1;; ++i) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 255u) == 0u) {
-      if (*abort_flag != 0) return false;
-      if (global_timer() - t0 > kWaitLimitNs) return false;
-    }
+  for (;;) {
+    if (mbar_try_wait_sleep(bar, parity)) return true;
+    if (*abort_flag != 0) return false;
+    if (global_timer() - t0 > kWaitLimitNs) return false;
   }
 }
 __device__ __forceinline__ void raise_abort(volatile int* abort_flag, unsigned* error) {
@@ -161,8 +174,8 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
         "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
         "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
       : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
+__device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
 // Shared-memory matrix descriptor: K-major operand, 128-byte rows, 128B
 // swizzle, 8-row groups 1024 bytes apart (Blackwell descriptor version 1).
@@ -210,7 +223,7 @@ __device__ __forceinline__ void tile_coords(int t, int num_m, int num_n, int& mt
 }
 
 template <int BN, int FMT, bool BF16>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(Cfg<BN, FMT>::kThreads, 1)
     fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                     KernelArgs p) {
   using C = Cfg<BN, FMT>;
@@ -239,7 +252,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(smem_u32(&tfull[a]), 1);
-      mbar_init(smem_u32(&tempty[a]), 4);
+      mbar_init(smem_u32(&tempty[a]), C::kEpiWarps);
     }
     mbar_init(smem_u32(drain), 1);
     *abort_flag = 0;
@@ -316,6 +329,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       int local = 0;
+      uint32_t ktile_count = 0;   // k-tiles issued so far: picks the scale-factor buffer
       bool ok = true;
       bool any_mma = false;
       for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x, ++local) {
@@ -340,10 +354,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
           const int kvalid = min(BK, p.K - kb * BK);
           const int atoms = (kvalid / FmtTraits<FMT>::kBlock + 3) / 4;
+          // alternate between two scale buffers so these copies never overwrite scales that the
+          // previous k-tile's MMAs may still be reading
+          const uint32_t sfa_col = C::kSfBase + (ktile_count & 1u) * kSfCols;
+          const uint32_t sfb_col = sfa_col + 16u;
+          ++ktile_count;
           for (int i = 0; i < atoms; ++i) {
-            tc_cp_sf(tmem + kSfaCol + 4u * i, desc_sf(smem_u32(sSFA + stage * C::kSfaBytes + i * 512)));
+            tc_cp_sf(tmem + sfa_col + 4u * i, desc_sf(smem_u32(sSFA + stage * C::kSfaBytes + i * 512)));
             for (int rb = 0; rb < BN / 128; ++rb)
-              tc_cp_sf(tmem + kSfbCol + 4u * (i * (BN / 128) + rb),
+              tc_cp_sf(tmem + sfb_col + 4u * (i * (BN / 128) + rb),
                        desc_sf(smem_u32(sSFB + stage * C::kSfbBytes + (rb * APK + i) * 512)));
           }
           const uint64_t adesc = desc_sw128(smem_u32(sA + stage * C::kABytes));
@@ -360,7 +379,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             const uint32_t idesc = idesc_base<BN, FMT>() | (sf_id << 29) | (sf_id << 4);
             tc_mma<FMT>(d_tmem, adesc + (uint64_t)(2 * j), bdesc + (uint64_t)(2 * j), idesc,
-                        tmem + kSfaCol + 4u * chunk, tmem + kSfbCol + 4u * chunk * (BN / 128),
+                        tmem + sfa_col + 4u * chunk, tmem + sfb_col + 4u * chunk * (BN / 128),
                         (kb > 0 || j > 0) ? 1u : 0u);
             any_mma = true;
           }
@@ -383,7 +402,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue --
-    const int q = warp & 3;                  // tensor-memory lane quadrant of this warp
+    // Warp w reads tensor-memory lanes 32*(w%4) .. +31 (its hardware quadrant) and
+    // 128 accumulator columns; all 128 values per thread are loaded before the
+    // accumulator is released, so the next tile's MMAs start while stores drain.
+    const int q = warp & 3;
+    const int col0 = ((warp - 2) / 4) * 128;
     const int row_in_tile = q * 32 + lane;
     const float alpha = FMT == FMT_NV ? __fmul_rn(*p.a_ts, *p.b_ts) : 1.0f;
     int local = 0;
@@ -400,19 +423,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
+      const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN + col0);
+      uint32_t r[4][32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32(tbase + (uint32_t)(32 * c), r[c]);
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&tempty[acc]));
       const int m = mt * BM + row_in_tile;
-      const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
-#pragma unroll 1
-      for (int c0 = 0; c0 < BN; c0 += 32) {
-        uint32_t r[32];
-        tmem_ld32(tbase + (uint32_t)c0, r);
-        if (c0 + 32 == BN) {
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(smem_u32(&tempty[acc]));
-        }
-        const int n0 = nt * BN + c0;
-        if (m < p.M && n0 < p.N) {
+      if (m < p.M) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const int n0 = nt * BN + col0 + 32 * c;
+          if (n0 >= p.N) break;
           if (BF16) {
             __nv_bfloat16* yr = reinterpret_cast<__nv_bfloat16*>(p.y) + (size_t)m * p.ldy + n0;
             if (p.vec_store && n0 + 32 <= p.N) {
@@ -421,8 +445,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 uint32_t w[4];
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
-                  const float lo = __fmul_rn(__uint_as_float(r[8 * v + 2 * i]), alpha);
-                  const float hi = __fmul_rn(__uint_as_float(r[8 * v + 2 * i + 1]), alpha);
+                  const float lo = __fmul_rn(__uint_as_float(r[c][8 * v + 2 * i]), alpha);
+                  const float hi = __fmul_rn(__uint_as_float(r[c][8 * v + 2 * i + 1]), alpha);
                   w[i] = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(lo)) |
                          ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(hi)) << 16);
                 }
@@ -431,20 +455,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             } else {
 #pragma unroll
               for (int i = 0; i < 32; ++i)
-                if (n0 + i < p.N) yr[i] = __float2bfloat16_rn(__fmul_rn(__uint_as_float(r[i]), alpha));
+                if (n0 + i < p.N) yr[i] = __float2bfloat16_rn(__fmul_rn(__uint_as_float(r[c][i]), alpha));
             }
           } else {
             float* yr = reinterpret_cast<float*>(p.y) + (size_t)m * p.ldy + n0;
             if (p.vec_store && n0 + 32 <= p.N) {
 #pragma unroll
               for (int v = 0; v < 8; ++v)
-                reinterpret_cast<float4*>(yr)[v] =
-                    make_float4(__fmul_rn(__uint_as_float(r[4 * v]), alpha), __fmul_rn(__uint_as_float(r[4 * v + 1]), alpha),
-                                __fmul_rn(__uint_as_float(r[4 * v + 2]), alpha), __fmul_rn(__uint_as_float(r[4 * v + 3]), alpha));
+                reinterpret_cast<float4*>(yr)[v] = make_float4(
+                    __fmul_rn(__uint_as_float(r[c][4 * v]), alpha), __fmul_rn(__uint_as_float(r[c][4 * v + 1]), alpha),
+                    __fmul_rn(__uint_as_float(r[c][4 * v + 2]), alpha), __fmul_rn(__uint_as_float(r[c][4 * v + 3]), alpha));
             } else {
 #pragma unroll
               for (int i = 0; i < 32; ++i)
-                if (n0 + i < p.N) yr[i] = __fmul_rn(__uint_as_float(r[i]), alpha);
+                if (n0 + i < p.N) yr[i] = __fmul_rn(__uint_as_float(r[c][i]), alpha);
             }
           }
         }
@@ -517,15 +541,27 @@ cudaError_t run(const GemmParams& gp, int num_sms, cudaStream_t st) {
   }
   const int tiles = ka.num_m * ka.num_n;
   const int grid = tiles < num_sms ? tiles : num_sms;
-  fp4_gemm_kernel<BN, FMT, BF16><<<grid, kThreads, C::kSmemBytes, st>>>(ta, tb, ka);
+  fp4_gemm_kernel<BN, FMT, BF16><<<grid, C::kThreads, C::kSmemBytes, st>>>(ta, tb, ka);
   return cudaGetLastError();
 }
 
 }  // namespace
 
+template <int BN>
+static cudaError_t dispatch_fmt(const GemmParams& p, int num_sms, cudaStream_t st) {
+  if (p.fmt == FMT_MX) return p.y_bf16 ? run<BN, FMT_MX, true>(p, num_sms, st) : run<BN, FMT_MX, false>(p, num_sms, st);
+  return p.y_bf16 ? run<BN, FMT_NV, true>(p, num_sms, st) : run<BN, FMT_NV, false>(p, num_sms, st);
+}
+
 cudaError_t launch_gemm(const GemmParams& p, int num_sms, cudaStream_t st) {
-  if (p.fmt == FMT_MX) return p.y_bf16 ? run<128, FMT_MX, true>(p, num_sms, st) : run<128, FMT_MX, false>(p, num_sms, st);
-  return p.y_bf16 ? run<128, FMT_NV, true>(p, num_sms, st) : run<128, FMT_NV, false>(p, num_sms, st);
+  // 128x256 tiles halve the operand traffic per FLOP; 128x128 tiles keep two accumulators in
+  // tensor memory and more CTAs busy when N is small.  FP4_GEMM_BN=128|256 overrides (tuning).
+  static const int forced = [] {
+    const char* e = getenv("FP4_GEMM_BN");
+    return e ? atoi(e) : 0;
+  }();
+  const int bn = forced == 128 || forced == 256 ? forced : (p.N >= 256 ? 256 : 128);
+  return bn == 256 ? dispatch_fmt<256>(p, num_sms, st) : dispatch_fmt<128>(p, num_sms, st);
 }
 
 }  // namespace fp4lib

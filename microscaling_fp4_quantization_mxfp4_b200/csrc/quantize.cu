@@ -44,11 +44,14 @@ __device__ __forceinline__ uint4 ld_stream(const void* p) {
 }
 
 // ============================================================= amax pass ===
+constexpr int kAmaxUnroll = 4;
+
 struct AmaxParams {
   const uint16_t* x;
   uint32_t rows_x_cpr;   // number of 8-element chunks
   FastDiv cpr;           // chunks per row
   int64_t ld;
+  int contig;            // ld == cols: chunk c starts at element 8c
   float* partials;
   unsigned* counter;
   float* out;
@@ -63,20 +66,27 @@ __global__ void __launch_bounds__(256) amax_kernel(AmaxParams p) {
   const uint32_t gwarp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const uint32_t nwarps = (gridDim.x * blockDim.x) >> 5;
   float m = 0.0f;
-  for (uint32_t t = gwarp; t < ntiles; t += nwarps) {
-    const uint32_t chunk = t * 32u + lane;
-    float x[8];
-    if (chunk < nchunks) {
-      const uint32_t row = fdiv(chunk, p.cpr);
-      const uint32_t c8 = chunk - row * p.cpr.d;
-      unpack8(ld_stream(p.x + (int64_t)row * p.ld + (int64_t)c8 * 8), x);
-    } else {
+  for (uint32_t t0 = gwarp; t0 < ntiles; t0 += nwarps * kAmaxUnroll) {
+    uint4 v[kAmaxUnroll];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) x[i] = 0.0f;
+    for (int u = 0; u < kAmaxUnroll; ++u) {
+      const uint32_t chunk = (t0 + (uint32_t)u * nwarps) * 32u + lane;
+      v[u] = make_uint4(0u, 0u, 0u, 0u);
+      if (t0 + (uint32_t)u * nwarps < ntiles && chunk < nchunks) {
+        const uint32_t row = p.contig ? 0u : fdiv(chunk, p.cpr);
+        const int64_t off = p.contig ? (int64_t)chunk * 8 : (int64_t)row * p.ld + (int64_t)(chunk - row * p.cpr.d) * 8;
+        v[u] = ld_stream(p.x + off);
+      }
     }
-    if (HAD) hadamard_rotate<HAD>(x, lane);
 #pragma unroll
-    for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(x[i]));
+    for (int u = 0; u < kAmaxUnroll; ++u) {
+      if (t0 + (uint32_t)u * nwarps >= ntiles) break;     // warp-uniform
+      float x[8];
+      unpack8(v[u], x);
+      if (HAD) hadamard_rotate<HAD>(x, lane);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(x[i]));
+    }
   }
   // non-negative floats order like their bit patterns
   uint32_t bits = __reduce_max_sync(0xFFFFFFFFu, __float_as_uint(m));
@@ -125,6 +135,7 @@ struct QRowParams {
   uint32_t nchunks;
   FastDiv cpr;           // chunks (8 elements) per row
   int64_t ld;
+  int contig;            // ld == cols
   uint32_t cols;
   uint32_t g4;           // padded k-groups / 4 (tensor-core scale layout)
   unsigned long long seed;
@@ -171,8 +182,20 @@ __device__ __forceinline__ void quantize_chunk(const QRowParams& p, const uint4 
     byte = e4m3_rn_sat(t);
     zero = (byte == 0u);
     const float S = zero ? 1.0f : __fmul_rn(e4m3_value(byte), s_t);
+    const float y = __frcp_rn(S);
+    bool ok = recip_usable(S);
 #pragma unroll
-    for (int i = 0; i < 8; ++i) v8[i] = __fdiv_rn(x[i], S);
+    for (int i = 0; i < 8; ++i) {
+      bool oki;
+      v8[i] = div_by_recip(x[i], S, y, oki);
+      ok = ok && oki;
+    }
+    if (__any_sync(0xFFFFFFFFu, !ok)) {       // rare: tiny values or scales -> IEEE division
+      if (!ok) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v8[i] = __fdiv_rn(x[i], S);
+      }
+    }
   }
   uint32_t packed;
   if (RND == RND_RTN) {
@@ -218,9 +241,13 @@ __global__ void __launch_bounds__(256) quantize_rows_kernel(QRowParams p) {
       const uint32_t t = t0 + (uint32_t)u * nwarps;
       chunk[u] = t * 32u + lane;
       if (t < ntiles && chunk[u] < p.nchunks) {
-        const uint32_t row = fdiv(chunk[u], p.cpr);
-        const uint32_t c8 = chunk[u] - row * p.cpr.d;
-        v[u] = ld_stream(p.x + (int64_t)row * p.ld + (int64_t)c8 * 8);
+        if (p.contig) {
+          v[u] = ld_stream(p.x + (int64_t)chunk[u] * 8);
+        } else {
+          const uint32_t row = fdiv(chunk[u], p.cpr);
+          const uint32_t c8 = chunk[u] - row * p.cpr.d;
+          v[u] = ld_stream(p.x + (int64_t)row * p.ld + (int64_t)c8 * 8);
+        }
       } else {
         v[u] = make_uint4(0u, 0u, 0u, 0u);
       }
@@ -294,7 +321,8 @@ __global__ void __launch_bounds__(256) quantize_cols_kernel(QColParams p) {
       for (int i = 0; i < BS; ++i) am = fmaxf(am, fabsf(xv[b * BS + i]));
       uint32_t byte;
       bool zero;
-      float inv = 1.0f, S = 1.0f;
+      float inv = 1.0f, S = 1.0f, y = 1.0f;
+      bool fast = true;
       if (FMT == FMT_MX) {
         byte = mx_scale_byte(am);
         inv = mx_inv_scale(byte);
@@ -304,6 +332,8 @@ __global__ void __launch_bounds__(256) quantize_cols_kernel(QColParams p) {
         byte = e4m3_rn_sat(tt);
         zero = (byte == 0u);
         S = zero ? 1.0f : __fmul_rn(e4m3_value(byte), s_t);
+        y = __frcp_rn(S);
+        fast = recip_usable(S);
       }
 #pragma unroll
       for (int w8 = 0; w8 < BS / 8; ++w8) {
@@ -311,7 +341,13 @@ __global__ void __launch_bounds__(256) quantize_cols_kernel(QColParams p) {
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           const float xi = xv[b * BS + w8 * 8 + i];
-          v8[i] = FMT == FMT_MX ? __fmul_rn(xi, inv) : __fdiv_rn(xi, S);
+          if (FMT == FMT_MX) {
+            v8[i] = __fmul_rn(xi, inv);
+          } else {
+            bool oki;
+            v8[i] = div_by_recip(xi, S, y, oki);
+            if (!(fast && oki)) v8[i] = __fdiv_rn(xi, S);
+          }
         }
         uint32_t packed;
         if (RND == RND_RTN) {
@@ -352,42 +388,58 @@ struct DeqParams {
 };
 
 template <int FMT, bool SFMMA, bool BF16>
-__global__ void __launch_bounds__(256) dequantize_kernel(DeqParams p) {
+__device__ __forceinline__ void dequantize_chunk(const DeqParams& p, uint32_t chunk, uint32_t w, float s_t) {
   constexpr int LPB = FMT == FMT_MX ? 4 : 2;
+  uint32_t byte;
+  if (SFMMA) {
+    const uint32_t row = fdiv(chunk, p.cpr);
+    byte = p.scales[sf_mma_offset(row, (chunk - row * p.cpr.d) / LPB, p.g4)];
+  } else {
+    byte = p.scales[chunk / LPB];
+  }
+  float y[8];
+  if (FMT == FMT_MX) {
+    const float sc = mx_scale_value(byte);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) y[i] = __fmul_rn(e2m1_value((w >> (4 * i)) & 0xFu), sc);
+  } else {
+    const float sb = e4m3_value(byte);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) y[i] = __fmul_rn(__fmul_rn(e2m1_value((w >> (4 * i)) & 0xFu), sb), s_t);
+  }
+  if (BF16) {
+    uint32_t o[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t lo = __bfloat16_as_ushort(__float2bfloat16_rn(y[2 * i]));
+      const uint32_t hi = __bfloat16_as_ushort(__float2bfloat16_rn(y[2 * i + 1]));
+      o[i] = lo | (hi << 16);
+    }
+    reinterpret_cast<uint4*>(p.out)[chunk] = make_uint4(o[0], o[1], o[2], o[3]);
+  } else {
+    float4* o = reinterpret_cast<float4*>(p.out) + (size_t)chunk * 2;
+    o[0] = make_float4(y[0], y[1], y[2], y[3]);
+    o[1] = make_float4(y[4], y[5], y[6], y[7]);
+  }
+}
+
+// Each thread takes two adjacent chunks (16 codes, one 8-byte load) per step;
+// the chunk count is even because rows hold a whole number of 16-element blocks.
+template <int FMT, bool SFMMA, bool BF16>
+__global__ void __launch_bounds__(256) dequantize_kernel(DeqParams p) {
   const float s_t = FMT == FMT_NV ? *p.ts : 1.0f;
+  const uint32_t npairs = p.nchunks / 2;
   const uint32_t stride = gridDim.x * blockDim.x;
-  for (uint32_t chunk = blockIdx.x * blockDim.x + threadIdx.x; chunk < p.nchunks; chunk += stride) {
-    const uint32_t w = __ldg(p.codes + chunk);
-    uint32_t byte;
-    if (SFMMA) {
-      const uint32_t row = fdiv(chunk, p.cpr);
-      byte = p.scales[sf_mma_offset(row, (chunk - row * p.cpr.d) / LPB, p.g4)];
-    } else {
-      byte = p.scales[chunk / LPB];
-    }
-    float y[8];
-    if (FMT == FMT_MX) {
-      const float sc = mx_scale_value(byte);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) y[i] = __fmul_rn(e2m1_value((w >> (4 * i)) & 0xFu), sc);
-    } else {
-      const float sb = e4m3_value(byte);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) y[i] = __fmul_rn(__fmul_rn(e2m1_value((w >> (4 * i)) & 0xFu), sb), s_t);
-    }
-    if (BF16) {
-      uint32_t o[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const uint32_t lo = __bfloat16_as_ushort(__float2bfloat16_rn(y[2 * i]));
-        const uint32_t hi = __bfloat16_as_ushort(__float2bfloat16_rn(y[2 * i + 1]));
-        o[i] = lo | (hi << 16);
-      }
-      reinterpret_cast<uint4*>(p.out)[chunk] = make_uint4(o[0], o[1], o[2], o[3]);
-    } else {
-      float4* o = reinterpret_cast<float4*>(p.out) + (size_t)chunk * 2;
-      o[0] = make_float4(y[0], y[1], y[2], y[3]);
-      o[1] = make_float4(y[4], y[5], y[6], y[7]);
+  for (uint32_t i = blockIdx.x * blockDim.x + threadIdx.x; i < npairs; i += 2 * stride) {
+    const uint2 a = __ldg(reinterpret_cast<const uint2*>(p.codes) + i);
+    const bool has2 = i + stride < npairs;
+    uint2 b = make_uint2(0u, 0u);
+    if (has2) b = __ldg(reinterpret_cast<const uint2*>(p.codes) + i + stride);
+    dequantize_chunk<FMT, SFMMA, BF16>(p, 2 * i, a.x, s_t);
+    dequantize_chunk<FMT, SFMMA, BF16>(p, 2 * i + 1, a.y, s_t);
+    if (has2) {
+      dequantize_chunk<FMT, SFMMA, BF16>(p, 2 * (i + stride), b.x, s_t);
+      dequantize_chunk<FMT, SFMMA, BF16>(p, 2 * (i + stride) + 1, b.y, s_t);
     }
   }
 }
@@ -403,7 +455,7 @@ static int resident_ctas(K kernel, int threads) {
 template <int HAD>
 static cudaError_t amax_launch(const AmaxParams& ap, uint32_t ntiles, int num_sms, cudaStream_t st) {
   static int occ = resident_ctas(amax_kernel<HAD>, 256);
-  uint32_t want = (ntiles + 7u) / 8u;
+  uint32_t want = (ntiles + 8u * kAmaxUnroll - 1u) / (8u * kAmaxUnroll);
   uint32_t grid = (uint32_t)num_sms * (uint32_t)occ;
   if (grid > (uint32_t)kMaxAmaxBlocks) grid = kMaxAmaxBlocks;
   if (want < grid) grid = want > 0 ? want : 1;
@@ -418,6 +470,7 @@ cudaError_t launch_amax(const void* x, int64_t rows, int64_t cols, int64_t ld, i
   ap.rows_x_cpr = (uint32_t)(rows * (cols / 8));
   ap.cpr = make_fastdiv((uint32_t)(cols / 8));
   ap.ld = ld;
+  ap.contig = (ld == cols);
   ap.partials = s.partials;
   ap.counter = s.counter;
   ap.out = out;
@@ -440,6 +493,7 @@ cudaError_t launch_amax_fixed_grid(const void* x, int64_t rows, int64_t cols, in
   ap.rows_x_cpr = (uint32_t)(rows * (cols / 8));
   ap.cpr = make_fastdiv((uint32_t)(cols / 8));
   ap.ld = ld;
+  ap.contig = (ld == cols);
   ap.partials = s.partials;
   ap.counter = s.counter;
   ap.out = out;
@@ -505,6 +559,7 @@ cudaError_t launch_quantize(const QuantizeParams& p, int num_sms, cudaStream_t s
     qp.nchunks = (uint32_t)(p.rows * (p.cols / 8));
     qp.cpr = make_fastdiv((uint32_t)(p.cols / 8));
     qp.ld = p.ld;
+    qp.contig = (p.ld == p.cols);
     qp.cols = (uint32_t)p.cols;
     qp.g4 = (uint32_t)((p.cols / bs + 3) / 4);
     qp.seed = p.seed;
@@ -541,7 +596,7 @@ cudaError_t launch_quantize(const QuantizeParams& p, int num_sms, cudaStream_t s
 template <int FMT, bool SFMMA, bool BF16>
 static cudaError_t deq_launch(const DeqParams& dp, int num_sms, cudaStream_t st) {
   static int occ = resident_ctas(dequantize_kernel<FMT, SFMMA, BF16>, 256);
-  uint32_t want = (dp.nchunks + 255u) / 256u;
+  uint32_t want = (dp.nchunks / 2 + 511u) / 512u;
   uint32_t grid = (uint32_t)num_sms * (uint32_t)occ;
   if (want < grid) grid = want > 0 ? want : 1;
   dequantize_kernel<FMT, SFMMA, BF16><<<grid, 256, 0, st>>>(dp);
