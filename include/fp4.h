@@ -127,7 +127,8 @@ fp4_status fp4_hadamard_quantize(const void* x, int64_t rows, int64_t cols, int6
  * fp4_dequantize -- codes + scales (+ s_t) back to floating point
  * ("FP4 All the Way", Abstract: the E2M1 values times their block scale).
  * MX: G[c] * 2^(b-127), exact in fp32.  NV: fp32(fp32(G[c] * sb) * s_t).
- *   codes  uint8 [rows, cols/2] (rows, cols = out_rows, L of the quantizer)
+ *   codes  uint8 [rows, cols/2] (rows, cols = out_rows, L of the quantizer),
+ *          16-byte aligned; out 16-byte aligned
  *   scales in `sf_layout`; tensor_scale device fp32 (NV), ignored for MX.
  *   out    fp32 or bf16 (RNE of the fp32 value) [rows, cols], row stride cols.
  */

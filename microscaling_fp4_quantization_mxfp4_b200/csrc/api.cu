@@ -52,6 +52,7 @@ fp4_status device_state(DeviceState** out) {
     d.scratch.partials = static_cast<float*>(mem);
     d.scratch.counter = reinterpret_cast<unsigned*>(static_cast<char*>(mem) + sizeof(float) * kMaxAmaxBlocks);
     d.scratch.error = d.scratch.counter + 1;
+    d.scratch.grid_arrive = d.scratch.counter + 2;
     d.num_sms = sms;
     d.ready = true;
   }
@@ -60,6 +61,15 @@ fp4_status device_state(DeviceState** out) {
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// FP4_SINGLE_PASS=0 forces the two-pass NVFP4 path (amax kernel, then quantize); for testing.
+bool single_pass_disabled() {
+  static const bool off = [] {
+    const char* e = getenv("FP4_SINGLE_PASS");
+    return e != nullptr && e[0] == '0';
+  }();
+  return off;
+}
 
 fp4_status check_format(int fmt, int block) {
   if (fmt == FP4_MXFP4 && block == 32) return FP4_OK;
@@ -114,6 +124,28 @@ fp4_status quantize_impl(const void* x, int64_t rows, int64_t cols, int64_t ld, 
     if (cudaMemsetAsync(scales, 0, (size_t)(round_up(orows, 128) * round_up(groups, 4)), st) != cudaSuccess)
       return FP4_ERR_CUDA;
   }
+  QuantizeParams p;
+  p.x = x;
+  p.rows = rows;
+  p.cols = cols;
+  p.ld = ld;
+  p.fmt = fmt == FP4_MXFP4 ? FMT_MX : FMT_NV;
+  p.axis = axis;
+  p.rnd = rnd == FP4_RTN ? RND_RTN : RND_SR;
+  p.seed = seed;
+  p.codes = codes;
+  p.scales = scales;
+  p.sf_mma = sf_layout == FP4_SF_MMA;
+  p.had = had;
+  p.rotated = rotated;
+  p.error = d->scratch.error;
+  size_t fused_smem = 0;
+  uint32_t fused_tiles = 0;
+  if (fmt == FP4_NVFP4 && ts_in == nullptr && axis == 1 && ld == cols && !single_pass_disabled() &&
+      fused_nv_fits(rows, cols, d->num_sms, &fused_smem, &fused_tiles)) {
+    // one HBM read: amax and quantize in a single cooperative launch
+    return from_cuda(launch_quantize_nv_fused(p, ts_out, d->scratch, d->num_sms, st));
+  }
   const float* ts_read = nullptr;
   float* ts_copy = nullptr;
   if (fmt == FP4_NVFP4) {
@@ -126,22 +158,8 @@ fp4_status quantize_impl(const void* x, int64_t rows, int64_t cols, int64_t ld, 
       ts_read = ts_out;
     }
   }
-  QuantizeParams p;
-  p.x = x;
-  p.rows = rows;
-  p.cols = cols;
-  p.ld = ld;
-  p.fmt = fmt == FP4_MXFP4 ? FMT_MX : FMT_NV;
-  p.axis = axis;
-  p.rnd = rnd == FP4_RTN ? RND_RTN : RND_SR;
-  p.seed = seed;
   p.ts = ts_read;
   p.ts_copy_out = ts_copy;
-  p.codes = codes;
-  p.scales = scales;
-  p.sf_mma = sf_layout == FP4_SF_MMA;
-  p.had = had;
-  p.rotated = rotated;
   return from_cuda(launch_quantize(p, d->num_sms, st));
 }
 
@@ -175,7 +193,7 @@ fp4_status fp4_dequantize(const uint8_t* codes, const uint8_t* scales, const flo
   if (out_dtype != FP4_OUT_F32 && out_dtype != FP4_OUT_BF16) return FP4_ERR_ARG;
   if (cols % block != 0) return FP4_ERR_SHAPE;
   if (rows * (cols / 8) >= (int64_t)1 << 32) return FP4_ERR_SHAPE;
-  if ((reinterpret_cast<uintptr_t>(codes) & 3u) != 0 || !aligned16(out)) return FP4_ERR_ALIGN;
+  if (!aligned16(codes) || !aligned16(out)) return FP4_ERR_ALIGN;
   DeviceState* d = nullptr;
   if ((s = device_state(&d)) != FP4_OK) return s;
   return from_cuda(launch_dequantize(codes, scales, tensor_scale, rows, cols, fmt == FP4_MXFP4 ? FMT_MX : FMT_NV,

@@ -155,6 +155,26 @@ __device__ __forceinline__ float e4m3_value(uint32_t b) {
   return __uint_as_float(((e + 120u) << 23) | (m << 20));                // (1 + m/8) * 2^(e-7)
 }
 
+// NVFP4 block-scale argument t = RN(RN(amax_b / 6) / s_t), bit-identical to two
+// IEEE divisions, from RN(1/6) and y_st = RN(1/s_t) (st_ok: recip_usable(s_t)).
+__device__ __forceinline__ float nv_scale_arg(float am, float s_t, float y_st, bool st_ok) {
+  bool ok1, ok2;
+  const float d6 = div_by_recip(am, 6.0f, 0x1.555556p-3f, ok1);     // 0x1.555556p-3 = RN(1/6)
+  const float t = div_by_recip(d6, s_t, y_st, ok2);
+  return (ok1 && ok2 && st_ok) ? t : __fdiv_rn(__fdiv_rn(am, 6.0f), s_t);
+}
+
+// Per-CTA table of the element divisor S = RN(e4m3(b) * s_t) and RN(1/S) for
+// every E4M3 byte b (b = 0 is the zero scale; its entry is unused).  A scale
+// whose reciprocal is out of the fast path's range gets y = 0, which makes
+// every quotient fail the `ok` test and take the IEEE division.
+__device__ __forceinline__ void nv_fill_scale_table(float2* tab, float s_t) {
+  for (int b = threadIdx.x; b < 128; b += blockDim.x) {
+    const float S = (b == 0 || b == 127) ? 1.0f : __fmul_rn(e4m3_value((uint32_t)b), s_t);
+    tab[b] = make_float2(S, recip_usable(S) ? __frcp_rn(S) : 0.0f);
+  }
+}
+
 // -------------------------------------------------------- E2M1 decoding -----
 __device__ __forceinline__ float e2m1_value(uint32_t c) {
   const uint32_t e = (c >> 1) & 3u, m = c & 1u;
@@ -199,5 +219,71 @@ __device__ __forceinline__ void hadamard_rotate(float (&x)[8], int lane) {
 #pragma unroll
   for (int i = 0; i < 8; ++i) x[i] = __fmul_rn(x[i], s);
 }
+
+// ------------------------------------------- bulk copies and mbarriers -----
+// Thin wrappers over the sm_90+/sm_100 bulk-copy engine (cp.async.bulk, no
+// tensor map, no multicast) and shared-memory mbarriers, used by the
+// streaming kernels to move whole tiles with one instruction.
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_init_fence() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity, uint32_t sleep_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(sleep_ns)
+      : "memory");
+  return ok != 0u;
+}
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+// Wait for phase `parity` of an mbarrier, giving up after ~2 s.
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity) {
+  if (mbar_test(bar, parity, 0u)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (;;) {
+    if (mbar_test(bar, parity, 10000u)) return true;
+    if (globaltimer_ns() - t0 > 2000000000ull) return false;
+  }
+}
+// global -> shared, completion counted on an mbarrier (addresses 16-byte aligned, size % 16 == 0).
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(src), "r"(bytes), "r"(bar)
+               : "memory");
+}
+// shared -> global in a bulk group of the issuing thread.
+__device__ __forceinline__ void bulk_s2g(void* dst, uint32_t src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(src), "r"(bytes)
+               : "memory");
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// Wait until at most N of this thread's bulk groups still read shared memory.
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+// Order this thread's generic-proxy shared-memory writes before later bulk copies.
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
 }  // namespace fp4dev

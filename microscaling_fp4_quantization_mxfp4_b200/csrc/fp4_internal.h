@@ -15,6 +15,7 @@ struct Scratch {
   float* partials;      // per-CTA maxima of the tensor-amax pass
   unsigned* counter;    // CTA ticket counter of the amax pass (self-resetting)
   unsigned* error;      // device error word set by bounded waits
+  unsigned* grid_arrive;  // arrivals at the single-pass NVFP4 quantizer's grid barrier
 };
 constexpr int kMaxAmaxBlocks = 2048;
 
@@ -37,6 +38,7 @@ struct QuantizeParams {
   int sf_mma;
   int had;                // 0 or Hadamard block size
   float* rotated;         // optional fp32 dump of the rotated input
+  unsigned* error;        // device error word
 };
 
 // amax pass: mode 0 writes max|x| (after rotation when had > 0) to `out`,
@@ -48,6 +50,11 @@ cudaError_t launch_amax_fixed_grid(const void* x, int64_t rows, int64_t cols, in
                                    const Scratch& s, uint32_t grid, cudaStream_t st);
 cudaError_t launch_nv_tensor_scale(const float* amax, float* out, cudaStream_t st);
 cudaError_t launch_quantize(const QuantizeParams& p, int num_sms, cudaStream_t st);
+// Single-pass NVFP4 quantize (axis 1, no caller-given s_t) for tensors that fit in shared memory
+// across the SMs; fused_nv_fits says whether it applies.  Writes s_t to ts_out.
+bool fused_nv_fits(int64_t rows, int64_t cols, int num_sms, size_t* smem, uint32_t* tiles_per_cta);
+cudaError_t launch_quantize_nv_fused(const QuantizeParams& p, float* ts_out, const Scratch& s, int num_sms,
+                                     cudaStream_t st);
 cudaError_t launch_dequantize(const uint8_t* codes, const uint8_t* scales, const float* ts, int64_t rows,
                               int64_t cols, int fmt, int sf_mma, void* out, int out_bf16, int num_sms,
                               cudaStream_t st);

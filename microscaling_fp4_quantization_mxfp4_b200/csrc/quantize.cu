@@ -144,13 +144,21 @@ struct QRowParams {
   uint32_t* codes;       // [rows, cols/8] 32-bit words of 8 nibbles
   uint8_t* scales;
   float* rotated;
+  unsigned* error;       // device error word (streaming kernels: bit 2 = a ring wait expired)
 };
 
 constexpr int kUnroll = 4;
 
+// Per-thread NVFP4 constants: the tensor scale, its reciprocal and the (S, 1/S) table.
+struct NvConsts {
+  float s_t, y_st;
+  bool st_ok;
+  const float2* tab;
+};
+
 template <int FMT, int RND, int HAD, bool SFMMA>
 __device__ __forceinline__ void quantize_chunk(const QRowParams& p, const uint4 v, uint32_t chunk, bool valid,
-                                               int lane, float s_t) {
+                                               int lane, const NvConsts& nv) {
   constexpr int LPB = FMT == FMT_MX ? 4 : 2;   // lanes per scale block
   float x[8];
   unpack8(v, x);
@@ -178,12 +186,11 @@ __device__ __forceinline__ void quantize_chunk(const QRowParams& p, const uint4 
     for (int i = 0; i < 8; ++i) v8[i] = __fmul_rn(x[i], inv);     // exact power-of-two scaling
     zero = (am == 0.0f);
   } else {
-    const float t = __fdiv_rn(__fdiv_rn(am, 6.0f), s_t);
-    byte = e4m3_rn_sat(t);
+    byte = e4m3_rn_sat(nv_scale_arg(am, nv.s_t, nv.y_st, nv.st_ok));
     zero = (byte == 0u);
-    const float S = zero ? 1.0f : __fmul_rn(e4m3_value(byte), s_t);
-    const float y = __frcp_rn(S);
-    bool ok = recip_usable(S);
+    const float2 sy = nv.tab[byte];
+    const float S = sy.x, y = sy.y;
+    bool ok = true;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       bool oki;
@@ -228,10 +235,15 @@ __global__ void __launch_bounds__(256) quantize_rows_kernel(QRowParams p) {
   const uint32_t ntiles = (p.nchunks + 31u) >> 5;
   const uint32_t gwarp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const uint32_t nwarps = (gridDim.x * blockDim.x) >> 5;
-  float s_t = 1.0f;
+  __shared__ float2 tab[128];
+  NvConsts nv{1.0f, 1.0f, true, tab};
   if (FMT == FMT_NV) {
-    s_t = *p.ts;
-    if (p.ts_copy_out != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *p.ts_copy_out = s_t;
+    nv.s_t = *p.ts;
+    nv.y_st = __frcp_rn(nv.s_t);
+    nv.st_ok = recip_usable(nv.s_t);
+    nv_fill_scale_table(tab, nv.s_t);
+    if (p.ts_copy_out != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *p.ts_copy_out = nv.s_t;
+    __syncthreads();
   }
   for (uint32_t t0 = gwarp; t0 < ntiles; t0 += nwarps * kUnroll) {
     uint4 v[kUnroll];
@@ -256,8 +268,317 @@ __global__ void __launch_bounds__(256) quantize_rows_kernel(QRowParams p) {
     for (int u = 0; u < kUnroll; ++u) {
       const uint32_t t = t0 + (uint32_t)u * nwarps;
       if (t < ntiles)   // warp-uniform: every lane of the warp takes the same branch
-        quantize_chunk<FMT, RND, HAD, SFMMA>(p, v[u], chunk[u], chunk[u] < p.nchunks, lane, s_t);
+        quantize_chunk<FMT, RND, HAD, SFMMA>(p, v[u], chunk[u], chunk[u] < p.nchunks, lane, nv);
     }
+  }
+}
+
+// ======================================= TMA-fed axis-1 quantize / amax ===
+// Contiguous inputs stream through a ring of 32 KB shared-memory stages filled
+// by the bulk-copy engine: one producer thread issues a cp.async.bulk per stage
+// (no per-thread load traffic, many bytes in flight), 16 consumer warps
+// quantize (or reduce) each stage and release it through an mbarrier.
+constexpr int kStreamChunks = 2048;                     // 8-element chunks per stage (32 KB of bf16)
+constexpr int kStreamStages = 6;
+constexpr int kStreamWarps = 16;                        // consumer warps
+constexpr int kStreamThreads = 32 * (kStreamWarps + 1);
+constexpr int kStreamSmem = kStreamStages * kStreamChunks * 16 + 2 * kStreamStages * 8;
+
+struct StreamRing {
+  uint4* data;
+  uint64_t* full;
+  uint64_t* empty;
+};
+
+__device__ __forceinline__ StreamRing stream_ring(uint8_t* smem) {
+  StreamRing r;
+  r.data = reinterpret_cast<uint4*>(smem);
+  r.full = reinterpret_cast<uint64_t*>(smem + kStreamStages * kStreamChunks * 16);
+  r.empty = r.full + kStreamStages;
+  return r;
+}
+
+__device__ __forceinline__ void stream_ring_init(const StreamRing& r) {
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStreamStages; ++s) {
+      mbar_init(smem_addr(&r.full[s]), 1);
+      mbar_init(smem_addr(&r.empty[s]), kStreamWarps);
+    }
+    mbar_init_fence();
+  }
+}
+
+// Producer (one thread): stage tiles blockIdx.x, +gridDim.x, ... of the chunk
+// range into the ring.  On an expired wait it flags the error, lets every copy
+// it issued land, and stops.
+__device__ void stream_produce(const StreamRing& r, const uint16_t* x, uint32_t nchunks, unsigned* error) {
+  const uint32_t nstage = (nchunks + kStreamChunks - 1) / kStreamChunks;
+  uint32_t stage = 0, phase = 0, issued = 0, parity_bits = 0;
+  for (uint32_t i = blockIdx.x; i < nstage; i += gridDim.x) {
+    if (!mbar_wait_bounded(smem_addr(&r.empty[stage]), phase ^ 1u)) {
+      if (error != nullptr) atomicOr(error, 4u);
+      for (int s = 0; s < kStreamStages; ++s)
+        if (issued & (1u << s)) mbar_wait_bounded(smem_addr(&r.full[s]), (parity_bits >> s) & 1u);
+      return;
+    }
+    const uint32_t c0 = i * kStreamChunks;
+    const uint32_t n = min((uint32_t)kStreamChunks, nchunks - c0);
+    const uint32_t fb = smem_addr(&r.full[stage]);
+    mbar_expect_tx(fb, n * 16u);
+    bulk_g2s(smem_addr(r.data + (size_t)stage * kStreamChunks), x + (size_t)c0 * 8, n * 16u, fb);
+    issued |= 1u << stage;
+    parity_bits = (parity_bits & ~(1u << stage)) | (phase << stage);
+    if (++stage == kStreamStages) {
+      stage = 0;
+      phase ^= 1u;
+    }
+  }
+}
+
+template <int FMT, int RND, int HAD, bool SFMMA>
+__global__ void __launch_bounds__(kStreamThreads, 1) quantize_stream_kernel(QRowParams p) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  __shared__ float2 tab[128];
+  const StreamRing r = stream_ring(smem);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  stream_ring_init(r);
+  NvConsts nv{1.0f, 1.0f, true, tab};
+  if (FMT == FMT_NV) {
+    nv.s_t = *p.ts;
+    nv.y_st = __frcp_rn(nv.s_t);
+    nv.st_ok = recip_usable(nv.s_t);
+    nv_fill_scale_table(tab, nv.s_t);
+    if (p.ts_copy_out != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *p.ts_copy_out = nv.s_t;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    if (lane == 0) stream_produce(r, p.x, p.nchunks, p.error);
+    return;
+  }
+  const int cw = warp - 1;
+  const uint32_t nstage = (p.nchunks + kStreamChunks - 1) / kStreamChunks;
+  uint32_t stage = 0, phase = 0;
+  for (uint32_t i = blockIdx.x; i < nstage; i += gridDim.x) {
+    int ok = 1;
+    if (lane == 0) ok = mbar_wait_bounded(smem_addr(&r.full[stage]), phase) ? 1 : 0;
+    if (!__shfl_sync(0xFFFFFFFFu, ok, 0)) {
+      if (lane == 0 && p.error != nullptr) atomicOr(p.error, 4u);
+      return;
+    }
+    const uint32_t c0 = i * kStreamChunks;
+    const uint32_t n = min((uint32_t)kStreamChunks, p.nchunks - c0);
+    const uint4* src = r.data + (size_t)stage * kStreamChunks;
+#pragma unroll
+    for (int k = 0; k < kStreamChunks / 32 / kStreamWarps; ++k) {
+      const uint32_t lt = (uint32_t)(cw + k * kStreamWarps);
+      if (lt * 32u >= n) break;                          // warp-uniform
+      const uint32_t local = lt * 32u + lane;
+      const bool valid = local < n;
+      const uint4 v = valid ? src[local] : make_uint4(0u, 0u, 0u, 0u);
+      quantize_chunk<FMT, RND, HAD, SFMMA>(p, v, c0 + local, valid, lane, nv);
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(smem_addr(&r.empty[stage]));
+    if (++stage == kStreamStages) {
+      stage = 0;
+      phase ^= 1u;
+    }
+  }
+}
+
+// The amax pass on the same ring (contiguous input).
+template <int HAD>
+__global__ void __launch_bounds__(kStreamThreads, 1) amax_stream_kernel(AmaxParams p, unsigned* error) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  __shared__ uint32_t wmax[kStreamWarps];
+  __shared__ bool is_last;
+  const StreamRing r = stream_ring(smem);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  stream_ring_init(r);
+  __syncthreads();
+  float m = 0.0f;
+  if (warp == 0) {
+    if (lane == 0) stream_produce(r, p.x, p.rows_x_cpr, error);
+  } else {
+    const int cw = warp - 1;
+    const uint32_t nstage = (p.rows_x_cpr + kStreamChunks - 1) / kStreamChunks;
+    uint32_t stage = 0, phase = 0;
+    for (uint32_t i = blockIdx.x; i < nstage; i += gridDim.x) {
+      int ok = 1;
+      if (lane == 0) ok = mbar_wait_bounded(smem_addr(&r.full[stage]), phase) ? 1 : 0;
+      if (!__shfl_sync(0xFFFFFFFFu, ok, 0)) {
+        if (lane == 0 && error != nullptr) atomicOr(error, 4u);
+        break;
+      }
+      const uint32_t n = min((uint32_t)kStreamChunks, p.rows_x_cpr - i * kStreamChunks);
+      const uint4* src = r.data + (size_t)stage * kStreamChunks;
+#pragma unroll
+      for (int k = 0; k < kStreamChunks / 32 / kStreamWarps; ++k) {
+        const uint32_t lt = (uint32_t)(cw + k * kStreamWarps);
+        if (lt * 32u >= n) break;
+        const uint32_t local = lt * 32u + lane;
+        const uint4 v = local < n ? src[local] : make_uint4(0u, 0u, 0u, 0u);
+        float x[8];
+        unpack8(v, x);
+        if (HAD) hadamard_rotate<HAD>(x, lane);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) m = fmaxf(m, fabsf(x[j]));
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_addr(&r.empty[stage]));
+      if (++stage == kStreamStages) {
+        stage = 0;
+        phase ^= 1u;
+      }
+    }
+    const uint32_t b = __reduce_max_sync(0xFFFFFFFFu, __float_as_uint(m));
+    if (lane == 0) wmax[cw] = b;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    uint32_t b = 0;
+    for (int w = 0; w < kStreamWarps; ++w) b = max(b, wmax[w]);
+    p.partials[blockIdx.x] = __uint_as_float(b);
+    __threadfence();
+    is_last = (atomicAdd(p.counter, 1u) == gridDim.x - 1);
+  }
+  __syncthreads();
+  if (!is_last || warp != 0) return;
+  uint32_t b = 0;
+  for (uint32_t i = lane; i < gridDim.x; i += 32u) b = max(b, __float_as_uint(__ldcg(p.partials + i)));
+  b = __reduce_max_sync(0xFFFFFFFFu, b);
+  if (lane == 0) {
+    const float amax = __uint_as_float(b);
+    *p.out = p.mode == 0 ? amax : (amax == 0.0f ? 1.0f : __fdiv_rn(amax, 2688.0f));
+    *p.counter = 0u;
+  }
+}
+
+// ============================================ single-pass NVFP4 quantize ===
+// NVFP4 needs the tensor amax before any block can be scaled.  When the whole
+// tensor fits in shared memory across the SMs (148 x ~227 KB on B200), one
+// cooperative launch reads it from HBM once: each CTA stages a contiguous run
+// of warp tiles in shared memory while reducing its amax, the CTAs meet at a
+// bounded grid barrier, and each quantizes its staged slice.
+struct FusedParams {
+  QRowParams q;
+  float* ts_out;          // s_t, written by CTA 0
+  float* partials;        // one partial amax per CTA
+  unsigned* arrive;       // grid-barrier arrivals (zeroed before the launch)
+  unsigned* error;        // device error word (bit 1: barrier wait expired)
+  uint32_t tiles_per_cta; // 32-chunk warp tiles staged by each CTA
+};
+
+constexpr int kFusedThreads = 32 * (kStreamWarps + 1);   // producer warp + 16 consumer warps
+constexpr int kFusedMaxSmem = 227 * 1024 - 2048;          // staged slice; room left for the static data
+constexpr int kFusedPieces = 8;                           // bulk copies (and mbarriers) per slice
+
+template <int RND, int HAD, bool SFMMA>
+__global__ void __launch_bounds__(kFusedThreads, 1) nv_quantize_fused_kernel(FusedParams fp) {
+  extern __shared__ __align__(1024) uint4 slice[];
+  __shared__ float2 tab[128];
+  __shared__ float red[kStreamWarps];
+  __shared__ float s_t_shared;
+  __shared__ __align__(8) uint64_t piece_bar[kFusedPieces];
+  const QRowParams& p = fp.q;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const uint32_t ntiles = (p.nchunks + 31u) >> 5;
+  const uint32_t t_begin = blockIdx.x * fp.tiles_per_cta;
+  const uint32_t t_end = min(ntiles, t_begin + fp.tiles_per_cta);
+  const uint32_t c_begin = t_begin * 32u;
+  const uint32_t c_end = min(p.nchunks, t_end * 32u);
+  const uint32_t nslice = c_end > c_begin ? c_end - c_begin : 0u;
+  const uint32_t piece = ((nslice + kFusedPieces - 1) / kFusedPieces + 31u) & ~31u;   // chunks, whole warp tiles
+  if (threadIdx.x == 0) {
+    for (int k = 0; k < kFusedPieces; ++k) mbar_init(smem_addr(&piece_bar[k]), 1);
+    mbar_init_fence();
+  }
+  __syncthreads();
+  // phase 1: the slice lands in shared memory as kFusedPieces bulk copies; consumers reduce the
+  // amax (of the rotated values when HAD > 0) of each piece as soon as it arrives
+  if (warp == 0) {
+    if (lane == 0) {
+      for (int k = 0; k < kFusedPieces; ++k) {
+        const uint32_t a = min(nslice, (uint32_t)k * piece), b = min(nslice, (uint32_t)(k + 1) * piece);
+        const uint32_t bar = smem_addr(&piece_bar[k]);
+        if (b > a) {
+          mbar_expect_tx(bar, (b - a) * 16u);
+          bulk_g2s(smem_addr(slice + a), p.x + (size_t)(c_begin + a) * 8, (b - a) * 16u, bar);
+        } else {
+          mbar_arrive(bar);                                  // empty piece: complete its phase
+        }
+      }
+    }
+  } else {
+    const int cw = warp - 1;
+    float m = 0.0f;
+    for (int k = 0; k < kFusedPieces; ++k) {
+      const uint32_t a = min(nslice, (uint32_t)k * piece), b = min(nslice, (uint32_t)(k + 1) * piece);
+      if (b <= a) continue;
+      int ok = 1;
+      if (lane == 0) ok = mbar_wait_bounded(smem_addr(&piece_bar[k]), 0u) ? 1 : 0;
+      if (!__shfl_sync(0xFFFFFFFFu, ok, 0)) {
+        if (lane == 0) atomicOr(fp.error, 4u);
+        break;
+      }
+      for (uint32_t lt = a / 32u + cw; lt * 32u < b; lt += kStreamWarps) {
+        const uint32_t local = lt * 32u + lane;
+        const uint4 v = local < b ? slice[local] : make_uint4(0u, 0u, 0u, 0u);
+        float x[8];
+        unpack8(v, x);
+        if (HAD) hadamard_rotate<HAD>(x, lane);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) m = fmaxf(m, fabsf(x[j]));
+      }
+    }
+    m = __uint_as_float(__reduce_max_sync(0xFFFFFFFFu, __float_as_uint(m)));
+    if (lane == 0) red[cw] = m;
+  }
+  __syncthreads();
+
+  // grid barrier: publish this CTA's maximum, wait (bounded) for every CTA
+  if (threadIdx.x == 0) {
+    float cm = 0.0f;
+    for (int w = 0; w < kStreamWarps; ++w) cm = fmaxf(cm, red[w]);
+    fp.partials[blockIdx.x] = cm;
+    __threadfence();
+    atomicAdd(fp.arrive, 1u);
+    const uint64_t t0 = globaltimer_ns();
+    for (;;) {
+      unsigned n;
+      asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(n) : "l"(fp.arrive) : "memory");
+      if (n >= gridDim.x) break;
+      if (globaltimer_ns() - t0 > 2000000000ull) {       // 2 s: give up, flag the error, finish anyway
+        atomicOr(fp.error, 2u);
+        break;
+      }
+      __nanosleep(64);
+    }
+  }
+  __syncthreads();
+  if (warp == 0) {
+    uint32_t b = 0u;
+    for (uint32_t i = lane; i < gridDim.x; i += 32u) b = max(b, __float_as_uint(__ldcg(fp.partials + i)));
+    b = __reduce_max_sync(0xFFFFFFFFu, b);
+    if (lane == 0) {
+      const float amax = __uint_as_float(b);
+      const float s_t = amax == 0.0f ? 1.0f : __fdiv_rn(amax, 2688.0f);
+      s_t_shared = s_t;
+      if (blockIdx.x == 0) *fp.ts_out = s_t;
+    }
+  }
+  __syncthreads();
+  NvConsts nv{s_t_shared, __frcp_rn(s_t_shared), recip_usable(s_t_shared), tab};
+  nv_fill_scale_table(tab, nv.s_t);
+  __syncthreads();
+  if (warp == 0) return;
+
+  // phase 2: quantize the staged slice
+  for (uint32_t lt = (uint32_t)(warp - 1); lt * 32u < nslice; lt += kStreamWarps) {
+    const uint32_t local = lt * 32u + lane;
+    const bool valid = local < nslice;
+    const uint4 v = valid ? slice[local] : make_uint4(0u, 0u, 0u, 0u);
+    quantize_chunk<FMT_NV, RND, HAD, SFMMA>(p, v, c_begin + local, valid, lane, nv);
   }
 }
 
@@ -282,11 +603,16 @@ struct QColParams {
 template <int FMT, int RND, bool SFMMA>
 __global__ void __launch_bounds__(256) quantize_cols_kernel(QColParams p) {
   __shared__ __align__(16) uint16_t tile[128][64];
+  __shared__ float2 tab[128];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t tiles_r = (p.R + 127u) / 128u, tiles_c = (p.C + 63u) / 64u;
-  float s_t = 1.0f;
+  float s_t = 1.0f, y_st = 1.0f;
+  bool st_ok = true;
   if (FMT == FMT_NV) {
     s_t = *p.ts;
+    y_st = __frcp_rn(s_t);
+    st_ok = recip_usable(s_t);
+    nv_fill_scale_table(tab, s_t);          // visible after the first __syncthreads of the tile loop
     if (p.ts_copy_out != nullptr && blockIdx.x == 0 && tid == 0) *p.ts_copy_out = s_t;
   }
   for (uint32_t t = blockIdx.x; t < tiles_r * tiles_c; t += gridDim.x) {
@@ -328,12 +654,12 @@ __global__ void __launch_bounds__(256) quantize_cols_kernel(QColParams p) {
         inv = mx_inv_scale(byte);
         zero = (am == 0.0f);
       } else {
-        const float tt = __fdiv_rn(__fdiv_rn(am, 6.0f), s_t);
-        byte = e4m3_rn_sat(tt);
+        byte = e4m3_rn_sat(nv_scale_arg(am, s_t, y_st, st_ok));
         zero = (byte == 0u);
-        S = zero ? 1.0f : __fmul_rn(e4m3_value(byte), s_t);
-        y = __frcp_rn(S);
-        fast = recip_usable(S);
+        const float2 sy = tab[byte];
+        S = sy.x;
+        y = sy.y;
+        fast = true;
       }
 #pragma unroll
       for (int w8 = 0; w8 < BS / 8; ++w8) {
@@ -388,7 +714,17 @@ struct DeqParams {
 };
 
 template <int FMT, bool SFMMA, bool BF16>
+__device__ __forceinline__ void dequantize_chunk_to(const DeqParams& p, uint32_t chunk, uint32_t slot, uint32_t w,
+                                                    float s_t);
+
+template <int FMT, bool SFMMA, bool BF16>
 __device__ __forceinline__ void dequantize_chunk(const DeqParams& p, uint32_t chunk, uint32_t w, float s_t) {
+  dequantize_chunk_to<FMT, SFMMA, BF16>(p, chunk, chunk, w, s_t);
+}
+
+template <int FMT, bool SFMMA, bool BF16>
+__device__ __forceinline__ void dequantize_chunk_to(const DeqParams& p, uint32_t chunk, uint32_t slot, uint32_t w,
+                                                    float s_t) {
   constexpr int LPB = FMT == FMT_MX ? 4 : 2;
   uint32_t byte;
   if (SFMMA) {
@@ -415,33 +751,89 @@ __device__ __forceinline__ void dequantize_chunk(const DeqParams& p, uint32_t ch
       const uint32_t hi = __bfloat16_as_ushort(__float2bfloat16_rn(y[2 * i + 1]));
       o[i] = lo | (hi << 16);
     }
-    reinterpret_cast<uint4*>(p.out)[chunk] = make_uint4(o[0], o[1], o[2], o[3]);
+    reinterpret_cast<uint4*>(p.out)[slot] = make_uint4(o[0], o[1], o[2], o[3]);
   } else {
-    float4* o = reinterpret_cast<float4*>(p.out) + (size_t)chunk * 2;
+    float4* o = reinterpret_cast<float4*>(p.out) + (size_t)slot * 2;
     o[0] = make_float4(y[0], y[1], y[2], y[3]);
     o[1] = make_float4(y[4], y[5], y[6], y[7]);
   }
 }
 
-// Each thread takes two adjacent chunks (16 codes, one 8-byte load) per step;
-// the chunk count is even because rows hold a whole number of 16-element blocks.
+// Each thread takes four adjacent chunks (32 codes, one 16-byte load) per step;
+// a ragged last quad falls back to 4-byte loads.
 template <int FMT, bool SFMMA, bool BF16>
 __global__ void __launch_bounds__(256) dequantize_kernel(DeqParams p) {
   const float s_t = FMT == FMT_NV ? *p.ts : 1.0f;
-  const uint32_t npairs = p.nchunks / 2;
+  const uint32_t nquads = (p.nchunks + 3u) / 4u;
   const uint32_t stride = gridDim.x * blockDim.x;
-  for (uint32_t i = blockIdx.x * blockDim.x + threadIdx.x; i < npairs; i += 2 * stride) {
-    const uint2 a = __ldg(reinterpret_cast<const uint2*>(p.codes) + i);
-    const bool has2 = i + stride < npairs;
-    uint2 b = make_uint2(0u, 0u);
-    if (has2) b = __ldg(reinterpret_cast<const uint2*>(p.codes) + i + stride);
-    dequantize_chunk<FMT, SFMMA, BF16>(p, 2 * i, a.x, s_t);
-    dequantize_chunk<FMT, SFMMA, BF16>(p, 2 * i + 1, a.y, s_t);
-    if (has2) {
-      dequantize_chunk<FMT, SFMMA, BF16>(p, 2 * (i + stride), b.x, s_t);
-      dequantize_chunk<FMT, SFMMA, BF16>(p, 2 * (i + stride) + 1, b.y, s_t);
+  for (uint32_t i = blockIdx.x * blockDim.x + threadIdx.x; i < nquads; i += stride) {
+    const uint32_t c0 = 4u * i;
+    if (c0 + 4u <= p.nchunks) {
+      const uint4 w = __ldg(reinterpret_cast<const uint4*>(p.codes) + i);
+      dequantize_chunk<FMT, SFMMA, BF16>(p, c0, w.x, s_t);
+      dequantize_chunk<FMT, SFMMA, BF16>(p, c0 + 1, w.y, s_t);
+      dequantize_chunk<FMT, SFMMA, BF16>(p, c0 + 2, w.z, s_t);
+      dequantize_chunk<FMT, SFMMA, BF16>(p, c0 + 3, w.w, s_t);
+    } else {
+      for (uint32_t c = c0; c < p.nchunks; ++c) dequantize_chunk<FMT, SFMMA, BF16>(p, c, __ldg(p.codes + c), s_t);
     }
   }
+}
+
+// Dequantize through shared memory: each CTA fills 512-chunk output tiles
+// (16 KB fp32 / 8 KB bf16) in a 4-deep staging ring and writes each tile back
+// with one bulk store, so the stores never queue behind per-thread traffic.
+constexpr int kDeqTileChunks = 512;
+constexpr int kDeqStages = 4;
+constexpr int kDeqThreads = 256;
+
+template <int FMT, bool SFMMA, bool BF16>
+__global__ void __launch_bounds__(kDeqThreads) dequantize_stream_kernel(DeqParams p) {
+  constexpr int kOut = BF16 ? 16 : 32;                   // output bytes per chunk
+  constexpr int kTileBytes = kDeqTileChunks * kOut;
+  extern __shared__ __align__(128) uint8_t stage_buf[];
+  const float s_t = FMT == FMT_NV ? *p.ts : 1.0f;
+  const uint32_t ntiles = (p.nchunks + kDeqTileChunks - 1) / kDeqTileChunks;
+  DeqParams q = p;
+  int it = 0;
+  uint32_t w_next[2] = {0u, 0u};
+  uint32_t i = blockIdx.x;
+  if (i < ntiles) {
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const uint32_t c = i * kDeqTileChunks + threadIdx.x + k * kDeqThreads;
+      if (c < p.nchunks) w_next[k] = __ldg(p.codes + c);
+    }
+  }
+  for (; i < ntiles; i += gridDim.x, ++it) {
+    const int stage = it % kDeqStages;
+    uint32_t w[2] = {w_next[0], w_next[1]};
+    const uint32_t inext = i + gridDim.x;
+    if (inext < ntiles) {                                 // prefetch the next tile's codes
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        const uint32_t c = inext * kDeqTileChunks + threadIdx.x + k * kDeqThreads;
+        w_next[k] = c < p.nchunks ? __ldg(p.codes + c) : 0u;
+      }
+    }
+    if (threadIdx.x == 0 && it >= kDeqStages) bulk_wait_read<kDeqStages - 1>();
+    __syncthreads();                                      // this stage's previous store has read its data
+    q.out = stage_buf + stage * kTileBytes;               // chunk-local output pointer
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const uint32_t local = threadIdx.x + k * kDeqThreads;
+      const uint32_t c = i * kDeqTileChunks + local;
+      if (c < p.nchunks) dequantize_chunk_to<FMT, SFMMA, BF16>(q, c, local, w[k], s_t);
+    }
+    fence_async_smem();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      const uint32_t n = min((uint32_t)kDeqTileChunks, p.nchunks - i * kDeqTileChunks);
+      bulk_s2g(static_cast<uint8_t*>(p.out) + (size_t)i * kTileBytes, smem_addr(stage_buf + stage * kTileBytes),
+               n * (uint32_t)kOut);
+    }
+  }
+  if (threadIdx.x == 0) bulk_wait_all();
 }
 
 // ============================================================== launchers ===
@@ -463,6 +855,19 @@ static cudaError_t amax_launch(const AmaxParams& ap, uint32_t ntiles, int num_sm
   return cudaGetLastError();
 }
 
+template <int HAD>
+static cudaError_t amax_stream_launch(const AmaxParams& ap, int num_sms, unsigned* error, cudaStream_t st) {
+  static const cudaError_t attr =
+      cudaFuncSetAttribute(amax_stream_kernel<HAD>, cudaFuncAttributeMaxDynamicSharedMemorySize, kStreamSmem);
+  if (attr != cudaSuccess) return attr;
+  const uint32_t nstage = (ap.rows_x_cpr + kStreamChunks - 1) / kStreamChunks;
+  uint32_t grid = (uint32_t)num_sms;
+  if (grid > (uint32_t)kMaxAmaxBlocks) grid = kMaxAmaxBlocks;
+  if (nstage < grid) grid = nstage > 0 ? nstage : 1;
+  amax_stream_kernel<HAD><<<grid, kStreamThreads, kStreamSmem, st>>>(ap, error);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_amax(const void* x, int64_t rows, int64_t cols, int64_t ld, int had, int mode, float* out,
                         const Scratch& s, int num_sms, cudaStream_t st) {
   AmaxParams ap;
@@ -476,6 +881,16 @@ cudaError_t launch_amax(const void* x, int64_t rows, int64_t cols, int64_t ld, i
   ap.out = out;
   ap.mode = mode;
   const uint32_t ntiles = (ap.rows_x_cpr + 31u) / 32u;
+  if (ap.contig) {
+    switch (had) {
+      case 0: return amax_stream_launch<0>(ap, num_sms, s.error, st);
+      case 16: return amax_stream_launch<16>(ap, num_sms, s.error, st);
+      case 32: return amax_stream_launch<32>(ap, num_sms, s.error, st);
+      case 64: return amax_stream_launch<64>(ap, num_sms, s.error, st);
+      case 128: return amax_stream_launch<128>(ap, num_sms, s.error, st);
+      default: return cudaErrorInvalidValue;
+    }
+  }
   switch (had) {
     case 0: return amax_launch<0>(ap, ntiles, num_sms, st);
     case 16: return amax_launch<16>(ap, ntiles, num_sms, st);
@@ -508,7 +923,21 @@ cudaError_t launch_nv_tensor_scale(const float* amax, float* out, cudaStream_t s
 }
 
 template <int FMT, int RND, int HAD, bool SFMMA>
+static cudaError_t rows_stream_launch(const QRowParams& qp, int num_sms, cudaStream_t st) {
+  auto kernel = quantize_stream_kernel<FMT, RND, HAD, SFMMA>;
+  static const cudaError_t attr =
+      cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kStreamSmem);
+  if (attr != cudaSuccess) return attr;
+  const uint32_t nstage = (qp.nchunks + kStreamChunks - 1) / kStreamChunks;
+  uint32_t grid = (uint32_t)num_sms;
+  if (nstage < grid) grid = nstage > 0 ? nstage : 1;
+  kernel<<<grid, kStreamThreads, kStreamSmem, st>>>(qp);
+  return cudaGetLastError();
+}
+
+template <int FMT, int RND, int HAD, bool SFMMA>
 static cudaError_t rows_launch(const QRowParams& qp, int num_sms, cudaStream_t st) {
+  if (qp.contig) return rows_stream_launch<FMT, RND, HAD, SFMMA>(qp, num_sms, st);
   static int occ = resident_ctas(quantize_rows_kernel<FMT, RND, HAD, SFMMA>, 256);
   const uint32_t ntiles = (qp.nchunks + 31u) / 32u;
   uint32_t want = (ntiles + 8u * kUnroll - 1u) / (8u * kUnroll);
@@ -533,6 +962,78 @@ static cudaError_t rows_dispatch_had(const QRowParams& qp, int had, bool sfmma, 
     case 128: return rows_dispatch_sf<FMT, RND, 128>(qp, sfmma, num_sms, st);
     default: return cudaErrorInvalidValue;
   }
+}
+
+template <int RND, int HAD, bool SFMMA>
+static cudaError_t fused_launch(const FusedParams& fp, uint32_t grid, size_t smem, cudaStream_t st) {
+  auto kernel = nv_quantize_fused_kernel<RND, HAD, SFMMA>;
+  static const cudaError_t attr =
+      cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kFusedMaxSmem);
+  if (attr != cudaSuccess) return attr;
+  FusedParams args = fp;
+  void* kargs[] = {&args};
+  return cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(kernel), dim3(grid), dim3(kFusedThreads), kargs,
+                                     smem, st);
+}
+
+template <int RND, int HAD>
+static cudaError_t fused_dispatch_sf(const FusedParams& fp, bool sfmma, uint32_t grid, size_t smem, cudaStream_t st) {
+  return sfmma ? fused_launch<RND, HAD, true>(fp, grid, smem, st) : fused_launch<RND, HAD, false>(fp, grid, smem, st);
+}
+
+bool fused_nv_fits(int64_t rows, int64_t cols, int num_sms, size_t* smem_out, uint32_t* tiles_per_cta) {
+  const uint64_t nchunks = (uint64_t)rows * (uint64_t)(cols / 8);
+  const uint64_t ntiles = (nchunks + 31u) / 32u;
+  const uint64_t per = (ntiles + (uint64_t)num_sms - 1) / (uint64_t)num_sms;
+  const size_t smem = (size_t)per * 32u * 16u;
+  if (smem > (size_t)kFusedMaxSmem || num_sms > kMaxAmaxBlocks) return false;
+  *smem_out = smem;
+  *tiles_per_cta = (uint32_t)per;
+  return true;
+}
+
+cudaError_t launch_quantize_nv_fused(const QuantizeParams& p, float* ts_out, const Scratch& s, int num_sms,
+                                     cudaStream_t st) {
+  size_t smem = 0;
+  uint32_t per = 0;
+  if (!fused_nv_fits(p.rows, p.cols, num_sms, &smem, &per)) return cudaErrorInvalidValue;
+  FusedParams fp;
+  QRowParams& qp = fp.q;
+  qp.x = static_cast<const uint16_t*>(p.x);
+  qp.nchunks = (uint32_t)(p.rows * (p.cols / 8));
+  qp.cpr = make_fastdiv((uint32_t)(p.cols / 8));
+  qp.ld = p.ld;
+  qp.contig = (p.ld == p.cols);
+  qp.cols = (uint32_t)p.cols;
+  qp.g4 = (uint32_t)((p.cols / 16 + 3) / 4);
+  qp.seed = p.seed;
+  qp.ts = nullptr;
+  qp.ts_copy_out = nullptr;
+  qp.codes = reinterpret_cast<uint32_t*>(p.codes);
+  qp.scales = p.scales;
+  qp.rotated = p.rotated;
+  qp.error = s.error;
+  fp.ts_out = ts_out;
+  fp.partials = s.partials;
+  fp.arrive = s.grid_arrive;
+  fp.error = s.error;
+  fp.tiles_per_cta = per;
+  const uint64_t ntiles = ((uint64_t)qp.nchunks + 31u) / 32u;
+  const uint32_t grid = (uint32_t)((ntiles + per - 1) / per);
+  if (cudaMemsetAsync(s.grid_arrive, 0, sizeof(unsigned), st) != cudaSuccess) return cudaErrorUnknown;
+  const bool sfmma = p.sf_mma != 0;
+#define FP4_FUSED_HAD(H)                                                                               \
+  return p.rnd == RND_RTN ? fused_dispatch_sf<RND_RTN, H>(fp, sfmma, grid, smem, st)                  \
+                          : fused_dispatch_sf<RND_SR, H>(fp, sfmma, grid, smem, st)
+  switch (p.had) {
+    case 0: FP4_FUSED_HAD(0);
+    case 16: FP4_FUSED_HAD(16);
+    case 32: FP4_FUSED_HAD(32);
+    case 64: FP4_FUSED_HAD(64);
+    case 128: FP4_FUSED_HAD(128);
+    default: return cudaErrorInvalidValue;
+  }
+#undef FP4_FUSED_HAD
 }
 
 template <int FMT, int RND, bool SFMMA>
@@ -568,6 +1069,7 @@ cudaError_t launch_quantize(const QuantizeParams& p, int num_sms, cudaStream_t s
     qp.codes = reinterpret_cast<uint32_t*>(p.codes);
     qp.scales = p.scales;
     qp.rotated = p.rotated;
+    qp.error = p.error;
     if (p.fmt == FMT_MX)
       return p.rnd == RND_RTN ? rows_dispatch_had<FMT_MX, RND_RTN>(qp, p.had, sfmma, num_sms, st)
                               : rows_dispatch_had<FMT_MX, RND_SR>(qp, p.had, sfmma, num_sms, st);
@@ -595,11 +1097,18 @@ cudaError_t launch_quantize(const QuantizeParams& p, int num_sms, cudaStream_t s
 
 template <int FMT, bool SFMMA, bool BF16>
 static cudaError_t deq_launch(const DeqParams& dp, int num_sms, cudaStream_t st) {
-  static int occ = resident_ctas(dequantize_kernel<FMT, SFMMA, BF16>, 256);
-  uint32_t want = (dp.nchunks / 2 + 511u) / 512u;
+  auto kernel = dequantize_stream_kernel<FMT, SFMMA, BF16>;
+  constexpr int smem = kDeqStages * kDeqTileChunks * (BF16 ? 16 : 32);
+  static const int occ = [&] {
+    int n = 0;
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) return 1;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, kDeqThreads, smem) != cudaSuccess || n < 1) n = 1;
+    return n;
+  }();
+  const uint32_t ntiles = (dp.nchunks + kDeqTileChunks - 1) / kDeqTileChunks;
   uint32_t grid = (uint32_t)num_sms * (uint32_t)occ;
-  if (want < grid) grid = want > 0 ? want : 1;
-  dequantize_kernel<FMT, SFMMA, BF16><<<grid, 256, 0, st>>>(dp);
+  if (ntiles < grid) grid = ntiles > 0 ? ntiles : 1;
+  kernel<<<grid, kDeqThreads, smem, st>>>(dp);
   return cudaGetLastError();
 }
 

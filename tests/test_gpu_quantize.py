@@ -194,3 +194,20 @@ def test_full_size_nvfp4_student_t_4096(rnd):
                 np.testing.assert_array_equal(scales[r:r + 1], ref["scales"])
         want = O.dequantize(codes[blk], scales[blk], fmt="nvfp4", tensor_scale=s_t)
         np.testing.assert_array_equal(deq[blk].view(np.uint32), want.view(np.uint32))
+
+
+def test_nv_two_pass_path_large_tensor():
+    """A 64 MiB tensor is larger than the SMs' shared memory, so NVFP4 without a given tensor scale
+    takes the two-pass path (amax kernel, then quantize); 64 sampled rows checked bit-exactly."""
+    from workloads import student_t_bf16
+    xb = student_t_bf16((8192, 4096), 3.0, 0.1, 7, 0)
+    x = dev_bf16(xb)
+    q = F.fp4_quantize(x, fmt="nvfp4", rnd="sr", seed=3)
+    x32 = bf16_to_f32(xb)
+    s_t = O.nv_tensor_scale(x32)
+    assert host_f32(q.tensor_scale)[0] == s_t
+    codes, scales = host_u8(q.codes), host_u8(q.scales)
+    for r in np.sort(np.random.default_rng(1).choice(8192, 64, replace=False)):
+        ref = O.quantize_values(x32[r:r + 1], fmt="nvfp4", rnd="sr", seed=3, tensor_scale=s_t, idx_base=int(r) * 4096)
+        np.testing.assert_array_equal(codes[r:r + 1], ref["codes"])
+        np.testing.assert_array_equal(scales[r:r + 1], ref["scales"])
