@@ -69,20 +69,26 @@ __device__ __forceinline__ uint32_t e2m1_sr(float v, uint32_t r) {
 // q0 = RN(x*y) is within 1.5 ulp of x/S; one FMA correction
 // q1 = RN(q0 + (x - S*q0)*y) is faithful, and a second correction with a
 // faithful quotient and y = RN(1/S) is correctly rounded (Markstein's
-// theorem).  The residuals x - S*q are exact while x, S and the quotient stay
-// well inside the normal range; `ok` is false otherwise and the caller then
-// uses the IEEE division.  copysign keeps the sign of a zero dividend.
-__device__ __forceinline__ float div_by_recip(float x, float S, float y, bool& ok) {
+// theorem).  The residual is formed as -(S*q - x), which keeps the sign of a
+// zero dividend through both corrections.  Valid when the residuals are exact
+// and the quotient normal: |x| >= 2^-103 or x == 0, with S in
+// [2^-125, 2^20] (recip_usable); callers check that per block and fall back
+// to the IEEE division otherwise.  The quotient must also stay far from
+// overflow (|x| * y < 2^64), or the corrections turn an infinite quotient into
+// NaN; the quantizers check the block maximum.
+__device__ __forceinline__ float div_by_recip(float x, float S, float y) {
   float q = __fmul_rn(x, y);
-  float r = __fmaf_rn(-q, S, x);
+  float r = -__fmaf_rn(q, S, -x);
   q = __fmaf_rn(r, y, q);
-  r = __fmaf_rn(-q, S, x);
-  q = __fmaf_rn(r, y, q);
-  const float ax = fabsf(x);
-  ok = (ax == 0.0f) || (ax >= 0x1p-100f && fabsf(q) >= 0x1p-120f);
-  return copysignf(q, x);
+  r = -__fmaf_rn(q, S, -x);
+  return __fmaf_rn(r, y, q);
 }
-__device__ __forceinline__ bool recip_usable(float S) { return S >= 0x1p-125f && S <= 0x1p+124f; }
+// Running minimum over a block of 2*|x| - 2 as an unsigned integer (zeros wrap
+// to the top): the block passes div_by_recip's |x| >= 2^-103 test iff the
+// minimum is >= 2*bits(2^-103) - 2.
+__device__ __forceinline__ uint32_t tiny_key(float x) { return (__float_as_uint(x) << 1) - 2u; }
+constexpr uint32_t kTinyKeyMin = (0x0C000000u << 1) - 2u;     // 2^-103 = biased exponent 24
+__device__ __forceinline__ bool recip_usable(float S) { return S >= 0x1p-125f && S <= 0x1p+20f; }
 
 // ---------------------------------------------------------------- Philox ----
 // Philox4x32 with 10 rounds (Salmon, Moraes, Dror, Shaw, SC'11): two 32x32
@@ -158,10 +164,10 @@ __device__ __forceinline__ float e4m3_value(uint32_t b) {
 // NVFP4 block-scale argument t = RN(RN(amax_b / 6) / s_t), bit-identical to two
 // IEEE divisions, from RN(1/6) and y_st = RN(1/s_t) (st_ok: recip_usable(s_t)).
 __device__ __forceinline__ float nv_scale_arg(float am, float s_t, float y_st, bool st_ok) {
-  bool ok1, ok2;
-  const float d6 = div_by_recip(am, 6.0f, 0x1.555556p-3f, ok1);     // 0x1.555556p-3 = RN(1/6)
-  const float t = div_by_recip(d6, s_t, y_st, ok2);
-  return (ok1 && ok2 && st_ok) ? t : __fdiv_rn(__fdiv_rn(am, 6.0f), s_t);
+  const float d6 = div_by_recip(am, 6.0f, 0x1.555556p-3f);          // 0x1.555556p-3 = RN(1/6)
+  const float t = div_by_recip(d6, s_t, y_st);
+  const bool ok = st_ok && (am == 0.0f || (am >= 0x1p-100f && d6 >= 0x1p-100f && __fmul_rn(d6, y_st) < 0x1p64f));
+  return ok ? t : __fdiv_rn(__fdiv_rn(am, 6.0f), s_t);
 }
 
 // Per-CTA table of the element divisor S = RN(e4m3(b) * s_t) and RN(1/S) for
@@ -218,6 +224,39 @@ __device__ __forceinline__ void hadamard_rotate(float (&x)[8], int lane) {
   const float s = HB == 16 ? 0.25f : HB == 32 ? 0.17677669529663687f : HB == 64 ? 0.125f : 0.08838834764831845f;
 #pragma unroll
   for (int i = 0; i < 8; ++i) x[i] = __fmul_rn(x[i], s);
+}
+
+// Same transform with one thread holding E consecutive elements (E = 16 or
+// 32, a whole scale block): butterflies inside the thread for distances < E,
+// then across HB/E consecutive lanes.  The stages run in the same order
+// (distance 1, 2, 4, ...) with the same operand order as hadamard_rotate, so
+// both layouts give bit-identical fp32 results.
+template <int HB, int E>
+__device__ __forceinline__ void hadamard_rotate_block(float (&x)[E], int lane) {
+  constexpr int IN = HB < E ? HB : E;
+#pragma unroll
+  for (int d = 1; d < IN; d <<= 1) {
+#pragma unroll
+    for (int i = 0; i < E; ++i) {
+      if ((i & d) == 0) {
+        const float a = x[i], b = x[i + d];
+        x[i] = __fadd_rn(a, b);
+        x[i + d] = __fsub_rn(a, b);
+      }
+    }
+  }
+#pragma unroll
+  for (int ld = 1; ld < HB / E; ld <<= 1) {
+    const bool upper = (lane & ld) != 0;
+#pragma unroll
+    for (int i = 0; i < E; ++i) {
+      const float p = __shfl_xor_sync(0xFFFFFFFFu, x[i], ld);
+      x[i] = upper ? __fsub_rn(p, x[i]) : __fadd_rn(x[i], p);
+    }
+  }
+  const float s = HB == 16 ? 0.25f : HB == 32 ? 0.17677669529663687f : HB == 64 ? 0.125f : 0.08838834764831845f;
+#pragma unroll
+  for (int i = 0; i < E; ++i) x[i] = __fmul_rn(x[i], s);
 }
 
 // ------------------------------------------- bulk copies and mbarriers -----

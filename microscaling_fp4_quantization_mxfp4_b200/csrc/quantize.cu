@@ -133,6 +133,8 @@ __global__ void nv_tensor_scale_kernel(const float* amax, float* out) {
 struct QRowParams {
   const uint16_t* x;
   uint32_t nchunks;
+  uint32_t nblocks;      // scale blocks (rows * cols / block)
+  FastDiv bpr;           // scale blocks per row
   FastDiv cpr;           // chunks (8 elements) per row
   int64_t ld;
   int contig;            // ld == cols
@@ -147,7 +149,6 @@ struct QRowParams {
   unsigned* error;       // device error word (streaming kernels: bit 2 = a ring wait expired)
 };
 
-constexpr int kUnroll = 4;
 
 // Per-thread NVFP4 constants: the tensor scale, its reciprocal and the (S, 1/S) table.
 struct NvConsts {
@@ -156,86 +157,101 @@ struct NvConsts {
   const float2* tab;
 };
 
+// One thread quantizes one whole scale block of E = 32 (MX) or 16 (NV)
+// elements held as E/8 uint4: the block maximum, the scale and every division
+// are computed once per block, with E independent element computations.
+template <int FMT>
+struct BlockShape {
+  static constexpr int E = FMT == FMT_MX ? 32 : 16;   // elements per block
+  static constexpr int V = E / 8;                      // uint4 per block
+};
+
 template <int FMT, int RND, int HAD, bool SFMMA>
-__device__ __forceinline__ void quantize_chunk(const QRowParams& p, const uint4 v, uint32_t chunk, bool valid,
-                                               int lane, const NvConsts& nv) {
-  constexpr int LPB = FMT == FMT_MX ? 4 : 2;   // lanes per scale block
-  float x[8];
-  unpack8(v, x);
+__device__ __forceinline__ void quantize_block(const QRowParams& p, const uint4 (&v)[BlockShape<FMT>::V], uint32_t blk,
+                                               bool valid, int lane, const NvConsts& nv) {
+  constexpr int E = BlockShape<FMT>::E, V = BlockShape<FMT>::V;
+  float x[E];
+#pragma unroll
+  for (int k = 0; k < V; ++k) {
+    float t8[8];
+    unpack8(v[k], t8);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) x[8 * k + i] = t8[i];
+  }
   if (HAD) {
-    hadamard_rotate<HAD>(x, lane);
+    hadamard_rotate_block<HAD, E>(x, lane);
     if (p.rotated != nullptr && valid) {
-      float4* r = reinterpret_cast<float4*>(p.rotated + (size_t)chunk * 8);
-      r[0] = make_float4(x[0], x[1], x[2], x[3]);
-      r[1] = make_float4(x[4], x[5], x[6], x[7]);
+      float4* r = reinterpret_cast<float4*>(p.rotated + (size_t)blk * E);
+#pragma unroll
+      for (int k = 0; k < E / 4; ++k) r[k] = make_float4(x[4 * k], x[4 * k + 1], x[4 * k + 2], x[4 * k + 3]);
     }
   }
   float am = 0.0f;
 #pragma unroll
-  for (int i = 0; i < 8; ++i) am = fmaxf(am, fabsf(x[i]));
-#pragma unroll
-  for (int o = 1; o < LPB; o <<= 1) am = fmaxf(am, __shfl_xor_sync(0xFFFFFFFFu, am, o));
-
+  for (int i = 0; i < E; ++i) am = fmaxf(am, fabsf(x[i]));
   uint32_t byte;
   bool zero;
-  float v8[8];
   if (FMT == FMT_MX) {
     byte = mx_scale_byte(am);
     const float inv = mx_inv_scale(byte);
 #pragma unroll
-    for (int i = 0; i < 8; ++i) v8[i] = __fmul_rn(x[i], inv);     // exact power-of-two scaling
+    for (int i = 0; i < E; ++i) x[i] = __fmul_rn(x[i], inv);          // exact power-of-two scaling
     zero = (am == 0.0f);
   } else {
     byte = e4m3_rn_sat(nv_scale_arg(am, nv.s_t, nv.y_st, nv.st_ok));
     zero = (byte == 0u);
     const float2 sy = nv.tab[byte];
-    const float S = sy.x, y = sy.y;
-    bool ok = true;
+    uint32_t kmin = 0xFFFFFFFFu;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      bool oki;
-      v8[i] = div_by_recip(x[i], S, y, oki);
-      ok = ok && oki;
-    }
-    if (__any_sync(0xFFFFFFFFu, !ok)) {       // rare: tiny values or scales -> IEEE division
-      if (!ok) {
+    for (int i = 0; i < E; ++i) kmin = min(kmin, tiny_key(x[i]));
+    if (sy.y != 0.0f && kmin >= kTinyKeyMin && __fmul_rn(am, sy.y) < 0x1p64f) {
 #pragma unroll
-        for (int i = 0; i < 8; ++i) v8[i] = __fdiv_rn(x[i], S);
-      }
+      for (int i = 0; i < E; ++i) x[i] = div_by_recip(x[i], sy.x, sy.y);
+    } else {                                     // rare: tiny operands or scales -> IEEE division
+#pragma unroll
+      for (int i = 0; i < E; ++i) x[i] = __fdiv_rn(x[i], sy.x);
     }
   }
-  uint32_t packed;
+  uint32_t w[E / 8];
   if (RND == RND_RTN) {
-    packed = pack8_rtn(v8);
-  } else {
-    uint32_t r[8];
-    philox_words8((unsigned long long)chunk * 8ull, p.seed, r);
-    packed = 0u;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) packed |= e2m1_sr(v8[i], r[i]) << (4 * i);
-  }
-  if (zero) packed = 0u;
-  if (valid) {
-    p.codes[chunk] = packed;
-    if ((lane & (LPB - 1)) == 0) {
-      if (SFMMA) {
-        const uint32_t row = fdiv(chunk, p.cpr);
-        const uint32_t g = (chunk - row * p.cpr.d) / LPB;
-        p.scales[sf_mma_offset(row, g, p.g4)] = (uint8_t)byte;
-      } else {
-        p.scales[chunk / LPB] = (uint8_t)byte;
-      }
+    for (int k = 0; k < E / 8; ++k)
+      w[k] = e2m1x4_rn(x[8 * k], x[8 * k + 1], x[8 * k + 2], x[8 * k + 3], x[8 * k + 4], x[8 * k + 5], x[8 * k + 6],
+                       x[8 * k + 7]);
+  } else {
+    const unsigned long long j0 = (unsigned long long)blk * (E / 4);     // Philox counter of element blk*E
+#pragma unroll
+    for (int k = 0; k < E / 8; ++k) {
+      const unsigned long long j = j0 + 2u * k;
+      const u32x4 a = philox4x32_10((uint32_t)j, (uint32_t)(j >> 32), (uint32_t)p.seed, (uint32_t)(p.seed >> 32));
+      const u32x4 b = philox4x32_10((uint32_t)(j + 1), (uint32_t)((j + 1) >> 32), (uint32_t)p.seed,
+                                    (uint32_t)(p.seed >> 32));
+      const float* xe = x + 8 * k;
+      w[k] = e2m1_sr(xe[0], a.x) | (e2m1_sr(xe[1], a.y) << 4) | (e2m1_sr(xe[2], a.z) << 8) |
+             (e2m1_sr(xe[3], a.w) << 12) | (e2m1_sr(xe[4], b.x) << 16) | (e2m1_sr(xe[5], b.y) << 20) |
+             (e2m1_sr(xe[6], b.z) << 24) | (e2m1_sr(xe[7], b.w) << 28);
     }
+  }
+  if (!valid) return;
+  if (FMT == FMT_MX) {
+    reinterpret_cast<uint4*>(p.codes)[blk] = zero ? make_uint4(0u, 0u, 0u, 0u) : make_uint4(w[0], w[1], w[2], w[3]);
+  } else {
+    reinterpret_cast<uint2*>(p.codes)[blk] = zero ? make_uint2(0u, 0u) : make_uint2(w[0], w[1]);
+  }
+  if (SFMMA) {
+    const uint32_t row = fdiv(blk, p.bpr);
+    p.scales[sf_mma_offset(row, blk - row * p.bpr.d, p.g4)] = (uint8_t)byte;
+  } else {
+    p.scales[blk] = (uint8_t)byte;
   }
 }
 
+// Strided inputs (ld != cols): one thread per scale block, loads straight from global memory.
 template <int FMT, int RND, int HAD, bool SFMMA>
 __global__ void __launch_bounds__(256) quantize_rows_kernel(QRowParams p) {
-  const int lane = threadIdx.x & 31;
-  const uint32_t ntiles = (p.nchunks + 31u) >> 5;
-  const uint32_t gwarp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const uint32_t nwarps = (gridDim.x * blockDim.x) >> 5;
+  constexpr int V = BlockShape<FMT>::V;
   __shared__ float2 tab[128];
+  const int lane = threadIdx.x & 31;
   NvConsts nv{1.0f, 1.0f, true, tab};
   if (FMT == FMT_NV) {
     nv.s_t = *p.ts;
@@ -245,31 +261,22 @@ __global__ void __launch_bounds__(256) quantize_rows_kernel(QRowParams p) {
     if (p.ts_copy_out != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *p.ts_copy_out = nv.s_t;
     __syncthreads();
   }
-  for (uint32_t t0 = gwarp; t0 < ntiles; t0 += nwarps * kUnroll) {
-    uint4 v[kUnroll];
-    uint32_t chunk[kUnroll];
+  const uint32_t nunits = (p.nblocks + 31u) >> 5;               // warp units of 32 blocks
+  const uint32_t gwarp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const uint32_t nwarps = (gridDim.x * blockDim.x) >> 5;
+  for (uint32_t u = gwarp; u < nunits; u += nwarps) {
+    const uint32_t blk = u * 32u + lane;
+    const bool valid = blk < p.nblocks;
+    uint4 v[V];
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      const uint32_t t = t0 + (uint32_t)u * nwarps;
-      chunk[u] = t * 32u + lane;
-      if (t < ntiles && chunk[u] < p.nchunks) {
-        if (p.contig) {
-          v[u] = ld_stream(p.x + (int64_t)chunk[u] * 8);
-        } else {
-          const uint32_t row = fdiv(chunk[u], p.cpr);
-          const uint32_t c8 = chunk[u] - row * p.cpr.d;
-          v[u] = ld_stream(p.x + (int64_t)row * p.ld + (int64_t)c8 * 8);
-        }
-      } else {
-        v[u] = make_uint4(0u, 0u, 0u, 0u);
-      }
-    }
+    for (int k = 0; k < V; ++k) v[k] = make_uint4(0u, 0u, 0u, 0u);
+    if (valid) {
+      const uint32_t row = fdiv(blk, p.bpr);
+      const uint16_t* src = p.x + (int64_t)row * p.ld + (int64_t)(blk - row * p.bpr.d) * (8 * V);
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      const uint32_t t = t0 + (uint32_t)u * nwarps;
-      if (t < ntiles)   // warp-uniform: every lane of the warp takes the same branch
-        quantize_chunk<FMT, RND, HAD, SFMMA>(p, v[u], chunk[u], chunk[u] < p.nchunks, lane, nv);
+      for (int k = 0; k < V; ++k) v[k] = ld_stream(src + 8 * k);
     }
+    quantize_block<FMT, RND, HAD, SFMMA>(p, v, blk, valid, lane, nv);
   }
 }
 
@@ -278,11 +285,20 @@ __global__ void __launch_bounds__(256) quantize_rows_kernel(QRowParams p) {
 // by the bulk-copy engine: one producer thread issues a cp.async.bulk per stage
 // (no per-thread load traffic, many bytes in flight), 16 consumer warps
 // quantize (or reduce) each stage and release it through an mbarrier.
-constexpr int kStreamChunks = 2048;                     // 8-element chunks per stage (32 KB of bf16)
-constexpr int kStreamStages = 6;
-constexpr int kStreamWarps = 16;                        // consumer warps
-constexpr int kStreamThreads = 32 * (kStreamWarps + 1);
+constexpr int kStreamChunks = 4096;                     // 8-element chunks per stage (64 KB of bf16)
+constexpr int kStreamStages = 3;
 constexpr int kStreamSmem = kStreamStages * kStreamChunks * 16 + 2 * kStreamStages * 8;
+// Consumer warps per CTA: 31 (with the producer, the 1024-thread maximum)
+// where a thread's live state is small (NVFP4's 16-element blocks, the amax),
+// 16 for MXFP4's 32-element blocks.  Units of a stage are dealt to the warps
+// round-robin, starting one place further on each stage, so that counts that
+// do not divide evenly still balance over a run.
+template <int FMT>
+struct StreamWarps {
+  static constexpr int kWarps = FMT == FMT_MX ? 16 : 31;    // producer + consumers <= 1024 threads
+  static constexpr int kThreads = 32 * (kWarps + 1);
+};
+constexpr int kAmaxWarps = 31;
 
 struct StreamRing {
   uint4* data;
@@ -298,11 +314,11 @@ __device__ __forceinline__ StreamRing stream_ring(uint8_t* smem) {
   return r;
 }
 
-__device__ __forceinline__ void stream_ring_init(const StreamRing& r) {
+__device__ __forceinline__ void stream_ring_init(const StreamRing& r, int consumer_warps) {
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStreamStages; ++s) {
       mbar_init(smem_addr(&r.full[s]), 1);
-      mbar_init(smem_addr(&r.empty[s]), kStreamWarps);
+      mbar_init(smem_addr(&r.empty[s]), (uint32_t)consumer_warps);
     }
     mbar_init_fence();
   }
@@ -336,12 +352,13 @@ __device__ void stream_produce(const StreamRing& r, const uint16_t* x, uint32_t 
 }
 
 template <int FMT, int RND, int HAD, bool SFMMA>
-__global__ void __launch_bounds__(kStreamThreads, 1) quantize_stream_kernel(QRowParams p) {
+__global__ void __launch_bounds__(StreamWarps<FMT>::kThreads, 1) quantize_stream_kernel(QRowParams p) {
+  constexpr int kStreamWarps = StreamWarps<FMT>::kWarps;
   extern __shared__ __align__(1024) uint8_t smem[];
   __shared__ float2 tab[128];
   const StreamRing r = stream_ring(smem);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  stream_ring_init(r);
+  stream_ring_init(r, kStreamWarps);
   NvConsts nv{1.0f, 1.0f, true, tab};
   if (FMT == FMT_NV) {
     nv.s_t = *p.ts;
@@ -368,14 +385,16 @@ __global__ void __launch_bounds__(kStreamThreads, 1) quantize_stream_kernel(QRow
     const uint32_t c0 = i * kStreamChunks;
     const uint32_t n = min((uint32_t)kStreamChunks, p.nchunks - c0);
     const uint4* src = r.data + (size_t)stage * kStreamChunks;
+    constexpr int V = BlockShape<FMT>::V;
+    constexpr uint32_t kUnits = kStreamChunks / (32 * V);                   // warp units per full stage
+    const uint32_t first = ((uint32_t)cw + kStreamWarps - (i / gridDim.x * kUnits) % kStreamWarps) % kStreamWarps;
+    for (uint32_t u = first; u * 32u * V < n; u += kStreamWarps) {         // warp-uniform
+      const uint32_t lb = u * 32u + lane;                                    // block within the stage
+      const bool valid = lb * V < n;
+      uint4 v[V];
 #pragma unroll
-    for (int k = 0; k < kStreamChunks / 32 / kStreamWarps; ++k) {
-      const uint32_t lt = (uint32_t)(cw + k * kStreamWarps);
-      if (lt * 32u >= n) break;                          // warp-uniform
-      const uint32_t local = lt * 32u + lane;
-      const bool valid = local < n;
-      const uint4 v = valid ? src[local] : make_uint4(0u, 0u, 0u, 0u);
-      quantize_chunk<FMT, RND, HAD, SFMMA>(p, v, c0 + local, valid, lane, nv);
+      for (int k = 0; k < V; ++k) v[k] = valid ? src[lb * V + k] : make_uint4(0u, 0u, 0u, 0u);
+      quantize_block<FMT, RND, HAD, SFMMA>(p, v, c0 / V + lb, valid, lane, nv);
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(smem_addr(&r.empty[stage]));
@@ -388,13 +407,14 @@ __global__ void __launch_bounds__(kStreamThreads, 1) quantize_stream_kernel(QRow
 
 // The amax pass on the same ring (contiguous input).
 template <int HAD>
-__global__ void __launch_bounds__(kStreamThreads, 1) amax_stream_kernel(AmaxParams p, unsigned* error) {
+__global__ void __launch_bounds__(32 * (kAmaxWarps + 1), 1) amax_stream_kernel(AmaxParams p, unsigned* error) {
+  constexpr int kStreamWarps = kAmaxWarps;
   extern __shared__ __align__(1024) uint8_t smem[];
   __shared__ uint32_t wmax[kStreamWarps];
   __shared__ bool is_last;
   const StreamRing r = stream_ring(smem);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  stream_ring_init(r);
+  stream_ring_init(r, kStreamWarps);
   __syncthreads();
   float m = 0.0f;
   if (warp == 0) {
@@ -469,7 +489,8 @@ struct FusedParams {
   uint32_t tiles_per_cta; // 32-chunk warp tiles staged by each CTA
 };
 
-constexpr int kFusedThreads = 32 * (kStreamWarps + 1);   // producer warp + 16 consumer warps
+constexpr int kFusedWarps = 31;                            // consumer warps (1024 threads in all)
+constexpr int kFusedThreads = 32 * (kFusedWarps + 1);
 constexpr int kFusedMaxSmem = 227 * 1024 - 2048;          // staged slice; room left for the static data
 constexpr int kFusedPieces = 8;                           // bulk copies (and mbarriers) per slice
 
@@ -477,7 +498,7 @@ template <int RND, int HAD, bool SFMMA>
 __global__ void __launch_bounds__(kFusedThreads, 1) nv_quantize_fused_kernel(FusedParams fp) {
   extern __shared__ __align__(1024) uint4 slice[];
   __shared__ float2 tab[128];
-  __shared__ float red[kStreamWarps];
+  __shared__ float red[kFusedWarps];
   __shared__ float s_t_shared;
   __shared__ __align__(8) uint64_t piece_bar[kFusedPieces];
   const QRowParams& p = fp.q;
@@ -521,7 +542,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) nv_quantize_fused_kernel(Fus
         if (lane == 0) atomicOr(fp.error, 4u);
         break;
       }
-      for (uint32_t lt = a / 32u + cw; lt * 32u < b; lt += kStreamWarps) {
+      for (uint32_t lt = a / 32u + cw; lt * 32u < b; lt += kFusedWarps) {
         const uint32_t local = lt * 32u + lane;
         const uint4 v = local < b ? slice[local] : make_uint4(0u, 0u, 0u, 0u);
         float x[8];
@@ -539,7 +560,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) nv_quantize_fused_kernel(Fus
   // grid barrier: publish this CTA's maximum, wait (bounded) for every CTA
   if (threadIdx.x == 0) {
     float cm = 0.0f;
-    for (int w = 0; w < kStreamWarps; ++w) cm = fmaxf(cm, red[w]);
+    for (int w = 0; w < kFusedWarps; ++w) cm = fmaxf(cm, red[w]);
     fp.partials[blockIdx.x] = cm;
     __threadfence();
     atomicAdd(fp.arrive, 1u);
@@ -573,12 +594,14 @@ __global__ void __launch_bounds__(kFusedThreads, 1) nv_quantize_fused_kernel(Fus
   __syncthreads();
   if (warp == 0) return;
 
-  // phase 2: quantize the staged slice
-  for (uint32_t lt = (uint32_t)(warp - 1); lt * 32u < nslice; lt += kStreamWarps) {
-    const uint32_t local = lt * 32u + lane;
-    const bool valid = local < nslice;
-    const uint4 v = valid ? slice[local] : make_uint4(0u, 0u, 0u, 0u);
-    quantize_chunk<FMT_NV, RND, HAD, SFMMA>(p, v, c_begin + local, valid, lane, nv);
+  // phase 2: quantize the staged slice, one thread per 16-element block
+  for (uint32_t u = (uint32_t)(warp - 1); u * 64u < nslice; u += kFusedWarps) {
+    const uint32_t lb = u * 32u + lane;
+    const bool valid = lb * 2u < nslice;
+    uint4 v[2];
+    v[0] = valid ? slice[lb * 2u] : make_uint4(0u, 0u, 0u, 0u);
+    v[1] = valid ? slice[lb * 2u + 1u] : make_uint4(0u, 0u, 0u, 0u);
+    quantize_block<FMT_NV, RND, HAD, SFMMA>(p, v, c_begin / 2u + lb, valid, lane, nv);
   }
 }
 
@@ -659,7 +682,10 @@ __global__ void __launch_bounds__(256) quantize_cols_kernel(QColParams p) {
         const float2 sy = tab[byte];
         S = sy.x;
         y = sy.y;
-        fast = true;
+        uint32_t kmin = 0xFFFFFFFFu;
+#pragma unroll
+        for (int i = 0; i < BS; ++i) kmin = min(kmin, tiny_key(xv[b * BS + i]));
+        fast = y != 0.0f && kmin >= kTinyKeyMin && __fmul_rn(am, y) < 0x1p64f;
       }
 #pragma unroll
       for (int w8 = 0; w8 < BS / 8; ++w8) {
@@ -670,9 +696,7 @@ __global__ void __launch_bounds__(256) quantize_cols_kernel(QColParams p) {
           if (FMT == FMT_MX) {
             v8[i] = __fmul_rn(xi, inv);
           } else {
-            bool oki;
-            v8[i] = div_by_recip(xi, S, y, oki);
-            if (!(fast && oki)) v8[i] = __fdiv_rn(xi, S);
+            v8[i] = fast ? div_by_recip(xi, S, y) : __fdiv_rn(xi, S);
           }
         }
         uint32_t packed;
@@ -713,18 +737,16 @@ struct DeqParams {
   void* out;
 };
 
-template <int FMT, bool SFMMA, bool BF16>
-__device__ __forceinline__ void dequantize_chunk_to(const DeqParams& p, uint32_t chunk, uint32_t slot, uint32_t w,
-                                                    float s_t);
-
-template <int FMT, bool SFMMA, bool BF16>
-__device__ __forceinline__ void dequantize_chunk(const DeqParams& p, uint32_t chunk, uint32_t w, float s_t) {
-  dequantize_chunk_to<FMT, SFMMA, BF16>(p, chunk, chunk, w, s_t);
+// E2M1 values of both nibbles of every code byte (low nibble first): a 2 KB
+// shared-memory table, so dequantizing 8 codes is 4 table loads.
+__device__ __forceinline__ void fill_pair_table(float2* pairs) {
+  for (int b = threadIdx.x; b < 256; b += blockDim.x)
+    pairs[b] = make_float2(e2m1_value((uint32_t)b & 0xFu), e2m1_value((uint32_t)b >> 4));
 }
 
 template <int FMT, bool SFMMA, bool BF16>
 __device__ __forceinline__ void dequantize_chunk_to(const DeqParams& p, uint32_t chunk, uint32_t slot, uint32_t w,
-                                                    float s_t) {
+                                                    float s_t, const float2* pairs) {
   constexpr int LPB = FMT == FMT_MX ? 4 : 2;
   uint32_t byte;
   if (SFMMA) {
@@ -734,14 +756,20 @@ __device__ __forceinline__ void dequantize_chunk_to(const DeqParams& p, uint32_t
     byte = p.scales[chunk / LPB];
   }
   float y[8];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const float2 g = pairs[(w >> (8 * k)) & 0xFFu];
+    y[2 * k] = g.x;
+    y[2 * k + 1] = g.y;
+  }
   if (FMT == FMT_MX) {
     const float sc = mx_scale_value(byte);
 #pragma unroll
-    for (int i = 0; i < 8; ++i) y[i] = __fmul_rn(e2m1_value((w >> (4 * i)) & 0xFu), sc);
+    for (int i = 0; i < 8; ++i) y[i] = __fmul_rn(y[i], sc);
   } else {
     const float sb = e4m3_value(byte);
 #pragma unroll
-    for (int i = 0; i < 8; ++i) y[i] = __fmul_rn(__fmul_rn(e2m1_value((w >> (4 * i)) & 0xFu), sb), s_t);
+    for (int i = 0; i < 8; ++i) y[i] = __fmul_rn(__fmul_rn(y[i], sb), s_t);
   }
   if (BF16) {
     uint32_t o[4];
@@ -759,27 +787,6 @@ __device__ __forceinline__ void dequantize_chunk_to(const DeqParams& p, uint32_t
   }
 }
 
-// Each thread takes four adjacent chunks (32 codes, one 16-byte load) per step;
-// a ragged last quad falls back to 4-byte loads.
-template <int FMT, bool SFMMA, bool BF16>
-__global__ void __launch_bounds__(256) dequantize_kernel(DeqParams p) {
-  const float s_t = FMT == FMT_NV ? *p.ts : 1.0f;
-  const uint32_t nquads = (p.nchunks + 3u) / 4u;
-  const uint32_t stride = gridDim.x * blockDim.x;
-  for (uint32_t i = blockIdx.x * blockDim.x + threadIdx.x; i < nquads; i += stride) {
-    const uint32_t c0 = 4u * i;
-    if (c0 + 4u <= p.nchunks) {
-      const uint4 w = __ldg(reinterpret_cast<const uint4*>(p.codes) + i);
-      dequantize_chunk<FMT, SFMMA, BF16>(p, c0, w.x, s_t);
-      dequantize_chunk<FMT, SFMMA, BF16>(p, c0 + 1, w.y, s_t);
-      dequantize_chunk<FMT, SFMMA, BF16>(p, c0 + 2, w.z, s_t);
-      dequantize_chunk<FMT, SFMMA, BF16>(p, c0 + 3, w.w, s_t);
-    } else {
-      for (uint32_t c = c0; c < p.nchunks; ++c) dequantize_chunk<FMT, SFMMA, BF16>(p, c, __ldg(p.codes + c), s_t);
-    }
-  }
-}
-
 // Dequantize through shared memory: each CTA fills 512-chunk output tiles
 // (16 KB fp32 / 8 KB bf16) in a 4-deep staging ring and writes each tile back
 // with one bulk store, so the stores never queue behind per-thread traffic.
@@ -792,6 +799,8 @@ __global__ void __launch_bounds__(kDeqThreads) dequantize_stream_kernel(DeqParam
   constexpr int kOut = BF16 ? 16 : 32;                   // output bytes per chunk
   constexpr int kTileBytes = kDeqTileChunks * kOut;
   extern __shared__ __align__(128) uint8_t stage_buf[];
+  __shared__ float2 pairs[256];
+  fill_pair_table(pairs);
   const float s_t = FMT == FMT_NV ? *p.ts : 1.0f;
   const uint32_t ntiles = (p.nchunks + kDeqTileChunks - 1) / kDeqTileChunks;
   DeqParams q = p;
@@ -823,7 +832,7 @@ __global__ void __launch_bounds__(kDeqThreads) dequantize_stream_kernel(DeqParam
     for (int k = 0; k < 2; ++k) {
       const uint32_t local = threadIdx.x + k * kDeqThreads;
       const uint32_t c = i * kDeqTileChunks + local;
-      if (c < p.nchunks) dequantize_chunk_to<FMT, SFMMA, BF16>(q, c, local, w[k], s_t);
+      if (c < p.nchunks) dequantize_chunk_to<FMT, SFMMA, BF16>(q, c, local, w[k], s_t, pairs);
     }
     fence_async_smem();
     __syncthreads();
@@ -864,7 +873,7 @@ static cudaError_t amax_stream_launch(const AmaxParams& ap, int num_sms, unsigne
   uint32_t grid = (uint32_t)num_sms;
   if (grid > (uint32_t)kMaxAmaxBlocks) grid = kMaxAmaxBlocks;
   if (nstage < grid) grid = nstage > 0 ? nstage : 1;
-  amax_stream_kernel<HAD><<<grid, kStreamThreads, kStreamSmem, st>>>(ap, error);
+  amax_stream_kernel<HAD><<<grid, 32 * (kAmaxWarps + 1), kStreamSmem, st>>>(ap, error);
   return cudaGetLastError();
 }
 
@@ -931,7 +940,7 @@ static cudaError_t rows_stream_launch(const QRowParams& qp, int num_sms, cudaStr
   const uint32_t nstage = (qp.nchunks + kStreamChunks - 1) / kStreamChunks;
   uint32_t grid = (uint32_t)num_sms;
   if (nstage < grid) grid = nstage > 0 ? nstage : 1;
-  kernel<<<grid, kStreamThreads, kStreamSmem, st>>>(qp);
+  kernel<<<grid, StreamWarps<FMT>::kThreads, kStreamSmem, st>>>(qp);
   return cudaGetLastError();
 }
 
@@ -939,8 +948,8 @@ template <int FMT, int RND, int HAD, bool SFMMA>
 static cudaError_t rows_launch(const QRowParams& qp, int num_sms, cudaStream_t st) {
   if (qp.contig) return rows_stream_launch<FMT, RND, HAD, SFMMA>(qp, num_sms, st);
   static int occ = resident_ctas(quantize_rows_kernel<FMT, RND, HAD, SFMMA>, 256);
-  const uint32_t ntiles = (qp.nchunks + 31u) / 32u;
-  uint32_t want = (ntiles + 8u * kUnroll - 1u) / (8u * kUnroll);
+  const uint32_t nunits = (qp.nblocks + 31u) / 32u;
+  uint32_t want = (nunits + 7u) / 8u;
   uint32_t grid = (uint32_t)num_sms * (uint32_t)occ;
   if (want < grid) grid = want > 0 ? want : 1;
   quantize_rows_kernel<FMT, RND, HAD, SFMMA><<<grid, 256, 0, st>>>(qp);
@@ -1001,6 +1010,8 @@ cudaError_t launch_quantize_nv_fused(const QuantizeParams& p, float* ts_out, con
   QRowParams& qp = fp.q;
   qp.x = static_cast<const uint16_t*>(p.x);
   qp.nchunks = (uint32_t)(p.rows * (p.cols / 8));
+  qp.nblocks = (uint32_t)(p.rows * (p.cols / 16));
+  qp.bpr = make_fastdiv((uint32_t)(p.cols / 16));
   qp.cpr = make_fastdiv((uint32_t)(p.cols / 8));
   qp.ld = p.ld;
   qp.contig = (p.ld == p.cols);
@@ -1058,6 +1069,8 @@ cudaError_t launch_quantize(const QuantizeParams& p, int num_sms, cudaStream_t s
     QRowParams qp;
     qp.x = static_cast<const uint16_t*>(p.x);
     qp.nchunks = (uint32_t)(p.rows * (p.cols / 8));
+    qp.nblocks = (uint32_t)(p.rows * (p.cols / bs));
+    qp.bpr = make_fastdiv((uint32_t)(p.cols / bs));
     qp.cpr = make_fastdiv((uint32_t)(p.cols / 8));
     qp.ld = p.ld;
     qp.contig = (p.ld == p.cols);

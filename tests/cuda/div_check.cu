@@ -17,12 +17,10 @@ __global__ void div_check_kernel(const float* scales, int n, unsigned long long*
   for (uint32_t b = blockIdx.x * blockDim.x + threadIdx.x; b < 65536u; b += gridDim.x * blockDim.x) {
     if (((b >> 7) & 0xFFu) == 0xFFu) continue;            // bf16 Inf/NaN
     const float x = __uint_as_float(b << 16);
-    bool ok;
-    float q = fp4dev::div_by_recip(x, S, y, ok);
-    if (!(ok && usable)) {
-      q = __fdiv_rn(x, S);
-      ++slow;
-    }
+    // the quantizer's per-block guard, applied to a one-element block
+    const bool ok = usable && fp4dev::tiny_key(x) >= fp4dev::kTinyKeyMin && __fmul_rn(fabsf(x), y) < 0x1p64f;
+    float q = ok ? fp4dev::div_by_recip(x, S, y) : __fdiv_rn(x, S);
+    if (!ok) ++slow;
     const float ref = __fdiv_rn(x, S);
     if (__float_as_uint(q) != __float_as_uint(ref)) ++bad;
   }
