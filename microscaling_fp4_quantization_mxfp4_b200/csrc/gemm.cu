@@ -109,6 +109,20 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parit
       : "memory");
   return ok != 0u;
 }
+// Critical-path wait (producer, MMA issuer): spin on try_wait, checking the
+// abort flag and the time limit every 1024 polls.
+__device__ __forceinline__ bool wait_spin(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 1023u) == 0u) {
+      if (*abort_flag != 0) return false;
+      if (global_timer() - t0 > kWaitLimitNs) return false;
+    }
+  }
+}
+// Long waits (epilogue warps): sleep in hardware between polls.
 __device__ __noinline__ bool wait_bounded(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer();
@@ -288,7 +302,7 @@ __global__ void __launch_bounds__(Cfg<BN, FMT>::kThreads, 1)
         tile_coords(t, p.num_m, p.num_n, mt, nt);
         const int rb_here = min(BN / 128, rb_total - nt * (BN / 128));
         for (int kb = 0; kb < nkb; ++kb) {
-          if (!wait_bounded(smem_u32(&empty[stage]), phase ^ 1u, abort_flag)) {
+          if (!wait_spin(smem_u32(&empty[stage]), phase ^ 1u, abort_flag)) {
             raise_abort(abort_flag, p.error);
             ok = false;
             break;
@@ -338,7 +352,7 @@ __global__ void __launch_bounds__(Cfg<BN, FMT>::kThreads, 1)
         (void)mt;
         const int acc = local % C::kAccStages;
         const uint32_t use = (uint32_t)(local / C::kAccStages);
-        if (!wait_bounded(smem_u32(&tempty[acc]), (use & 1u) ^ 1u, abort_flag)) {
+        if (!wait_spin(smem_u32(&tempty[acc]), (use & 1u) ^ 1u, abort_flag)) {
           raise_abort(abort_flag, p.error);
           ok = false;
           break;
@@ -346,7 +360,7 @@ __global__ void __launch_bounds__(Cfg<BN, FMT>::kThreads, 1)
         tc_fence_after();
         const uint32_t d_tmem = tmem + (uint32_t)(acc * BN);
         for (int kb = 0; kb < nkb; ++kb) {
-          if (!wait_bounded(smem_u32(&full[stage]), phase, abort_flag)) {
+          if (!wait_spin(smem_u32(&full[stage]), phase, abort_flag)) {
             raise_abort(abort_flag, p.error);
             ok = false;
             break;
@@ -483,6 +497,321 @@ __global__ void __launch_bounds__(Cfg<BN, FMT>::kThreads, 1)
   }
 }
 
+// =========================================== SM-pair (cta_group::2) kernel ===
+// A cluster of two CTAs on neighbouring SMs computes a 256 x 256 output tile
+// with M = 256 MMAs issued by the even ("leader") CTA.  Each CTA stages its own
+// 128 rows of A and 128 of B's 256 rows (the MMA reads A and B from both CTAs'
+// shared memory at the same offsets), the scale factors of its A rows, and the
+// scale factors of all 256 B rows (each CTA's tensor memory holds its 128 x 256
+// accumulator).  Operand bytes per SM per MMA are half those of the 128 x 256
+// single-SM tile, and one MMA instruction does twice the work.
+//   - Both CTAs' TMA loads signal the leader's full barrier (cta_group::2 form);
+//     only the leader's producer posts the expected byte count of the pair.
+//   - The leader's MMA commits multicast to both CTAs' empty / accumulator-full
+//     barriers; both CTAs' epilogue warps arrive on the leader's
+//     accumulator-empty barrier (the follower remotely).
+//   - Every role falls through to one cluster barrier before tensor memory is
+//     freed, and every wait is bounded.
+// No load uses TMA multicast.
+namespace pair {
+
+constexpr int kEpiWarps = 8;
+constexpr int kThreads = 64 + 32 * kEpiWarps;
+
+template <int FMT>
+struct Cfg2 {
+  static constexpr int kApk = FmtTraits<FMT>::kAtomsPerKTile;
+  static constexpr int kABytes = 128 * BK_BYTES;
+  static constexpr int kBBytes = 128 * BK_BYTES;
+  static constexpr int kSfaBytes = kApk * 512;
+  static constexpr int kSfbBytes = 2 * kApk * 512;
+  static constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;
+  static constexpr int kStages = (220 * 1024) / kStageBytes > 8 ? 8 : (220 * 1024) / kStageBytes;
+  static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + 1024;
+  static constexpr uint32_t kSfBase = 256;     // scale buffers after the 256-column accumulator
+};
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// shared::cluster address of the same shared-memory location in CTA `rank` of the cluster
+__device__ __forceinline__ uint32_t map_rank(uint32_t addr, uint32_t rank) {
+  uint32_t d;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(d) : "r"(addr), "r"(rank));
+  return d;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::
+          "r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t bar_cluster) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster) : "memory");
+}
+__device__ __forceinline__ void tc_commit_pair(uint32_t bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(bar),
+      "h"((uint16_t)3)
+      : "memory");
+}
+__device__ __forceinline__ void tc_cp_sf_pair(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+template <int FMT>
+__device__ __forceinline__ void tc_mma_pair(uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t sfa,
+                                            uint32_t sfb, uint32_t accumulate) {
+  if (FMT == FMT_MX) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::mxf4.block_scale.scale_vec::2X [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+        : "memory");
+  } else {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.scale_vec::4X [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
+            d),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+        : "memory");
+  }
+}
+
+template <int FMT, bool BF16>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+    fp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
+                         const __grid_constant__ CUtensorMap tmap_sfa, const __grid_constant__ CUtensorMap tmap_sfb,
+                         KernelArgs p) {
+  using C = Cfg2<FMT>;
+  constexpr int S = C::kStages;
+  constexpr int APK = C::kApk;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = sA + S * C::kABytes;
+  uint8_t* sSFA = sB + S * C::kBBytes;
+  uint8_t* sSFB = sSFA + S * C::kSfaBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sSFB + S * C::kSfbBytes);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + S;
+  uint64_t* tfull = bars + 2 * S;
+  uint64_t* tempty = bars + 2 * S + 1;
+  uint64_t* drain = bars + 2 * S + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 3);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();
+  const bool leader = rank == 0;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(smem_u32(&full[s]), 1);
+      mbar_init(smem_u32(&empty[s]), 1);
+    }
+    mbar_init(smem_u32(tfull), 1);
+    mbar_init(smem_u32(tempty), 2 * kEpiWarps);
+    mbar_init(smem_u32(drain), 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  cluster_sync_all();                  // barriers of both CTAs initialised before any remote signal
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  const int num_tiles = p.num_m * p.num_n;            // 256 x 256 tiles
+  const int cluster = blockIdx.x >> 1, nclusters = gridDim.x >> 1;
+  const int nkb = p.K / BK;                           // K % 256 == 0 on this path
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer --
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int t = cluster; t < num_tiles && ok; t += nclusters) {
+        int mt, nt;
+        tile_coords(t, p.num_m, p.num_n, mt, nt);
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!wait_spin(smem_u32(&empty[stage]), phase ^ 1u, abort_flag)) {
+            raise_abort(abort_flag, p.error);
+            ok = false;
+            break;
+          }
+          const uint32_t fb = map_rank(smem_u32(&full[stage]), 0);
+          if (leader) mbar_expect_tx(smem_u32(&full[stage]), 2u * (uint32_t)C::kStageBytes);
+          tma_load_2d_pair(smem_u32(sA + stage * C::kABytes), &tmap_a, kb * BK_BYTES, mt * 256 + (int)rank * 128, fb);
+          tma_load_2d_pair(smem_u32(sB + stage * C::kBBytes), &tmap_b, kb * BK_BYTES, nt * 256 + (int)rank * 128, fb);
+          tma_load_2d_pair(smem_u32(sSFA + stage * C::kSfaBytes), &tmap_sfa, 0,
+                           (mt * 2 + (int)rank) * p.g4 + kb * APK, fb);
+#pragma unroll
+          for (int rb = 0; rb < 2; ++rb)
+            tma_load_2d_pair(smem_u32(sSFB + stage * C::kSfbBytes + rb * APK * 512), &tmap_sfb, 0,
+                             (nt * 2 + rb) * p.g4 + kb * APK, fb);
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------- MMA issuer (leader) --
+    if (leader && lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int local = 0;
+      uint32_t ktile_count = 0;
+      bool ok = true, any_mma = false;
+      for (int t = cluster; t < num_tiles && ok; t += nclusters, ++local) {
+        if (!wait_spin(smem_u32(tempty), ((uint32_t)local & 1u) ^ 1u, abort_flag)) {
+          raise_abort(abort_flag, p.error);
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!wait_spin(smem_u32(&full[stage]), phase, abort_flag)) {
+            raise_abort(abort_flag, p.error);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sfa_col = C::kSfBase + (ktile_count & 1u) * kSfCols;
+          const uint32_t sfb_col = sfa_col + 16u;
+          ++ktile_count;
+#pragma unroll
+          for (int i = 0; i < APK; ++i) {
+            tc_cp_sf_pair(tmem + sfa_col + 4u * i, desc_sf(smem_u32(sSFA + stage * C::kSfaBytes + i * 512)));
+#pragma unroll
+            for (int rb = 0; rb < 2; ++rb)
+              tc_cp_sf_pair(tmem + sfb_col + 4u * (i * 2 + rb),
+                            desc_sf(smem_u32(sSFB + stage * C::kSfbBytes + (rb * APK + i) * 512)));
+          }
+          const uint64_t adesc = desc_sw128(smem_u32(sA + stage * C::kABytes));
+          const uint64_t bdesc = desc_sw128(smem_u32(sB + stage * C::kBBytes));
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const uint32_t chunk = FMT == FMT_MX ? (uint32_t)(j >> 1) : (uint32_t)j;
+            const uint32_t sf_id = FMT == FMT_MX ? (uint32_t)((j & 1) * 2) : 0u;
+            const uint32_t idesc = (1u << 7) | (1u << 10) | ((uint32_t)(256 >> 3) << 17) |
+                                   ((FMT == FMT_MX ? 1u : 0u) << 23) | ((uint32_t)(256 >> 4) << 24) | (sf_id << 29) |
+                                   (sf_id << 4);
+            tc_mma_pair<FMT>(tmem, adesc + (uint64_t)(2 * j), bdesc + (uint64_t)(2 * j), idesc,
+                             tmem + sfa_col + 4u * chunk, tmem + sfb_col + 8u * chunk, (kb > 0 || j > 0) ? 1u : 0u);
+            any_mma = true;
+          }
+          tc_commit_pair(smem_u32(&empty[stage]));
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        tc_commit_pair(smem_u32(tfull));
+      }
+      if (!ok && any_mma) {
+        tc_commit_pair(smem_u32(drain));
+        volatile int never = 0;
+        wait_bounded(smem_u32(drain), 0u, &never);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue --
+    const int q = warp & 3;
+    const int col0 = ((warp - 2) / 4) * 128;
+    const int row_in_tile = (int)rank * 128 + q * 32 + lane;
+    const float alpha = FMT == FMT_NV ? __fmul_rn(*p.a_ts, *p.b_ts) : 1.0f;
+    const uint32_t tempty_leader = map_rank(smem_u32(tempty), 0);
+    int local = 0;
+    for (int t = cluster; t < num_tiles; t += nclusters, ++local) {
+      int mt, nt;
+      tile_coords(t, p.num_m, p.num_n, mt, nt);
+      int ok = 1;
+      if (lane == 0) ok = wait_bounded(smem_u32(tfull), (uint32_t)local & 1u, abort_flag) ? 1 : 0;
+      ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+      if (!ok) {
+        if (lane == 0) raise_abort(abort_flag, p.error);
+        break;
+      }
+      tc_fence_after();
+      const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)col0;
+      uint32_t r[4][32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32(tbase + (uint32_t)(32 * c), r[c]);
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_remote(tempty_leader);
+      const int m = mt * 256 + row_in_tile;
+      if (m < p.M) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const int n0 = nt * 256 + col0 + 32 * c;
+          if (n0 >= p.N) break;
+          if (BF16) {
+            __nv_bfloat16* yr = reinterpret_cast<__nv_bfloat16*>(p.y) + (size_t)m * p.ldy + n0;
+            if (p.vec_store && n0 + 32 <= p.N) {
+#pragma unroll
+              for (int v = 0; v < 4; ++v) {
+                uint32_t w[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                  const float lo = __fmul_rn(__uint_as_float(r[c][8 * v + 2 * i]), alpha);
+                  const float hi = __fmul_rn(__uint_as_float(r[c][8 * v + 2 * i + 1]), alpha);
+                  w[i] = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(lo)) |
+                         ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(hi)) << 16);
+                }
+                reinterpret_cast<uint4*>(yr)[v] = make_uint4(w[0], w[1], w[2], w[3]);
+              }
+            } else {
+#pragma unroll
+              for (int i = 0; i < 32; ++i)
+                if (n0 + i < p.N) yr[i] = __float2bfloat16_rn(__fmul_rn(__uint_as_float(r[c][i]), alpha));
+            }
+          } else {
+            float* yr = reinterpret_cast<float*>(p.y) + (size_t)m * p.ldy + n0;
+            if (p.vec_store && n0 + 32 <= p.N) {
+#pragma unroll
+              for (int v = 0; v < 8; ++v)
+                reinterpret_cast<float4*>(yr)[v] = make_float4(
+                    __fmul_rn(__uint_as_float(r[c][4 * v]), alpha), __fmul_rn(__uint_as_float(r[c][4 * v + 1]), alpha),
+                    __fmul_rn(__uint_as_float(r[c][4 * v + 2]), alpha), __fmul_rn(__uint_as_float(r[c][4 * v + 3]), alpha));
+            } else {
+#pragma unroll
+              for (int i = 0; i < 32; ++i)
+                if (n0 + i < p.N) yr[i] = __fmul_rn(__uint_as_float(r[c][i]), alpha);
+            }
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();                  // neither CTA frees tensor memory or exits while the pair is busy
+  tc_fence_after();
+  if (warp == 1) {
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
+  }
+}
+
+}  // namespace pair
+
 // ------------------------------------------------------------------ host ---
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 std::once_flag g_encode_once;
@@ -509,6 +838,60 @@ bool make_code_map(CUtensorMap* map, const uint8_t* base, int64_t rows, int64_t 
   return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(base), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Scale factors in the tensor-core layout viewed as [atoms, 128] uint32 (512 B
+// per atom), box = `box_atoms` consecutive atoms.
+bool make_sf_map(CUtensorMap* map, const uint8_t* base, int64_t atoms, int box_atoms) {
+  auto enc = encode_fn();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[2] = {128, (cuuint64_t)atoms};
+  cuuint64_t strides[1] = {512};
+  cuuint32_t box[2] = {128, (cuuint32_t)box_atoms};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint8_t*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int FMT, bool BF16>
+cudaError_t run_pair(const GemmParams& gp, int num_sms, cudaStream_t st) {
+  using C = pair::Cfg2<FMT>;
+  static_assert(C::kStages >= 2, "shared memory too small for two stages");
+  auto kernel = pair::fp4_gemm_pair_kernel<FMT, BF16>;
+  static const cudaError_t attr =
+      cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+  if (attr != cudaSuccess) return attr;
+  const int bs = FmtTraits<FMT>::kBlock;
+  const int64_t g4 = (gp.K / bs + 3) / 4;
+  CUtensorMap ta, tb, tsa, tsb;
+  if (!make_code_map(&ta, gp.a, gp.M, gp.K / 2, 128)) return cudaErrorNotSupported;
+  if (!make_code_map(&tb, gp.b, gp.N, gp.K / 2, 128)) return cudaErrorNotSupported;
+  if (!make_sf_map(&tsa, gp.a_sf, (gp.M + 127) / 128 * g4, C::kApk)) return cudaErrorNotSupported;
+  if (!make_sf_map(&tsb, gp.b_sf, (gp.N + 127) / 128 * g4, C::kApk)) return cudaErrorNotSupported;
+  KernelArgs ka;
+  ka.a_sf = gp.a_sf;
+  ka.b_sf = gp.b_sf;
+  ka.a_ts = gp.a_ts;
+  ka.b_ts = gp.b_ts;
+  ka.y = gp.y;
+  ka.ldy = gp.ldy;
+  ka.M = (int)gp.M;
+  ka.N = (int)gp.N;
+  ka.K = (int)gp.K;
+  ka.num_m = (int)((gp.M + 255) / 256);
+  ka.num_n = (int)((gp.N + 255) / 256);
+  ka.g4 = (int)g4;
+  ka.error = gp.error;
+  {
+    const int64_t esz = gp.y_bf16 ? 2 : 4;
+    ka.vec_store = ((gp.ldy * esz) % 16 == 0 && (reinterpret_cast<uintptr_t>(gp.y) & 15u) == 0) ? 1 : 0;
+  }
+  const int tiles = ka.num_m * ka.num_n;
+  int clusters = num_sms / 2;
+  if (tiles < clusters) clusters = tiles;
+  kernel<<<2 * clusters, pair::kThreads, C::kSmemBytes, st>>>(ta, tb, tsa, tsb, ka);
+  return cudaGetLastError();
 }
 
 template <int BN, int FMT, bool BF16>
@@ -560,6 +943,18 @@ cudaError_t launch_gemm(const GemmParams& p, int num_sms, cudaStream_t st) {
     const char* e = getenv("FP4_GEMM_BN");
     return e ? atoi(e) : 0;
   }();
+  // SM-pair 256 x 256 tiles when the problem has enough of them (K a multiple of 256 keeps every
+  // scale box inside its row block); FP4_GEMM_PAIR=0 disables them (tuning).
+  // FP4_GEMM_PAIR=1 forces them whenever K allows (testing).
+  static const int pair_mode = [] {
+    const char* e = getenv("FP4_GEMM_PAIR");
+    return e == nullptr ? -1 : (e[0] == '0' ? 0 : 1);
+  }();
+  const bool pair_auto = p.M >= 256 && p.N >= 256 && ((p.M + 255) / 256) * ((p.N + 255) / 256) >= num_sms / 2;
+  if (pair_mode != 0 && forced == 0 && p.K % 256 == 0 && (pair_mode == 1 || pair_auto)) {
+    if (p.fmt == FMT_MX) return p.y_bf16 ? run_pair<FMT_MX, true>(p, num_sms, st) : run_pair<FMT_MX, false>(p, num_sms, st);
+    return p.y_bf16 ? run_pair<FMT_NV, true>(p, num_sms, st) : run_pair<FMT_NV, false>(p, num_sms, st);
+  }
   const int bn = forced == 128 || forced == 256 ? forced : (p.N >= 256 ? 256 : 128);
   return bn == 256 ? dispatch_fmt<256>(p, num_sms, st) : dispatch_fmt<128>(p, num_sms, st);
 }
