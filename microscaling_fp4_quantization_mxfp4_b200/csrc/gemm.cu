@@ -515,20 +515,25 @@ __global__ void __launch_bounds__(Cfg<BN, FMT>::kThreads, 1)
 // No load uses TMA multicast.
 namespace pair {
 
-constexpr int kEpiWarps = 8;
-constexpr int kThreads = 64 + 32 * kEpiWarps;
-
-template <int FMT>
+// BN = 256: 256 x 256 cluster tiles, one 256-column accumulator, 8 epilogue
+// warps.  BN = 128: 256 x 128 tiles, two 128-column accumulators so the next
+// tile's MMAs overlap the epilogue (better when K is short), 4 epilogue warps.
+template <int BN, int FMT>
 struct Cfg2 {
   static constexpr int kApk = FmtTraits<FMT>::kAtomsPerKTile;
+  static constexpr int kAccStages = BN == 128 ? 2 : 1;
+  static constexpr int kEpiWarps = BN == 256 ? 8 : 4;
+  static constexpr int kThreads = 64 + 32 * kEpiWarps;
+  static constexpr int kBRows = BN / 2;                  // B rows staged by each CTA
+  static constexpr int kSfbBlocks = BN / 128;            // 128-row scale blocks of B per tile
   static constexpr int kABytes = 128 * BK_BYTES;
-  static constexpr int kBBytes = 128 * BK_BYTES;
+  static constexpr int kBBytes = kBRows * BK_BYTES;
   static constexpr int kSfaBytes = kApk * 512;
-  static constexpr int kSfbBytes = 2 * kApk * 512;
+  static constexpr int kSfbBytes = kSfbBlocks * kApk * 512;
   static constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;
   static constexpr int kStages = (220 * 1024) / kStageBytes > 8 ? 8 : (220 * 1024) / kStageBytes;
   static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + 1024;
-  static constexpr uint32_t kSfBase = 256;     // scale buffers after the 256-column accumulator
+  static constexpr uint32_t kSfBase = (uint32_t)(kAccStages * BN);   // scale buffers after the accumulators
 };
 
 __device__ __forceinline__ uint32_t cluster_rank() {
@@ -583,14 +588,15 @@ __device__ __forceinline__ void tc_mma_pair(uint32_t d, uint64_t adesc, uint64_t
   }
 }
 
-template <int FMT, bool BF16>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+template <int BN, int FMT, bool BF16>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg2<BN, FMT>::kThreads, 1)
     fp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                          const __grid_constant__ CUtensorMap tmap_sfa, const __grid_constant__ CUtensorMap tmap_sfb,
                          KernelArgs p) {
-  using C = Cfg2<FMT>;
+  using C = Cfg2<BN, FMT>;
   constexpr int S = C::kStages;
   constexpr int APK = C::kApk;
+  constexpr int kEpiWarps = C::kEpiWarps;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
@@ -601,9 +607,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   uint64_t* full = bars;
   uint64_t* empty = bars + S;
   uint64_t* tfull = bars + 2 * S;
-  uint64_t* tempty = bars + 2 * S + 1;
-  uint64_t* drain = bars + 2 * S + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 3);
+  uint64_t* tempty = bars + 2 * S + 2;
+  uint64_t* drain = bars + 2 * S + 4;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 5);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -614,8 +620,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       mbar_init(smem_u32(&full[s]), 1);
       mbar_init(smem_u32(&empty[s]), 1);
     }
-    mbar_init(smem_u32(tfull), 1);
-    mbar_init(smem_u32(tempty), 2 * kEpiWarps);
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(smem_u32(&tfull[a]), 1);
+      mbar_init(smem_u32(&tempty[a]), 2 * kEpiWarps);
+    }
     mbar_init(smem_u32(drain), 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -631,7 +639,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  const int num_tiles = p.num_m * p.num_n;            // 256 x 256 tiles
+  const int num_tiles = p.num_m * p.num_n;            // 256 x BN tiles
   const int cluster = blockIdx.x >> 1, nclusters = gridDim.x >> 1;
   const int nkb = p.K / BK;                           // K % 256 == 0 on this path
 
@@ -653,13 +661,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           const uint32_t fb = map_rank(smem_u32(&full[stage]), 0);
           if (leader) mbar_expect_tx(smem_u32(&full[stage]), 2u * (uint32_t)C::kStageBytes);
           tma_load_2d_pair(smem_u32(sA + stage * C::kABytes), &tmap_a, kb * BK_BYTES, mt * 256 + (int)rank * 128, fb);
-          tma_load_2d_pair(smem_u32(sB + stage * C::kBBytes), &tmap_b, kb * BK_BYTES, nt * 256 + (int)rank * 128, fb);
+          tma_load_2d_pair(smem_u32(sB + stage * C::kBBytes), &tmap_b, kb * BK_BYTES,
+                           nt * BN + (int)rank * C::kBRows, fb);
           tma_load_2d_pair(smem_u32(sSFA + stage * C::kSfaBytes), &tmap_sfa, 0,
                            (mt * 2 + (int)rank) * p.g4 + kb * APK, fb);
 #pragma unroll
-          for (int rb = 0; rb < 2; ++rb)
+          for (int rb = 0; rb < C::kSfbBlocks; ++rb)
             tma_load_2d_pair(smem_u32(sSFB + stage * C::kSfbBytes + rb * APK * 512), &tmap_sfb, 0,
-                             (nt * 2 + rb) * p.g4 + kb * APK, fb);
+                             (nt * C::kSfbBlocks + rb) * p.g4 + kb * APK, fb);
           if (++stage == S) {
             stage = 0;
             phase ^= 1u;
@@ -677,12 +686,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       uint32_t ktile_count = 0;
       bool ok = true, any_mma = false;
       for (int t = cluster; t < num_tiles && ok; t += nclusters, ++local) {
-        if (!wait_spin(smem_u32(tempty), ((uint32_t)local & 1u) ^ 1u, abort_flag)) {
+        const int acc = local % C::kAccStages;
+        const uint32_t use = (uint32_t)(local / C::kAccStages);
+        if (!wait_spin(smem_u32(&tempty[acc]), (use & 1u) ^ 1u, abort_flag)) {
           raise_abort(abort_flag, p.error);
           ok = false;
           break;
         }
         tc_fence_after();
+        const uint32_t d_tmem = tmem + (uint32_t)(acc * BN);
         for (int kb = 0; kb < nkb; ++kb) {
           if (!wait_spin(smem_u32(&full[stage]), phase, abort_flag)) {
             raise_abort(abort_flag, p.error);
@@ -697,8 +709,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           for (int i = 0; i < APK; ++i) {
             tc_cp_sf_pair(tmem + sfa_col + 4u * i, desc_sf(smem_u32(sSFA + stage * C::kSfaBytes + i * 512)));
 #pragma unroll
-            for (int rb = 0; rb < 2; ++rb)
-              tc_cp_sf_pair(tmem + sfb_col + 4u * (i * 2 + rb),
+            for (int rb = 0; rb < C::kSfbBlocks; ++rb)
+              tc_cp_sf_pair(tmem + sfb_col + 4u * (i * C::kSfbBlocks + rb),
                             desc_sf(smem_u32(sSFB + stage * C::kSfbBytes + (rb * APK + i) * 512)));
           }
           const uint64_t adesc = desc_sw128(smem_u32(sA + stage * C::kABytes));
@@ -707,11 +719,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           for (int j = 0; j < 4; ++j) {
             const uint32_t chunk = FMT == FMT_MX ? (uint32_t)(j >> 1) : (uint32_t)j;
             const uint32_t sf_id = FMT == FMT_MX ? (uint32_t)((j & 1) * 2) : 0u;
-            const uint32_t idesc = (1u << 7) | (1u << 10) | ((uint32_t)(256 >> 3) << 17) |
+            const uint32_t idesc = (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
                                    ((FMT == FMT_MX ? 1u : 0u) << 23) | ((uint32_t)(256 >> 4) << 24) | (sf_id << 29) |
                                    (sf_id << 4);
-            tc_mma_pair<FMT>(tmem, adesc + (uint64_t)(2 * j), bdesc + (uint64_t)(2 * j), idesc,
-                             tmem + sfa_col + 4u * chunk, tmem + sfb_col + 8u * chunk, (kb > 0 || j > 0) ? 1u : 0u);
+            tc_mma_pair<FMT>(d_tmem, adesc + (uint64_t)(2 * j), bdesc + (uint64_t)(2 * j), idesc,
+                             tmem + sfa_col + 4u * chunk, tmem + sfb_col + 4u * C::kSfbBlocks * chunk,
+                             (kb > 0 || j > 0) ? 1u : 0u);
             any_mma = true;
           }
           tc_commit_pair(smem_u32(&empty[stage]));
@@ -721,7 +734,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           }
         }
         if (!ok) break;
-        tc_commit_pair(smem_u32(tfull));
+        tc_commit_pair(smem_u32(&tfull[acc]));
       }
       if (!ok && any_mma) {
         tc_commit_pair(smem_u32(drain));
@@ -736,20 +749,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const int col0 = ((warp - 2) / 4) * 128;
     const int row_in_tile = (int)rank * 128 + q * 32 + lane;
     const float alpha = FMT == FMT_NV ? __fmul_rn(*p.a_ts, *p.b_ts) : 1.0f;
-    const uint32_t tempty_leader = map_rank(smem_u32(tempty), 0);
     int local = 0;
     for (int t = cluster; t < num_tiles; t += nclusters, ++local) {
       int mt, nt;
       tile_coords(t, p.num_m, p.num_n, mt, nt);
+      const int acc = local % C::kAccStages;
+      const uint32_t use = (uint32_t)(local / C::kAccStages);
+      const uint32_t tempty_leader = map_rank(smem_u32(&tempty[acc]), 0);
       int ok = 1;
-      if (lane == 0) ok = wait_bounded(smem_u32(tfull), (uint32_t)local & 1u, abort_flag) ? 1 : 0;
+      if (lane == 0) ok = wait_bounded(smem_u32(&tfull[acc]), use & 1u, abort_flag) ? 1 : 0;
       ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
       if (!ok) {
         if (lane == 0) raise_abort(abort_flag, p.error);
         break;
       }
       tc_fence_after();
-      const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)col0;
+      const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN + col0);
       uint32_t r[4][32];
 #pragma unroll
       for (int c = 0; c < 4; ++c) tmem_ld32(tbase + (uint32_t)(32 * c), r[c]);
@@ -761,7 +776,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       if (m < p.M) {
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-          const int n0 = nt * 256 + col0 + 32 * c;
+          const int n0 = nt * BN + col0 + 32 * c;
           if (n0 >= p.N) break;
           if (BF16) {
             __nv_bfloat16* yr = reinterpret_cast<__nv_bfloat16*>(p.y) + (size_t)m * p.ldy + n0;
@@ -854,11 +869,11 @@ bool make_sf_map(CUtensorMap* map, const uint8_t* base, int64_t atoms, int box_a
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int FMT, bool BF16>
+template <int BN, int FMT, bool BF16>
 cudaError_t run_pair(const GemmParams& gp, int num_sms, cudaStream_t st) {
-  using C = pair::Cfg2<FMT>;
+  using C = pair::Cfg2<BN, FMT>;
   static_assert(C::kStages >= 2, "shared memory too small for two stages");
-  auto kernel = pair::fp4_gemm_pair_kernel<FMT, BF16>;
+  auto kernel = pair::fp4_gemm_pair_kernel<BN, FMT, BF16>;
   static const cudaError_t attr =
       cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (attr != cudaSuccess) return attr;
@@ -866,7 +881,7 @@ cudaError_t run_pair(const GemmParams& gp, int num_sms, cudaStream_t st) {
   const int64_t g4 = (gp.K / bs + 3) / 4;
   CUtensorMap ta, tb, tsa, tsb;
   if (!make_code_map(&ta, gp.a, gp.M, gp.K / 2, 128)) return cudaErrorNotSupported;
-  if (!make_code_map(&tb, gp.b, gp.N, gp.K / 2, 128)) return cudaErrorNotSupported;
+  if (!make_code_map(&tb, gp.b, gp.N, gp.K / 2, C::kBRows)) return cudaErrorNotSupported;
   if (!make_sf_map(&tsa, gp.a_sf, (gp.M + 127) / 128 * g4, C::kApk)) return cudaErrorNotSupported;
   if (!make_sf_map(&tsb, gp.b_sf, (gp.N + 127) / 128 * g4, C::kApk)) return cudaErrorNotSupported;
   KernelArgs ka;
@@ -880,7 +895,7 @@ cudaError_t run_pair(const GemmParams& gp, int num_sms, cudaStream_t st) {
   ka.N = (int)gp.N;
   ka.K = (int)gp.K;
   ka.num_m = (int)((gp.M + 255) / 256);
-  ka.num_n = (int)((gp.N + 255) / 256);
+  ka.num_n = (int)((gp.N + BN - 1) / BN);
   ka.g4 = (int)g4;
   ka.error = gp.error;
   {
@@ -890,7 +905,7 @@ cudaError_t run_pair(const GemmParams& gp, int num_sms, cudaStream_t st) {
   const int tiles = ka.num_m * ka.num_n;
   int clusters = num_sms / 2;
   if (tiles < clusters) clusters = tiles;
-  kernel<<<2 * clusters, pair::kThreads, C::kSmemBytes, st>>>(ta, tb, tsa, tsb, ka);
+  kernel<<<2 * clusters, C::kThreads, C::kSmemBytes, st>>>(ta, tb, tsa, tsb, ka);
   return cudaGetLastError();
 }
 
@@ -936,26 +951,34 @@ static cudaError_t dispatch_fmt(const GemmParams& p, int num_sms, cudaStream_t s
   return p.y_bf16 ? run<BN, FMT_NV, true>(p, num_sms, st) : run<BN, FMT_NV, false>(p, num_sms, st);
 }
 
+template <int BN>
+static cudaError_t dispatch_pair(const GemmParams& p, int num_sms, cudaStream_t st) {
+  if (p.fmt == FMT_MX)
+    return p.y_bf16 ? run_pair<BN, FMT_MX, true>(p, num_sms, st) : run_pair<BN, FMT_MX, false>(p, num_sms, st);
+  return p.y_bf16 ? run_pair<BN, FMT_NV, true>(p, num_sms, st) : run_pair<BN, FMT_NV, false>(p, num_sms, st);
+}
+
 cudaError_t launch_gemm(const GemmParams& p, int num_sms, cudaStream_t st) {
-  // 128x256 tiles halve the operand traffic per FLOP; 128x128 tiles keep two accumulators in
-  // tensor memory and more CTAs busy when N is small.  FP4_GEMM_BN=128|256 overrides (tuning).
-  static const int forced = [] {
+  // Tuning overrides: FP4_GEMM_BN=128|256 (tile width), FP4_GEMM_PAIR=0|1 (SM-pair kernel off/forced).
+  static const int forced_bn = [] {
     const char* e = getenv("FP4_GEMM_BN");
-    return e ? atoi(e) : 0;
+    const int v = e ? atoi(e) : 0;
+    return v == 128 || v == 256 ? v : 0;
   }();
-  // SM-pair 256 x 256 tiles when the problem has enough of them (K a multiple of 256 keeps every
-  // scale box inside its row block); FP4_GEMM_PAIR=0 disables them (tuning).
-  // FP4_GEMM_PAIR=1 forces them whenever K allows (testing).
   static const int pair_mode = [] {
     const char* e = getenv("FP4_GEMM_PAIR");
     return e == nullptr ? -1 : (e[0] == '0' ? 0 : 1);
   }();
-  const bool pair_auto = p.M >= 256 && p.N >= 256 && ((p.M + 255) / 256) * ((p.N + 255) / 256) >= num_sms / 2;
-  if (pair_mode != 0 && forced == 0 && p.K % 256 == 0 && (pair_mode == 1 || pair_auto)) {
-    if (p.fmt == FMT_MX) return p.y_bf16 ? run_pair<FMT_MX, true>(p, num_sms, st) : run_pair<FMT_MX, false>(p, num_sms, st);
-    return p.y_bf16 ? run_pair<FMT_NV, true>(p, num_sms, st) : run_pair<FMT_NV, false>(p, num_sms, st);
-  }
-  const int bn = forced == 128 || forced == 256 ? forced : (p.N >= 256 ? 256 : 128);
+  // SM-pair 256 x 256 tiles when K is a multiple of 256 (every scale box then stays inside its row
+  // block), long enough (>= 2048) for the single accumulator's epilogue to hide behind the mainloop,
+  // and the problem has enough tiles to occupy the SM pairs.  Shorter K runs on single-SM 128 x 256
+  // tiles (measured faster at K = 768).  256 x 128 pair tiles are only used when forced.
+  const int pair_bn = forced_bn ? forced_bn : 256;
+  const bool pair_auto = p.K >= 2048 && p.M >= 256 && p.N >= 256 &&
+                         ((p.M + 255) / 256) * ((p.N + pair_bn - 1) / pair_bn) >= num_sms / 2;
+  if (pair_mode != 0 && p.K % 256 == 0 && (pair_mode == 1 || pair_auto))
+    return pair_bn == 256 ? dispatch_pair<256>(p, num_sms, st) : dispatch_pair<128>(p, num_sms, st);
+  const int bn = forced_bn ? forced_bn : (p.N >= 256 ? 256 : 128);
   return bn == 256 ? dispatch_fmt<256>(p, num_sms, st) : dispatch_fmt<128>(p, num_sms, st);
 }
 
