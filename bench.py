@@ -233,9 +233,11 @@ def _dist_setup(torch):
 
 
 def _max_over_ranks(torch, pg, value: float) -> float:
+    """Max of a per-rank scalar over the process group (device time: the slowest rank counts)."""
     if pg is None:
         return value
-    t = torch.tensor([value], dtype=torch.float64, device="cuda")
+    dev = "cuda" if pg.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
     pg.all_reduce(t, op=pg.ReduceOp.MAX)
     return float(t.item())
 
