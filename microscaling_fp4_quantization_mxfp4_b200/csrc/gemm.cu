@@ -12,13 +12,19 @@
 //   warp 0      TMA producer: A/B code tiles (128-byte rows, 128B swizzle) and
 //               the scale-factor atoms (plain bulk copies) into a STAGES-deep
 //               shared-memory ring guarded by full/empty mbarriers.
-//   warp 1      allocates tensor memory; one thread copies each stage's scale
-//               factors to tensor memory (tcgen05.cp 32x128b.warpx4) and
-//               issues 4 block-scaled MMAs (K = 64 each) per 256-wide k-tile,
-//               committing to the stage's empty barrier.
-//   warps 2..5  epilogue: tcgen05.ld the fp32 accumulator (two accumulator
-//               buffers in tensor memory so the next tile's MMAs overlap the
-//               stores), multiply by alpha, store fp32 or bf16.
+//   warp 1      allocates tensor memory; one thread issues 4 block-scaled MMAs
+//               (K = 64 each) per 256-wide k-tile, committing to the stage's
+//               empty barrier and to the scale buffer's empty barrier.
+//   last warp   scale-factor copier: one thread copies each stage's scale
+//               atoms to one of four tensor-memory scale buffers
+//               (tcgen05.cp 32x128b.warpx4) ahead of the MMAs.  The copies
+//               run on their own path, so issuing them from a separate thread
+//               lets them overlap the previous k-tiles' MMAs instead of
+//               queueing between them (measured: 22-28% faster than copying
+//               from the MMA thread).
+//   other warps epilogue: tcgen05.ld the fp32 accumulator (two accumulator
+//               buffers in tensor memory when BN = 128 so the next tile's MMAs
+//               overlap the stores), multiply by alpha, store fp32 or bf16.
 // Every mbarrier wait is bounded; on expiry the CTA raises a shared abort
 // flag and a device error word, drains its own copies and MMAs, frees tensor
 // memory and returns.
@@ -41,6 +47,7 @@ constexpr int BK = 256;               // fp4 elements per k-tile (128 bytes per 
 constexpr int BK_BYTES = BK / 2;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kSfCols = 48;      // one scale-factor buffer: SFA (<= 16 cols) then SFB (<= 32 cols)
+constexpr uint32_t kSfBufs = 4;       // scale buffers in tensor memory (after the accumulators)
 constexpr unsigned long long kWaitLimitNs = 4000000000ull;   // 4 s per wait
 
 template <int FMT>
@@ -53,8 +60,10 @@ template <int BN, int FMT>
 struct Cfg {
   static constexpr int kAccStages = BN == 128 ? 2 : 1;
   static constexpr int kEpiWarps = BN == 256 ? 8 : 4;          // each epilogue warp drains 128 columns
-  static constexpr int kThreads = 64 + 32 * kEpiWarps;
-  static constexpr uint32_t kSfBase = (uint32_t)(kAccStages * BN);   // two scale buffers after the accumulators
+  static constexpr int kThreads = 96 + 32 * kEpiWarps;        // producer, MMA, epilogue warps, scale copier
+  static constexpr int kSfWarp = 2 + kEpiWarps;
+  static constexpr uint32_t kSfBase = (uint32_t)(kAccStages * BN);   // scale buffers after the accumulators
+  static_assert(kSfBase + kSfBufs * kSfCols <= kTmemCols, "tensor memory budget");
   static constexpr int kApk = FmtTraits<FMT>::kAtomsPerKTile;
   static constexpr int kABytes = BM * BK_BYTES;
   static constexpr int kBBytes = BN * BK_BYTES;
@@ -189,7 +198,19 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
         "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
       : "r"(taddr));
 }
-__device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+// Waits for this thread's tensor-memory loads into r[4][32].  The registers are in-out operands of
+// the wait (and of an empty statement right after it), so the compiler cannot schedule any use of
+// them ahead of the wait.
+__device__ __forceinline__ void tmem_ld_wait(uint32_t (&r)[4][32]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+r"(r[0][0]), "+r"(r[0][1]), "+r"(r[0][2]), "+r"(r[0][3]), "+r"(r[0][4]), "+r"(r[0][5]), "+r"(r[0][6]), "+r"(r[0][7]), "+r"(r[0][8]), "+r"(r[0][9]), "+r"(r[0][10]), "+r"(r[0][11]), "+r"(r[0][12]), "+r"(r[0][13]), "+r"(r[0][14]), "+r"(r[0][15]), "+r"(r[0][16]), "+r"(r[0][17]), "+r"(r[0][18]), "+r"(r[0][19]), "+r"(r[0][20]), "+r"(r[0][21]), "+r"(r[0][22]), "+r"(r[0][23]), "+r"(r[0][24]), "+r"(r[0][25]), "+r"(r[0][26]), "+r"(r[0][27]), "+r"(r[0][28]), "+r"(r[0][29]), "+r"(r[0][30]), "+r"(r[0][31]),
+                 "+r"(r[1][0]), "+r"(r[1][1]), "+r"(r[1][2]), "+r"(r[1][3]), "+r"(r[1][4]), "+r"(r[1][5]), "+r"(r[1][6]), "+r"(r[1][7]), "+r"(r[1][8]), "+r"(r[1][9]), "+r"(r[1][10]), "+r"(r[1][11]), "+r"(r[1][12]), "+r"(r[1][13]), "+r"(r[1][14]), "+r"(r[1][15]), "+r"(r[1][16]), "+r"(r[1][17]), "+r"(r[1][18]), "+r"(r[1][19]), "+r"(r[1][20]), "+r"(r[1][21]), "+r"(r[1][22]), "+r"(r[1][23]), "+r"(r[1][24]), "+r"(r[1][25]), "+r"(r[1][26]), "+r"(r[1][27]), "+r"(r[1][28]), "+r"(r[1][29]), "+r"(r[1][30]), "+r"(r[1][31])
+               :
+               : "memory");
+  asm volatile(""
+               : "+r"(r[2][0]), "+r"(r[2][1]), "+r"(r[2][2]), "+r"(r[2][3]), "+r"(r[2][4]), "+r"(r[2][5]), "+r"(r[2][6]), "+r"(r[2][7]), "+r"(r[2][8]), "+r"(r[2][9]), "+r"(r[2][10]), "+r"(r[2][11]), "+r"(r[2][12]), "+r"(r[2][13]), "+r"(r[2][14]), "+r"(r[2][15]), "+r"(r[2][16]), "+r"(r[2][17]), "+r"(r[2][18]), "+r"(r[2][19]), "+r"(r[2][20]), "+r"(r[2][21]), "+r"(r[2][22]), "+r"(r[2][23]), "+r"(r[2][24]), "+r"(r[2][25]), "+r"(r[2][26]), "+r"(r[2][27]), "+r"(r[2][28]), "+r"(r[2][29]), "+r"(r[2][30]), "+r"(r[2][31]),
+                 "+r"(r[3][0]), "+r"(r[3][1]), "+r"(r[3][2]), "+r"(r[3][3]), "+r"(r[3][4]), "+r"(r[3][5]), "+r"(r[3][6]), "+r"(r[3][7]), "+r"(r[3][8]), "+r"(r[3][9]), "+r"(r[3][10]), "+r"(r[3][11]), "+r"(r[3][12]), "+r"(r[3][13]), "+r"(r[3][14]), "+r"(r[3][15]), "+r"(r[3][16]), "+r"(r[3][17]), "+r"(r[3][18]), "+r"(r[3][19]), "+r"(r[3][20]), "+r"(r[3][21]), "+r"(r[3][22]), "+r"(r[3][23]), "+r"(r[3][24]), "+r"(r[3][25]), "+r"(r[3][26]), "+r"(r[3][27]), "+r"(r[3][28]), "+r"(r[3][29]), "+r"(r[3][30]), "+r"(r[3][31]));
+}
 
 // Shared-memory matrix descriptor: K-major operand, 128-byte rows, 128B
 // swizzle, 8-row groups 1024 bytes apart (Blackwell descriptor version 1).
@@ -255,7 +276,10 @@ __global__ void __launch_bounds__(Cfg<BN, FMT>::kThreads, 1)
   uint64_t* tfull = bars + 2 * S;
   uint64_t* tempty = bars + 2 * S + 2;
   uint64_t* drain = bars + 2 * S + 4;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 5);
+  uint64_t* sfdrain = bars + 2 * S + 5;
+  uint64_t* sf_full = bars + 2 * S + 6;                 // scale buffer b written (copies landed)
+  uint64_t* sf_empty = sf_full + kSfBufs;               // scale buffer b free (its MMAs done)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sf_empty + kSfBufs);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -269,6 +293,11 @@ __global__ void __launch_bounds__(Cfg<BN, FMT>::kThreads, 1)
       mbar_init(smem_u32(&tempty[a]), C::kEpiWarps);
     }
     mbar_init(smem_u32(drain), 1);
+    mbar_init(smem_u32(sfdrain), 1);
+    for (uint32_t b = 0; b < kSfBufs; ++b) {
+      mbar_init(smem_u32(&sf_full[b]), 1);
+      mbar_init(smem_u32(&sf_empty[b]), 1);
+    }
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -343,7 +372,7 @@ __global__ void __launch_bounds__(Cfg<BN, FMT>::kThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       int local = 0;
-      uint32_t ktile_count = 0;   // k-tiles issued so far: picks the scale-factor buffer
+      uint32_t ktile_count = 0;   // k-tiles issued so far: picks the scale buffer
       bool ok = true;
       bool any_mma = false;
       for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x, ++local) {
@@ -360,25 +389,19 @@ __global__ void __launch_bounds__(Cfg<BN, FMT>::kThreads, 1)
         tc_fence_after();
         const uint32_t d_tmem = tmem + (uint32_t)(acc * BN);
         for (int kb = 0; kb < nkb; ++kb) {
-          if (!wait_spin(smem_u32(&full[stage]), phase, abort_flag)) {
+          const uint32_t b = ktile_count % kSfBufs, use_b = ktile_count / kSfBufs;
+          ++ktile_count;
+          // the scale buffer's copies landed (the copier waited for this stage first)
+          if (!wait_spin(smem_u32(&sf_full[b]), use_b & 1u, abort_flag) ||
+              !wait_spin(smem_u32(&full[stage]), phase, abort_flag)) {
             raise_abort(abort_flag, p.error);
             ok = false;
             break;
           }
           tc_fence_after();
           const int kvalid = min(BK, p.K - kb * BK);
-          const int atoms = (kvalid / FmtTraits<FMT>::kBlock + 3) / 4;
-          // alternate between two scale buffers so these copies never overwrite scales that the
-          // previous k-tile's MMAs may still be reading
-          const uint32_t sfa_col = C::kSfBase + (ktile_count & 1u) * kSfCols;
+          const uint32_t sfa_col = C::kSfBase + b * kSfCols;
           const uint32_t sfb_col = sfa_col + 16u;
-          ++ktile_count;
-          for (int i = 0; i < atoms; ++i) {
-            tc_cp_sf(tmem + sfa_col + 4u * i, desc_sf(smem_u32(sSFA + stage * C::kSfaBytes + i * 512)));
-            for (int rb = 0; rb < BN / 128; ++rb)
-              tc_cp_sf(tmem + sfb_col + 4u * (i * (BN / 128) + rb),
-                       desc_sf(smem_u32(sSFB + stage * C::kSfbBytes + (rb * APK + i) * 512)));
-          }
           const uint64_t adesc = desc_sw128(smem_u32(sA + stage * C::kABytes));
           const uint64_t bdesc = desc_sw128(smem_u32(sB + stage * C::kBBytes));
           const int nmma = kvalid / 64;
@@ -398,6 +421,7 @@ __global__ void __launch_bounds__(Cfg<BN, FMT>::kThreads, 1)
             any_mma = true;
           }
           tc_commit(smem_u32(&empty[stage]));
+          tc_commit(smem_u32(&sf_empty[b]));
           if (++stage == S) {
             stage = 0;
             phase ^= 1u;
@@ -411,6 +435,51 @@ __global__ void __launch_bounds__(Cfg<BN, FMT>::kThreads, 1)
         tc_commit(smem_u32(drain));
         volatile int never = 0;
         wait_bounded(smem_u32(drain), 0u, &never);
+      }
+    }
+    __syncwarp();
+  } else if (warp == C::kSfWarp) {
+    // ------------------------------------------------------ scale copier --
+    // k-tile n's scale atoms go to buffer n % kSfBufs once the stage has landed and the MMAs
+    // that last read that buffer have completed; the commit tells the MMA issuer.
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0, kt = 0;
+      bool ok = true, any_cp = false;
+      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+        for (int kb = 0; kb < nkb; ++kb) {
+          const uint32_t b = kt % kSfBufs, use_b = kt / kSfBufs;
+          ++kt;
+          if (!wait_spin(smem_u32(&full[stage]), phase, abort_flag) ||
+              !wait_spin(smem_u32(&sf_empty[b]), (use_b & 1u) ^ 1u, abort_flag)) {
+            raise_abort(abort_flag, p.error);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const int kvalid = min(BK, p.K - kb * BK);
+          const int atoms = (kvalid / FmtTraits<FMT>::kBlock + 3) / 4;
+          const uint32_t sfa_col = C::kSfBase + b * kSfCols;
+          const uint32_t sfb_col = sfa_col + 16u;
+          for (int i = 0; i < atoms; ++i) {
+            tc_cp_sf(tmem + sfa_col + 4u * i, desc_sf(smem_u32(sSFA + stage * C::kSfaBytes + i * 512)));
+            for (int rb = 0; rb < BN / 128; ++rb)
+              tc_cp_sf(tmem + sfb_col + 4u * (i * (BN / 128) + rb),
+                       desc_sf(smem_u32(sSFB + stage * C::kSfbBytes + (rb * APK + i) * 512)));
+          }
+          tc_commit(smem_u32(&sf_full[b]));
+          any_cp = true;
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok && any_cp) {
+        // copies already issued complete before tensor memory is released
+        tc_commit(smem_u32(sfdrain));
+        volatile int never = 0;
+        wait_bounded(smem_u32(sfdrain), 0u, &never);
       }
     }
     __syncwarp();
@@ -441,7 +510,7 @@ __global__ void __launch_bounds__(Cfg<BN, FMT>::kThreads, 1)
       uint32_t r[4][32];
 #pragma unroll
       for (int c = 0; c < 4; ++c) tmem_ld32(tbase + (uint32_t)(32 * c), r[c]);
-      tmem_ld_wait();
+      tmem_ld_wait(r);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&tempty[acc]));
@@ -523,7 +592,8 @@ struct Cfg2 {
   static constexpr int kApk = FmtTraits<FMT>::kAtomsPerKTile;
   static constexpr int kAccStages = BN == 128 ? 2 : 1;
   static constexpr int kEpiWarps = BN == 256 ? 8 : 4;
-  static constexpr int kThreads = 64 + 32 * kEpiWarps;
+  static constexpr int kThreads = 96 + 32 * kEpiWarps;  // producer, MMA, epilogue warps, scale copier
+  static constexpr int kSfWarp = 2 + kEpiWarps;
   static constexpr int kBRows = BN / 2;                  // B rows staged by each CTA
   static constexpr int kSfbBlocks = BN / 128;            // 128-row scale blocks of B per tile
   static constexpr int kABytes = 128 * BK_BYTES;
@@ -534,6 +604,7 @@ struct Cfg2 {
   static constexpr int kStages = (220 * 1024) / kStageBytes > 8 ? 8 : (220 * 1024) / kStageBytes;
   static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + 1024;
   static constexpr uint32_t kSfBase = (uint32_t)(kAccStages * BN);   // scale buffers after the accumulators
+  static_assert(kSfBase + kSfBufs * kSfCols <= kTmemCols, "tensor memory budget");
 };
 
 __device__ __forceinline__ uint32_t cluster_rank() {
@@ -565,6 +636,10 @@ __device__ __forceinline__ void tc_commit_pair(uint32_t bar) {
       "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(bar),
       "h"((uint16_t)3)
       : "memory");
+}
+// commit of the pair's tensor-core work to a barrier of this CTA only
+__device__ __forceinline__ void tc_commit_pair_local(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
 }
 __device__ __forceinline__ void tc_cp_sf_pair(uint32_t taddr, uint64_t sdesc) {
   asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
@@ -609,7 +684,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg2<BN, FMT>::kThre
   uint64_t* tfull = bars + 2 * S;
   uint64_t* tempty = bars + 2 * S + 2;
   uint64_t* drain = bars + 2 * S + 4;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 5);
+  uint64_t* sfdrain = bars + 2 * S + 5;
+  uint64_t* sf_full = bars + 2 * S + 6;                 // scale buffer b written (copies landed)
+  uint64_t* sf_empty = sf_full + kSfBufs;               // scale buffer b free (its MMAs done)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sf_empty + kSfBufs);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -625,6 +703,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg2<BN, FMT>::kThre
       mbar_init(smem_u32(&tempty[a]), 2 * kEpiWarps);
     }
     mbar_init(smem_u32(drain), 1);
+    mbar_init(smem_u32(sfdrain), 1);
+    for (uint32_t b = 0; b < kSfBufs; ++b) {
+      mbar_init(smem_u32(&sf_full[b]), 1);
+      mbar_init(smem_u32(&sf_empty[b]), 1);
+    }
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -696,23 +779,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg2<BN, FMT>::kThre
         tc_fence_after();
         const uint32_t d_tmem = tmem + (uint32_t)(acc * BN);
         for (int kb = 0; kb < nkb; ++kb) {
-          if (!wait_spin(smem_u32(&full[stage]), phase, abort_flag)) {
+          const uint32_t b = ktile_count % kSfBufs, use_b = ktile_count / kSfBufs;
+          ++ktile_count;
+          if (!wait_spin(smem_u32(&sf_full[b]), use_b & 1u, abort_flag) ||
+              !wait_spin(smem_u32(&full[stage]), phase, abort_flag)) {
             raise_abort(abort_flag, p.error);
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t sfa_col = C::kSfBase + (ktile_count & 1u) * kSfCols;
+          const uint32_t sfa_col = C::kSfBase + b * kSfCols;
           const uint32_t sfb_col = sfa_col + 16u;
-          ++ktile_count;
-#pragma unroll
-          for (int i = 0; i < APK; ++i) {
-            tc_cp_sf_pair(tmem + sfa_col + 4u * i, desc_sf(smem_u32(sSFA + stage * C::kSfaBytes + i * 512)));
-#pragma unroll
-            for (int rb = 0; rb < C::kSfbBlocks; ++rb)
-              tc_cp_sf_pair(tmem + sfb_col + 4u * (i * C::kSfbBlocks + rb),
-                            desc_sf(smem_u32(sSFB + stage * C::kSfbBytes + (rb * APK + i) * 512)));
-          }
           const uint64_t adesc = desc_sw128(smem_u32(sA + stage * C::kABytes));
           const uint64_t bdesc = desc_sw128(smem_u32(sB + stage * C::kBBytes));
 #pragma unroll
@@ -728,6 +805,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg2<BN, FMT>::kThre
             any_mma = true;
           }
           tc_commit_pair(smem_u32(&empty[stage]));
+          tc_commit_pair_local(smem_u32(&sf_empty[b]));
           if (++stage == S) {
             stage = 0;
             phase ^= 1u;
@@ -740,6 +818,50 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg2<BN, FMT>::kThre
         tc_commit_pair(smem_u32(drain));
         volatile int never = 0;
         wait_bounded(smem_u32(drain), 0u, &never);
+      }
+    }
+    __syncwarp();
+  } else if (warp == C::kSfWarp) {
+    // ------------------------------------------------ scale copier (leader) --
+    // The leader's cta_group::2 copies fill the same scale buffer in both CTAs' tensor memory,
+    // each from its own shared memory.
+    if (leader && lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0, kt = 0;
+      bool ok = true, any_cp = false;
+      for (int t = cluster; t < num_tiles && ok; t += nclusters) {
+        for (int kb = 0; kb < nkb; ++kb) {
+          const uint32_t b = kt % kSfBufs, use_b = kt / kSfBufs;
+          ++kt;
+          if (!wait_spin(smem_u32(&full[stage]), phase, abort_flag) ||
+              !wait_spin(smem_u32(&sf_empty[b]), (use_b & 1u) ^ 1u, abort_flag)) {
+            raise_abort(abort_flag, p.error);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sfa_col = C::kSfBase + b * kSfCols;
+          const uint32_t sfb_col = sfa_col + 16u;
+#pragma unroll
+          for (int i = 0; i < APK; ++i) {
+            tc_cp_sf_pair(tmem + sfa_col + 4u * i, desc_sf(smem_u32(sSFA + stage * C::kSfaBytes + i * 512)));
+#pragma unroll
+            for (int rb = 0; rb < C::kSfbBlocks; ++rb)
+              tc_cp_sf_pair(tmem + sfb_col + 4u * (i * C::kSfbBlocks + rb),
+                            desc_sf(smem_u32(sSFB + stage * C::kSfbBytes + (rb * APK + i) * 512)));
+          }
+          tc_commit_pair_local(smem_u32(&sf_full[b]));
+          any_cp = true;
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok && any_cp) {
+        tc_commit_pair_local(smem_u32(sfdrain));
+        volatile int never = 0;
+        wait_bounded(smem_u32(sfdrain), 0u, &never);
       }
     }
     __syncwarp();
@@ -768,7 +890,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg2<BN, FMT>::kThre
       uint32_t r[4][32];
 #pragma unroll
       for (int c = 0; c < 4; ++c) tmem_ld32(tbase + (uint32_t)(32 * c), r[c]);
-      tmem_ld_wait();
+      tmem_ld_wait(r);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_remote(tempty_leader);
