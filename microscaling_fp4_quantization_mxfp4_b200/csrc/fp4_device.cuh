@@ -47,18 +47,20 @@ __device__ __forceinline__ uint32_t pack8_rtn(const float (&v)[8]) {
 // Stochastic rounding of one scaled value with a 32-bit random word:
 // lo <= |v| < hi adjacent grid points, p = (|v| - lo) / (hi - lo) (exact in
 // fp32), round up iff r < ceil(p * 2^32); |v| >= 6 gives 6; sign kept.
-// Branch-free: on [0,2), [2,4), [4,6) the grid step is 0.5, 1, 2, so with
-// s = |v| / step (exact) the lower grid point is floor(s) steps in and p is
-// the fractional part of s.
+// On [0,2), [2,4), [4,6) the grid step is 0.5, 1, 2, so with s = |v| / step
+// (exact, s < 4) the lower grid point is floor(s) steps in and p is the
+// fractional part of s.  floor(s) comes from one round-toward-zero addition
+// of 2^23 (the sum's last significand bits are the integer part), so the only
+// conversion left per element is the threshold's.
 __device__ __forceinline__ uint32_t e2m1_sr(float v, uint32_t r) {
   const float a = fabsf(v);
   const float inv_step = a < 2.0f ? 2.0f : (a < 4.0f ? 1.0f : 0.5f);
   const uint32_t base = a < 2.0f ? 0u : (a < 4.0f ? 2u : 4u);
   const float s = __fmul_rn(a, inv_step);
-  const float fl = floorf(s);
-  const float p = __fsub_rn(s, fl);
+  const float t = __fadd_rz(s, 8388608.0f);                        // 2^23 + floor(s)
+  const float p = __fsub_rn(s, __fsub_rn(t, 8388608.0f));          // exact fractional part
   const uint32_t thr = __float2uint_ru(__fmul_rn(p, 4294967296.0f));   // < 2^32 since p < 1
-  uint32_t code = (uint32_t)fl + base + (r < thr ? 1u : 0u);
+  uint32_t code = (__float_as_uint(t) - 0x4B000000u) + base + (r < thr ? 1u : 0u);
   code = a < 6.0f ? code : 7u;
   return code | ((__float_as_uint(v) >> 31) << 3);
 }

@@ -606,11 +606,35 @@ __global__ void __launch_bounds__(kFusedThreads, 1) nv_quantize_fused_kernel(Fus
 }
 
 // ======================================================== axis-0 quantize ===
+// 4 x 4 transpose of 32-bit words across the four lanes of a quad: on entry
+// lane q holds row q (w[0..3]); on return t[s] is word q of row s.  In round
+// k lane q reads from lane s = (q + k) & 3, which sends its word (s - k) & 3,
+// that is word q.  Every lane of the warp must call it.
+__device__ __forceinline__ void quad_transpose4(const uint32_t (&w)[4], uint32_t (&t)[4], int lane) {
+  const int q = lane & 3;
+  t[0] = t[1] = t[2] = t[3] = 0u;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int si = (q - k) & 3;
+    const uint32_t send = si == 0 ? w[0] : (si == 1 ? w[1] : (si == 2 ? w[2] : w[3]));
+    const uint32_t recv = __shfl_sync(0xFFFFFFFFu, send, (lane & ~3) | ((q + k) & 3));
+    const int row = (q + k) & 3;
+    t[0] = row == 0 ? recv : t[0];
+    t[1] = row == 1 ? recv : t[1];
+    t[2] = row == 2 ? recv : t[2];
+    t[3] = row == 3 ? recv : t[3];
+  }
+}
+
 // Blocks run down the columns of x[R, C]; the output is written transposed
 // (codes [C, R/2]).  A CTA stages a 128-row x 64-column bf16 tile in shared
 // memory with coalesced 128-bit loads; each thread then owns one column and a
 // 32-row segment (one MX block / two NV blocks) and writes its packed codes
-// as one contiguous run of the output row.
+// as one contiguous run of the output row.  For stochastic rounding the four
+// lanes of a quad hold four adjacent columns (C is a multiple of 8), which
+// share one Philox counter per row: each lane draws the block of one row and
+// a quad transpose hands every lane its column's word, one Philox4x32-10
+// evaluation per four elements as on axis 1.
 struct QColParams {
   const uint16_t* x;
   uint32_t R, C;
@@ -654,7 +678,8 @@ __global__ void __launch_bounds__(256) quantize_cols_kernel(QColParams p) {
     const uint32_t c = c0 + 32u * (warp & 1) + lane;
     const uint32_t seg = warp >> 1;
     const uint32_t rbase = r0 + 32u * seg;
-    if (c >= p.C || rbase >= p.R) continue;
+    if (rbase >= p.R) continue;                  // warp-uniform; lanes past C stay for the shuffles
+    const bool col_ok = c < p.C;
     float xv[32];
 #pragma unroll
     for (int i = 0; i < 32; ++i) xv[i] = __uint_as_float((uint32_t)tile[32 * seg + i][32 * (warp & 1) + lane] << 16);
@@ -703,15 +728,27 @@ __global__ void __launch_bounds__(256) quantize_cols_kernel(QColParams p) {
         if (RND == RND_RTN) {
           packed = pack8_rtn(v8);
         } else {
+          // rows rb + 8*w8 + 4h + q (q = lane & 3): word (c & 3) of row i's block goes to element i
+          uint32_t rw[8];
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const unsigned long long row = rb + w8 * 8 + 4 * h + (lane & 3);
+            const unsigned long long j = (row * p.C + (c & ~3u)) >> 2;
+            const u32x4 ph = philox4x32_10((uint32_t)j, (uint32_t)(j >> 32), (uint32_t)p.seed,
+                                           (uint32_t)(p.seed >> 32));
+            const uint32_t w[4] = {ph.x, ph.y, ph.z, ph.w};
+            uint32_t t[4];
+            quad_transpose4(w, t, lane);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) rw[4 * h + i] = t[i];
+          }
           packed = 0u;
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const unsigned long long idx = (unsigned long long)(rb + w8 * 8 + i) * p.C + c;
-            packed |= e2m1_sr(v8[i], philox_word(idx, p.seed)) << (4 * i);
-          }
+          for (int i = 0; i < 8; ++i) packed |= e2m1_sr(v8[i], rw[i]) << (4 * i);
         }
         words[b * (BS / 8) + w8] = zero ? 0u : packed;
       }
+      if (!col_ok) continue;
       const uint32_t g = rb / BS;
       if (SFMMA) p.scales[sf_mma_offset(c, g, p.g4)] = (uint8_t)byte;
       else p.scales[(size_t)c * p.G + g] = (uint8_t)byte;
@@ -719,7 +756,7 @@ __global__ void __launch_bounds__(256) quantize_cols_kernel(QColParams p) {
         *reinterpret_cast<uint2*>(p.codes + (size_t)c * (p.R / 2) + rb / 2) = make_uint2(words[2 * b], words[2 * b + 1]);
       }
     }
-    if (FMT == FMT_MX) {
+    if (FMT == FMT_MX && col_ok) {
       *reinterpret_cast<uint4*>(p.codes + (size_t)c * (p.R / 2) + rbase / 2) =
           make_uint4(words[0], words[1], words[2], words[3]);
     }

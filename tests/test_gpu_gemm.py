@@ -8,8 +8,8 @@ import torch
 import oracle as O
 import microscaling_fp4_quantization_mxfp4_b200 as F
 from gpu_utils import dev_bf16, host_f32, host_u8
-from workloads import (bf16_to_f32, hadamard_acts, hadamard_weights, mx_linear_128x512, vit_layer,
-                       normal_bf16)
+from workloads import (bf16_to_f32, hadamard_acts, hadamard_weights, llama_acts, llama_weights,
+                       mx_linear_128x512, vit_layer, normal_bf16)
 
 pytestmark = pytest.mark.gpu
 
@@ -117,10 +117,11 @@ def test_full_size_hadamard_mxfp4_8192x11008x4096(had):
     F.fp4_check_device_errors()
 
 
-def test_vit_qkv_fwd_dgrad_wgrad_full_size():
-    """ViT-B/16 qkv linear, M = 50432: forward (RTN), dgrad and wgrad with SR-quantized dY,
+@pytest.mark.parametrize("layer", ["qkv", "fc1", "fc2"])
+def test_vit_fwd_dgrad_wgrad_full_size(layer):
+    """ViT-B/16 linear (qkv 768->2304, fc1 768->3072, fc2 3072->768), M = 50432: forward (RTN), dgrad and wgrad with SR-quantized dY,
     each operand quantized along its own contraction axis (axis 0 = transposed blocks)."""
-    xb, wb, dyb = vit_layer("qkv")
+    xb, wb, dyb = vit_layer(layer)
     M, K = xb.shape
     N = wb.shape[0]
     x, w, dy = dev_bf16(xb), dev_bf16(wb), dev_bf16(dyb)
@@ -151,4 +152,47 @@ def test_vit_qkv_fwd_dgrad_wgrad_full_size():
         np.testing.assert_array_equal(host_u8(qdyt.codes[c:c + 1]), ref["codes"])
         np.testing.assert_array_equal(
             O.sf_from_mma(host_u8(qdyt.scales), N, M // 32)[c:c + 1], ref["scales"])
+    F.fp4_check_device_errors()
+
+
+@pytest.mark.parametrize("kn", [(4096, 4096), (4096, 11008), (11008, 4096)])
+def test_llama_nvfp4_sweep(kn):
+    """Llama-7B shapes, NVFP4: X[:M] (0.5% channels x20, generated at 16384 rows) amax + quantize
+    along K, W quantized once; M = 1, 16, 128, 1024, 4096, 16384.  Per M: the tensor scale equals
+    the oracle's, sampled rows of codes and scales are bit-exact, and sampled output rows (all
+    rows for M <= 128) and columns (M <= 4096) of the fp32 GEMM meet the bound."""
+    K, N = kn
+    xb = llama_acts(K, 16384, seed=4)
+    wb = llama_weights(K, N, seed=4)
+    x, w = dev_bf16(xb), dev_bf16(wb)
+    qw = _gpu_quant(w, "nvfp4")
+    ob = _as_oracle(qw, "nvfp4", N, K)
+    w32 = bf16_to_f32(wb)
+    assert ob["tensor_scale"] == O.nv_tensor_scale(w32)
+    g = np.random.default_rng(K + N)
+    wr = np.sort(g.choice(N, 16, replace=False))
+    ref = O.quantize_values(w32[wr], fmt="nvfp4", tensor_scale=ob["tensor_scale"])
+    np.testing.assert_array_equal(ob["codes"][wr], ref["codes"])
+    np.testing.assert_array_equal(ob["scales"][wr], ref["scales"])
+    x32 = bf16_to_f32(xb)
+    for M in (1, 16, 128, 1024, 4096, 16384):
+        qx = _gpu_quant(x[:M], "nvfp4")
+        oa = _as_oracle(qx, "nvfp4", M, K)
+        assert oa["tensor_scale"] == O.nv_tensor_scale(x32[:M]), M
+        rows = np.arange(M) if M <= 128 else np.sort(g.choice(M, 32, replace=False))
+        sample = rows[:16]
+        ref = O.quantize_values(x32[sample], fmt="nvfp4", tensor_scale=oa["tensor_scale"])
+        np.testing.assert_array_equal(oa["codes"][sample], ref["codes"])
+        np.testing.assert_array_equal(oa["scales"][sample], ref["scales"])
+        y = F.fp4_gemm(qx.codes, qx.scales, qw.codes, qw.scales, fmt="nvfp4", a_tensor_scale=qx.tensor_scale,
+                       b_tensor_scale=qw.tensor_scale, out_dtype="f32")
+        yr, bd = O.gemm_ref_rows(oa, ob, "nvfp4", rows)
+        _check(y[torch.from_numpy(rows).cuda()].cpu().numpy(), yr, bd)
+        if M <= 4096:
+            cols = np.sort(g.choice(N, 16, replace=False))
+            yc, bc = O.gemm_ref_cols(oa, ob, "nvfp4", cols)
+            _check(y[:, torch.from_numpy(cols).cuda()].cpu().numpy(), yc, bc)
+        y16 = F.fp4_gemm(qx.codes, qx.scales, qw.codes, qw.scales, fmt="nvfp4", a_tensor_scale=qx.tensor_scale,
+                         b_tensor_scale=qw.tensor_scale, out_dtype="bf16")
+        _bf16_ulp_check(y16[torch.from_numpy(rows).cuda()], y[torch.from_numpy(rows).cuda()].cpu().numpy())
     F.fp4_check_device_errors()

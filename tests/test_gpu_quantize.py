@@ -211,3 +211,41 @@ def test_nv_two_pass_path_large_tensor():
         ref = O.quantize_values(x32[r:r + 1], fmt="nvfp4", rnd="sr", seed=3, tensor_scale=s_t, idx_base=int(r) * 4096)
         np.testing.assert_array_equal(codes[r:r + 1], ref["codes"])
         np.testing.assert_array_equal(scales[r:r + 1], ref["scales"])
+
+
+def _sr_edge_blocks(rows: int, cols: int, seed: int) -> np.ndarray:
+    """MX blocks whose amax (7.5 or 6) fixes the scale at 1, so the scaled values are the inputs:
+    zeros of both signs, bf16 subnormals, tiny normals on both sides of 2^-9 (where the fixed-point
+    split of the stochastic rounding changes path), every grid point, midpoints, values just
+    below 2, 4 and 6, values above 6 (saturating), and random values over many binades."""
+    from workloads import bf16_bits
+    g = np.random.default_rng(seed)
+    edge = np.array([0.0, -0.0, 2.0 ** -133, -2.0 ** -130, 2.0 ** -126, 2.0 ** -11, 2.0 ** -10, 2.0 ** -9,
+                     3 * 2.0 ** -10, 2.0 ** -8, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0, 0.25, 0.75, 1.25, 1.75,
+                     2.5, 3.5, 5.0, 1.9921875, 3.984375, 5.96875, 6.5, 7.0, -7.5, -5.0, -0.001],
+                    dtype=np.float32)
+    x = np.empty((rows, cols), dtype=np.float32)
+    for r in range(rows):
+        for b in range(cols // 32):
+            if (r + b) % 2 == 0:
+                blk = g.permutation(edge).copy()
+            else:
+                blk = (g.standard_normal(32) * np.exp2(g.integers(-14, 3, 32))).astype(np.float32)
+            blk[0] = 7.5 if (r + b) % 3 else 6.0
+            x[r, 32 * b:32 * b + 32] = blk
+    return bf16_bits(np.clip(x, -7.5, 7.5))
+
+
+@pytest.mark.parametrize("axis", [1, 0])
+@pytest.mark.parametrize("seed", [1, 0xDEADBEEFCAFEF00D])
+def test_sr_edge_values_mx(axis, seed):
+    """Stochastic rounding at the edges of its arithmetic, bit-exact against the oracle, along
+    both axes (axis 0 transposes the edge blocks, so they are built column-wise there)."""
+    xb = _sr_edge_blocks(64, 256, seed & 0xFFFF)
+    if axis == 0:
+        xb = np.ascontiguousarray(xb.T)
+    q = F.fp4_quantize(dev_bf16(xb), fmt="mxfp4", axis=axis, rnd="sr", seed=seed)
+    ref = O.quantize(xb, fmt="mxfp4", axis=axis, rnd="sr", seed=seed)
+    np.testing.assert_array_equal(host_u8(q.scales), ref["scales"])
+    np.testing.assert_array_equal(host_u8(q.codes), ref["codes"])
+    F.fp4_check_device_errors()
