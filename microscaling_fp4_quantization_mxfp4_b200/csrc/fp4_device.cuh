@@ -44,25 +44,41 @@ __device__ __forceinline__ uint32_t pack8_rtn(const float (&v)[8]) {
   return e2m1x4_rn(v[0], v[1], v[2], v[3], v[4], v[5], v[6], v[7]);
 }
 
-// Stochastic rounding of one scaled value with a 32-bit random word:
-// lo <= |v| < hi adjacent grid points, p = (|v| - lo) / (hi - lo) (exact in
-// fp32), round up iff r < ceil(p * 2^32); |v| >= 6 gives 6; sign kept.
-// On [0,2), [2,4), [4,6) the grid step is 0.5, 1, 2, so with s = |v| / step
-// (exact, s < 4) the lower grid point is floor(s) steps in and p is the
-// fractional part of s.  floor(s) comes from one round-toward-zero addition
-// of 2^23 (the sum's last significand bits are the integer part), so the only
-// conversion left per element is the threshold's.
+// a * b + c on the integer multiply-add path (keeps shifts-and-ors of packing
+// and key arithmetic off the ALU pipe, which the stochastic-rounding kernels saturate).
+__device__ __forceinline__ uint32_t mad_u32(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("mad.lo.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+
+// Stochastic rounding of one scaled value with a 32-bit random word; returns
+// the 4-bit code with the sign in bit 3.  lo <= |v| < hi adjacent grid points,
+// p = (|v| - lo) / (hi - lo) (exact in fp32), round up iff r < ceil(p * 2^32);
+// |v| >= 6 gives 6; sign kept.
+// On [0,2), [2,4), [4,8) the grid step is 0.5, 1, 2 = 2^(m-128) with m the
+// biased exponent of |v| clamped to [127, 129], and the lower grid point's code
+// is 2 (m - 127) + floor(s) for s = |v| / step (exact).  floor(s) comes from one
+// round-toward-zero addition of 2^23 (the sum's last significand bits are the
+// integer part), p is the exact remainder, and codes past 6 (|v| >= 6, where s
+// reaches 3 on the top binade) clamp to 7.
 __device__ __forceinline__ uint32_t e2m1_sr(float v, uint32_t r) {
-  const float a = fabsf(v);
-  const float inv_step = a < 2.0f ? 2.0f : (a < 4.0f ? 1.0f : 0.5f);
-  const uint32_t base = a < 2.0f ? 0u : (a < 4.0f ? 2u : 4u);
-  const float s = __fmul_rn(a, inv_step);
+  const uint32_t vb = __float_as_uint(v);
+  const uint32_t m = min(max((vb >> 23) & 0xFFu, 127u), 129u);
+  const float inv_step = __uint_as_float(mad_u32(m, 0xFF800000u, 0x7F800000u));   // (255 - m) << 23
+  const float s = __fmul_rn(fabsf(v), inv_step);
   const float t = __fadd_rz(s, 8388608.0f);                        // 2^23 + floor(s)
   const float p = __fsub_rn(s, __fsub_rn(t, 8388608.0f));          // exact fractional part
   const uint32_t thr = __float2uint_ru(__fmul_rn(p, 4294967296.0f));   // < 2^32 since p < 1
-  uint32_t code = (__float_as_uint(t) - 0x4B000000u) + base + (r < thr ? 1u : 0u);
-  code = a < 6.0f ? code : 7u;
-  return code | ((__float_as_uint(v) >> 31) << 3);
+  const uint32_t code = min(mad_u32(m, 2u, __float_as_uint(t)) - (0x4B000000u + 254u) + (r < thr ? 1u : 0u), 7u);
+  return code | ((vb >> 28) & 8u);
+}
+
+// Eight 4-bit codes, element i in nibble i, packed with multiply-adds.
+__device__ __forceinline__ uint32_t pack8_nibbles(const uint32_t (&n)[8]) {
+  const uint32_t a = mad_u32(n[1], 16u, n[0]), b = mad_u32(n[3], 16u, n[2]);
+  const uint32_t c = mad_u32(n[5], 16u, n[4]), d = mad_u32(n[7], 16u, n[6]);
+  return mad_u32(mad_u32(d, 256u, c), 65536u, mad_u32(b, 256u, a));
 }
 
 // ------------------------------------------------------- scale division -----
@@ -88,7 +104,7 @@ __device__ __forceinline__ float div_by_recip(float x, float S, float y) {
 // Running minimum over a block of 2*|x| - 2 as an unsigned integer (zeros wrap
 // to the top): the block passes div_by_recip's |x| >= 2^-103 test iff the
 // minimum is >= 2*bits(2^-103) - 2.
-__device__ __forceinline__ uint32_t tiny_key(float x) { return (__float_as_uint(x) << 1) - 2u; }
+__device__ __forceinline__ uint32_t tiny_key(float x) { return mad_u32(__float_as_uint(x), 2u, 0xFFFFFFFEu); }
 constexpr uint32_t kTinyKeyMin = (0x0C000000u << 1) - 2u;     // 2^-103 = biased exponent 24
 __device__ __forceinline__ bool recip_usable(float S) { return S >= 0x1p-125f && S <= 0x1p+20f; }
 

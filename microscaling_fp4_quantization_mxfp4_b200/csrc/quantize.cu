@@ -227,9 +227,9 @@ __device__ __forceinline__ void quantize_block(const QRowParams& p, const uint4 
       const u32x4 b = philox4x32_10((uint32_t)(j + 1), (uint32_t)((j + 1) >> 32), (uint32_t)p.seed,
                                     (uint32_t)(p.seed >> 32));
       const float* xe = x + 8 * k;
-      w[k] = e2m1_sr(xe[0], a.x) | (e2m1_sr(xe[1], a.y) << 4) | (e2m1_sr(xe[2], a.z) << 8) |
-             (e2m1_sr(xe[3], a.w) << 12) | (e2m1_sr(xe[4], b.x) << 16) | (e2m1_sr(xe[5], b.y) << 20) |
-             (e2m1_sr(xe[6], b.z) << 24) | (e2m1_sr(xe[7], b.w) << 28);
+      const uint32_t n[8] = {e2m1_sr(xe[0], a.x), e2m1_sr(xe[1], a.y), e2m1_sr(xe[2], a.z), e2m1_sr(xe[3], a.w),
+                             e2m1_sr(xe[4], b.x), e2m1_sr(xe[5], b.y), e2m1_sr(xe[6], b.z), e2m1_sr(xe[7], b.w)};
+      w[k] = pack8_nibbles(n);
     }
   }
   if (!valid) return;
@@ -281,21 +281,24 @@ __global__ void __launch_bounds__(256) quantize_rows_kernel(QRowParams p) {
 }
 
 // ======================================= TMA-fed axis-1 quantize / amax ===
-// Contiguous inputs stream through a ring of 32 KB shared-memory stages filled
+// Contiguous inputs stream through a ring of 64 KB shared-memory stages filled
 // by the bulk-copy engine: one producer thread issues a cp.async.bulk per stage
-// (no per-thread load traffic, many bytes in flight), 16 consumer warps
+// (no per-thread load traffic, many bytes in flight), 15 to 31 consumer warps
 // quantize (or reduce) each stage and release it through an mbarrier.
 constexpr int kStreamChunks = 4096;                     // 8-element chunks per stage (64 KB of bf16)
 constexpr int kStreamStages = 3;
 constexpr int kStreamSmem = kStreamStages * kStreamChunks * 16 + 2 * kStreamStages * 8;
-// Consumer warps per CTA: 31 (with the producer, the 1024-thread maximum)
-// where a thread's live state is small (NVFP4's 16-element blocks, the amax),
-// 16 for MXFP4's 32-element blocks.  Units of a stage are dealt to the warps
-// round-robin, starting one place further on each stage, so that counts that
-// do not divide evenly still balance over a run.
-template <int FMT>
+// Consumer warps per CTA (measured): 31 for NVFP4 and the amax (with the
+// producer, the 1024-thread maximum, so at most 64 registers a thread, which
+// their 16-element blocks fit); 16 for MXFP4 round-to-nearest, with or
+// without rotation (31 warps ran 10-20 % slower); 15 for MXFP4 stochastic
+// rounding, whose 32-element blocks with their eight Philox blocks want about
+// 124 registers.  Units of a stage are dealt to the warps round-robin,
+// starting one place further on each stage, so that counts that do not divide
+// evenly still balance over a run.
+template <int FMT, int RND>
 struct StreamWarps {
-  static constexpr int kWarps = FMT == FMT_MX ? 16 : 31;    // producer + consumers <= 1024 threads
+  static constexpr int kWarps = FMT == FMT_NV ? 31 : (RND == RND_SR ? 15 : 16);   // producer + consumers <= 1024
   static constexpr int kThreads = 32 * (kWarps + 1);
 };
 constexpr int kAmaxWarps = 31;
@@ -324,21 +327,35 @@ __device__ __forceinline__ void stream_ring_init(const StreamRing& r, int consum
   }
 }
 
-// Producer (one thread): stage tiles blockIdx.x, +gridDim.x, ... of the chunk
-// range into the ring.  On an expired wait it flags the error, lets every copy
-// it issued land, and stops.
+// The CTA's share of the chunk range: whole 512-chunk granules (4096 elements,
+// so stage starts stay aligned to scale blocks, Hadamard blocks and warp
+// units), split as evenly as the granules allow, so that every SM gets the same
+// work within one granule instead of whole 64 KB stages dealt round-robin.
+struct StreamRange {
+  uint32_t lo, hi;
+};
+__device__ __forceinline__ StreamRange stream_range(uint32_t nchunks) {
+  constexpr uint32_t kGranule = 512;
+  const uint32_t ng = (nchunks + kGranule - 1) / kGranule;
+  const uint32_t g0 = (uint32_t)(((unsigned long long)ng * blockIdx.x) / gridDim.x);
+  const uint32_t g1 = (uint32_t)(((unsigned long long)ng * (blockIdx.x + 1u)) / gridDim.x);
+  return {min(g0 * kGranule, nchunks), min(g1 * kGranule, nchunks)};
+}
+
+// Producer (one thread): stage the CTA's range into the ring, kStreamChunks at
+// a time.  On an expired wait it flags the error, lets every copy it issued
+// land, and stops.
 __device__ void stream_produce(const StreamRing& r, const uint16_t* x, uint32_t nchunks, unsigned* error) {
-  const uint32_t nstage = (nchunks + kStreamChunks - 1) / kStreamChunks;
+  const StreamRange rg = stream_range(nchunks);
   uint32_t stage = 0, phase = 0, issued = 0, parity_bits = 0;
-  for (uint32_t i = blockIdx.x; i < nstage; i += gridDim.x) {
+  for (uint32_t c0 = rg.lo; c0 < rg.hi; c0 += kStreamChunks) {
     if (!mbar_wait_bounded(smem_addr(&r.empty[stage]), phase ^ 1u)) {
       if (error != nullptr) atomicOr(error, 4u);
       for (int s = 0; s < kStreamStages; ++s)
         if (issued & (1u << s)) mbar_wait_bounded(smem_addr(&r.full[s]), (parity_bits >> s) & 1u);
       return;
     }
-    const uint32_t c0 = i * kStreamChunks;
-    const uint32_t n = min((uint32_t)kStreamChunks, nchunks - c0);
+    const uint32_t n = min((uint32_t)kStreamChunks, rg.hi - c0);
     const uint32_t fb = smem_addr(&r.full[stage]);
     mbar_expect_tx(fb, n * 16u);
     bulk_g2s(smem_addr(r.data + (size_t)stage * kStreamChunks), x + (size_t)c0 * 8, n * 16u, fb);
@@ -352,8 +369,8 @@ __device__ void stream_produce(const StreamRing& r, const uint16_t* x, uint32_t 
 }
 
 template <int FMT, int RND, int HAD, bool SFMMA>
-__global__ void __launch_bounds__(StreamWarps<FMT>::kThreads, 1) quantize_stream_kernel(QRowParams p) {
-  constexpr int kStreamWarps = StreamWarps<FMT>::kWarps;
+__global__ void __launch_bounds__(StreamWarps<FMT, RND>::kThreads, 1) quantize_stream_kernel(QRowParams p) {
+  constexpr int kStreamWarps = StreamWarps<FMT, RND>::kWarps;
   extern __shared__ __align__(1024) uint8_t smem[];
   __shared__ float2 tab[128];
   const StreamRing r = stream_ring(smem);
@@ -373,21 +390,20 @@ __global__ void __launch_bounds__(StreamWarps<FMT>::kThreads, 1) quantize_stream
     return;
   }
   const int cw = warp - 1;
-  const uint32_t nstage = (p.nchunks + kStreamChunks - 1) / kStreamChunks;
-  uint32_t stage = 0, phase = 0;
-  for (uint32_t i = blockIdx.x; i < nstage; i += gridDim.x) {
+  const StreamRange rg = stream_range(p.nchunks);
+  uint32_t stage = 0, phase = 0, j = 0;
+  for (uint32_t c0 = rg.lo; c0 < rg.hi; c0 += kStreamChunks, ++j) {
     int ok = 1;
     if (lane == 0) ok = mbar_wait_bounded(smem_addr(&r.full[stage]), phase) ? 1 : 0;
     if (!__shfl_sync(0xFFFFFFFFu, ok, 0)) {
       if (lane == 0 && p.error != nullptr) atomicOr(p.error, 4u);
       return;
     }
-    const uint32_t c0 = i * kStreamChunks;
-    const uint32_t n = min((uint32_t)kStreamChunks, p.nchunks - c0);
+    const uint32_t n = min((uint32_t)kStreamChunks, rg.hi - c0);
     const uint4* src = r.data + (size_t)stage * kStreamChunks;
     constexpr int V = BlockShape<FMT>::V;
     constexpr uint32_t kUnits = kStreamChunks / (32 * V);                   // warp units per full stage
-    const uint32_t first = ((uint32_t)cw + kStreamWarps - (i / gridDim.x * kUnits) % kStreamWarps) % kStreamWarps;
+    const uint32_t first = ((uint32_t)cw + kStreamWarps - (j * kUnits) % kStreamWarps) % kStreamWarps;
     for (uint32_t u = first; u * 32u * V < n; u += kStreamWarps) {         // warp-uniform
       const uint32_t lb = u * 32u + lane;                                    // block within the stage
       const bool valid = lb * V < n;
@@ -421,16 +437,16 @@ __global__ void __launch_bounds__(32 * (kAmaxWarps + 1), 1) amax_stream_kernel(A
     if (lane == 0) stream_produce(r, p.x, p.rows_x_cpr, error);
   } else {
     const int cw = warp - 1;
-    const uint32_t nstage = (p.rows_x_cpr + kStreamChunks - 1) / kStreamChunks;
+    const StreamRange rg = stream_range(p.rows_x_cpr);
     uint32_t stage = 0, phase = 0;
-    for (uint32_t i = blockIdx.x; i < nstage; i += gridDim.x) {
+    for (uint32_t c0 = rg.lo; c0 < rg.hi; c0 += kStreamChunks) {
       int ok = 1;
       if (lane == 0) ok = mbar_wait_bounded(smem_addr(&r.full[stage]), phase) ? 1 : 0;
       if (!__shfl_sync(0xFFFFFFFFu, ok, 0)) {
         if (lane == 0 && error != nullptr) atomicOr(error, 4u);
         break;
       }
-      const uint32_t n = min((uint32_t)kStreamChunks, p.rows_x_cpr - i * kStreamChunks);
+      const uint32_t n = min((uint32_t)kStreamChunks, rg.hi - c0);
       const uint4* src = r.data + (size_t)stage * kStreamChunks;
 #pragma unroll
       for (int k = 0; k < kStreamChunks / 32 / kStreamWarps; ++k) {
@@ -742,9 +758,10 @@ __global__ void __launch_bounds__(256) quantize_cols_kernel(QColParams p) {
 #pragma unroll
             for (int i = 0; i < 4; ++i) rw[4 * h + i] = t[i];
           }
-          packed = 0u;
+          uint32_t n[8];
 #pragma unroll
-          for (int i = 0; i < 8; ++i) packed |= e2m1_sr(v8[i], rw[i]) << (4 * i);
+          for (int i = 0; i < 8; ++i) n[i] = e2m1_sr(v8[i], rw[i]);
+          packed = pack8_nibbles(n);
         }
         words[b * (BS / 8) + w8] = zero ? 0u : packed;
       }
@@ -781,17 +798,20 @@ __device__ __forceinline__ void fill_pair_table(float2* pairs) {
     pairs[b] = make_float2(e2m1_value((uint32_t)b & 0xFu), e2m1_value((uint32_t)b >> 4));
 }
 
-template <int FMT, bool SFMMA, bool BF16>
-__device__ __forceinline__ void dequantize_chunk_to(const DeqParams& p, uint32_t chunk, uint32_t slot, uint32_t w,
-                                                    float s_t, const float2* pairs) {
-  constexpr int LPB = FMT == FMT_MX ? 4 : 2;
-  uint32_t byte;
+// Address of the scale byte of a chunk (8 codes) in either scale layout.
+template <int FMT, bool SFMMA>
+__device__ __forceinline__ const uint8_t* deq_scale_ptr(const DeqParams& p, uint32_t chunk) {
+  constexpr int LPB = FMT == FMT_MX ? 4 : 2;             // chunks per scale block
   if (SFMMA) {
     const uint32_t row = fdiv(chunk, p.cpr);
-    byte = p.scales[sf_mma_offset(row, (chunk - row * p.cpr.d) / LPB, p.g4)];
-  } else {
-    byte = p.scales[chunk / LPB];
+    return p.scales + sf_mma_offset(row, (chunk - row * p.cpr.d) / LPB, p.g4);
   }
+  return p.scales + chunk / LPB;
+}
+
+template <int FMT, bool BF16>
+__device__ __forceinline__ void dequantize_chunk_to(const DeqParams& p, uint32_t byte, uint32_t slot, uint32_t w,
+                                                    float s_t, const float2* pairs) {
   float y[8];
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
@@ -827,6 +847,8 @@ __device__ __forceinline__ void dequantize_chunk_to(const DeqParams& p, uint32_t
 // Dequantize through shared memory: each CTA fills 512-chunk output tiles
 // (16 KB fp32 / 8 KB bf16) in a 4-deep staging ring and writes each tile back
 // with one bulk store, so the stores never queue behind per-thread traffic.
+// A CTA owns a contiguous, evenly sized run of tiles, and the codes and scale
+// bytes of the next tile are loaded while the current one is converted.
 constexpr int kDeqTileChunks = 512;
 constexpr int kDeqStages = 4;
 constexpr int kDeqThreads = 256;
@@ -840,28 +862,26 @@ __global__ void __launch_bounds__(kDeqThreads) dequantize_stream_kernel(DeqParam
   fill_pair_table(pairs);
   const float s_t = FMT == FMT_NV ? *p.ts : 1.0f;
   const uint32_t ntiles = (p.nchunks + kDeqTileChunks - 1) / kDeqTileChunks;
+  const uint32_t t0 = (uint32_t)(((unsigned long long)ntiles * blockIdx.x) / gridDim.x);
+  const uint32_t t1 = (uint32_t)(((unsigned long long)ntiles * (blockIdx.x + 1u)) / gridDim.x);
   DeqParams q = p;
-  int it = 0;
-  uint32_t w_next[2] = {0u, 0u};
-  uint32_t i = blockIdx.x;
-  if (i < ntiles) {
+  uint32_t w_next[2] = {0u, 0u}, b_next[2] = {0u, 0u};
+  auto prefetch = [&](uint32_t tile) {
 #pragma unroll
     for (int k = 0; k < 2; ++k) {
-      const uint32_t c = i * kDeqTileChunks + threadIdx.x + k * kDeqThreads;
-      if (c < p.nchunks) w_next[k] = __ldg(p.codes + c);
-    }
-  }
-  for (; i < ntiles; i += gridDim.x, ++it) {
-    const int stage = it % kDeqStages;
-    uint32_t w[2] = {w_next[0], w_next[1]};
-    const uint32_t inext = i + gridDim.x;
-    if (inext < ntiles) {                                 // prefetch the next tile's codes
-#pragma unroll
-      for (int k = 0; k < 2; ++k) {
-        const uint32_t c = inext * kDeqTileChunks + threadIdx.x + k * kDeqThreads;
-        w_next[k] = c < p.nchunks ? __ldg(p.codes + c) : 0u;
+      const uint32_t c = tile * kDeqTileChunks + threadIdx.x + k * kDeqThreads;
+      if (c < p.nchunks) {
+        w_next[k] = __ldg(p.codes + c);
+        b_next[k] = __ldg(deq_scale_ptr<FMT, SFMMA>(p, c));
       }
     }
+  };
+  if (t0 < t1) prefetch(t0);
+  int it = 0;
+  for (uint32_t i = t0; i < t1; ++i, ++it) {
+    const int stage = it % kDeqStages;
+    const uint32_t w[2] = {w_next[0], w_next[1]}, sb[2] = {b_next[0], b_next[1]};
+    if (i + 1u < t1) prefetch(i + 1u);
     if (threadIdx.x == 0 && it >= kDeqStages) bulk_wait_read<kDeqStages - 1>();
     __syncthreads();                                      // this stage's previous store has read its data
     q.out = stage_buf + stage * kTileBytes;               // chunk-local output pointer
@@ -869,7 +889,7 @@ __global__ void __launch_bounds__(kDeqThreads) dequantize_stream_kernel(DeqParam
     for (int k = 0; k < 2; ++k) {
       const uint32_t local = threadIdx.x + k * kDeqThreads;
       const uint32_t c = i * kDeqTileChunks + local;
-      if (c < p.nchunks) dequantize_chunk_to<FMT, SFMMA, BF16>(q, c, local, w[k], s_t, pairs);
+      if (c < p.nchunks) dequantize_chunk_to<FMT, BF16>(q, sb[k], local, w[k], s_t, pairs);
     }
     fence_async_smem();
     __syncthreads();
@@ -906,10 +926,10 @@ static cudaError_t amax_stream_launch(const AmaxParams& ap, int num_sms, unsigne
   static const cudaError_t attr =
       cudaFuncSetAttribute(amax_stream_kernel<HAD>, cudaFuncAttributeMaxDynamicSharedMemorySize, kStreamSmem);
   if (attr != cudaSuccess) return attr;
-  const uint32_t nstage = (ap.rows_x_cpr + kStreamChunks - 1) / kStreamChunks;
+  const uint32_t ngran = (ap.rows_x_cpr + 511u) / 512u;      // stream_range's granules
   uint32_t grid = (uint32_t)num_sms;
   if (grid > (uint32_t)kMaxAmaxBlocks) grid = kMaxAmaxBlocks;
-  if (nstage < grid) grid = nstage > 0 ? nstage : 1;
+  if (ngran < grid) grid = ngran > 0 ? ngran : 1;
   amax_stream_kernel<HAD><<<grid, 32 * (kAmaxWarps + 1), kStreamSmem, st>>>(ap, error);
   return cudaGetLastError();
 }
@@ -974,10 +994,10 @@ static cudaError_t rows_stream_launch(const QRowParams& qp, int num_sms, cudaStr
   static const cudaError_t attr =
       cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kStreamSmem);
   if (attr != cudaSuccess) return attr;
-  const uint32_t nstage = (qp.nchunks + kStreamChunks - 1) / kStreamChunks;
+  const uint32_t ngran = (qp.nchunks + 511u) / 512u;         // stream_range's granules
   uint32_t grid = (uint32_t)num_sms;
-  if (nstage < grid) grid = nstage > 0 ? nstage : 1;
-  kernel<<<grid, StreamWarps<FMT>::kThreads, kStreamSmem, st>>>(qp);
+  if (ngran < grid) grid = ngran > 0 ? ngran : 1;
+  kernel<<<grid, StreamWarps<FMT, RND>::kThreads, kStreamSmem, st>>>(qp);
   return cudaGetLastError();
 }
 
