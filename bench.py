@@ -496,7 +496,7 @@ class LlamaNvfp4(GemmWorkload):
         self.outs = [t.empty((m, n), dtype=t.bfloat16, device=device) for k, n, m in self.cases]
         self.timers = {k: KernelTimer(t) for k in ("amax+quantize", "gemm")}
         self.case_timers = [KernelTimer(t) for _ in self.cases]
-        self.flush = t.empty((256 * 1024 * 1024,), dtype=t.uint8, device=device)
+        self.flush = t.zeros((64 * 1024 * 1024,), dtype=t.int32, device=device)
         self.dev_in = {k: t.empty_like(v) for k, v in self.x.items()}
 
     def single_kernel(self):
@@ -526,9 +526,13 @@ class LlamaNvfp4(GemmWorkload):
 
     def step(self, i, timed=False, use_e2e_inputs=False):
         x = self.dev_in if use_e2e_inputs else self.x
+        if timed:
+            # ~2 ms of GPU sleep (untimed) while the host enqueues the step's 18 cases, so that no
+            # case's events also measure the host's launch latency
+            self.t.cuda._sleep(4_000_000)
         for ci in range(len(self.cases)):
             if self.flush_between_cases:
-                self.flush.fill_(i & 0xFF)       # between timed cases: evict the previous case from L2
+                self.flush.max()                 # between timed cases: a 256 MB read evicts the previous case from L2
             self._case(ci, x, timed)
 
     def timed_ms_total(self):
@@ -561,7 +565,8 @@ class LlamaNvfp4(GemmWorkload):
                 "format": "nvfp4", "block": 16, "activations": "N(0,1), 0.5% channels x20, seed 4",
                 "weights": "N(0,0.02), quantized offline (untimed)", "out": "bf16",
                 "gemm_flops_per_step": self.step_flops,
-                "l2": "256 MB write between cases (untimed); ms_per_step sums the per-case event times"}
+                "l2": "256 MB read between cases (untimed) and a GPU sleep while the host enqueues a step; "
+                      "ms_per_step sums the per-case event times"}
 
     def oracle_setup(self):
         from workloads import llama_acts, llama_weights

@@ -35,6 +35,7 @@
 #include <stdint.h>
 #include <stdlib.h>
 
+#include <algorithm>
 #include <mutex>
 
 #include "fp4_internal.h"
@@ -949,6 +950,317 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg2<BN, FMT>::kThre
 
 }  // namespace pair
 
+// ================================== split-K clusters (too few output tiles) ===
+// When the 128 x BN output tiles cannot fill the SMs (small M, as in
+// single-token or short-batch linears), each tile is computed by a cluster of
+// `split` CTAs that divide its k-tiles evenly.  Every CTA runs the single-SM
+// roles (TMA producer, scale copier, MMA thread) over its k-range into its own
+// tensor-memory accumulator; the epilogue warps then park the fp32 partial tile
+// in the CTA's (now idle) shared-memory ring, the cluster synchronises, and
+// every CTA sums one slice of the tile across all partials through distributed
+// shared memory, in rank order (deterministic), scales by alpha and stores it.
+// A second cluster barrier keeps every partial alive until all slices are
+// read.  Both cluster barriers are reached on every path, errors included.
+namespace splitk {
+
+constexpr int kMaxSplit = 8;
+
+template <int BN>
+struct Part {
+  static constexpr int kStride = BN + 4;                       // floats per row (padding spreads banks)
+  static constexpr int kBytes = 128 * kStride * 4;
+};
+
+// Called only between the two cluster barriers, which order it against the partials' stores.
+__device__ __forceinline__ float4 ld_cluster_f4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(addr));
+  return v;
+}
+
+template <int BN, int FMT, bool BF16>
+__global__ void __launch_bounds__(Cfg<BN, FMT>::kThreads, 1)
+    fp4_gemm_splitk_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
+                           KernelArgs p, int split) {
+  using C = Cfg<BN, FMT>;
+  constexpr int S = C::kStages;
+  constexpr int APK = C::kApk;
+  static_assert(Part<BN>::kBytes <= S * C::kStageBytes, "partial tile must fit in the stage ring");
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = sA + S * C::kABytes;
+  uint8_t* sSFA = sB + S * C::kBBytes;
+  uint8_t* sSFB = sSFA + S * C::kSfaBytes;
+  float* part = reinterpret_cast<float*>(smem);               // reuses the ring after the last MMA
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sSFB + S * C::kSfbBytes);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + S;
+  uint64_t* tfull = bars + 2 * S;
+  uint64_t* drain = bars + 2 * S + 1;
+  uint64_t* sfdrain = bars + 2 * S + 2;
+  uint64_t* sf_full = bars + 2 * S + 3;
+  uint64_t* sf_empty = sf_full + kSfBufs;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sf_empty + kSfBufs);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = pair::cluster_rank();
+  const int tile = (int)(blockIdx.x / (uint32_t)split);
+  int mt, nt;
+  tile_coords(tile, p.num_m, p.num_n, mt, nt);
+  const int nkb = (p.K + BK - 1) / BK;
+  const int kb0 = (int)((int64_t)nkb * rank / split), kb1 = (int)((int64_t)nkb * (rank + 1) / split);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(smem_u32(&full[s]), 1);
+      mbar_init(smem_u32(&empty[s]), 1);
+    }
+    mbar_init(smem_u32(tfull), 1);
+    mbar_init(smem_u32(drain), 1);
+    mbar_init(smem_u32(sfdrain), 1);
+    for (uint32_t b = 0; b < kSfBufs; ++b) {
+      mbar_init(smem_u32(&sf_full[b]), 1);
+      mbar_init(smem_u32(&sf_empty[b]), 1);
+    }
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  bool have_part = false;                                        // this thread wrote its partial rows
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer --
+    if (lane == 0) {
+      const int rb_total = (p.N + 127) / 128;
+      const int rb_here = min(BN / 128, rb_total - nt * (BN / 128));
+      int stage = 0;
+      uint32_t phase = 0, issued = 0, issued_parity = 0;
+      bool ok = true;
+      for (int kb = kb0; kb < kb1; ++kb) {
+        if (!wait_spin(smem_u32(&empty[stage]), phase ^ 1u, abort_flag)) {
+          raise_abort(abort_flag, p.error);
+          ok = false;
+          break;
+        }
+        const int kvalid = min(BK, p.K - kb * BK);
+        const int atoms = (kvalid / FmtTraits<FMT>::kBlock + 3) / 4;
+        const uint32_t fb = smem_u32(&full[stage]);
+        mbar_expect_tx(fb, (uint32_t)(C::kABytes + C::kBBytes + atoms * 512 * (1 + rb_here)));
+        tma_load_2d(smem_u32(sA + stage * C::kABytes), &tmap_a, kb * BK_BYTES, mt * BM, fb);
+        tma_load_2d(smem_u32(sB + stage * C::kBBytes), &tmap_b, kb * BK_BYTES, nt * BN, fb);
+        bulk_load(smem_u32(sSFA + stage * C::kSfaBytes), p.a_sf + ((size_t)mt * p.g4 + (size_t)kb * APK) * 512,
+                  (uint32_t)atoms * 512u, fb);
+        for (int rb = 0; rb < rb_here; ++rb)
+          bulk_load(smem_u32(sSFB + stage * C::kSfbBytes + rb * APK * 512),
+                    p.b_sf + ((size_t)(nt * (BN / 128) + rb) * p.g4 + (size_t)kb * APK) * 512, (uint32_t)atoms * 512u,
+                    fb);
+        issued |= 1u << stage;
+        issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
+        if (++stage == S) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      if (!ok) {
+        for (int s = 0; s < S; ++s)
+          if (issued & (1u << s)) {
+            volatile int never = 0;
+            wait_bounded(smem_u32(&full[s]), (issued_parity >> s) & 1u, &never);
+          }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer --
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true, any_mma = false;
+      for (int kb = kb0; kb < kb1; ++kb) {
+        const uint32_t n = (uint32_t)(kb - kb0), b = n % kSfBufs, use_b = n / kSfBufs;
+        if (!wait_spin(smem_u32(&sf_full[b]), use_b & 1u, abort_flag) ||
+            !wait_spin(smem_u32(&full[stage]), phase, abort_flag)) {
+          raise_abort(abort_flag, p.error);
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const int kvalid = min(BK, p.K - kb * BK);
+        const uint32_t sfa_col = C::kSfBase + b * kSfCols;
+        const uint32_t sfb_col = sfa_col + 16u;
+        const uint64_t adesc = desc_sw128(smem_u32(sA + stage * C::kABytes));
+        const uint64_t bdesc = desc_sw128(smem_u32(sB + stage * C::kBBytes));
+        const int nmma = kvalid / 64;
+        for (int j = 0; j < nmma; ++j) {
+          const uint32_t chunk = FMT == FMT_MX ? (uint32_t)(j >> 1) : (uint32_t)j;
+          const uint32_t sf_id = FMT == FMT_MX ? (uint32_t)((j & 1) * 2) : 0u;
+          const uint32_t idesc = idesc_base<BN, FMT>() | (sf_id << 29) | (sf_id << 4);
+          tc_mma<FMT>(tmem, adesc + (uint64_t)(2 * j), bdesc + (uint64_t)(2 * j), idesc, tmem + sfa_col + 4u * chunk,
+                      tmem + sfb_col + 4u * chunk * (BN / 128), (kb > kb0 || j > 0) ? 1u : 0u);
+          any_mma = true;
+        }
+        tc_commit(smem_u32(&empty[stage]));
+        tc_commit(smem_u32(&sf_empty[b]));
+        if (++stage == S) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      if (ok) {
+        tc_commit(smem_u32(tfull));
+      } else if (any_mma) {
+        tc_commit(smem_u32(drain));
+        volatile int never = 0;
+        wait_bounded(smem_u32(drain), 0u, &never);
+      }
+    }
+    __syncwarp();
+  } else if (warp == C::kSfWarp) {
+    // ------------------------------------------------------ scale copier --
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true, any_cp = false;
+      for (int kb = kb0; kb < kb1; ++kb) {
+        const uint32_t n = (uint32_t)(kb - kb0), b = n % kSfBufs, use_b = n / kSfBufs;
+        if (!wait_spin(smem_u32(&full[stage]), phase, abort_flag) ||
+            !wait_spin(smem_u32(&sf_empty[b]), (use_b & 1u) ^ 1u, abort_flag)) {
+          raise_abort(abort_flag, p.error);
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const int kvalid = min(BK, p.K - kb * BK);
+        const int atoms = (kvalid / FmtTraits<FMT>::kBlock + 3) / 4;
+        const uint32_t sfa_col = C::kSfBase + b * kSfCols;
+        const uint32_t sfb_col = sfa_col + 16u;
+        for (int i = 0; i < atoms; ++i) {
+          tc_cp_sf(tmem + sfa_col + 4u * i, desc_sf(smem_u32(sSFA + stage * C::kSfaBytes + i * 512)));
+          for (int rb = 0; rb < BN / 128; ++rb)
+            tc_cp_sf(tmem + sfb_col + 4u * (i * (BN / 128) + rb),
+                     desc_sf(smem_u32(sSFB + stage * C::kSfbBytes + (rb * APK + i) * 512)));
+        }
+        tc_commit(smem_u32(&sf_full[b]));
+        any_cp = true;
+        if (++stage == S) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      if (!ok && any_cp) {
+        tc_commit(smem_u32(sfdrain));
+        volatile int never = 0;
+        wait_bounded(smem_u32(sfdrain), 0u, &never);
+      }
+    }
+    __syncwarp();
+  } else {
+    // -------------------------------------------------- partial tile out --
+    const int q = warp & 3;
+    const int col0 = ((warp - 2) / 4) * 128;
+    int ok = 1;
+    if (lane == 0) ok = wait_bounded(smem_u32(tfull), 0u, abort_flag) ? 1 : 0;
+    ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+    if (!ok) {
+      if (lane == 0) raise_abort(abort_flag, p.error);
+    } else {
+      tc_fence_after();
+      uint32_t r[4][32];
+      const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)col0;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32(tbase + (uint32_t)(32 * c), r[c]);
+      tmem_ld_wait(r);
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // ring bytes last touched by the async proxy
+      float4* row = reinterpret_cast<float4*>(part + (size_t)(q * 32 + lane) * Part<BN>::kStride + col0);
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+#pragma unroll
+        for (int v = 0; v < 8; ++v)
+          row[c * 8 + v] = make_float4(__uint_as_float(r[c][4 * v]), __uint_as_float(r[c][4 * v + 1]),
+                                       __uint_as_float(r[c][4 * v + 2]), __uint_as_float(r[c][4 * v + 3]));
+      have_part = true;
+    }
+  }
+  (void)have_part;
+  tc_fence_before();
+  __syncthreads();
+  pair::cluster_sync_all();                 // every CTA's partial tile is in its shared memory
+
+  // ------------------------------------------- reduce one slice across ranks --
+  {
+    const int rows = min(128, p.M - mt * BM);
+    constexpr int kC4 = BN / 4;                                   // float4 columns per row
+    const int items = rows * kC4;
+    const int i0 = (int)((int64_t)items * rank / split), i1 = (int)((int64_t)items * (rank + 1) / split);
+    const float alpha = FMT == FMT_NV ? __fmul_rn(*p.a_ts, *p.b_ts) : 1.0f;
+    const uint32_t part_base = smem_u32(part);
+    for (int it = i0 + (int)threadIdx.x; it < i1; it += (int)blockDim.x) {
+      const int row = it / kC4, c4 = it - row * kC4;
+      const uint32_t addr = part_base + (uint32_t)((row * Part<BN>::kStride + 4 * c4) * 4);
+      float4 v[kMaxSplit];                                       // all remote loads in flight at once
+#pragma unroll
+      for (int s = 0; s < kMaxSplit; ++s)
+        if (s < split) v[s] = ld_cluster_f4(pair::map_rank(addr, (uint32_t)s));
+      float4 acc = v[0];
+#pragma unroll
+      for (int s = 1; s < kMaxSplit; ++s)
+        if (s < split) {
+          acc.x = __fadd_rn(acc.x, v[s].x);
+          acc.y = __fadd_rn(acc.y, v[s].y);
+          acc.z = __fadd_rn(acc.z, v[s].z);
+          acc.w = __fadd_rn(acc.w, v[s].w);
+        }
+      const float y4[4] = {__fmul_rn(acc.x, alpha), __fmul_rn(acc.y, alpha), __fmul_rn(acc.z, alpha),
+                           __fmul_rn(acc.w, alpha)};
+      const int m = mt * BM + row;
+      const int n0 = nt * BN + 4 * c4;
+      if (BF16) {
+        __nv_bfloat16* yr = reinterpret_cast<__nv_bfloat16*>(p.y) + (size_t)m * p.ldy + n0;
+        if (p.vec_store && n0 + 4 <= p.N) {
+          const uint32_t lo = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(y4[0])) |
+                              ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(y4[1])) << 16);
+          const uint32_t hi = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(y4[2])) |
+                              ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(y4[3])) << 16);
+          *reinterpret_cast<uint2*>(yr) = make_uint2(lo, hi);
+        } else {
+          for (int i = 0; i < 4; ++i)
+            if (n0 + i < p.N) yr[i] = __float2bfloat16_rn(y4[i]);
+        }
+      } else {
+        float* yr = reinterpret_cast<float*>(p.y) + (size_t)m * p.ldy + n0;
+        if (p.vec_store && n0 + 4 <= p.N) {
+          *reinterpret_cast<float4*>(yr) = make_float4(y4[0], y4[1], y4[2], y4[3]);
+        } else {
+          for (int i = 0; i < 4; ++i)
+            if (n0 + i < p.N) yr[i] = y4[i];
+        }
+      }
+    }
+  }
+  pair::cluster_sync_all();                 // no CTA leaves while a peer may still read its partial
+  tc_fence_after();
+  if (warp == 1) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
+  }
+}
+
+}  // namespace splitk
+
+
 // ------------------------------------------------------------------ host ---
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 std::once_flag g_encode_once;
@@ -1065,7 +1377,94 @@ cudaError_t run(const GemmParams& gp, int num_sms, cudaStream_t st) {
   return cudaGetLastError();
 }
 
+// Clusters of `split` CTAs of this kernel that the device can hold at once (0 if unknown).
+template <int BN, int FMT, bool BF16>
+int splitk_max_clusters(int split) {
+  using C = Cfg<BN, FMT>;
+  static int cache[splitk::kMaxSplit + 1] = {};
+  static std::mutex mu;
+  std::lock_guard<std::mutex> lock(mu);
+  if (split < 1 || split > splitk::kMaxSplit) return 0;
+  if (cache[split] == 0) {
+    auto kernel = splitk::fp4_gemm_splitk_kernel<BN, FMT, BF16>;
+    int n = 0;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)split, 1, 1);
+    cfg.blockDim = dim3((unsigned)C::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = (size_t)C::kSmemBytes;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = (unsigned)split;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess ||
+        cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) != cudaSuccess)
+      n = -1;
+    cache[split] = n;
+  }
+  return cache[split] > 0 ? cache[split] : 0;
+}
+
+template <int BN, int FMT, bool BF16>
+cudaError_t run_splitk(const GemmParams& gp, int split, cudaStream_t st) {
+  using C = Cfg<BN, FMT>;
+  auto kernel = splitk::fp4_gemm_splitk_kernel<BN, FMT, BF16>;
+  static const cudaError_t attr = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                       C::kSmemBytes);
+  if (attr != cudaSuccess) return attr;
+  CUtensorMap ta, tb;
+  if (!make_code_map(&ta, gp.a, gp.M, gp.K / 2, BM)) return cudaErrorNotSupported;
+  if (!make_code_map(&tb, gp.b, gp.N, gp.K / 2, BN)) return cudaErrorNotSupported;
+  KernelArgs ka;
+  ka.a_sf = gp.a_sf;
+  ka.b_sf = gp.b_sf;
+  ka.a_ts = gp.a_ts;
+  ka.b_ts = gp.b_ts;
+  ka.y = gp.y;
+  ka.ldy = gp.ldy;
+  ka.M = (int)gp.M;
+  ka.N = (int)gp.N;
+  ka.K = (int)gp.K;
+  ka.num_m = (int)((gp.M + BM - 1) / BM);
+  ka.num_n = (int)((gp.N + BN - 1) / BN);
+  ka.g4 = (int)((gp.K / FmtTraits<FMT>::kBlock + 3) / 4);
+  ka.error = gp.error;
+  {
+    const int64_t esz = gp.y_bf16 ? 2 : 4;
+    ka.vec_store = ((gp.ldy * esz) % 16 == 0 && (reinterpret_cast<uintptr_t>(gp.y) & 15u) == 0) ? 1 : 0;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(ka.num_m * ka.num_n * split), 1, 1);
+  cfg.blockDim = dim3((unsigned)C::kThreads, 1, 1);
+  cfg.dynamicSmemBytes = (size_t)C::kSmemBytes;
+  cfg.stream = st;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = (unsigned)split;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, ta, tb, ka, split);
+}
+
 }  // namespace
+
+template <int BN>
+static int splitk_fit(const GemmParams& p, int split) {
+  if (p.fmt == FMT_MX)
+    return p.y_bf16 ? splitk_max_clusters<BN, FMT_MX, true>(split) : splitk_max_clusters<BN, FMT_MX, false>(split);
+  return p.y_bf16 ? splitk_max_clusters<BN, FMT_NV, true>(split) : splitk_max_clusters<BN, FMT_NV, false>(split);
+}
+
+template <int BN>
+static cudaError_t dispatch_splitk(const GemmParams& p, int split, cudaStream_t st) {
+  if (p.fmt == FMT_MX)
+    return p.y_bf16 ? run_splitk<BN, FMT_MX, true>(p, split, st) : run_splitk<BN, FMT_MX, false>(p, split, st);
+  return p.y_bf16 ? run_splitk<BN, FMT_NV, true>(p, split, st) : run_splitk<BN, FMT_NV, false>(p, split, st);
+}
 
 template <int BN>
 static cudaError_t dispatch_fmt(const GemmParams& p, int num_sms, cudaStream_t st) {
@@ -1101,6 +1500,25 @@ cudaError_t launch_gemm(const GemmParams& p, int num_sms, cudaStream_t st) {
   if (pair_mode != 0 && p.K % 256 == 0 && (pair_mode == 1 || pair_auto))
     return pair_bn == 256 ? dispatch_pair<256>(p, num_sms, st) : dispatch_pair<128>(p, num_sms, st);
   const int bn = forced_bn ? forced_bn : (p.N >= 256 ? 256 : 128);
+  // Too few output tiles to fill the SMs (small M): split each tile's k-range over a cluster of up
+  // to 8 CTAs, as many as keep the launch within one CTA per SM.  FP4_GEMM_SPLIT=1 turns it off.
+  static const int split_mode = [] {
+    const char* e = getenv("FP4_GEMM_SPLIT");
+    return e == nullptr ? -1 : atoi(e);
+  }();
+  const int64_t tiles = ((p.M + BM - 1) / BM) * ((p.N + bn - 1) / bn);
+  const int64_t nkb = (p.K + BK - 1) / BK;
+  int64_t split = tiles > 0 ? num_sms / tiles : 1;
+  if (split > splitk::kMaxSplit) split = splitk::kMaxSplit;
+  if (split > nkb) split = nkb;
+  if (split_mode >= 1) split = std::min<int64_t>(std::min<int64_t>(split_mode, splitk::kMaxSplit), nkb);
+  // every cluster must be resident at once: shrink the clusters until the device holds them all
+  // (clusters of 8 x 220 KB CTAs need 8 free SMs in one GPC)
+  while (split >= 2 &&
+         tiles > (bn == 256 ? splitk_fit<256>(p, (int)split) : splitk_fit<128>(p, (int)split)))
+    --split;
+  if (split >= 2)
+    return bn == 256 ? dispatch_splitk<256>(p, (int)split, st) : dispatch_splitk<128>(p, (int)split, st);
   return bn == 256 ? dispatch_fmt<256>(p, num_sms, st) : dispatch_fmt<128>(p, num_sms, st);
 }
 
