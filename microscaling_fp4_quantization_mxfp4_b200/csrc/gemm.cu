@@ -24,7 +24,10 @@
 //               from the MMA thread).
 //   other warps epilogue: tcgen05.ld the fp32 accumulator (two accumulator
 //               buffers in tensor memory when BN = 128 so the next tile's MMAs
-//               overlap the stores), multiply by alpha, store fp32 or bf16.
+//               overlap the stores), release it, multiply by alpha and store:
+//               bf16 through a 4 KB 128B-swizzled shared-memory box per warp
+//               and TMA stores (full-line writes; short-K shapes are bound by
+//               the output write), fp32 or unaligned rows with direct stores.
 // Every mbarrier wait is bounded; on expiry the CTA raises a shared abort
 // flag and a device error word, drains its own copies and MMAs, frees tensor
 // memory and returns.
@@ -34,6 +37,7 @@
 #include <cudaTypedefs.h>
 #include <stdint.h>
 #include <stdlib.h>
+#include <string.h>
 
 #include <algorithm>
 #include <mutex>
@@ -50,6 +54,8 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kSfCols = 48;      // one scale-factor buffer: SFA (<= 16 cols) then SFB (<= 32 cols)
 constexpr uint32_t kSfBufs = 4;       // scale buffers in tensor memory (after the accumulators)
 constexpr unsigned long long kWaitLimitNs = 4000000000ull;   // 4 s per wait
+constexpr int kSmemRing = 220 * 1024;   // operand stages + output staging, below the 227 KB a CTA can have
+constexpr int kEpiStage = 4096;         // one 32-row x 64-column bf16 box, 128B-swizzled
 
 template <int FMT>
 struct FmtTraits {
@@ -57,7 +63,7 @@ struct FmtTraits {
   static constexpr int kAtomsPerKTile = BK / kBlock / 4;     // 128x4 scale atoms per 128 rows per k-tile
 };
 
-template <int BN, int FMT>
+template <int BN, int FMT, bool EPI = true>
 struct Cfg {
   static constexpr int kAccStages = BN == 128 ? 2 : 1;
   static constexpr int kEpiWarps = BN == 256 ? 8 : 4;          // each epilogue warp drains 128 columns
@@ -71,9 +77,12 @@ struct Cfg {
   static constexpr int kSfaBytes = kApk * 512;
   static constexpr int kSfbBytes = (BN / 128) * kApk * 512;
   static constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;
-  static constexpr int kStages = (220 * 1024) / kStageBytes > 8 ? 8 : (220 * 1024) / kStageBytes;
+  // bf16 output staging for TMA stores: 4 KB (32 rows x 128 bytes) per epilogue warp
+  static constexpr int kEpiBytes = EPI ? kEpiWarps * kEpiStage : 0;
+  static constexpr int kRing = kSmemRing - kEpiBytes;
+  static constexpr int kStages = kRing / kStageBytes > 8 ? 8 : kRing / kStageBytes;
   static constexpr int kBarrierBytes = 1024;
-  static constexpr int kSmemBytes = 1024 /*alignment slack*/ + kStages * kStageBytes + kBarrierBytes;
+  static constexpr int kSmemBytes = 1024 /*alignment slack*/ + kStages * kStageBytes + kEpiBytes + kBarrierBytes;
 };
 
 // ------------------------------------------------------------ PTX wrappers --
@@ -215,6 +224,52 @@ __device__ __forceinline__ void tmem_ld_wait(uint32_t (&r)[4][32]) {
 
 // Shared-memory matrix descriptor: K-major operand, 128-byte rows, 128B
 // swizzle, 8-row groups 1024 bytes apart (Blackwell descriptor version 1).
+// TMA store of one box from shared memory, and bulk-group completion.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t src, int x, int y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(src), "r"(x), "r"(y)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+// One epilogue warp's 32 rows x 128 accumulator columns (r[c][i] = column 32c + i of row
+// y0 + lane) -> alpha * value in bf16 -> two 32 x 64 boxes through the warp's 4 KB staging
+// buffer (1024-byte aligned, 128B-swizzled: 16-byte chunk j of row i at chunk j ^ (i & 7), the
+// layout the tensor map's SWIZZLE_128B expects) -> TMA stores, which clip rows >= M and columns
+// >= N.  The buffer is reused for the second box once the first store has read it.
+__device__ __forceinline__ void epi_store_bf16_tma(const CUtensorMap* tmap_y, uint8_t* stg, const uint32_t (&r)[4][32],
+                                                   float alpha, int x0, int y0, int M, int N, int lane) {
+  const uint32_t base = smem_u32(stg) + (uint32_t)lane * 128u;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    if (lane == 0) bulk_wait_read0();        // the previous box's store has read the buffer
+    __syncwarp();
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      uint32_t w[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float lo = __fmul_rn(__uint_as_float(r[2 * h + (j >> 2)][(j & 3) * 8 + 2 * i]), alpha);
+        const float hi = __fmul_rn(__uint_as_float(r[2 * h + (j >> 2)][(j & 3) * 8 + 2 * i + 1]), alpha);
+        w[i] = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(lo)) |
+               ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(hi)) << 16);
+      }
+      const uint32_t dst = base + (uint32_t)(((j ^ (lane & 7)) & 7) * 16);
+      asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3])
+                   : "memory");
+    }
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // generic writes -> async-proxy reads
+    __syncwarp();
+    if (lane == 0 && x0 + 64 * h < N && y0 < M) {       // boxes wholly past the edge are skipped
+      tma_store_2d(tmap_y, smem_u32(stg), x0 + 64 * h, y0);
+      bulk_commit_group();
+    }
+  }
+}
+
 __device__ __forceinline__ uint64_t desc_sw128(uint32_t addr) {
   return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)1u << 16) | ((uint64_t)(1024u >> 4) << 32) |
          ((uint64_t)1u << 46) | ((uint64_t)2u << 61);
@@ -245,6 +300,7 @@ struct KernelArgs {
   int num_m, num_n;
   int g4;                 // padded k-groups / 4 of both scale tensors
   int vec_store;          // output rows 16-byte aligned: 128-bit stores
+  int tma_store;          // bf16 output through shared memory and TMA stores (tensor map valid)
   unsigned* error;
 };
 
@@ -261,7 +317,7 @@ __device__ __forceinline__ void tile_coords(int t, int num_m, int num_n, int& mt
 template <int BN, int FMT, bool BF16>
 __global__ void __launch_bounds__(Cfg<BN, FMT>::kThreads, 1)
     fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
-                    KernelArgs p) {
+                    const __grid_constant__ CUtensorMap tmap_y, KernelArgs p) {
   using C = Cfg<BN, FMT>;
   constexpr int S = C::kStages;
   constexpr int APK = C::kApk;
@@ -271,7 +327,8 @@ __global__ void __launch_bounds__(Cfg<BN, FMT>::kThreads, 1)
   uint8_t* sB = sA + S * C::kABytes;
   uint8_t* sSFA = sB + S * C::kBBytes;
   uint8_t* sSFB = sSFA + S * C::kSfaBytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sSFB + S * C::kSfbBytes);
+  uint8_t* sEpi = sSFB + S * C::kSfbBytes;                       // 1024-byte aligned
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sEpi + C::kEpiBytes);
   uint64_t* full = bars;
   uint64_t* empty = bars + S;
   uint64_t* tfull = bars + 2 * S;
@@ -515,6 +572,11 @@ __global__ void __launch_bounds__(Cfg<BN, FMT>::kThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&tempty[acc]));
+      if (BF16 && p.tma_store) {
+        epi_store_bf16_tma(&tmap_y, sEpi + (warp - 2) * kEpiStage, r, alpha, nt * BN + col0, mt * BM + q * 32, p.M,
+                           p.N, lane);
+        continue;
+      }
       const int m = mt * BM + row_in_tile;
       if (m < p.M) {
 #pragma unroll
@@ -558,6 +620,7 @@ __global__ void __launch_bounds__(Cfg<BN, FMT>::kThreads, 1)
         }
       }
     }
+    if (BF16 && p.tma_store && lane == 0) bulk_wait_all0();     // stores done before the CTA exits
   }
   tc_fence_before();
   __syncthreads();
@@ -602,7 +665,9 @@ struct Cfg2 {
   static constexpr int kSfaBytes = kApk * 512;
   static constexpr int kSfbBytes = kSfbBlocks * kApk * 512;
   static constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;
-  static constexpr int kStages = (220 * 1024) / kStageBytes > 8 ? 8 : (220 * 1024) / kStageBytes;
+  // No output staging: with K >= 2048 the direct stores hide behind the next tile's MMAs, and the
+  // 32 KB a TMA-store staging buffer takes would cost a stage (measured 2-3 % slower).
+  static constexpr int kStages = kSmemRing / kStageBytes > 8 ? 8 : kSmemRing / kStageBytes;
   static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + 1024;
   static constexpr uint32_t kSfBase = (uint32_t)(kAccStages * BN);   // scale buffers after the accumulators
   static_assert(kSfBase + kSfBufs * kSfCols <= kTmemCols, "tensor memory budget");
@@ -981,10 +1046,10 @@ __device__ __forceinline__ float4 ld_cluster_f4(uint32_t addr) {
 }
 
 template <int BN, int FMT, bool BF16>
-__global__ void __launch_bounds__(Cfg<BN, FMT>::kThreads, 1)
+__global__ void __launch_bounds__(Cfg<BN, FMT, false>::kThreads, 1)
     fp4_gemm_splitk_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                            KernelArgs p, int split) {
-  using C = Cfg<BN, FMT>;
+  using C = Cfg<BN, FMT, false>;
   constexpr int S = C::kStages;
   constexpr int APK = C::kApk;
   static_assert(Part<BN>::kBytes <= S * C::kStageBytes, "partial tile must fit in the stage ring");
@@ -1303,6 +1368,22 @@ bool make_sf_map(CUtensorMap* map, const uint8_t* base, int64_t atoms, int box_a
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// bf16 output Y[M, N] (row stride ldy elements) for TMA stores: 32-row x 64-column boxes,
+// 128B swizzle.  Returns false (caller falls back to direct stores) when Y is fp32, its rows are
+// not 16-byte multiples or its base is not 16-byte aligned.
+bool make_y_map(CUtensorMap* map, const GemmParams& gp) {
+  if (!gp.y_bf16 || (gp.ldy * 2) % 16 != 0 || (reinterpret_cast<uintptr_t>(gp.y) & 15u) != 0) return false;
+  auto enc = encode_fn();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)gp.N, (cuuint64_t)gp.M};
+  cuuint64_t strides[1] = {(cuuint64_t)(gp.ldy * 2)};
+  cuuint32_t box[2] = {64, 32};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, gp.y, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int BN, int FMT, bool BF16>
 cudaError_t run_pair(const GemmParams& gp, int num_sms, cudaStream_t st) {
   using C = pair::Cfg2<BN, FMT>;
@@ -1336,6 +1417,7 @@ cudaError_t run_pair(const GemmParams& gp, int num_sms, cudaStream_t st) {
     const int64_t esz = gp.y_bf16 ? 2 : 4;
     ka.vec_store = ((gp.ldy * esz) % 16 == 0 && (reinterpret_cast<uintptr_t>(gp.y) & 15u) == 0) ? 1 : 0;
   }
+  ka.tma_store = 0;
   const int tiles = ka.num_m * ka.num_n;
   int clusters = num_sms / 2;
   if (tiles < clusters) clusters = tiles;
@@ -1371,16 +1453,19 @@ cudaError_t run(const GemmParams& gp, int num_sms, cudaStream_t st) {
     const int64_t esz = gp.y_bf16 ? 2 : 4;
     ka.vec_store = ((gp.ldy * esz) % 16 == 0 && (reinterpret_cast<uintptr_t>(gp.y) & 15u) == 0) ? 1 : 0;
   }
+  CUtensorMap ty;
+  memset(&ty, 0, sizeof(ty));
+  ka.tma_store = make_y_map(&ty, gp) ? 1 : 0;
   const int tiles = ka.num_m * ka.num_n;
   const int grid = tiles < num_sms ? tiles : num_sms;
-  fp4_gemm_kernel<BN, FMT, BF16><<<grid, C::kThreads, C::kSmemBytes, st>>>(ta, tb, ka);
+  fp4_gemm_kernel<BN, FMT, BF16><<<grid, C::kThreads, C::kSmemBytes, st>>>(ta, tb, ty, ka);
   return cudaGetLastError();
 }
 
 // Clusters of `split` CTAs of this kernel that the device can hold at once (0 if unknown).
 template <int BN, int FMT, bool BF16>
 int splitk_max_clusters(int split) {
-  using C = Cfg<BN, FMT>;
+  using C = Cfg<BN, FMT, false>;
   static int cache[splitk::kMaxSplit + 1] = {};
   static std::mutex mu;
   std::lock_guard<std::mutex> lock(mu);
@@ -1409,7 +1494,7 @@ int splitk_max_clusters(int split) {
 
 template <int BN, int FMT, bool BF16>
 cudaError_t run_splitk(const GemmParams& gp, int split, cudaStream_t st) {
-  using C = Cfg<BN, FMT>;
+  using C = Cfg<BN, FMT, false>;
   auto kernel = splitk::fp4_gemm_splitk_kernel<BN, FMT, BF16>;
   static const cudaError_t attr = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                        C::kSmemBytes);
@@ -1435,6 +1520,7 @@ cudaError_t run_splitk(const GemmParams& gp, int split, cudaStream_t st) {
     const int64_t esz = gp.y_bf16 ? 2 : 4;
     ka.vec_store = ((gp.ldy * esz) % 16 == 0 && (reinterpret_cast<uintptr_t>(gp.y) & 15u) == 0) ? 1 : 0;
   }
+  ka.tma_store = 0;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(ka.num_m * ka.num_n * split), 1, 1);
   cfg.blockDim = dim3((unsigned)C::kThreads, 1, 1);
