@@ -166,6 +166,24 @@ struct BlockShape {
   static constexpr int V = E / 8;                      // uint4 per block
 };
 
+// Whether a block may divide by its scale S with div_by_recip (exact IEEE quotients) instead of
+// __fdiv_rn.  Both need y = RN(1/S) usable (S in [2^-125, 2^20], y != 0) and quotients below
+// 2^64.  Stochastic rounding uses the exact quotient of every element, so it also needs every
+// |x| >= 2^-103 (or 0), where the residuals are exact.  Round-to-nearest only needs the codes:
+// with S >= 2^-100 an element below 2^-103 has |x/S| < 2^-3, and div_by_recip keeps such a
+// quotient below 0.13 with the sign of x, so it rounds to a signed zero code exactly like the
+// correctly rounded quotient, while every larger element is divided exactly; that saves the
+// per-element test.
+template <int RND, int E>
+__device__ __forceinline__ bool nv_fast_division(const float (&x)[E], float am, float S, float y) {
+  if (y == 0.0f || !(__fmul_rn(am, y) < 0x1p64f)) return false;
+  if (RND == RND_RTN) return S >= 0x1p-100f;
+  uint32_t kmin = 0xFFFFFFFFu;
+#pragma unroll
+  for (int i = 0; i < E; ++i) kmin = min(kmin, tiny_key(x[i]));
+  return kmin >= kTinyKeyMin;
+}
+
 template <int FMT, int RND, int HAD, bool SFMMA>
 __device__ __forceinline__ void quantize_block(const QRowParams& p, const uint4 (&v)[BlockShape<FMT>::V], uint32_t blk,
                                                bool valid, int lane, const NvConsts& nv) {
@@ -201,10 +219,7 @@ __device__ __forceinline__ void quantize_block(const QRowParams& p, const uint4 
     byte = e4m3_rn_sat(nv_scale_arg(am, nv.s_t, nv.y_st, nv.st_ok));
     zero = (byte == 0u);
     const float2 sy = nv.tab[byte];
-    uint32_t kmin = 0xFFFFFFFFu;
-#pragma unroll
-    for (int i = 0; i < E; ++i) kmin = min(kmin, tiny_key(x[i]));
-    if (sy.y != 0.0f && kmin >= kTinyKeyMin && __fmul_rn(am, sy.y) < 0x1p64f) {
+    if (nv_fast_division<RND, E>(x, am, sy.x, sy.y)) {
 #pragma unroll
       for (int i = 0; i < E; ++i) x[i] = div_by_recip(x[i], sy.x, sy.y);
     } else {                                     // rare: tiny operands or scales -> IEEE division
@@ -723,10 +738,10 @@ __global__ void __launch_bounds__(256) quantize_cols_kernel(QColParams p) {
         const float2 sy = tab[byte];
         S = sy.x;
         y = sy.y;
-        uint32_t kmin = 0xFFFFFFFFu;
+        float xb[BS];
 #pragma unroll
-        for (int i = 0; i < BS; ++i) kmin = min(kmin, tiny_key(xv[b * BS + i]));
-        fast = y != 0.0f && kmin >= kTinyKeyMin && __fmul_rn(am, y) < 0x1p64f;
+        for (int i = 0; i < BS; ++i) xb[i] = xv[b * BS + i];
+        fast = nv_fast_division<RND, BS>(xb, am, S, y);
       }
 #pragma unroll
       for (int w8 = 0; w8 < BS / 8; ++w8) {
@@ -848,7 +863,7 @@ __device__ __forceinline__ void dequantize_chunk_to(const DeqParams& p, uint32_t
 // (16 KB fp32 / 8 KB bf16) in a 4-deep staging ring and writes each tile back
 // with one bulk store, so the stores never queue behind per-thread traffic.
 // A CTA owns a contiguous, evenly sized run of tiles, and the codes and scale
-// bytes of the next tile are loaded while the current one is converted.
+// bytes of the next three tiles are in flight while the current one is converted.
 constexpr int kDeqTileChunks = 512;
 constexpr int kDeqStages = 4;
 constexpr int kDeqThreads = 256;
@@ -865,23 +880,36 @@ __global__ void __launch_bounds__(kDeqThreads) dequantize_stream_kernel(DeqParam
   const uint32_t t0 = (uint32_t)(((unsigned long long)ntiles * blockIdx.x) / gridDim.x);
   const uint32_t t1 = (uint32_t)(((unsigned long long)ntiles * (blockIdx.x + 1u)) / gridDim.x);
   DeqParams q = p;
-  uint32_t w_next[2] = {0u, 0u}, b_next[2] = {0u, 0u};
-  auto prefetch = [&](uint32_t tile) {
+  // codes and scale bytes of the next kDeqAhead tiles are in flight while a tile is converted
+  constexpr int kDeqAhead = 3;
+  uint32_t wq[kDeqAhead][2], bq[kDeqAhead][2];
+  auto fetch = [&](uint32_t tile, uint32_t (&w)[2], uint32_t (&b)[2]) {
 #pragma unroll
     for (int k = 0; k < 2; ++k) {
       const uint32_t c = tile * kDeqTileChunks + threadIdx.x + k * kDeqThreads;
-      if (c < p.nchunks) {
-        w_next[k] = __ldg(p.codes + c);
-        b_next[k] = __ldg(deq_scale_ptr<FMT, SFMMA>(p, c));
+      w[k] = 0u;
+      b[k] = 0u;
+      if (tile < t1 && c < p.nchunks) {
+        w[k] = __ldg(p.codes + c);
+        b[k] = __ldg(deq_scale_ptr<FMT, SFMMA>(p, c));
       }
     }
   };
-  if (t0 < t1) prefetch(t0);
+#pragma unroll
+  for (int a = 0; a < kDeqAhead; ++a) fetch(t0 + (uint32_t)a, wq[a], bq[a]);
   int it = 0;
   for (uint32_t i = t0; i < t1; ++i, ++it) {
     const int stage = it % kDeqStages;
-    const uint32_t w[2] = {w_next[0], w_next[1]}, sb[2] = {b_next[0], b_next[1]};
-    if (i + 1u < t1) prefetch(i + 1u);
+    const uint32_t w[2] = {wq[0][0], wq[0][1]}, sb[2] = {bq[0][0], bq[0][1]};
+#pragma unroll
+    for (int a = 0; a + 1 < kDeqAhead; ++a) {
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        wq[a][k] = wq[a + 1][k];
+        bq[a][k] = bq[a + 1][k];
+      }
+    }
+    fetch(i + (uint32_t)kDeqAhead, wq[kDeqAhead - 1], bq[kDeqAhead - 1]);
     if (threadIdx.x == 0 && it >= kDeqStages) bulk_wait_read<kDeqStages - 1>();
     __syncthreads();                                      // this stage's previous store has read its data
     q.out = stage_buf + stage * kTileBytes;               // chunk-local output pointer

@@ -249,3 +249,27 @@ def test_sr_edge_values_mx(axis, seed):
     np.testing.assert_array_equal(host_u8(q.scales), ref["scales"])
     np.testing.assert_array_equal(host_u8(q.codes), ref["codes"])
     F.fp4_check_device_errors()
+
+
+@pytest.mark.parametrize("rnd", ["rtn", "sr"])
+@pytest.mark.parametrize("scale", [1.0, 1e-32])
+def test_nv_tiny_elements(rnd, scale):
+    """NVFP4 blocks holding elements far below the block maximum (down to bf16 subnormals and
+    signed zeros), in a tensor of ordinary magnitude (scales S >= 2^-100: the fast division path
+    without a per-element test for RTN) and in an all-tiny tensor (S < 2^-100: IEEE division);
+    codes and scales bit-exact against the oracle."""
+    from workloads import bf16_bits
+    g = np.random.default_rng(7)
+    x = (g.standard_normal((64, 256)) * scale).astype(np.float32)
+    tiny = np.array([1e-35, -1e-35, 2.0 ** -120, -(2.0 ** -126), 2.0 ** -133, -(2.0 ** -133), 0.0, -0.0, 1e-38,
+                     2.0 ** -104, -(2.0 ** -103), 2.0 ** -102], dtype=np.float32)
+    for r in range(0, 64, 3):
+        cols = g.choice(256, 12, replace=False)
+        x[r, cols] = tiny
+    xb = bf16_bits(x)
+    q = F.fp4_quantize(dev_bf16(xb), fmt="nvfp4", rnd=rnd, seed=99)
+    ref = O.quantize(xb, fmt="nvfp4", rnd=rnd, seed=99)
+    assert host_f32(q.tensor_scale)[0] == ref["tensor_scale"]
+    np.testing.assert_array_equal(host_u8(q.scales), ref["scales"])
+    np.testing.assert_array_equal(host_u8(q.codes), ref["codes"])
+    F.fp4_check_device_errors()
