@@ -53,6 +53,7 @@ fp4_status device_state(DeviceState** out) {
     d.scratch.counter = reinterpret_cast<unsigned*>(static_cast<char*>(mem) + sizeof(float) * kMaxAmaxBlocks);
     d.scratch.error = d.scratch.counter + 1;
     d.scratch.grid_arrive = d.scratch.counter + 2;
+    d.scratch.grid_depart = d.scratch.counter + 3;
     d.num_sms = sms;
     d.ready = true;
   }
@@ -61,6 +62,19 @@ fp4_status device_state(DeviceState** out) {
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+
+// FP4_PDL=0 launches without programmatic dependent launch (for debugging and comparison).
+bool fp4lib::pdl_enabled() {
+  static const bool on = [] {
+    const char* e = getenv("FP4_PDL");
+    return !(e != nullptr && e[0] == '0');
+  }();
+  return on;
+}
+
+namespace {
 
 // FP4_SINGLE_PASS=0 forces the two-pass NVFP4 path (amax kernel, then quantize); for testing.
 bool single_pass_disabled() {
@@ -277,8 +291,10 @@ fp4_status fp4_check_device_errors(void* stream) {
   unsigned word = 0;
   if (cudaMemcpy(&word, d->scratch.error, sizeof(unsigned), cudaMemcpyDeviceToHost) != cudaSuccess) return FP4_ERR_CUDA;
   if (word != 0) {
-    const unsigned zero = 0;
-    if (cudaMemcpy(d->scratch.error, &zero, sizeof(unsigned), cudaMemcpyHostToDevice) != cudaSuccess)
+    // clear the error word and the single-pass quantizer's barrier counters, which a timed-out
+    // launch may have left off zero
+    const unsigned zero[3] = {0u, 0u, 0u};
+    if (cudaMemcpy(d->scratch.error, zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess)
       return FP4_ERR_CUDA;
     return FP4_ERR_TIMEOUT;
   }

@@ -7,6 +7,52 @@
 
 namespace fp4lib {
 
+// Programmatic dependent launch.  Every kernel of the library is launched with programmatic
+// stream serialization (unless FP4_PDL=0), so its CTAs may be scheduled -- and run their
+// shared-memory, barrier and tensor-memory setup -- while the previous kernel in the stream
+// drains.  Each kernel calls pdl_wait() before its first global-memory access (that returns once
+// the previous grid has completed and its writes are visible) and pdl_trigger() at entry, so that
+// the next kernel may be scheduled as soon as every CTA of this one has started.
+#ifdef __CUDACC__
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+#endif
+bool pdl_enabled();
+
+// cudaLaunchKernelEx with the programmatic-serialization attribute, plus optional cooperative
+// launch and cluster width.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_kernel(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                          bool cooperative, unsigned cluster_x, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute at[3];
+  unsigned n = 0;
+  if (pdl_enabled()) {
+    at[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+  }
+  if (cooperative) {
+    at[n].id = cudaLaunchAttributeCooperative;
+    at[n].val.cooperative = 1;
+    ++n;
+  }
+  if (cluster_x > 1) {
+    at[n].id = cudaLaunchAttributeClusterDimension;
+    at[n].val.clusterDim.x = cluster_x;
+    at[n].val.clusterDim.y = 1;
+    at[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  cfg.attrs = at;
+  cfg.numAttrs = n;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 enum { FMT_MX = 0, FMT_NV = 1 };
 enum { RND_RTN = 0, RND_SR = 1 };
 
@@ -15,7 +61,8 @@ struct Scratch {
   float* partials;      // per-CTA maxima of the tensor-amax pass
   unsigned* counter;    // CTA ticket counter of the amax pass (self-resetting)
   unsigned* error;      // device error word set by bounded waits
-  unsigned* grid_arrive;  // arrivals at the single-pass NVFP4 quantizer's grid barrier
+  unsigned* grid_arrive;  // arrivals at the single-pass NVFP4 quantizer's grid barrier (self-resetting)
+  unsigned* grid_depart;  // departures from it; the last CTA out zeroes both
 };
 constexpr int kMaxAmaxBlocks = 2048;
 

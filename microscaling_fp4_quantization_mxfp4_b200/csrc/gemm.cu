@@ -318,6 +318,7 @@ template <int BN, int FMT, bool BF16>
 __global__ void __launch_bounds__(Cfg<BN, FMT>::kThreads, 1)
     fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                     const __grid_constant__ CUtensorMap tmap_y, KernelArgs p) {
+  pdl_trigger();
   using C = Cfg<BN, FMT>;
   constexpr int S = C::kStages;
   constexpr int APK = C::kApk;
@@ -370,6 +371,7 @@ __global__ void __launch_bounds__(Cfg<BN, FMT>::kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  pdl_wait();                               // the previous kernel's outputs (our operands) are complete
 
   const int num_tiles = p.num_m * p.num_n;
   const int nkb = (p.K + BK - 1) / BK;
@@ -734,6 +736,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg2<BN, FMT>::kThre
     fp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                          const __grid_constant__ CUtensorMap tmap_sfa, const __grid_constant__ CUtensorMap tmap_sfb,
                          KernelArgs p) {
+  pdl_trigger();
   using C = Cfg2<BN, FMT>;
   constexpr int S = C::kStages;
   constexpr int APK = C::kApk;
@@ -787,6 +790,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg2<BN, FMT>::kThre
   cluster_sync_all();                  // barriers of both CTAs initialised before any remote signal
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  pdl_wait();                          // the previous kernel's outputs (our operands) are complete
 
   const int num_tiles = p.num_m * p.num_n;            // 256 x BN tiles
   const int cluster = blockIdx.x >> 1, nclusters = gridDim.x >> 1;
@@ -1049,6 +1053,7 @@ template <int BN, int FMT, bool BF16>
 __global__ void __launch_bounds__(Cfg<BN, FMT, false>::kThreads, 1)
     fp4_gemm_splitk_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                            KernelArgs p, int split) {
+  pdl_trigger();
   using C = Cfg<BN, FMT, false>;
   constexpr int S = C::kStages;
   constexpr int APK = C::kApk;
@@ -1105,6 +1110,7 @@ __global__ void __launch_bounds__(Cfg<BN, FMT, false>::kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  pdl_wait();                               // the previous kernel's outputs (our operands) are complete
   bool have_part = false;                                        // this thread wrote its partial rows
 
   if (warp == 0) {
@@ -1421,8 +1427,8 @@ cudaError_t run_pair(const GemmParams& gp, int num_sms, cudaStream_t st) {
   const int tiles = ka.num_m * ka.num_n;
   int clusters = num_sms / 2;
   if (tiles < clusters) clusters = tiles;
-  kernel<<<2 * clusters, C::kThreads, C::kSmemBytes, st>>>(ta, tb, tsa, tsb, ka);
-  return cudaGetLastError();
+  return launch_kernel(kernel, dim3(2 * clusters), dim3(C::kThreads), C::kSmemBytes, st, false, 1u, ta, tb, tsa, tsb,
+                       ka);
 }
 
 template <int BN, int FMT, bool BF16>
@@ -1458,8 +1464,8 @@ cudaError_t run(const GemmParams& gp, int num_sms, cudaStream_t st) {
   ka.tma_store = make_y_map(&ty, gp) ? 1 : 0;
   const int tiles = ka.num_m * ka.num_n;
   const int grid = tiles < num_sms ? tiles : num_sms;
-  fp4_gemm_kernel<BN, FMT, BF16><<<grid, C::kThreads, C::kSmemBytes, st>>>(ta, tb, ty, ka);
-  return cudaGetLastError();
+  return launch_kernel(fp4_gemm_kernel<BN, FMT, BF16>, dim3(grid), dim3(C::kThreads), C::kSmemBytes, st, false, 1u,
+                       ta, tb, ty, ka);
 }
 
 // Clusters of `split` CTAs of this kernel that the device can hold at once (0 if unknown).
@@ -1521,19 +1527,8 @@ cudaError_t run_splitk(const GemmParams& gp, int split, cudaStream_t st) {
     ka.vec_store = ((gp.ldy * esz) % 16 == 0 && (reinterpret_cast<uintptr_t>(gp.y) & 15u) == 0) ? 1 : 0;
   }
   ka.tma_store = 0;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)(ka.num_m * ka.num_n * split), 1, 1);
-  cfg.blockDim = dim3((unsigned)C::kThreads, 1, 1);
-  cfg.dynamicSmemBytes = (size_t)C::kSmemBytes;
-  cfg.stream = st;
-  cudaLaunchAttribute at[1];
-  at[0].id = cudaLaunchAttributeClusterDimension;
-  at[0].val.clusterDim.x = (unsigned)split;
-  at[0].val.clusterDim.y = 1;
-  at[0].val.clusterDim.z = 1;
-  cfg.attrs = at;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kernel, ta, tb, ka, split);
+  return launch_kernel(kernel, dim3((unsigned)(ka.num_m * ka.num_n * split)), dim3(C::kThreads), C::kSmemBytes, st,
+                       false, (unsigned)split, ta, tb, ka, split);
 }
 
 }  // namespace

@@ -60,6 +60,8 @@ struct AmaxParams {
 
 template <int HAD>
 __global__ void __launch_bounds__(256) amax_kernel(AmaxParams p) {
+  pdl_trigger();
+  pdl_wait();
   const int lane = threadIdx.x & 31;
   const uint32_t nchunks = p.rows_x_cpr;
   const uint32_t ntiles = (nchunks + 31u) >> 5;
@@ -125,6 +127,8 @@ __global__ void __launch_bounds__(256) amax_kernel(AmaxParams p) {
 }
 
 __global__ void nv_tensor_scale_kernel(const float* amax, float* out) {
+  pdl_trigger();
+  pdl_wait();
   const float a = *amax;
   *out = (a == 0.0f) ? 1.0f : __fdiv_rn(a, 2688.0f);
 }
@@ -264,9 +268,11 @@ __device__ __forceinline__ void quantize_block(const QRowParams& p, const uint4 
 // Strided inputs (ld != cols): one thread per scale block, loads straight from global memory.
 template <int FMT, int RND, int HAD, bool SFMMA>
 __global__ void __launch_bounds__(256) quantize_rows_kernel(QRowParams p) {
+  pdl_trigger();
   constexpr int V = BlockShape<FMT>::V;
   __shared__ float2 tab[128];
   const int lane = threadIdx.x & 31;
+  pdl_wait();
   NvConsts nv{1.0f, 1.0f, true, tab};
   if (FMT == FMT_NV) {
     nv.s_t = *p.ts;
@@ -388,9 +394,11 @@ __global__ void __launch_bounds__(StreamWarps<FMT, RND>::kThreads, 1) quantize_s
   constexpr int kStreamWarps = StreamWarps<FMT, RND>::kWarps;
   extern __shared__ __align__(1024) uint8_t smem[];
   __shared__ float2 tab[128];
+  pdl_trigger();
   const StreamRing r = stream_ring(smem);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   stream_ring_init(r, kStreamWarps);
+  pdl_wait();
   NvConsts nv{1.0f, 1.0f, true, tab};
   if (FMT == FMT_NV) {
     nv.s_t = *p.ts;
@@ -443,9 +451,11 @@ __global__ void __launch_bounds__(32 * (kAmaxWarps + 1), 1) amax_stream_kernel(A
   extern __shared__ __align__(1024) uint8_t smem[];
   __shared__ uint32_t wmax[kStreamWarps];
   __shared__ bool is_last;
+  pdl_trigger();
   const StreamRing r = stream_ring(smem);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   stream_ring_init(r, kStreamWarps);
+  pdl_wait();
   __syncthreads();
   float m = 0.0f;
   if (warp == 0) {
@@ -515,7 +525,8 @@ struct FusedParams {
   QRowParams q;
   float* ts_out;          // s_t, written by CTA 0
   float* partials;        // one partial amax per CTA
-  unsigned* arrive;       // grid-barrier arrivals (zeroed before the launch)
+  unsigned* arrive;       // grid-barrier arrivals (zero at launch: the previous launch reset it)
+  unsigned* depart;       // grid-barrier departures
   unsigned* error;        // device error word (bit 1: barrier wait expired)
   uint32_t tiles_per_cta; // 32-chunk warp tiles staged by each CTA
 };
@@ -541,10 +552,12 @@ __global__ void __launch_bounds__(kFusedThreads, 1) nv_quantize_fused_kernel(Fus
   const uint32_t c_end = min(p.nchunks, t_end * 32u);
   const uint32_t nslice = c_end > c_begin ? c_end - c_begin : 0u;
   const uint32_t piece = ((nslice + kFusedPieces - 1) / kFusedPieces + 31u) & ~31u;   // chunks, whole warp tiles
+  pdl_trigger();
   if (threadIdx.x == 0) {
     for (int k = 0; k < kFusedPieces; ++k) mbar_init(smem_addr(&piece_bar[k]), 1);
     mbar_init_fence();
   }
+  pdl_wait();
   __syncthreads();
   // phase 1: the slice lands in shared memory as kFusedPieces bulk copies; consumers reduce the
   // amax (of the rotated values when HAD > 0) of each piece as soon as it arrives
@@ -605,6 +618,12 @@ __global__ void __launch_bounds__(kFusedThreads, 1) nv_quantize_fused_kernel(Fus
         break;
       }
       __nanosleep(64);
+    }
+    // the last CTA to leave zeroes both counters for the next launch (every CTA has seen the
+    // full count by then)
+    if (atomicAdd(fp.depart, 1u) == gridDim.x - 1u) {
+      atomicExch(fp.arrive, 0u);
+      atomicExch(fp.depart, 0u);
     }
   }
   __syncthreads();
@@ -680,9 +699,11 @@ struct QColParams {
 
 template <int FMT, int RND, bool SFMMA>
 __global__ void __launch_bounds__(256) quantize_cols_kernel(QColParams p) {
+  pdl_trigger();
   __shared__ __align__(16) uint16_t tile[128][64];
   __shared__ float2 tab[128];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  pdl_wait();
   const uint32_t tiles_r = (p.R + 127u) / 128u, tiles_c = (p.C + 63u) / 64u;
   float s_t = 1.0f, y_st = 1.0f;
   bool st_ok = true;
@@ -874,7 +895,9 @@ __global__ void __launch_bounds__(kDeqThreads) dequantize_stream_kernel(DeqParam
   constexpr int kTileBytes = kDeqTileChunks * kOut;
   extern __shared__ __align__(128) uint8_t stage_buf[];
   __shared__ float2 pairs[256];
+  pdl_trigger();
   fill_pair_table(pairs);
+  pdl_wait();
   const float s_t = FMT == FMT_NV ? *p.ts : 1.0f;
   const uint32_t ntiles = (p.nchunks + kDeqTileChunks - 1) / kDeqTileChunks;
   const uint32_t t0 = (uint32_t)(((unsigned long long)ntiles * blockIdx.x) / gridDim.x);
@@ -945,8 +968,7 @@ static cudaError_t amax_launch(const AmaxParams& ap, uint32_t ntiles, int num_sm
   uint32_t grid = (uint32_t)num_sms * (uint32_t)occ;
   if (grid > (uint32_t)kMaxAmaxBlocks) grid = kMaxAmaxBlocks;
   if (want < grid) grid = want > 0 ? want : 1;
-  amax_kernel<HAD><<<grid, 256, 0, st>>>(ap);
-  return cudaGetLastError();
+  return launch_kernel(amax_kernel<HAD>, dim3(grid), dim3(256), 0, st, false, 1u, ap);
 }
 
 template <int HAD>
@@ -958,8 +980,8 @@ static cudaError_t amax_stream_launch(const AmaxParams& ap, int num_sms, unsigne
   uint32_t grid = (uint32_t)num_sms;
   if (grid > (uint32_t)kMaxAmaxBlocks) grid = kMaxAmaxBlocks;
   if (ngran < grid) grid = ngran > 0 ? ngran : 1;
-  amax_stream_kernel<HAD><<<grid, 32 * (kAmaxWarps + 1), kStreamSmem, st>>>(ap, error);
-  return cudaGetLastError();
+  return launch_kernel(amax_stream_kernel<HAD>, dim3(grid), dim3(32 * (kAmaxWarps + 1)), kStreamSmem, st, false, 1u,
+                       ap, error);
 }
 
 cudaError_t launch_amax(const void* x, int64_t rows, int64_t cols, int64_t ld, int had, int mode, float* out,
@@ -1007,13 +1029,11 @@ cudaError_t launch_amax_fixed_grid(const void* x, int64_t rows, int64_t cols, in
   ap.counter = s.counter;
   ap.out = out;
   ap.mode = 0;
-  amax_kernel<0><<<grid, 256, 0, st>>>(ap);
-  return cudaGetLastError();
+  return launch_kernel(amax_kernel<0>, dim3(grid), dim3(256), 0, st, false, 1u, ap);
 }
 
 cudaError_t launch_nv_tensor_scale(const float* amax, float* out, cudaStream_t st) {
-  nv_tensor_scale_kernel<<<1, 1, 0, st>>>(amax, out);
-  return cudaGetLastError();
+  return launch_kernel(nv_tensor_scale_kernel, dim3(1), dim3(1), 0, st, false, 1u, amax, out);
 }
 
 template <int FMT, int RND, int HAD, bool SFMMA>
@@ -1025,8 +1045,7 @@ static cudaError_t rows_stream_launch(const QRowParams& qp, int num_sms, cudaStr
   const uint32_t ngran = (qp.nchunks + 511u) / 512u;         // stream_range's granules
   uint32_t grid = (uint32_t)num_sms;
   if (ngran < grid) grid = ngran > 0 ? ngran : 1;
-  kernel<<<grid, StreamWarps<FMT, RND>::kThreads, kStreamSmem, st>>>(qp);
-  return cudaGetLastError();
+  return launch_kernel(kernel, dim3(grid), dim3(StreamWarps<FMT, RND>::kThreads), kStreamSmem, st, false, 1u, qp);
 }
 
 template <int FMT, int RND, int HAD, bool SFMMA>
@@ -1037,8 +1056,7 @@ static cudaError_t rows_launch(const QRowParams& qp, int num_sms, cudaStream_t s
   uint32_t want = (nunits + 7u) / 8u;
   uint32_t grid = (uint32_t)num_sms * (uint32_t)occ;
   if (want < grid) grid = want > 0 ? want : 1;
-  quantize_rows_kernel<FMT, RND, HAD, SFMMA><<<grid, 256, 0, st>>>(qp);
-  return cudaGetLastError();
+  return launch_kernel(quantize_rows_kernel<FMT, RND, HAD, SFMMA>, dim3(grid), dim3(256), 0, st, false, 1u, qp);
 }
 
 template <int FMT, int RND, int HAD>
@@ -1064,10 +1082,7 @@ static cudaError_t fused_launch(const FusedParams& fp, uint32_t grid, size_t sme
   static const cudaError_t attr =
       cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kFusedMaxSmem);
   if (attr != cudaSuccess) return attr;
-  FusedParams args = fp;
-  void* kargs[] = {&args};
-  return cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(kernel), dim3(grid), dim3(kFusedThreads), kargs,
-                                     smem, st);
+  return launch_kernel(kernel, dim3(grid), dim3(kFusedThreads), smem, st, true, 1u, fp);
 }
 
 template <int RND, int HAD>
@@ -1112,11 +1127,11 @@ cudaError_t launch_quantize_nv_fused(const QuantizeParams& p, float* ts_out, con
   fp.ts_out = ts_out;
   fp.partials = s.partials;
   fp.arrive = s.grid_arrive;
+  fp.depart = s.grid_depart;
   fp.error = s.error;
   fp.tiles_per_cta = per;
   const uint64_t ntiles = ((uint64_t)qp.nchunks + 31u) / 32u;
   const uint32_t grid = (uint32_t)((ntiles + per - 1) / per);
-  if (cudaMemsetAsync(s.grid_arrive, 0, sizeof(unsigned), st) != cudaSuccess) return cudaErrorUnknown;
   const bool sfmma = p.sf_mma != 0;
 #define FP4_FUSED_HAD(H)                                                                               \
   return p.rnd == RND_RTN ? fused_dispatch_sf<RND_RTN, H>(fp, sfmma, grid, smem, st)                  \
@@ -1138,8 +1153,7 @@ static cudaError_t cols_launch(const QColParams& qp, int num_sms, cudaStream_t s
   const uint32_t ntiles = ((qp.R + 127u) / 128u) * ((qp.C + 63u) / 64u);
   uint32_t grid = (uint32_t)num_sms * (uint32_t)occ;
   if (ntiles < grid) grid = ntiles > 0 ? ntiles : 1;
-  quantize_cols_kernel<FMT, RND, SFMMA><<<grid, 256, 0, st>>>(qp);
-  return cudaGetLastError();
+  return launch_kernel(quantize_cols_kernel<FMT, RND, SFMMA>, dim3(grid), dim3(256), 0, st, false, 1u, qp);
 }
 
 template <int FMT, int RND>
@@ -1206,8 +1220,7 @@ static cudaError_t deq_launch(const DeqParams& dp, int num_sms, cudaStream_t st)
   const uint32_t ntiles = (dp.nchunks + kDeqTileChunks - 1) / kDeqTileChunks;
   uint32_t grid = (uint32_t)num_sms * (uint32_t)occ;
   if (ntiles < grid) grid = ntiles > 0 ? ntiles : 1;
-  kernel<<<grid, kDeqThreads, smem, st>>>(dp);
-  return cudaGetLastError();
+  return launch_kernel(kernel, dim3(grid), dim3(kDeqThreads), (size_t)smem, st, false, 1u, dp);
 }
 
 cudaError_t launch_dequantize(const uint8_t* codes, const uint8_t* scales, const float* ts, int64_t rows,
