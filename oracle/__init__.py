@@ -29,8 +29,9 @@ the plainest reading (OCP MX v1.0 E2M1/E8M0/E4M3 conventions, Philox4x32-10 of
 Salmon et al. SC'11, Sylvester Hadamard) and each module says which.
 
 Modules: `formats` (E2M1/E4M3/E8M0), `philox`, `quantize` (MX/NV, RTN/SR,
-axis 0/1, packing, dequantize), `hadamard`, `layout` (tensor-core scale-factor
-layout), `gemm` (fp64 reference and error bound).
+axis 0/1, packing, dequantize), `quantize2d` (square-tile 2-D blocks),
+`hadamard`, `layout` (tensor-core scale-factor layout), `gemm` (fp64 reference
+and error bound).
 """
 from .formats import (E2M1_GRID, e2m1_decode, e2m1_rtn, e2m1_sr, e4m3_decode, e4m3_rne_sat,
                       mx_scale_exponent)
@@ -39,11 +40,12 @@ from .hadamard import sylvester, block_hadamard
 from .quantize import quantize, quantize_values, dequantize, pack_nibbles, unpack_nibbles, nv_tensor_scale
 from .layout import sf_to_mma, sf_from_mma, sf_mma_bytes
 from .gemm import gemm_ref, gemm_ref_rows, gemm_ref_cols, deq_for_gemm
+from .quantize2d import quantize_2d
 
 __all__ = [
     "E2M1_GRID", "e2m1_decode", "e2m1_rtn", "e2m1_sr", "e4m3_decode", "e4m3_rne_sat",
     "mx_scale_exponent", "philox4x32_10", "philox_words", "sylvester", "block_hadamard",
     "quantize", "quantize_values", "dequantize", "pack_nibbles", "unpack_nibbles", "nv_tensor_scale",
     "sf_to_mma", "sf_from_mma", "sf_mma_bytes", "gemm_ref", "gemm_ref_rows", "gemm_ref_cols",
-    "deq_for_gemm",
+    "deq_for_gemm", "quantize_2d",
 ]
