@@ -124,6 +124,30 @@ fp4_status fp4_hadamard_quantize(const void* x, int64_t rows, int64_t cols, int6
                                  int had_block, float* rotated_out, void* stream);
 
 /*
+ * fp4_quantize_2d -- square-tile block quantization of a matrix
+ * ("Pretraining Large Language Models with NVFP4", Abstract: a two-dimensional
+ * quantization gives weights one consistent representation in the forward and
+ * backward passes).  A block x block tile (16 x 16 NVFP4, 32 x 32 MXFP4)
+ * shares one scale, computed from the tile's amax as fp4_quantize computes a
+ * block's; each element is scaled and rounded once (SR: Philox word of its
+ * row-major index in x), so W's codes along its rows and W^T's codes along its
+ * rows are the same codes transposed, every segment carrying its tile's scale.
+ *   x          bf16 [rows, cols], row stride ld; rows and cols multiples of the
+ *              block; alignment as fp4_quantize.
+ *   fmt,block,rnd,seed,tensor_scale_in,tensor_scale_out,sf_layout
+ *              as fp4_quantize (NV without tensor_scale_in runs an amax pass).
+ *   codes, scales      W along its rows: as fp4_quantize axis 1 (required).
+ *   codes_t, scales_t  W^T along its rows, i.e. x quantized along axis 0:
+ *              as fp4_quantize axis 0 ([cols, rows/2], 16-byte aligned); both
+ *              null to skip, or both given.
+ */
+fp4_status fp4_quantize_2d(const void* x, int64_t rows, int64_t cols, int64_t ld,
+                           int fmt, int block, int rnd, uint64_t seed,
+                           const float* tensor_scale_in, float* tensor_scale_out,
+                           uint8_t* codes, uint8_t* scales, uint8_t* codes_t, uint8_t* scales_t,
+                           int sf_layout, void* stream);
+
+/*
  * fp4_dequantize -- codes + scales (+ s_t) back to floating point
  * ("FP4 All the Way", Abstract: the E2M1 values times their block scale).
  * MX: G[c] * 2^(b-127), exact in fp32.  NV: fp32(fp32(G[c] * sb) * s_t).

@@ -127,6 +127,28 @@ def fp4_hadamard_quantize(x: torch.Tensor, had_block: int, fmt="mxfp4", axis: in
     return Fp4Quantized(codes, scales, ts_out if f == NVFP4 else None)
 
 
+def fp4_quantize_2d(x: torch.Tensor, fmt="nvfp4", rnd="rtn", seed: int = 0,
+                    tensor_scale_in: Optional[torch.Tensor] = None, sf_layout="rowmajor", transposed: bool = True,
+                    *, codes=None, scales=None, codes_t=None, scales_t=None, tensor_scale_out=None,
+                    stream=None):
+    """Square-tile (2-D) quantization (see fp4_quantize_2d in include/fp4.h).  Returns
+    (W along its rows, W^T along its rows or None) as Fp4Quantized, sharing one tensor scale."""
+    _bf16_matrix(x)
+    f, r, sf = _FMT[fmt], _RND[rnd], _SF[sf_layout]
+    codes, scales, ts_out = _alloc_quant_outputs(x, f, 1, sf, codes, scales, tensor_scale_out)
+    if transposed:
+        codes_t, scales_t, _ = _alloc_quant_outputs(x, f, 0, sf, codes_t, scales_t, ts_out)
+    else:
+        codes_t = scales_t = None
+    st = _lib.load().fp4_quantize_2d(
+        x.data_ptr(), x.shape[0], x.shape[1], x.stride(0), f, BLOCK[f], r, seed & (2 ** 64 - 1),
+        _ptr(tensor_scale_in), _ptr(ts_out), codes.data_ptr(), scales.data_ptr(), _ptr(codes_t), _ptr(scales_t),
+        sf, _stream(stream))
+    _check(st, "fp4_quantize_2d")
+    ts = ts_out if f == NVFP4 else None
+    return Fp4Quantized(codes, scales, ts), (Fp4Quantized(codes_t, scales_t, ts) if transposed else None)
+
+
 def fp4_dequantize(codes: torch.Tensor, scales: torch.Tensor, tensor_scale=None, fmt="mxfp4",
                    sf_layout="rowmajor", out_dtype="f32", *, out=None, stream=None) -> torch.Tensor:
     """Codes + scales (+ tensor scale) back to fp32 or bf16 [rows, 2 * codes.shape[1]]."""

@@ -197,6 +197,62 @@ fp4_status fp4_hadamard_quantize(const void* x, int64_t rows, int64_t cols, int6
                        scales, sf_layout, had_block, rotated_out, static_cast<cudaStream_t>(stream));
 }
 
+fp4_status fp4_quantize_2d(const void* x, int64_t rows, int64_t cols, int64_t ld, int fmt, int block, int rnd,
+                           uint64_t seed, const float* tensor_scale_in, float* tensor_scale_out, uint8_t* codes,
+                           uint8_t* scales, uint8_t* codes_t, uint8_t* scales_t, int sf_layout, void* stream) {
+  fp4_status s = check_format(fmt, block);
+  if (s != FP4_OK) return s;
+  if ((s = check_input(x, rows, cols, ld)) != FP4_OK) return s;
+  if (rnd != FP4_RTN && rnd != FP4_SR) return FP4_ERR_ARG;
+  if (sf_layout != FP4_SF_ROWMAJOR && sf_layout != FP4_SF_MMA) return FP4_ERR_ARG;
+  if (codes == nullptr || scales == nullptr) return FP4_ERR_ARG;
+  if ((codes_t == nullptr) != (scales_t == nullptr)) return FP4_ERR_ARG;
+  if (fmt == FP4_NVFP4 && tensor_scale_out == nullptr) return FP4_ERR_ARG;
+  if (rows % block != 0 || cols % block != 0) return FP4_ERR_SHAPE;
+  if (!aligned16(codes) || (codes_t != nullptr && !aligned16(codes_t))) return FP4_ERR_ALIGN;
+  DeviceState* d = nullptr;
+  if ((s = device_state(&d)) != FP4_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (sf_layout == FP4_SF_MMA) {
+    // padding bytes of the tensor-core layout must read as scale 0
+    const int64_t g = cols / block, gt = rows / block;
+    if ((rows % 128 != 0 || g % 4 != 0) &&
+        cudaMemsetAsync(scales, 0, (size_t)(round_up(rows, 128) * round_up(g, 4)), st) != cudaSuccess)
+      return FP4_ERR_CUDA;
+    if (scales_t != nullptr && (cols % 128 != 0 || gt % 4 != 0) &&
+        cudaMemsetAsync(scales_t, 0, (size_t)(round_up(cols, 128) * round_up(gt, 4)), st) != cudaSuccess)
+      return FP4_ERR_CUDA;
+  }
+  QuantizeParams p;
+  p.x = x;
+  p.rows = rows;
+  p.cols = cols;
+  p.ld = ld;
+  p.fmt = fmt == FP4_MXFP4 ? FMT_MX : FMT_NV;
+  p.axis = 1;
+  p.rnd = rnd == FP4_RTN ? RND_RTN : RND_SR;
+  p.seed = seed;
+  p.codes = codes;
+  p.scales = scales;
+  p.sf_mma = sf_layout == FP4_SF_MMA;
+  p.had = 0;
+  p.rotated = nullptr;
+  p.error = d->scratch.error;
+  p.ts = nullptr;
+  p.ts_copy_out = nullptr;
+  if (fmt == FP4_NVFP4) {
+    if (tensor_scale_in != nullptr) {
+      p.ts = tensor_scale_in;
+      p.ts_copy_out = (tensor_scale_out != tensor_scale_in) ? tensor_scale_out : nullptr;
+    } else {
+      if (launch_amax(x, rows, cols, ld, 0, 1, tensor_scale_out, d->scratch, d->num_sms, st) != cudaSuccess)
+        return FP4_ERR_CUDA;
+      p.ts = tensor_scale_out;
+    }
+  }
+  return from_cuda(launch_quantize_2d(p, codes_t, scales_t, d->num_sms, st));
+}
+
 fp4_status fp4_dequantize(const uint8_t* codes, const uint8_t* scales, const float* tensor_scale, int64_t rows,
                           int64_t cols, int fmt, int block, int sf_layout, void* out, int out_dtype, void* stream) {
   fp4_status s = check_format(fmt, block);

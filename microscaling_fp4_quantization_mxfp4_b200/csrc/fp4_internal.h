@@ -97,6 +97,10 @@ cudaError_t launch_amax_fixed_grid(const void* x, int64_t rows, int64_t cols, in
                                    const Scratch& s, uint32_t grid, cudaStream_t st);
 cudaError_t launch_nv_tensor_scale(const float* amax, float* out, cudaStream_t st);
 cudaError_t launch_quantize(const QuantizeParams& p, int num_sms, cudaStream_t st);
+// Square-tile (2-D) quantize along axis 1 (codes/scales) and, when codes_t is not null, the same
+// codes transposed with the same tile scales (codes_t/scales_t).  rows, cols multiples of the block.
+cudaError_t launch_quantize_2d(const QuantizeParams& p, uint8_t* codes_t, uint8_t* scales_t, int num_sms,
+                               cudaStream_t st);
 // Single-pass NVFP4 quantize (axis 1, no caller-given s_t) for tensors that fit in shared memory
 // across the SMs; fused_nv_fits says whether it applies.  Writes s_t to ts_out.
 bool fused_nv_fits(int64_t rows, int64_t cols, int num_sms, size_t* smem, uint32_t* tiles_per_cta);

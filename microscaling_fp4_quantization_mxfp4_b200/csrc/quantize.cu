@@ -816,6 +816,176 @@ __global__ void __launch_bounds__(256) quantize_cols_kernel(QColParams p) {
   }
 }
 
+// ===================================================== 2-D (square-tile) quantize ===
+// "Pretraining Large Language Models with NVFP4", Abstract: a two-dimensional
+// scheme gives weights one consistent representation forward and backward.
+// A block x block tile (16 x 16 NVFP4, 32 x 32 MXFP4) shares one scale; every
+// element is scaled and rounded once, and its code goes both to W's codes
+// (packed along rows, [R, C/2]) and, when asked, to W^T's codes (packed along
+// W's columns, [C, R/2]), each row or column segment carrying the tile's
+// scale byte.  A CTA stages a (4 x block) x 64 bf16 tile in shared memory;
+// `block` consecutive threads own one square tile, one row segment each: the
+// tile amax is a shuffle reduction over them, and the row segment is quantized
+// like a 1-D block (same Philox indices).  The codes are parked in shared
+// memory one per byte; then one thread per tile row writes W's 32 code bytes
+// of that row and one thread per tile column packs and writes W^T's.
+struct Q2Params {
+  const uint16_t* x;
+  uint32_t R, C;
+  int64_t ld;
+  unsigned long long seed;
+  const float* ts;
+  float* ts_copy_out;
+  uint8_t* codes;        // [R, C/2]
+  uint8_t* scales;       // [R, C/bs] or tensor-core layout (R rows, C/bs groups)
+  uint8_t* codes_t;      // [C, R/2] or null
+  uint8_t* scales_t;     // [C, R/bs] or tensor-core layout (C rows, R/bs groups)
+  uint32_t g4, g4_t;     // padded groups / 4 of the two scale tensors (tensor-core layout)
+};
+
+template <int FMT, int RND, bool SFMMA>
+__global__ void __launch_bounds__(256) quantize_2d_kernel(Q2Params p) {
+  pdl_trigger();
+  constexpr int BS = FMT == FMT_MX ? 32 : 16;
+  constexpr int TR = 4 * BS, TC = 64;                     // CTA tile: (4 x block) rows x 64 columns
+  constexpr int SPR = TC / BS;                            // square tiles across the CTA tile
+  __shared__ __align__(16) uint16_t tile[TR][TC + 8];     // 144-byte rows: 16-byte loads of 16 rows hit 2-way
+  __shared__ __align__(16) uint8_t code_sm[TR][TC + 4];    // 68-byte rows
+  __shared__ uint8_t tile_byte[4][SPR];
+  __shared__ float2 tab[128];
+  const int tid = threadIdx.x;
+  const int sq = tid / BS, rr = tid % BS;                 // square tile of the thread, its row in it
+  const int sq_r = sq / SPR, sq_c = sq % SPR;
+  pdl_wait();
+  float s_t = 1.0f, y_st = 1.0f;
+  bool st_ok = true;
+  if (FMT == FMT_NV) {
+    s_t = *p.ts;
+    y_st = __frcp_rn(s_t);
+    st_ok = recip_usable(s_t);
+    nv_fill_scale_table(tab, s_t);                        // visible after the tile loop's first barrier
+    if (p.ts_copy_out != nullptr && blockIdx.x == 0 && tid == 0) *p.ts_copy_out = s_t;
+  }
+  const uint32_t tiles_r = (p.R + TR - 1) / TR, tiles_c = (p.C + TC - 1) / TC;
+  for (uint32_t t = blockIdx.x; t < tiles_r * tiles_c; t += gridDim.x) {
+    const uint32_t r0 = (t / tiles_c) * TR, c0 = (t % tiles_c) * TC;
+    __syncthreads();                                      // the previous tile's shared data is consumed
+    for (int i = tid; i < TR * (TC / 8); i += 256) {
+      const int row = i / (TC / 8), ch = i % (TC / 8);
+      const uint32_t gr = r0 + row, gc = c0 + ch * 8;
+      uint4 v = make_uint4(0u, 0u, 0u, 0u);
+      if (gr < p.R && gc < p.C) v = ld_stream(p.x + (int64_t)gr * p.ld + gc);
+      *reinterpret_cast<uint4*>(&tile[row][ch * 8]) = v;
+    }
+    __syncthreads();
+    const uint32_t row = r0 + sq_r * BS + rr, col = c0 + sq_c * BS;   // this thread's row segment
+    float x[BS];
+#pragma unroll
+    for (int i = 0; i < BS; ++i) x[i] = __uint_as_float((uint32_t)tile[sq_r * BS + rr][sq_c * BS + i] << 16);
+    float am = 0.0f;
+#pragma unroll
+    for (int i = 0; i < BS; ++i) am = fmaxf(am, fabsf(x[i]));
+#pragma unroll
+    for (int off = BS / 2; off > 0; off >>= 1) am = fmaxf(am, __shfl_xor_sync(0xFFFFFFFFu, am, off));
+    uint32_t byte;
+    bool zero;
+    if (FMT == FMT_MX) {
+      byte = mx_scale_byte(am);
+      const float inv = mx_inv_scale(byte);
+#pragma unroll
+      for (int i = 0; i < BS; ++i) x[i] = __fmul_rn(x[i], inv);
+      zero = (am == 0.0f);
+    } else {
+      byte = e4m3_rn_sat(nv_scale_arg(am, s_t, y_st, st_ok));
+      zero = (byte == 0u);
+      const float2 sy = tab[byte];
+      if (nv_fast_division<RND, BS>(x, am, sy.x, sy.y)) {
+#pragma unroll
+        for (int i = 0; i < BS; ++i) x[i] = div_by_recip(x[i], sy.x, sy.y);
+      } else {
+#pragma unroll
+        for (int i = 0; i < BS; ++i) x[i] = __fdiv_rn(x[i], sy.x);
+      }
+    }
+    uint32_t w[BS / 8];
+    if (RND == RND_RTN) {
+#pragma unroll
+      for (int k = 0; k < BS / 8; ++k)
+        w[k] = e2m1x4_rn(x[8 * k], x[8 * k + 1], x[8 * k + 2], x[8 * k + 3], x[8 * k + 4], x[8 * k + 5], x[8 * k + 6],
+                         x[8 * k + 7]);
+    } else {
+      const unsigned long long j0 = ((unsigned long long)row * p.C + col) >> 2;   // col % 4 == 0
+#pragma unroll
+      for (int k = 0; k < BS / 8; ++k) {
+        const unsigned long long j = j0 + 2u * k;
+        const u32x4 a = philox4x32_10((uint32_t)j, (uint32_t)(j >> 32), (uint32_t)p.seed, (uint32_t)(p.seed >> 32));
+        const u32x4 b = philox4x32_10((uint32_t)(j + 1), (uint32_t)((j + 1) >> 32), (uint32_t)p.seed,
+                                      (uint32_t)(p.seed >> 32));
+        const float* xe = x + 8 * k;
+        const uint32_t n[8] = {e2m1_sr(xe[0], a.x), e2m1_sr(xe[1], a.y), e2m1_sr(xe[2], a.z), e2m1_sr(xe[3], a.w),
+                               e2m1_sr(xe[4], b.x), e2m1_sr(xe[5], b.y), e2m1_sr(xe[6], b.z), e2m1_sr(xe[7], b.w)};
+        w[k] = pack8_nibbles(n);
+      }
+    }
+    if (zero) {
+#pragma unroll
+      for (int k = 0; k < BS / 8; ++k) w[k] = 0u;
+    }
+    // park the codes one per byte (row rr of the square tile) and the tile's scale byte
+#pragma unroll
+    for (int k = 0; k < BS / 8; ++k)
+#pragma unroll
+      for (int i = 0; i < 8; ++i) code_sm[sq_r * BS + rr][sq_c * BS + 8 * k + i] = (uint8_t)((w[k] >> (4 * i)) & 0xFu);
+    if (rr == 0) tile_byte[sq_r][sq_c] = (uint8_t)byte;
+    __syncthreads();
+    // write-out: one thread per tile row (W, 32 code bytes per row) and, when asked, one per tile
+    // column (W^T, TR/2 code bytes per column): whole sectors instead of 8-byte pieces
+    const uint32_t vcols = min((uint32_t)TC, p.C > c0 ? p.C - c0 : 0u);      // multiple of the block
+    const uint32_t vrows = min((uint32_t)TR, p.R > r0 ? p.R - r0 : 0u);
+    if (tid < TR) {
+      const uint32_t lr = (uint32_t)tid;
+      if (lr < vrows) {
+        uint8_t* dst = p.codes + (size_t)(r0 + lr) * (p.C / 2) + c0 / 2;
+        for (uint32_t c = 0; c < vcols; c += 16) {                              // 8 bytes per 16 codes
+          uint32_t lo = 0u, hi = 0u;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            lo |= (uint32_t)code_sm[lr][c + i] << (4 * i);
+            hi |= (uint32_t)code_sm[lr][c + 8 + i] << (4 * i);
+          }
+          *reinterpret_cast<uint2*>(dst + c / 2) = make_uint2(lo, hi);
+        }
+        for (uint32_t c = 0; c < vcols; c += BS) {
+          const uint8_t b = tile_byte[lr / BS][c / BS];
+          const uint32_t g = (c0 + c) / BS;
+          if (SFMMA) p.scales[sf_mma_offset(r0 + lr, g, p.g4)] = b;
+          else p.scales[(size_t)(r0 + lr) * (p.C / BS) + g] = b;
+        }
+      }
+    } else if (p.codes_t != nullptr && tid < TR + TC) {
+      const uint32_t lc = (uint32_t)(tid - TR);
+      if (lc < vcols) {
+        uint8_t* dst = p.codes_t + (size_t)(c0 + lc) * (p.R / 2) + r0 / 2;
+        for (uint32_t r = 0; r < vrows; r += 16) {
+          uint32_t lo = 0u, hi = 0u;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            lo |= (uint32_t)code_sm[r + i][lc] << (4 * i);
+            hi |= (uint32_t)code_sm[r + 8 + i][lc] << (4 * i);
+          }
+          *reinterpret_cast<uint2*>(dst + r / 2) = make_uint2(lo, hi);
+        }
+        for (uint32_t r = 0; r < vrows; r += BS) {
+          const uint8_t b = tile_byte[r / BS][lc / BS];
+          const uint32_t g = (r0 + r) / BS;
+          if (SFMMA) p.scales_t[sf_mma_offset(c0 + lc, g, p.g4_t)] = b;
+          else p.scales_t[(size_t)(c0 + lc) * (p.R / BS) + g] = b;
+        }
+      }
+    }
+  }
+}
+
 // ============================================================ dequantize ===
 struct DeqParams {
   const uint32_t* codes;  // 32-bit words of 8 nibbles
@@ -1205,6 +1375,46 @@ cudaError_t launch_quantize(const QuantizeParams& p, int num_sms, cudaStream_t s
                             : cols_dispatch<FMT_MX, RND_SR>(qp, sfmma, num_sms, st);
   return p.rnd == RND_RTN ? cols_dispatch<FMT_NV, RND_RTN>(qp, sfmma, num_sms, st)
                           : cols_dispatch<FMT_NV, RND_SR>(qp, sfmma, num_sms, st);
+}
+
+template <int FMT, int RND, bool SFMMA>
+static cudaError_t q2d_launch(const Q2Params& qp, int num_sms, cudaStream_t st) {
+  auto kernel = quantize_2d_kernel<FMT, RND, SFMMA>;
+  static int occ = resident_ctas(kernel, 256);
+  constexpr uint32_t TR = FMT == FMT_MX ? 128 : 64;
+  const uint64_t tiles = (uint64_t)((qp.R + TR - 1) / TR) * ((qp.C + 63) / 64);
+  uint64_t grid = (uint64_t)num_sms * (uint64_t)occ;
+  if (tiles < grid) grid = tiles > 0 ? tiles : 1;
+  return launch_kernel(kernel, dim3((unsigned)grid), dim3(256), 0, st, false, 1u, qp);
+}
+
+template <int FMT>
+static cudaError_t q2d_dispatch(const Q2Params& qp, int rnd, bool sfmma, int num_sms, cudaStream_t st) {
+  if (rnd == RND_RTN)
+    return sfmma ? q2d_launch<FMT, RND_RTN, true>(qp, num_sms, st) : q2d_launch<FMT, RND_RTN, false>(qp, num_sms, st);
+  return sfmma ? q2d_launch<FMT, RND_SR, true>(qp, num_sms, st) : q2d_launch<FMT, RND_SR, false>(qp, num_sms, st);
+}
+
+cudaError_t launch_quantize_2d(const QuantizeParams& p, uint8_t* codes_t, uint8_t* scales_t, int num_sms,
+                               cudaStream_t st) {
+  const int bs = p.fmt == FMT_MX ? 32 : 16;
+  Q2Params qp;
+  qp.x = static_cast<const uint16_t*>(p.x);
+  qp.R = (uint32_t)p.rows;
+  qp.C = (uint32_t)p.cols;
+  qp.ld = p.ld;
+  qp.seed = p.seed;
+  qp.ts = p.ts;
+  qp.ts_copy_out = p.ts_copy_out;
+  qp.codes = p.codes;
+  qp.scales = p.scales;
+  qp.codes_t = codes_t;
+  qp.scales_t = scales_t;
+  qp.g4 = (uint32_t)((p.cols / bs + 3) / 4);
+  qp.g4_t = (uint32_t)((p.rows / bs + 3) / 4);
+  const bool sfmma = p.sf_mma != 0;
+  return p.fmt == FMT_MX ? q2d_dispatch<FMT_MX>(qp, p.rnd, sfmma, num_sms, st)
+                         : q2d_dispatch<FMT_NV>(qp, p.rnd, sfmma, num_sms, st);
 }
 
 template <int FMT, bool SFMMA, bool BF16>

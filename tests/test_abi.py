@@ -91,3 +91,8 @@ def test_other_entry_points_reject_before_launch(lib):
     assert lib.fp4_amax(None, 4, 64, 64, FAKE, None) == -1
     assert lib.fp4_amax_noalloc(FAKE, 8192, 8200, 8200, FAKE, None) == -2                # beyond its scratch
     assert lib.fp4_nv_tensor_scale(None, FAKE, None) == -1
+    # fp4_quantize_2d: rows not a multiple of the tile, half of the transposed pair, NV without s_t out
+    assert lib.fp4_quantize_2d(FAKE, 40, 64, 64, 0, 32, 0, 0, None, None, FAKE, FAKE, None, None, 0, None) == -2
+    assert lib.fp4_quantize_2d(FAKE, 64, 64, 64, 0, 32, 0, 0, None, None, FAKE, FAKE, FAKE, None, 0, None) == -1
+    assert lib.fp4_quantize_2d(FAKE, 64, 64, 64, 1, 16, 0, 0, None, None, FAKE, FAKE, None, None, 0, None) == -1
+    assert lib.fp4_quantize_2d(FAKE, 64, 64, 64, 0, 32, 0, 0, None, None, FAKE + 4, FAKE, None, None, 0, None) == -3

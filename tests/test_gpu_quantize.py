@@ -273,3 +273,57 @@ def test_nv_tiny_elements(rnd, scale):
     np.testing.assert_array_equal(host_u8(q.scales), ref["scales"])
     np.testing.assert_array_equal(host_u8(q.codes), ref["codes"])
     F.fp4_check_device_errors()
+
+
+@pytest.mark.parametrize("sf", ["rowmajor", "mma"])
+@pytest.mark.parametrize("rnd", ["rtn", "sr"])
+@pytest.mark.parametrize("fmt", ["mxfp4", "nvfp4"])
+@pytest.mark.parametrize("shape", [(64, 64), (96, 160), (256, 4096), (4096, 512)])
+def test_quantize_2d(shape, fmt, rnd, sf):
+    """Square-tile quantization: W's codes/scales along its rows and W^T's along its rows,
+    bit-exact against the oracle (tensor-core layout compared after the oracle's permutation)."""
+    rows, cols = shape
+    bs = 32 if fmt == "mxfp4" else 16
+    if rows % bs or cols % bs:
+        pytest.skip("shape not a multiple of the tile")
+    xb = mixed_input(rows, cols, rows * 3 + cols, fmt)
+    q, qt = F.fp4_quantize_2d(dev_bf16(xb), fmt=fmt, rnd=rnd, seed=77, sf_layout=sf)
+    ref = O.quantize_2d(xb, fmt=fmt, rnd=rnd, seed=77)
+    if fmt == "nvfp4":
+        assert host_f32(q.tensor_scale)[0] == ref["tensor_scale"]
+    np.testing.assert_array_equal(host_u8(q.codes), ref["codes"])
+    np.testing.assert_array_equal(host_u8(qt.codes), ref["codes_t"])
+    if sf == "rowmajor":
+        np.testing.assert_array_equal(host_u8(q.scales), ref["scales"])
+        np.testing.assert_array_equal(host_u8(qt.scales), ref["scales_t"])
+    else:
+        np.testing.assert_array_equal(host_u8(q.scales), O.sf_to_mma(ref["scales"]))
+        np.testing.assert_array_equal(host_u8(qt.scales), O.sf_to_mma(ref["scales_t"]))
+    F.fp4_check_device_errors()
+
+
+def test_quantize_2d_feeds_forward_and_dgrad_gemms():
+    """The same 2-D-quantized W serves the forward GEMM (W along K) and the dgrad GEMM (W^T along
+    N) without requantization: both against the oracle's fp64 products of the dequantized operands."""
+    from workloads import normal_bf16
+    M, K, N = 256, 512, 384
+    xb = normal_bf16((M, K), 1.0, 5, 0)
+    wb = normal_bf16((N, K), 0.02, 5, 1)
+    dyb = normal_bf16((M, N), 1e-3, 5, 2)
+    qw, qwt = F.fp4_quantize_2d(dev_bf16(wb), fmt="nvfp4", sf_layout="mma")
+    qx = F.fp4_quantize(dev_bf16(xb), fmt="nvfp4", sf_layout="mma")
+    qdy = F.fp4_quantize(dev_bf16(dyb), fmt="nvfp4", rnd="sr", seed=3, sf_layout="mma")
+    y = F.fp4_gemm(qx.codes, qx.scales, qw.codes, qw.scales, fmt="nvfp4", a_tensor_scale=qx.tensor_scale,
+                   b_tensor_scale=qw.tensor_scale, out_dtype="f32")
+    dx = F.fp4_gemm(qdy.codes, qdy.scales, qwt.codes, qwt.scales, fmt="nvfp4", a_tensor_scale=qdy.tensor_scale,
+                    b_tensor_scale=qwt.tensor_scale, out_dtype="f32")
+    ow = O.quantize_2d(wb, fmt="nvfp4")
+    ox = O.quantize(xb, fmt="nvfp4")
+    ody = O.quantize(dyb, fmt="nvfp4", rnd="sr", seed=3)
+    yr, bd = O.gemm_ref(ox, {"codes": ow["codes"], "scales": ow["scales"], "tensor_scale": ow["tensor_scale"]},
+                        "nvfp4")
+    assert np.all(np.abs(host_f32(y) - yr) <= 1e-5 * bd)
+    dr, bd2 = O.gemm_ref(ody, {"codes": ow["codes_t"], "scales": ow["scales_t"], "tensor_scale": ow["tensor_scale"]},
+                         "nvfp4")
+    assert np.all(np.abs(host_f32(dx) - dr) <= 1e-5 * bd2)
+    F.fp4_check_device_errors()
