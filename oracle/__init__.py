@@ -29,7 +29,8 @@ the plainest reading (OCP MX v1.0 E2M1/E8M0/E4M3 conventions, Philox4x32-10 of
 Salmon et al. SC'11, Sylvester Hadamard) and each module says which.
 
 Modules: `formats` (E2M1/E4M3/E8M0), `philox`, `quantize` (MX/NV, RTN/SR,
-axis 0/1, packing, dequantize), `quantize2d` (square-tile 2-D blocks),
+axis 0/1, packing, dequantize; fmt "nvfp4_4o6" via `four_over_six`),
+`quantize2d` (square-tile 2-D blocks),
 `hadamard`, `layout` (tensor-core scale-factor layout), `gemm` (fp64 reference
 and error bound).
 """

@@ -104,7 +104,10 @@ def quantize_values(x32, fmt: str = "mxfp4", block: int | None = None, axis: int
     The Philox index of element (r, c) is idx_base + r * idx_cols + c (idx_cols
     defaults to cols), so a row slice of a larger tensor can be quantized with
     its global indices.  For NVFP4 without `tensor_scale`, s_t comes from x32.
+    fmt "nvfp4_4o6" is NVFP4 with four-over-six block scales (`four_over_six`).
     """
+    four_six = fmt == "nvfp4_4o6"
+    fmt = "nvfp4" if four_six else fmt
     bs = block or FMT_BLOCK[fmt]
     if (fmt, bs) not in (("mxfp4", 32), ("nvfp4", 16)):
         raise ValueError("supported: (mxfp4, 32), (nvfp4, 16)")
@@ -119,8 +122,12 @@ def quantize_values(x32, fmt: str = "mxfp4", block: int | None = None, axis: int
     s_t = None
     if fmt == "nvfp4":
         s_t = np.float32(tensor_scale) if tensor_scale is not None else nv_tensor_scale(x)
-    codes, scales = _quantize_rows(np.ascontiguousarray(xw), np.ascontiguousarray(idxw),
-                                   fmt, bs, rnd, seed, s_t)
+    if four_six:
+        from .four_over_six import quantize_rows_46
+        codes, scales = quantize_rows_46(np.ascontiguousarray(xw), np.ascontiguousarray(idxw), rnd, seed, s_t)
+    else:
+        codes, scales = _quantize_rows(np.ascontiguousarray(xw), np.ascontiguousarray(idxw),
+                                       fmt, bs, rnd, seed, s_t)
     return {"codes": pack_nibbles(codes), "scales": scales, "tensor_scale": s_t}
 
 
