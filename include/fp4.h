@@ -79,6 +79,13 @@ enum {
 };
 
 enum { FP4_MXFP4 = 0, FP4_NVFP4 = 1 };              /* fp4_format    */
+/* Quantizer-only format: NVFP4 codes and E4M3 scales whose block scale is, per
+ * block, the one of max->6 (standard) and max->4 with the lower round-to-nearest
+ * squared error ("Four Over Six: More Accurate NVFP4 Quantization with Adaptive
+ * Block Scaling", Abstract; error in fp64, terms added in element order, ties
+ * keep max->6).  Accepted by fp4_quantize and fp4_hadamard_quantize with block
+ * 16; their outputs are plain NVFP4 (dequantize and GEMM with FP4_NVFP4). */
+enum { FP4_NVFP4_4O6 = 2 };
 enum { FP4_RTN = 0, FP4_SR = 1 };                   /* fp4_round     */
 enum { FP4_SF_ROWMAJOR = 0, FP4_SF_MMA = 1 };       /* fp4_sf_layout */
 enum { FP4_OUT_F32 = 0, FP4_OUT_BF16 = 1 };         /* fp4_dtype     */
@@ -91,7 +98,7 @@ enum { FP4_OUT_F32 = 0, FP4_OUT_BF16 = 1 };         /* fp4_dtype     */
  *
  *   x          bf16 [rows, cols], row stride `ld` elements (ld >= cols).
  *              16-byte aligned; cols and ld multiples of 8.
- *   fmt,block  (FP4_MXFP4, 32) or (FP4_NVFP4, 16).
+ *   fmt,block  (FP4_MXFP4, 32), (FP4_NVFP4, 16) or (FP4_NVFP4_4O6, 16).
  *   axis       1: blocks along cols (cols % block == 0);
  *              0: blocks along rows (rows % block == 0), output transposed.
  *   rnd, seed  FP4_RTN, or FP4_SR with the 64-bit Philox key `seed`.

@@ -14,17 +14,17 @@ import torch
 
 from . import _lib
 
-MXFP4, NVFP4 = 0, 1
+MXFP4, NVFP4, NVFP4_4O6 = 0, 1, 2
 RTN, SR = 0, 1
 SF_ROWMAJOR, SF_MMA = 0, 1
 OUT_F32, OUT_BF16 = 0, 1
 
-_FMT = {"mxfp4": MXFP4, "nvfp4": NVFP4, MXFP4: MXFP4, NVFP4: NVFP4}
+_FMT = {"mxfp4": MXFP4, "nvfp4": NVFP4, "nvfp4_4o6": NVFP4_4O6, MXFP4: MXFP4, NVFP4: NVFP4, NVFP4_4O6: NVFP4_4O6}
 _RND = {"rtn": RTN, "sr": SR, RTN: RTN, SR: SR}
 _SF = {"rowmajor": SF_ROWMAJOR, "mma": SF_MMA, SF_ROWMAJOR: SF_ROWMAJOR, SF_MMA: SF_MMA}
 _OUT = {"f32": OUT_F32, "bf16": OUT_BF16, torch.float32: OUT_F32, torch.bfloat16: OUT_BF16,
         OUT_F32: OUT_F32, OUT_BF16: OUT_BF16}
-BLOCK = {MXFP4: 32, NVFP4: 16}
+BLOCK = {MXFP4: 32, NVFP4: 16, NVFP4_4O6: 16}
 
 
 class Fp4Error(RuntimeError):
@@ -93,7 +93,7 @@ def _alloc_quant_outputs(x, fmt, axis, sf, codes, scales, ts_out):
             raise ValueError("shape not quantizable with this block size along this axis")
         shape = (orows, qlen // BLOCK[fmt]) if sf == SF_ROWMAJOR else (nbytes,)
         scales = torch.empty(shape, dtype=torch.uint8, device=x.device)
-    if fmt == NVFP4 and ts_out is None:
+    if fmt in (NVFP4, NVFP4_4O6) and ts_out is None:
         ts_out = torch.empty((1,), dtype=torch.float32, device=x.device)
     return codes, scales, ts_out
 
@@ -109,7 +109,7 @@ def fp4_quantize(x: torch.Tensor, fmt="mxfp4", axis: int = 1, rnd="rtn", seed: i
         x.data_ptr(), x.shape[0], x.shape[1], x.stride(0), f, BLOCK[f], axis, r, seed & (2 ** 64 - 1),
         _ptr(tensor_scale_in), _ptr(ts_out), codes.data_ptr(), scales.data_ptr(), sf, _stream(stream))
     _check(st, "fp4_quantize")
-    return Fp4Quantized(codes, scales, ts_out if f == NVFP4 else None)
+    return Fp4Quantized(codes, scales, ts_out if f in (NVFP4, NVFP4_4O6) else None)
 
 
 def fp4_hadamard_quantize(x: torch.Tensor, had_block: int, fmt="mxfp4", axis: int = 1, rnd="rtn",
@@ -124,7 +124,7 @@ def fp4_hadamard_quantize(x: torch.Tensor, had_block: int, fmt="mxfp4", axis: in
         _ptr(tensor_scale_in), _ptr(ts_out), codes.data_ptr(), scales.data_ptr(), sf, had_block,
         _ptr(rotated_out), _stream(stream))
     _check(st, "fp4_hadamard_quantize")
-    return Fp4Quantized(codes, scales, ts_out if f == NVFP4 else None)
+    return Fp4Quantized(codes, scales, ts_out if f in (NVFP4, NVFP4_4O6) else None)
 
 
 def fp4_quantize_2d(x: torch.Tensor, fmt="nvfp4", rnd="rtn", seed: int = 0,

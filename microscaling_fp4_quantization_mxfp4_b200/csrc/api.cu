@@ -109,6 +109,12 @@ fp4_status check_input(const void* x, int64_t rows, int64_t cols, int64_t ld) {
 fp4_status quantize_impl(const void* x, int64_t rows, int64_t cols, int64_t ld, int fmt, int block, int axis,
                          int rnd, uint64_t seed, const float* ts_in, float* ts_out, uint8_t* codes, uint8_t* scales,
                          int sf_layout, int had, float* rotated, cudaStream_t st) {
+  int four_six = 0;
+  if (fmt == FP4_NVFP4_4O6) {        // NVFP4 codes and scales with four-over-six block scales
+    if (block != 16) return FP4_ERR_UNSUPPORTED;
+    fmt = FP4_NVFP4;
+    four_six = 1;
+  }
   fp4_status s = check_format(fmt, block);
   if (s != FP4_OK) return s;
   if ((s = check_input(x, rows, cols, ld)) != FP4_OK) return s;
@@ -123,7 +129,7 @@ fp4_status quantize_impl(const void* x, int64_t rows, int64_t cols, int64_t ld, 
   if (!aligned16(codes)) return FP4_ERR_ALIGN;
   if (had != 0) {
     if (had != 16 && had != 32 && had != 64 && had != 128) return FP4_ERR_ARG;
-    if (axis != 1) return FP4_ERR_UNSUPPORTED;
+    if (axis != 1 || four_six) return FP4_ERR_UNSUPPORTED;
     if (cols % had != 0) return FP4_ERR_SHAPE;
     if (rotated != nullptr && !aligned16(rotated)) return FP4_ERR_ALIGN;
   }
@@ -153,6 +159,7 @@ fp4_status quantize_impl(const void* x, int64_t rows, int64_t cols, int64_t ld, 
   p.had = had;
   p.rotated = rotated;
   p.error = d->scratch.error;
+  p.four_six = four_six;
   size_t fused_smem = 0;
   uint32_t fused_tiles = 0;
   if (fmt == FP4_NVFP4 && ts_in == nullptr && axis == 1 && ld == cols && !single_pass_disabled() &&

@@ -188,6 +188,14 @@ __device__ __forceinline__ float nv_scale_arg(float am, float s_t, float y_st, b
   return ok ? t : __fdiv_rn(__fdiv_rn(am, 6.0f), s_t);
 }
 
+// Four-over-six candidate t4 = RN(RN(amax_b / 4) / s_t) (RN(amax_b / 4) = amax_b * 0.25, rounded).
+__device__ __forceinline__ float nv_scale_arg4(float am, float s_t, float y_st, bool st_ok) {
+  const float d4 = __fmul_rn(am, 0.25f);
+  const float t = div_by_recip(d4, s_t, y_st);
+  const bool ok = st_ok && (am == 0.0f || (d4 >= 0x1p-100f && __fmul_rn(d4, y_st) < 0x1p64f));
+  return ok ? t : __fdiv_rn(d4, s_t);
+}
+
 // Per-CTA table of the element divisor S = RN(e4m3(b) * s_t) and RN(1/S) for
 // every E4M3 byte b (b = 0 is the zero scale; its entry is unused).  A scale
 // whose reciprocal is out of the fast path's range gets y = 0, which makes
@@ -204,6 +212,15 @@ __device__ __forceinline__ float e2m1_value(uint32_t c) {
   const uint32_t e = (c >> 1) & 3u, m = c & 1u;
   float mag = (e == 0u) ? (m ? 0.5f : 0.0f) : __uint_as_float(((e + 126u) << 23) | (m << 22));
   return (c & 8u) ? -mag : mag;
+}
+
+// One pair of scaled values -> their RTN codes, `a` in bits 0-3, `b` in bits 4-7.
+__device__ __forceinline__ uint32_t e2m1x2_rn(float a, float b) {
+  uint32_t out;
+  asm("{\n\t.reg .b8 q;\n\tcvt.rn.satfinite.e2m1x2.f32 q, %2, %1;\n\tcvt.u32.u8 %0, q;\n\t}"
+      : "=r"(out)
+      : "f"(a), "f"(b));
+  return out;
 }
 
 // -------------------------------------------------- scale-factor offsets ----

@@ -53,7 +53,8 @@ cudaError_t launch_kernel(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_
   return cudaLaunchKernelEx(&cfg, kernel, args...);
 }
 
-enum { FMT_MX = 0, FMT_NV = 1 };
+// FMT_NV46: NVFP4 with four-over-six block scales (quantizer kernels only; its outputs are NVFP4)
+enum { FMT_MX = 0, FMT_NV = 1, FMT_NV46 = 2 };
 enum { RND_RTN = 0, RND_SR = 1 };
 
 // Per-device scratch owned by the library (allocated once per device).
@@ -86,6 +87,7 @@ struct QuantizeParams {
   int had;                // 0 or Hadamard block size
   float* rotated;         // optional fp32 dump of the rotated input
   unsigned* error;        // device error word
+  int four_six = 0;       // NVFP4: four-over-six block scales
 };
 
 // amax pass: mode 0 writes max|x| (after rotation when had > 0) to `out`,

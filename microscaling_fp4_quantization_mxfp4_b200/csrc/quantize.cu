@@ -188,6 +188,46 @@ __device__ __forceinline__ bool nv_fast_division(const float (&x)[E], float am, 
   return kmin >= kTinyKeyMin;
 }
 
+// Four-over-six (NVFP4): squared error of a block's round-to-nearest result under scale byte sb,
+// fp64 terms (x - dequantized code)^2 added in element order; a zero scale dequantizes to 0.
+template <int E>
+__device__ __forceinline__ double nv_rtn_sq_error(const float (&x)[E], float am, uint32_t sb, float s_t,
+                                               const float2* tab) {
+  double acc = 0.0;
+  if (sb == 0u) {
+#pragma unroll
+    for (int i = 0; i < E; ++i) acc = __dadd_rn(acc, __dmul_rn((double)x[i], (double)x[i]));
+    return acc;
+  }
+  const float2 sy = tab[sb];
+  const float sbv = e4m3_value(sb);
+  const bool fast = nv_fast_division<RND_RTN, E>(x, am, sy.x, sy.y);
+#pragma unroll
+  for (int i = 0; i < E; i += 2) {
+    const float v0 = fast ? div_by_recip(x[i], sy.x, sy.y) : __fdiv_rn(x[i], sy.x);
+    const float v1 = fast ? div_by_recip(x[i + 1], sy.x, sy.y) : __fdiv_rn(x[i + 1], sy.x);
+    const uint32_t c = e2m1x2_rn(v0, v1);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const float d = __fmul_rn(__fmul_rn(e2m1_value((c >> (4 * h)) & 0xFu), sbv), s_t);
+      const double e = __dsub_rn((double)x[i + h], (double)d);
+      acc = __dadd_rn(acc, __dmul_rn(e, e));
+    }
+  }
+  return acc;
+}
+
+// The scale byte among max->6 (byte6, the standard NVFP4 byte) and max->4 with the lower
+// round-to-nearest squared error ("Four Over Six", Abstract); ties keep byte6, and a zero or
+// identical max->4 byte is never taken.
+template <int E>
+__device__ __forceinline__ uint32_t nv_four_over_six(const float (&x)[E], float am, uint32_t byte6, float s_t,
+                                                     float y_st, bool st_ok, const float2* tab) {
+  const uint32_t byte4 = e4m3_rn_sat(nv_scale_arg4(am, s_t, y_st, st_ok));
+  if (byte4 == byte6 || byte4 == 0u) return byte6;
+  return nv_rtn_sq_error<E>(x, am, byte4, s_t, tab) < nv_rtn_sq_error<E>(x, am, byte6, s_t, tab) ? byte4 : byte6;
+}
+
 template <int FMT, int RND, int HAD, bool SFMMA>
 __device__ __forceinline__ void quantize_block(const QRowParams& p, const uint4 (&v)[BlockShape<FMT>::V], uint32_t blk,
                                                bool valid, int lane, const NvConsts& nv) {
@@ -221,6 +261,7 @@ __device__ __forceinline__ void quantize_block(const QRowParams& p, const uint4 
     zero = (am == 0.0f);
   } else {
     byte = e4m3_rn_sat(nv_scale_arg(am, nv.s_t, nv.y_st, nv.st_ok));
+    if (FMT == FMT_NV46) byte = nv_four_over_six<E>(x, am, byte, nv.s_t, nv.y_st, nv.st_ok, nv.tab);
     zero = (byte == 0u);
     const float2 sy = nv.tab[byte];
     if (nv_fast_division<RND, E>(x, am, sy.x, sy.y)) {
@@ -274,7 +315,7 @@ __global__ void __launch_bounds__(256) quantize_rows_kernel(QRowParams p) {
   const int lane = threadIdx.x & 31;
   pdl_wait();
   NvConsts nv{1.0f, 1.0f, true, tab};
-  if (FMT == FMT_NV) {
+  if (FMT != FMT_MX) {
     nv.s_t = *p.ts;
     nv.y_st = __frcp_rn(nv.s_t);
     nv.st_ok = recip_usable(nv.s_t);
@@ -314,12 +355,13 @@ constexpr int kStreamSmem = kStreamStages * kStreamChunks * 16 + 2 * kStreamStag
 // their 16-element blocks fit); 16 for MXFP4 round-to-nearest, with or
 // without rotation (31 warps ran 10-20 % slower); 15 for MXFP4 stochastic
 // rounding, whose 32-element blocks with their eight Philox blocks want about
-// 124 registers.  Units of a stage are dealt to the warps round-robin,
-// starting one place further on each stage, so that counts that do not divide
-// evenly still balance over a run.
+// 124 registers; 15 for four-over-six NVFP4, whose second candidate scale and
+// fp64 error sums do not fit in 64 registers.  Units of a stage are dealt to
+// the warps round-robin, starting one place further on each stage, so that
+// counts that do not divide evenly still balance over a run.
 template <int FMT, int RND>
 struct StreamWarps {
-  static constexpr int kWarps = FMT == FMT_NV ? 31 : (RND == RND_SR ? 15 : 16);   // producer + consumers <= 1024
+  static constexpr int kWarps = FMT == FMT_NV ? 31 : (FMT == FMT_NV46 || RND == RND_SR ? 15 : 16);
   static constexpr int kThreads = 32 * (kWarps + 1);
 };
 constexpr int kAmaxWarps = 31;
@@ -400,7 +442,7 @@ __global__ void __launch_bounds__(StreamWarps<FMT, RND>::kThreads, 1) quantize_s
   stream_ring_init(r, kStreamWarps);
   pdl_wait();
   NvConsts nv{1.0f, 1.0f, true, tab};
-  if (FMT == FMT_NV) {
+  if (FMT != FMT_MX) {
     nv.s_t = *p.ts;
     nv.y_st = __frcp_rn(nv.s_t);
     nv.st_ok = recip_usable(nv.s_t);
@@ -536,7 +578,7 @@ constexpr int kFusedThreads = 32 * (kFusedWarps + 1);
 constexpr int kFusedMaxSmem = 227 * 1024 - 2048;          // staged slice; room left for the static data
 constexpr int kFusedPieces = 8;                           // bulk copies (and mbarriers) per slice
 
-template <int RND, int HAD, bool SFMMA>
+template <int FMT, int RND, int HAD, bool SFMMA>
 __global__ void __launch_bounds__(kFusedThreads, 1) nv_quantize_fused_kernel(FusedParams fp) {
   extern __shared__ __align__(1024) uint4 slice[];
   __shared__ float2 tab[128];
@@ -651,7 +693,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) nv_quantize_fused_kernel(Fus
     uint4 v[2];
     v[0] = valid ? slice[lb * 2u] : make_uint4(0u, 0u, 0u, 0u);
     v[1] = valid ? slice[lb * 2u + 1u] : make_uint4(0u, 0u, 0u, 0u);
-    quantize_block<FMT_NV, RND, HAD, SFMMA>(p, v, c_begin / 2u + lb, valid, lane, nv);
+    quantize_block<FMT, RND, HAD, SFMMA>(p, v, c_begin / 2u + lb, valid, lane, nv);
   }
 }
 
@@ -707,7 +749,7 @@ __global__ void __launch_bounds__(256) quantize_cols_kernel(QColParams p) {
   const uint32_t tiles_r = (p.R + 127u) / 128u, tiles_c = (p.C + 63u) / 64u;
   float s_t = 1.0f, y_st = 1.0f;
   bool st_ok = true;
-  if (FMT == FMT_NV) {
+  if (FMT != FMT_MX) {
     s_t = *p.ts;
     y_st = __frcp_rn(s_t);
     st_ok = recip_usable(s_t);
@@ -754,14 +796,15 @@ __global__ void __launch_bounds__(256) quantize_cols_kernel(QColParams p) {
         inv = mx_inv_scale(byte);
         zero = (am == 0.0f);
       } else {
+        float xb[BS];
+#pragma unroll
+        for (int i = 0; i < BS; ++i) xb[i] = xv[b * BS + i];
         byte = e4m3_rn_sat(nv_scale_arg(am, s_t, y_st, st_ok));
+        if (FMT == FMT_NV46) byte = nv_four_over_six<BS>(xb, am, byte, s_t, y_st, st_ok, tab);
         zero = (byte == 0u);
         const float2 sy = tab[byte];
         S = sy.x;
         y = sy.y;
-        float xb[BS];
-#pragma unroll
-        for (int i = 0; i < BS; ++i) xb[i] = xv[b * BS + i];
         fast = nv_fast_division<RND, BS>(xb, am, S, y);
       }
 #pragma unroll
@@ -805,7 +848,7 @@ __global__ void __launch_bounds__(256) quantize_cols_kernel(QColParams p) {
       const uint32_t g = rb / BS;
       if (SFMMA) p.scales[sf_mma_offset(c, g, p.g4)] = (uint8_t)byte;
       else p.scales[(size_t)c * p.G + g] = (uint8_t)byte;
-      if (FMT == FMT_NV) {
+      if (FMT != FMT_MX) {
         *reinterpret_cast<uint2*>(p.codes + (size_t)c * (p.R / 2) + rb / 2) = make_uint2(words[2 * b], words[2 * b + 1]);
       }
     }
@@ -859,7 +902,7 @@ __global__ void __launch_bounds__(256) quantize_2d_kernel(Q2Params p) {
   pdl_wait();
   float s_t = 1.0f, y_st = 1.0f;
   bool st_ok = true;
-  if (FMT == FMT_NV) {
+  if (FMT != FMT_MX) {
     s_t = *p.ts;
     y_st = __frcp_rn(s_t);
     st_ok = recip_usable(s_t);
@@ -1246,18 +1289,19 @@ static cudaError_t rows_dispatch_had(const QRowParams& qp, int had, bool sfmma, 
   }
 }
 
-template <int RND, int HAD, bool SFMMA>
+template <int FMT, int RND, int HAD, bool SFMMA>
 static cudaError_t fused_launch(const FusedParams& fp, uint32_t grid, size_t smem, cudaStream_t st) {
-  auto kernel = nv_quantize_fused_kernel<RND, HAD, SFMMA>;
+  auto kernel = nv_quantize_fused_kernel<FMT, RND, HAD, SFMMA>;
   static const cudaError_t attr =
       cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kFusedMaxSmem);
   if (attr != cudaSuccess) return attr;
   return launch_kernel(kernel, dim3(grid), dim3(kFusedThreads), smem, st, true, 1u, fp);
 }
 
-template <int RND, int HAD>
+template <int RND, int HAD, int FMT = FMT_NV>
 static cudaError_t fused_dispatch_sf(const FusedParams& fp, bool sfmma, uint32_t grid, size_t smem, cudaStream_t st) {
-  return sfmma ? fused_launch<RND, HAD, true>(fp, grid, smem, st) : fused_launch<RND, HAD, false>(fp, grid, smem, st);
+  return sfmma ? fused_launch<FMT, RND, HAD, true>(fp, grid, smem, st)
+               : fused_launch<FMT, RND, HAD, false>(fp, grid, smem, st);
 }
 
 bool fused_nv_fits(int64_t rows, int64_t cols, int num_sms, size_t* smem_out, uint32_t* tiles_per_cta) {
@@ -1303,6 +1347,11 @@ cudaError_t launch_quantize_nv_fused(const QuantizeParams& p, float* ts_out, con
   const uint64_t ntiles = ((uint64_t)qp.nchunks + 31u) / 32u;
   const uint32_t grid = (uint32_t)((ntiles + per - 1) / per);
   const bool sfmma = p.sf_mma != 0;
+  if (p.four_six) {
+    if (p.had != 0) return cudaErrorInvalidValue;
+    return p.rnd == RND_RTN ? fused_dispatch_sf<RND_RTN, 0, FMT_NV46>(fp, sfmma, grid, smem, st)
+                            : fused_dispatch_sf<RND_SR, 0, FMT_NV46>(fp, sfmma, grid, smem, st);
+  }
 #define FP4_FUSED_HAD(H)                                                                               \
   return p.rnd == RND_RTN ? fused_dispatch_sf<RND_RTN, H>(fp, sfmma, grid, smem, st)                  \
                           : fused_dispatch_sf<RND_SR, H>(fp, sfmma, grid, smem, st)
@@ -1355,6 +1404,11 @@ cudaError_t launch_quantize(const QuantizeParams& p, int num_sms, cudaStream_t s
     if (p.fmt == FMT_MX)
       return p.rnd == RND_RTN ? rows_dispatch_had<FMT_MX, RND_RTN>(qp, p.had, sfmma, num_sms, st)
                               : rows_dispatch_had<FMT_MX, RND_SR>(qp, p.had, sfmma, num_sms, st);
+    if (p.four_six) {
+      if (p.had != 0) return cudaErrorInvalidValue;
+      return p.rnd == RND_RTN ? rows_dispatch_sf<FMT_NV46, RND_RTN, 0>(qp, sfmma, num_sms, st)
+                              : rows_dispatch_sf<FMT_NV46, RND_SR, 0>(qp, sfmma, num_sms, st);
+    }
     return p.rnd == RND_RTN ? rows_dispatch_had<FMT_NV, RND_RTN>(qp, p.had, sfmma, num_sms, st)
                             : rows_dispatch_had<FMT_NV, RND_SR>(qp, p.had, sfmma, num_sms, st);
   }
@@ -1373,6 +1427,9 @@ cudaError_t launch_quantize(const QuantizeParams& p, int num_sms, cudaStream_t s
   if (p.fmt == FMT_MX)
     return p.rnd == RND_RTN ? cols_dispatch<FMT_MX, RND_RTN>(qp, sfmma, num_sms, st)
                             : cols_dispatch<FMT_MX, RND_SR>(qp, sfmma, num_sms, st);
+  if (p.four_six)
+    return p.rnd == RND_RTN ? cols_dispatch<FMT_NV46, RND_RTN>(qp, sfmma, num_sms, st)
+                            : cols_dispatch<FMT_NV46, RND_SR>(qp, sfmma, num_sms, st);
   return p.rnd == RND_RTN ? cols_dispatch<FMT_NV, RND_RTN>(qp, sfmma, num_sms, st)
                           : cols_dispatch<FMT_NV, RND_SR>(qp, sfmma, num_sms, st);
 }

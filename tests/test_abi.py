@@ -96,3 +96,9 @@ def test_other_entry_points_reject_before_launch(lib):
     assert lib.fp4_quantize_2d(FAKE, 64, 64, 64, 0, 32, 0, 0, None, None, FAKE, FAKE, FAKE, None, 0, None) == -1
     assert lib.fp4_quantize_2d(FAKE, 64, 64, 64, 1, 16, 0, 0, None, None, FAKE, FAKE, None, None, 0, None) == -1
     assert lib.fp4_quantize_2d(FAKE, 64, 64, 64, 0, 32, 0, 0, None, None, FAKE + 4, FAKE, None, None, 0, None) == -3
+    # four-over-six NVFP4 (fmt 2): block 16 only, needs s_t out, no Hadamard, quantizer entry points only
+    assert lib.fp4_quantize(FAKE, 4, 64, 64, 2, 32, 1, 0, 0, None, None, FAKE, FAKE, 0, None) == -4
+    assert lib.fp4_quantize(FAKE, 4, 64, 64, 2, 16, 1, 0, 0, None, None, FAKE, FAKE, 0, None) == -1
+    assert lib.fp4_hadamard_quantize(FAKE, 4, 64, 64, 2, 16, 1, 0, 0, None, FAKE, FAKE, FAKE, 0, 16, None, None) == -4
+    assert lib.fp4_dequantize(FAKE, FAKE, FAKE, 4, 64, 2, 16, 0, FAKE, 0, None) == -1
+    assert lib.fp4_gemm(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 4, 64, 2, 16, FAKE, 4, 0, None) == -1

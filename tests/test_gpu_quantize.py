@@ -327,3 +327,73 @@ def test_quantize_2d_feeds_forward_and_dgrad_gemms():
                          "nvfp4")
     assert np.all(np.abs(host_f32(dx) - dr) <= 1e-5 * bd2)
     F.fp4_check_device_errors()
+
+
+def _four_six_check(q, xb, axis, rnd, seed, sf, ts=None):
+    """Bit-exact against the oracle's four-over-six, and not vacuous: some block took max->4."""
+    ref = O.quantize(xb, fmt="nvfp4_4o6", axis=axis, rnd=rnd, seed=seed, tensor_scale=ts)
+    _check_against_oracle(q, ref, "nvfp4", axis, *xb.shape, sf)
+    plain = O.quantize(xb, fmt="nvfp4", axis=axis, rnd=rnd, seed=seed, tensor_scale=ts)
+    assert np.any(ref["scales"] != plain["scales"])
+
+
+@pytest.mark.parametrize("sf", ["rowmajor", "mma"])
+@pytest.mark.parametrize("rnd", ["rtn", "sr"])
+@pytest.mark.parametrize("axis, shape", [(1, (7, 64)), (1, (200, 384)), (1, (129, 4096)), (1, (33, 1056)),
+                                         (0, (96, 200)), (0, (384, 136)), (0, (48, 24))])
+def test_quantize_four_over_six(axis, shape, rnd, sf):
+    """Four-over-six NVFP4 (per block the lower-error of the max->6 and max->4 scales): codes, scales
+    and s_t bit-exact, along both axes, both roundings and both scale layouts.  Axis-1 tensors this
+    small take the single-pass (fused amax) kernel."""
+    rows, cols = shape
+    xb = mixed_input(rows, cols, rows * 11 + cols, "nvfp4")
+    q = F.fp4_quantize(dev_bf16(xb), fmt="nvfp4_4o6", axis=axis, rnd=rnd, seed=77, sf_layout=sf)
+    _four_six_check(q, xb, axis, rnd, 77, sf)
+    F.fp4_check_device_errors()
+
+
+@pytest.mark.parametrize("rnd", ["rtn", "sr"])
+def test_quantize_four_over_six_given_scale_and_strided(rnd):
+    """The streaming kernel (caller's s_t) and the strided-rows kernel (ld > cols)."""
+    xb_full = mixed_input(256, 640, 5, "nvfp4")
+    xb = np.ascontiguousarray(xb_full[:, :512])
+    ts = np.float32(O.nv_tensor_scale(bf16_to_f32(xb)) * np.float32(1.5))
+    ts_dev = torch.tensor([ts], dtype=torch.float32, device="cuda")
+    q = F.fp4_quantize(dev_bf16(xb), fmt="nvfp4_4o6", rnd=rnd, seed=9, tensor_scale_in=ts_dev)
+    _four_six_check(q, xb, 1, rnd, 9, "rowmajor", ts=ts)
+    q2 = F.fp4_quantize(dev_bf16(xb_full)[:, :512], fmt="nvfp4_4o6", rnd=rnd, seed=9, sf_layout="mma")
+    _four_six_check(q2, xb, 1, rnd, 9, "mma")
+    F.fp4_check_device_errors()
+
+
+def test_quantize_four_over_six_two_pass_large_tensor():
+    """A 64 MiB tensor takes the amax kernel then the streaming four-over-six kernel; 64 sampled rows
+    checked bit-exactly against the oracle with the whole tensor's s_t."""
+    from workloads import student_t_bf16
+    xb = student_t_bf16((8192, 4096), 3.0, 0.1, 7, 0)
+    q = F.fp4_quantize(dev_bf16(xb), fmt="nvfp4_4o6", rnd="sr", seed=3)
+    x32 = bf16_to_f32(xb)
+    s_t = O.nv_tensor_scale(x32)
+    assert host_f32(q.tensor_scale)[0] == s_t
+    codes, scales = host_u8(q.codes), host_u8(q.scales)
+    for r in np.sort(np.random.default_rng(2).choice(8192, 64, replace=False)):
+        ref = O.quantize_values(x32[r:r + 1], fmt="nvfp4_4o6", rnd="sr", seed=3, tensor_scale=s_t,
+                                idx_base=int(r) * 4096)
+        np.testing.assert_array_equal(codes[r:r + 1], ref["codes"])
+        np.testing.assert_array_equal(scales[r:r + 1], ref["scales"])
+
+
+def test_four_over_six_feeds_nvfp4_gemm():
+    """Four-over-six outputs are ordinary NVFP4 operands for the block-scaled GEMM."""
+    from workloads import normal_bf16
+    M, K, N = 256, 512, 384
+    xb = normal_bf16((M, K), 1.0, 6, 0)
+    wb = normal_bf16((N, K), 0.02, 6, 1)
+    qx = F.fp4_quantize(dev_bf16(xb), fmt="nvfp4_4o6", sf_layout="mma")
+    qw = F.fp4_quantize(dev_bf16(wb), fmt="nvfp4_4o6", sf_layout="mma")
+    y = F.fp4_gemm(qx.codes, qx.scales, qw.codes, qw.scales, fmt="nvfp4", a_tensor_scale=qx.tensor_scale,
+                   b_tensor_scale=qw.tensor_scale, out_dtype="f32")
+    ox, ow = O.quantize(xb, fmt="nvfp4_4o6"), O.quantize(wb, fmt="nvfp4_4o6")
+    yr, bd = O.gemm_ref(ox, ow, "nvfp4")
+    assert np.all(np.abs(host_f32(y) - yr) <= 1e-5 * bd)
+    F.fp4_check_device_errors()
