@@ -149,6 +149,7 @@ class NvfpStudentT(Workload):
     """NVFP4 quantize (RTN, then Philox SR) + fp32 dequantize of 0.1*Student-t(3), 4096x4096."""
 
     name = "nvfp4_student_t_4096"
+    fmt = "nvfp4"                # the quantizer's format ("nvfp4_4o6": four-over-six block scales)
     rows = cols = 4096
     n_inputs = 4                 # rotating input copies: 128 MB of inputs, each step writes ~146 MB
     launches_per_step = 4        # single-pass amax+quantize RTN, dequantize, quantize SR, dequantize
@@ -195,12 +196,12 @@ class NvfpStudentT(Workload):
             return T[key].around(fn) if T is not None else fn()
 
         # RTN: tensor amax + quantize (one entry point), then dequantize
-        run("amax+quantize_rtn", lambda: F.fp4_quantize(x, fmt="nvfp4", rnd="rtn", codes=self.codes[0],
+        run("amax+quantize_rtn", lambda: F.fp4_quantize(x, fmt=self.fmt, rnd="rtn", codes=self.codes[0],
                                                    scales=self.scales[0], tensor_scale_out=self.ts))
         run("dequantize", lambda: F.fp4_dequantize(self.codes[0], self.scales[0], self.ts, fmt="nvfp4",
                                                    out=self.deq[0]))
         # SR with the same tensor scale, then dequantize
-        run("quantize_sr", lambda: F.fp4_quantize(x, fmt="nvfp4", rnd="sr", seed=1, tensor_scale_in=self.ts,
+        run("quantize_sr", lambda: F.fp4_quantize(x, fmt=self.fmt, rnd="sr", seed=1, tensor_scale_in=self.ts,
                                                   codes=self.codes[1], scales=self.scales[1],
                                                   tensor_scale_out=self.ts_sr))
         run("dequantize", lambda: F.fp4_dequantize(self.codes[1], self.scales[1], self.ts_sr, fmt="nvfp4",
@@ -227,7 +228,7 @@ class NvfpStudentT(Workload):
         return self.step_bytes * n_ranks / (ms_per_step * 1e-3) / 1e9
 
     def config(self):
-        return {"workload": self.name, "shape": [self.rows, self.cols], "format": "nvfp4", "block": 16,
+        return {"workload": self.name, "shape": [self.rows, self.cols], "format": self.fmt, "block": 16,
                 "distribution": "0.1*student_t(3)", "seed": 1, "rounding": ["rtn", "sr(philox4x32-10, seed 1)"],
                 "dequantize": "f32", "algorithmic_bytes_per_step": self.step_bytes,
                 "l2": f"{self.n_inputs} rotating input copies (128 MB) and ~146 MB written per step"}
@@ -242,9 +243,9 @@ class NvfpStudentT(Workload):
         from workloads import bf16_to_f32
         x32 = bf16_to_f32(self.host_bits[:rows]) if rows < self.rows else bf16_to_f32(self.host_bits)
         s_t = O.nv_tensor_scale(bf16_to_f32(self.host_bits))
-        r = O.quantize_values(x32, fmt="nvfp4", rnd="rtn", tensor_scale=s_t)
+        r = O.quantize_values(x32, fmt=self.fmt, rnd="rtn", tensor_scale=s_t)
         O.dequantize(r["codes"], r["scales"], fmt="nvfp4", tensor_scale=s_t)
-        r = O.quantize_values(x32, fmt="nvfp4", rnd="sr", seed=1, tensor_scale=s_t)
+        r = O.quantize_values(x32, fmt=self.fmt, rnd="sr", seed=1, tensor_scale=s_t)
         O.dequantize(r["codes"], r["scales"], fmt="nvfp4", tensor_scale=s_t)
         return rows * self.cols * (2 * (2 + 0.5 + 1 / 16) + 2 * (0.5 + 1 / 16 + 4))
 
@@ -253,6 +254,112 @@ class NvfpStudentT(Workload):
 
     def reference_sample(self):
         return 256, f"256 of {self.rows} rows per step (global tensor scale), NumPy 1 thread"
+
+
+class NvfpStudentT46(NvfpStudentT):
+    """The same step with four-over-six block scales (per block the lower-error of max->6 and
+    max->4); its codes and scales are NVFP4, dequantized as such."""
+
+    name = "nvfp4_4o6_student_t_4096"
+    fmt = "nvfp4_4o6"
+
+    def cpu_sample(self):
+        return 512, f"512 of {self.rows} rows (global tensor scale), NumPy elementwise (1 thread)"
+
+    def reference_sample(self):
+        return 64, f"64 of {self.rows} rows per step (global tensor scale), NumPy 1 thread"
+
+
+class Nvfp2dWeight(Workload):
+    """Square-tile (16x16) NVFP4 quantization of a Llama MLP weight W[11008, 4096] ~ N(0, 0.02), RTN:
+    W's codes along K and W^T's codes along N from one rounding, one scale per tile."""
+
+    name = "nvfp4_2d_weight_11008x4096"
+    rows, cols = 11008, 4096
+    n_inputs = 2                 # two rotating weight copies (180 MB > L2)
+    launches_per_step = 3        # tensor amax, s_t = amax / 2688, 2-D quantize
+    unit = "GB/s"
+
+    def __init__(self, torch, F):
+        self.t, self.F = torch, F
+        n = self.rows * self.cols
+        # bf16 in; codes and E4M3 scales out twice (W and W^T); the amax pass is a second read of W
+        self.step_bytes = n * (2 + 2 * (0.5 + 1 / 16))
+        self.amax_bytes = n * 2.0
+
+    def _bits(self):
+        from workloads import normal_bf16
+        return normal_bf16((self.rows, self.cols), 0.02, 11, 0)
+
+    def setup(self, device):
+        t = self.t
+        bits = self._bits()
+        self.host_in = _pinned_bf16(t, bits)
+        self.x = [self.host_in.to(device).clone() for _ in range(self.n_inputs)]
+        self.dev_in = t.empty_like(self.x[0])
+        q, qt = self.F.fp4_quantize_2d(self.x[0], fmt="nvfp4", sf_layout="mma")
+        self.q, self.qt = q, qt
+        self.amax = t.empty((1,), dtype=t.float32, device=device)
+        self.timers = {k: KernelTimer(t) for k in ("amax", "quantize_2d")}
+
+    def single_kernel(self):
+        return ("quantize_2d",)
+
+    def step(self, i, timed=False, x=None):
+        F = self.F
+        x = self.x[i % self.n_inputs] if x is None else x
+        T = self.timers if timed else None
+
+        def run(key, fn):
+            return T[key].around(fn) if T is not None else fn()
+
+        def amax():
+            F.fp4_amax(x, out=self.amax)
+            F.fp4_nv_tensor_scale(self.amax, out=self.q.tensor_scale)
+
+        run("amax", amax)
+        run("quantize_2d", lambda: F.fp4_quantize_2d(
+            x, fmt="nvfp4", sf_layout="mma", tensor_scale_in=self.q.tensor_scale, codes=self.q.codes,
+            scales=self.q.scales, codes_t=self.qt.codes, scales_t=self.qt.scales,
+            tensor_scale_out=self.q.tensor_scale))
+
+    def outputs(self):
+        return [self.q.codes, self.q.scales, self.qt.codes, self.qt.scales, self.q.tensor_scale]
+
+    def e2e_step(self, host_outs):
+        self.dev_in.copy_(self.host_in, non_blocking=True)
+        self.step(0, x=self.dev_in)
+        for h, o in zip(host_outs, self.outputs()):
+            h.copy_(o, non_blocking=True)
+        return (self.host_in.numel() * 2, sum(o.numel() * o.element_size() for o in self.outputs()))
+
+    def family_work(self, key):
+        return {"amax": self.amax_bytes, "quantize_2d": self.step_bytes}[key]
+
+    def value_from_ms(self, ms_per_step, n_ranks):
+        return self.step_bytes * n_ranks / (ms_per_step * 1e-3) / 1e9
+
+    def config(self):
+        return {"workload": self.name, "shape": [self.rows, self.cols], "format": "nvfp4", "block": "16x16",
+                "distribution": "normal(0, 0.02)", "seed": 11, "rounding": "rtn", "outputs": "W and W^T",
+                "sf_layout": "mma", "algorithmic_bytes_per_step": self.step_bytes,
+                "l2": f"{self.n_inputs} rotating weight copies (180 MB)"}
+
+    def oracle_setup(self):
+        self.host_bits = self._bits()
+
+    def oracle_step(self, rows):
+        import oracle as O
+        from workloads import bf16_to_f32
+        s_t = O.nv_tensor_scale(bf16_to_f32(self.host_bits))
+        O.quantize_2d(self.host_bits[:rows], fmt="nvfp4", tensor_scale=s_t)
+        return rows * self.cols * (2 + 2 * (0.5 + 1 / 16))
+
+    def cpu_sample(self):
+        return 2048, f"2048 of {self.rows} rows (global tensor scale), NumPy (1 thread)"
+
+    def reference_sample(self):
+        return 512, f"512 of {self.rows} rows per step (global tensor scale), NumPy 1 thread"
 
 
 def _dev_bf16(torch, bits, device):
@@ -658,7 +765,8 @@ class MxLinear128(GemmWorkload):
         return 128, "the whole workload: quantize X and W, fp64 GEMM (NumPy)"
 
 
-WORKLOADS = {W.name: W for W in (NvfpStudentT, HadamardMxGemm, VitLinears, LlamaNvfp4, MxLinear128)}
+WORKLOADS = {W.name: W for W in (NvfpStudentT, NvfpStudentT46, Nvfp2dWeight, HadamardMxGemm, VitLinears,
+                                  LlamaNvfp4, MxLinear128)}
 
 
 # ------------------------------------------------------------------ arms ---

@@ -12,6 +12,7 @@
 // All of these are HBM-bound streaming kernels: 128-bit coalesced loads of
 // bf16, warp-shuffle block maxima, packed 32-bit code stores.
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -188,44 +189,100 @@ __device__ __forceinline__ bool nv_fast_division(const float (&x)[E], float am, 
   return kmin >= kTinyKeyMin;
 }
 
-// Four-over-six (NVFP4): squared error of a block's round-to-nearest result under scale byte sb,
-// fp64 terms (x - dequantized code)^2 added in element order; a zero scale dequantizes to 0.
-template <int E>
-__device__ __forceinline__ double nv_rtn_sq_error(const float (&x)[E], float am, uint32_t sb, float s_t,
-                                               const float2* tab) {
-  double acc = 0.0;
-  if (sb == 0u) {
+// Quotients q = x / S of one NVFP4 block under the divisor S = sy.x (sy.y = RN(1/S)): div_by_recip
+// when the block passes nv_fast_division's test for this rounding, IEEE division otherwise.  q may
+// alias x.
+template <int RND, int E>
+__device__ __forceinline__ void nv_divide_block(const float (&x)[E], float am, float2 sy, float (&q)[E]) {
+  if (nv_fast_division<RND, E>(x, am, sy.x, sy.y)) {
 #pragma unroll
-    for (int i = 0; i < E; ++i) acc = __dadd_rn(acc, __dmul_rn((double)x[i], (double)x[i]));
-    return acc;
+    for (int i = 0; i < E; ++i) q[i] = div_by_recip(x[i], sy.x, sy.y);
+  } else {                                       // rare: tiny operands or scales
+#pragma unroll
+    for (int i = 0; i < E; ++i) q[i] = __fdiv_rn(x[i], sy.x);
   }
-  const float2 sy = tab[sb];
-  const float sbv = e4m3_value(sb);
-  const bool fast = nv_fast_division<RND_RTN, E>(x, am, sy.x, sy.y);
-#pragma unroll
-  for (int i = 0; i < E; i += 2) {
-    const float v0 = fast ? div_by_recip(x[i], sy.x, sy.y) : __fdiv_rn(x[i], sy.x);
-    const float v1 = fast ? div_by_recip(x[i + 1], sy.x, sy.y) : __fdiv_rn(x[i + 1], sy.x);
-    const uint32_t c = e2m1x2_rn(v0, v1);
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const float d = __fmul_rn(__fmul_rn(e2m1_value((c >> (4 * h)) & 0xFu), sbv), s_t);
-      const double e = __dsub_rn((double)x[i + h], (double)d);
-      acc = __dadd_rn(acc, __dmul_rn(e, e));
-    }
-  }
-  return acc;
 }
 
-// The scale byte among max->6 (byte6, the standard NVFP4 byte) and max->4 with the lower
-// round-to-nearest squared error ("Four Over Six", Abstract); ties keep byte6, and a zero or
-// identical max->4 byte is never taken.
-template <int E>
-__device__ __forceinline__ uint32_t nv_four_over_six(const float (&x)[E], float am, uint32_t byte6, float s_t,
+// Round-to-nearest dequantization of two quotients: fp32(fp32(G[c] * sbv) * s_t) for each, where
+// c is the E2M1 code of the quotient and g holds the block scale sbv in both halves.  G[c] * sbv
+// has at most 6 significant bits and lies in [2^-10, 2688], so the f16 product is exact.
+__device__ __forceinline__ float2 nv_rtn_dequant2(float q0, float q1, __half2 g, float s_t) {
+  uint32_t h;
+  asm("{\n\t.reg .b8 c;\n\tcvt.rn.satfinite.e2m1x2.f32 c, %2, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, c;\n\t}"
+      : "=r"(h)
+      : "f"(q0), "f"(q1));
+  const float2 v = __half22float2(__hmul2(*reinterpret_cast<const __half2*>(&h), g));
+  return make_float2(__fmul_rn(v.x, s_t), __fmul_rn(v.y, s_t));
+}
+
+// Four-over-six ("Four Over Six", Abstract): of the standard scale byte byte6 (block max -> 6) and
+// the max -> 4 byte, the block takes the one whose round-to-nearest result has the lower squared
+// error, sum over the block of (x - dequantized)^2 in fp64 added in element order; ties keep
+// byte6, and a zero or identical max -> 4 byte is never taken.  x is replaced by its quotients
+// under the chosen scale (exact where the rounding mode needs them) and the byte is returned.
+//
+// The two sums are first screened in fp32 (one fma per element and candidate).  Each fp32 sum is
+// within 18 u (u = 2^-24) of the exact one, relatively, plus 16 * 2^-150 from underflow; each
+// fp64 sum within 15 * 2^-53 (its terms are exact: x has 8 significant bits, the dequantized d at
+// most 24, a non-zero d lies within a factor of 2 of x, so x - d has at most 26 bits and its
+// square at most 52).  A screen gap above 2^-17 of the sums plus 2^-120 therefore decides the
+// fp64 comparison; anything closer (near-ties, non-finite or tiny sums) takes the fp64 sums.
+template <int RND, int E>
+__device__ __forceinline__ uint32_t nv_four_over_six(float (&x)[E], float am, uint32_t byte6, float s_t,
                                                      float y_st, bool st_ok, const float2* tab) {
+  float q6[E];
+  nv_divide_block<RND, E>(x, am, tab[byte6], q6);
   const uint32_t byte4 = e4m3_rn_sat(nv_scale_arg4(am, s_t, y_st, st_ok));
-  if (byte4 == byte6 || byte4 == 0u) return byte6;
-  return nv_rtn_sq_error<E>(x, am, byte4, s_t, tab) < nv_rtn_sq_error<E>(x, am, byte6, s_t, tab) ? byte4 : byte6;
+  bool pick4 = false;
+  if (byte4 != byte6 && byte4 != 0u) {
+    float q4[E];
+    nv_divide_block<RND, E>(x, am, tab[byte4], q4);
+    const __half2 g6 = __float2half2_rn(e4m3_value(byte6)), g4 = __float2half2_rn(e4m3_value(byte4));
+    float f6 = 0.0f, f4 = 0.0f;
+#pragma unroll
+    for (int i = 0; i < E; i += 2) {
+      const float2 d6 = nv_rtn_dequant2(q6[i], q6[i + 1], g6, s_t);
+      const float2 d4 = nv_rtn_dequant2(q4[i], q4[i + 1], g4, s_t);
+      float e = __fsub_rn(x[i], d6.x);
+      f6 = __fmaf_rn(e, e, f6);
+      e = __fsub_rn(x[i], d4.x);
+      f4 = __fmaf_rn(e, e, f4);
+      e = __fsub_rn(x[i + 1], d6.y);
+      f6 = __fmaf_rn(e, e, f6);
+      e = __fsub_rn(x[i + 1], d4.y);
+      f4 = __fmaf_rn(e, e, f4);
+    }
+    const float tol = __fmaf_rn(__fadd_rn(f4, f6), 0x1p-17f, 0x1p-120f);
+    if (__fadd_rn(f4, tol) < f6) {
+      pick4 = true;
+    } else if (!(__fadd_rn(f6, tol) < f4)) {     // too close to call in fp32: the fp64 sums
+      double acc6 = 0.0, acc4 = 0.0;
+#pragma unroll
+      for (int i = 0; i < E; i += 2) {
+        const float2 d6 = nv_rtn_dequant2(q6[i], q6[i + 1], g6, s_t);
+        const float2 d4 = nv_rtn_dequant2(q4[i], q4[i + 1], g4, s_t);
+        const double x0 = (double)x[i], x1 = (double)x[i + 1];
+        double e = __dsub_rn(x0, (double)d6.x);
+        acc6 = __fma_rn(e, e, acc6);
+        e = __dsub_rn(x0, (double)d4.x);
+        acc4 = __fma_rn(e, e, acc4);
+        e = __dsub_rn(x1, (double)d6.y);
+        acc6 = __fma_rn(e, e, acc6);
+        e = __dsub_rn(x1, (double)d4.y);
+        acc4 = __fma_rn(e, e, acc4);
+      }
+      pick4 = acc4 < acc6;
+    }
+    if (pick4) {
+#pragma unroll
+      for (int i = 0; i < E; ++i) x[i] = q4[i];
+    }
+  }
+  if (!pick4) {
+#pragma unroll
+    for (int i = 0; i < E; ++i) x[i] = q6[i];
+  }
+  return pick4 ? byte4 : byte6;
 }
 
 template <int FMT, int RND, int HAD, bool SFMMA>
@@ -261,16 +318,12 @@ __device__ __forceinline__ void quantize_block(const QRowParams& p, const uint4 
     zero = (am == 0.0f);
   } else {
     byte = e4m3_rn_sat(nv_scale_arg(am, nv.s_t, nv.y_st, nv.st_ok));
-    if (FMT == FMT_NV46) byte = nv_four_over_six<E>(x, am, byte, nv.s_t, nv.y_st, nv.st_ok, nv.tab);
-    zero = (byte == 0u);
-    const float2 sy = nv.tab[byte];
-    if (nv_fast_division<RND, E>(x, am, sy.x, sy.y)) {
-#pragma unroll
-      for (int i = 0; i < E; ++i) x[i] = div_by_recip(x[i], sy.x, sy.y);
-    } else {                                     // rare: tiny operands or scales -> IEEE division
-#pragma unroll
-      for (int i = 0; i < E; ++i) x[i] = __fdiv_rn(x[i], sy.x);
+    if (FMT == FMT_NV46) {
+      byte = nv_four_over_six<RND, E>(x, am, byte, nv.s_t, nv.y_st, nv.st_ok, nv.tab);
+    } else {
+      nv_divide_block<RND, E>(x, am, nv.tab[byte], x);
     }
+    zero = (byte == 0u);
   }
   uint32_t w[E / 8];
   if (RND == RND_RTN) {
@@ -573,13 +626,19 @@ struct FusedParams {
   uint32_t tiles_per_cta; // 32-chunk warp tiles staged by each CTA
 };
 
-constexpr int kFusedWarps = 31;                            // consumer warps (1024 threads in all)
-constexpr int kFusedThreads = 32 * (kFusedWarps + 1);
+// Consumer warps: 31 (1024 threads in all, 64 registers a thread) for NVFP4; 15 for four-over-six,
+// whose two candidate scales need about 100 registers.
+template <int FMT>
+struct FusedWarps {
+  static constexpr int kWarps = FMT == FMT_NV46 ? 15 : 31;
+  static constexpr int kThreads = 32 * (kWarps + 1);
+};
 constexpr int kFusedMaxSmem = 227 * 1024 - 2048;          // staged slice; room left for the static data
 constexpr int kFusedPieces = 8;                           // bulk copies (and mbarriers) per slice
 
 template <int FMT, int RND, int HAD, bool SFMMA>
-__global__ void __launch_bounds__(kFusedThreads, 1) nv_quantize_fused_kernel(FusedParams fp) {
+__global__ void __launch_bounds__(FusedWarps<FMT>::kThreads, 1) nv_quantize_fused_kernel(FusedParams fp) {
+  constexpr int kFusedWarps = FusedWarps<FMT>::kWarps;
   extern __shared__ __align__(1024) uint4 slice[];
   __shared__ float2 tab[128];
   __shared__ float red[kFusedWarps];
@@ -740,7 +799,7 @@ struct QColParams {
 };
 
 template <int FMT, int RND, bool SFMMA>
-__global__ void __launch_bounds__(256) quantize_cols_kernel(QColParams p) {
+__global__ void __launch_bounds__(256, FMT == FMT_NV46 ? 2 : 1) quantize_cols_kernel(QColParams p) {
   pdl_trigger();
   __shared__ __align__(16) uint16_t tile[128][64];
   __shared__ float2 tab[128];
@@ -800,12 +859,17 @@ __global__ void __launch_bounds__(256) quantize_cols_kernel(QColParams p) {
 #pragma unroll
         for (int i = 0; i < BS; ++i) xb[i] = xv[b * BS + i];
         byte = e4m3_rn_sat(nv_scale_arg(am, s_t, y_st, st_ok));
-        if (FMT == FMT_NV46) byte = nv_four_over_six<BS>(xb, am, byte, s_t, y_st, st_ok, tab);
+        if (FMT == FMT_NV46) {
+          byte = nv_four_over_six<RND, BS>(xb, am, byte, s_t, y_st, st_ok, tab);
+#pragma unroll
+          for (int i = 0; i < BS; ++i) xv[b * BS + i] = xb[i];     // quotients under the chosen scale
+        } else {
+          const float2 sy = tab[byte];
+          S = sy.x;
+          y = sy.y;
+          fast = nv_fast_division<RND, BS>(xb, am, S, y);
+        }
         zero = (byte == 0u);
-        const float2 sy = tab[byte];
-        S = sy.x;
-        y = sy.y;
-        fast = nv_fast_division<RND, BS>(xb, am, S, y);
       }
 #pragma unroll
       for (int w8 = 0; w8 < BS / 8; ++w8) {
@@ -815,6 +879,8 @@ __global__ void __launch_bounds__(256) quantize_cols_kernel(QColParams p) {
           const float xi = xv[b * BS + w8 * 8 + i];
           if (FMT == FMT_MX) {
             v8[i] = __fmul_rn(xi, inv);
+          } else if (FMT == FMT_NV46) {
+            v8[i] = xi;
           } else {
             v8[i] = fast ? div_by_recip(xi, S, y) : __fdiv_rn(xi, S);
           }
@@ -1295,7 +1361,7 @@ static cudaError_t fused_launch(const FusedParams& fp, uint32_t grid, size_t sme
   static const cudaError_t attr =
       cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kFusedMaxSmem);
   if (attr != cudaSuccess) return attr;
-  return launch_kernel(kernel, dim3(grid), dim3(kFusedThreads), smem, st, true, 1u, fp);
+  return launch_kernel(kernel, dim3(grid), dim3(FusedWarps<FMT>::kThreads), smem, st, true, 1u, fp);
 }
 
 template <int RND, int HAD, int FMT = FMT_NV>

@@ -397,3 +397,40 @@ def test_four_over_six_feeds_nvfp4_gemm():
     yr, bd = O.gemm_ref(ox, ow, "nvfp4")
     assert np.all(np.abs(host_f32(y) - yr) <= 1e-5 * bd)
     F.fp4_check_device_errors()
+
+
+def _tie_blocks(nblocks: int, seed: int) -> np.ndarray:
+    """fp32 [nblocks, 16] blocks whose two four-over-six candidates have exactly equal errors under
+    s_t = 1: all +-24 (both exact: 24/4 = 6 on the 6-grid, 24/6 = 4 on the 4-grid) or 24 with +-5
+    elsewhere (5/4 = 1.25 ties to 1 -> error 1; 5/6 -> 1 -> error 1)."""
+    g = np.random.default_rng(seed)
+    x = np.full((nblocks, 16), 24.0, dtype=np.float32)
+    x[1::2, 1:] = 5.0
+    return x * np.where(g.random((nblocks, 16)) < 0.5, -1.0, 1.0).astype(np.float32)
+
+
+@pytest.mark.parametrize("rnd", ["rtn", "sr"])
+def test_four_over_six_ties_and_extreme_magnitudes(rnd):
+    """Blocks the kernels cannot decide in fp32 and settle with the fp64 sums: exact ties (keep the
+    max->6 scale), error sums that underflow fp32 (values near 1e-30) or overflow it (near 1e30),
+    plus Student-t blocks, some of which tie naturally.  Bit-exact against the oracle."""
+    from workloads import bf16_bits, student_t_bf16
+    ties = bf16_bits(_tie_blocks(256, 3).reshape(64, 64))
+    xb = np.concatenate([ties, student_t_bf16((448, 64), 3.0, 0.1, 8, 0)], axis=0)
+    x32 = bf16_to_f32(xb)
+    ts = torch.ones(1, dtype=torch.float32, device="cuda")
+    q = F.fp4_quantize(dev_bf16(xb), fmt="nvfp4_4o6", rnd=rnd, seed=5, tensor_scale_in=ts)
+    ref = O.quantize(xb, fmt="nvfp4_4o6", rnd=rnd, seed=5, tensor_scale=np.float32(1.0))
+    _check_against_oracle(q, ref, "nvfp4", 1, *xb.shape, "rowmajor")
+    plain = O.quantize(xb, fmt="nvfp4", rnd=rnd, seed=5, tensor_scale=np.float32(1.0))
+    np.testing.assert_array_equal(ref["scales"][:64], plain["scales"][:64])          # ties keep max->6
+    from oracle.four_over_six import nv_block_candidates, _rtn_sq_error
+    xs = x32[64:].reshape(-1, 16)
+    sb6, sb4 = nv_block_candidates(np.max(np.abs(xs), axis=-1), np.float32(1.0))
+    live = (sb4 != sb6) & (sb4 != 0)
+    assert np.any(live & (_rtn_sq_error(xs, sb6, np.float32(1.0)) == _rtn_sq_error(xs, sb4, np.float32(1.0))))
+    for mult in (1e-30, 1e30):                       # squared errors far outside fp32's range
+        xe = student_t_bf16((128, 256), 3.0, mult, 9, 1)
+        q = F.fp4_quantize(dev_bf16(xe), fmt="nvfp4_4o6", rnd=rnd, seed=6)
+        _four_six_check(q, xe, 1, rnd, 6, "rowmajor")
+    F.fp4_check_device_errors()
