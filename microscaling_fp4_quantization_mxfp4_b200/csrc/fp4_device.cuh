@@ -128,6 +128,26 @@ __device__ __forceinline__ u32x4 philox4x32_10(uint32_t c0, uint32_t c1, uint32_
   return {c0, c1, c2, c3};
 }
 
+// The same generator with its key schedule (k0 + i * 0x9E3779B9, k1 + i * 0xBB67AE85 for round
+// i = 0..9, interleaved) precomputed on the host and read from kernel parameters: the rounds then
+// take their keys straight from the constant bank instead of adding them up per call.
+struct PhiloxKeys {
+  uint32_t k[20];
+};
+
+__device__ __forceinline__ u32x4 philox4x32_10(uint32_t c0, uint32_t c1, const PhiloxKeys& ks) {
+  uint32_t c2 = 0u, c3 = 0u;
+#pragma unroll
+  for (int i = 0; i < 10; ++i) {
+    const unsigned long long p0 = (unsigned long long)0xD2511F53u * c0;
+    const unsigned long long p1 = (unsigned long long)0xCD9E8D57u * c2;
+    const uint32_t n0 = (uint32_t)(p1 >> 32) ^ c1 ^ ks.k[2 * i];
+    const uint32_t n2 = (uint32_t)(p0 >> 32) ^ c3 ^ ks.k[2 * i + 1];
+    c0 = n0; c1 = (uint32_t)p1; c2 = n2; c3 = (uint32_t)p0;
+  }
+  return {c0, c1, c2, c3};
+}
+
 // Random words for 8 consecutive elements starting at linear index idx0
 // (idx0 % 8 == 0): two counters, words in index order.
 __device__ __forceinline__ void philox_words8(unsigned long long idx0, unsigned long long seed,

@@ -146,6 +146,7 @@ struct QRowParams {
   uint32_t cols;
   uint32_t g4;           // padded k-groups / 4 (tensor-core scale layout)
   unsigned long long seed;
+  PhiloxKeys keys;      // the seed's Philox key schedule
   const float* ts;
   float* ts_copy_out;
   uint32_t* codes;       // [rows, cols/8] 32-bit words of 8 nibbles
@@ -336,9 +337,8 @@ __device__ __forceinline__ void quantize_block(const QRowParams& p, const uint4 
 #pragma unroll
     for (int k = 0; k < E / 8; ++k) {
       const unsigned long long j = j0 + 2u * k;
-      const u32x4 a = philox4x32_10((uint32_t)j, (uint32_t)(j >> 32), (uint32_t)p.seed, (uint32_t)(p.seed >> 32));
-      const u32x4 b = philox4x32_10((uint32_t)(j + 1), (uint32_t)((j + 1) >> 32), (uint32_t)p.seed,
-                                    (uint32_t)(p.seed >> 32));
+      const u32x4 a = philox4x32_10((uint32_t)j, (uint32_t)(j >> 32), p.keys);
+      const u32x4 b = philox4x32_10((uint32_t)(j + 1), (uint32_t)((j + 1) >> 32), p.keys);
       const float* xe = x + 8 * k;
       const uint32_t n[8] = {e2m1_sr(xe[0], a.x), e2m1_sr(xe[1], a.y), e2m1_sr(xe[2], a.z), e2m1_sr(xe[3], a.w),
                              e2m1_sr(xe[4], b.x), e2m1_sr(xe[5], b.y), e2m1_sr(xe[6], b.z), e2m1_sr(xe[7], b.w)};
@@ -792,6 +792,7 @@ struct QColParams {
   int64_t ld;
   uint32_t G, g4;        // k-groups per output row (R / block) and padded/4
   unsigned long long seed;
+  PhiloxKeys keys;      // the seed's Philox key schedule
   const float* ts;
   float* ts_copy_out;
   uint8_t* codes;
@@ -799,7 +800,7 @@ struct QColParams {
 };
 
 template <int FMT, int RND, bool SFMMA>
-__global__ void __launch_bounds__(256, FMT == FMT_NV46 ? 2 : 1) quantize_cols_kernel(QColParams p) {
+__global__ void __launch_bounds__(256, 2) quantize_cols_kernel(QColParams p) {
   pdl_trigger();
   __shared__ __align__(16) uint16_t tile[128][64];
   __shared__ float2 tab[128];
@@ -895,8 +896,7 @@ __global__ void __launch_bounds__(256, FMT == FMT_NV46 ? 2 : 1) quantize_cols_ke
           for (int h = 0; h < 2; ++h) {
             const unsigned long long row = rb + w8 * 8 + 4 * h + (lane & 3);
             const unsigned long long j = (row * p.C + (c & ~3u)) >> 2;
-            const u32x4 ph = philox4x32_10((uint32_t)j, (uint32_t)(j >> 32), (uint32_t)p.seed,
-                                           (uint32_t)(p.seed >> 32));
+            const u32x4 ph = philox4x32_10((uint32_t)j, (uint32_t)(j >> 32), p.keys);
             const uint32_t w[4] = {ph.x, ph.y, ph.z, ph.w};
             uint32_t t[4];
             quad_transpose4(w, t, lane);
@@ -943,6 +943,7 @@ struct Q2Params {
   uint32_t R, C;
   int64_t ld;
   unsigned long long seed;
+  PhiloxKeys keys;      // the seed's Philox key schedule
   const float* ts;
   float* ts_copy_out;
   uint8_t* codes;        // [R, C/2]
@@ -1027,9 +1028,8 @@ __global__ void __launch_bounds__(256) quantize_2d_kernel(Q2Params p) {
 #pragma unroll
       for (int k = 0; k < BS / 8; ++k) {
         const unsigned long long j = j0 + 2u * k;
-        const u32x4 a = philox4x32_10((uint32_t)j, (uint32_t)(j >> 32), (uint32_t)p.seed, (uint32_t)(p.seed >> 32));
-        const u32x4 b = philox4x32_10((uint32_t)(j + 1), (uint32_t)((j + 1) >> 32), (uint32_t)p.seed,
-                                      (uint32_t)(p.seed >> 32));
+        const u32x4 a = philox4x32_10((uint32_t)j, (uint32_t)(j >> 32), p.keys);
+        const u32x4 b = philox4x32_10((uint32_t)(j + 1), (uint32_t)((j + 1) >> 32), p.keys);
         const float* xe = x + 8 * k;
         const uint32_t n[8] = {e2m1_sr(xe[0], a.x), e2m1_sr(xe[1], a.y), e2m1_sr(xe[2], a.z), e2m1_sr(xe[3], a.w),
                                e2m1_sr(xe[4], b.x), e2m1_sr(xe[5], b.y), e2m1_sr(xe[6], b.z), e2m1_sr(xe[7], b.w)};
@@ -1311,6 +1311,19 @@ cudaError_t launch_amax_fixed_grid(const void* x, int64_t rows, int64_t cols, in
   return launch_kernel(amax_kernel<0>, dim3(grid), dim3(256), 0, st, false, 1u, ap);
 }
 
+// Philox4x32-10 key schedule of a 64-bit seed: round i uses (lo + i * 0x9E3779B9, hi + i * 0xBB67AE85).
+static PhiloxKeys philox_keys(unsigned long long seed) {
+  PhiloxKeys ks;
+  uint32_t k0 = (uint32_t)seed, k1 = (uint32_t)(seed >> 32);
+  for (int i = 0; i < 10; ++i) {
+    ks.k[2 * i] = k0;
+    ks.k[2 * i + 1] = k1;
+    k0 += 0x9E3779B9u;
+    k1 += 0xBB67AE85u;
+  }
+  return ks;
+}
+
 cudaError_t launch_nv_tensor_scale(const float* amax, float* out, cudaStream_t st) {
   return launch_kernel(nv_tensor_scale_kernel, dim3(1), dim3(1), 0, st, false, 1u, amax, out);
 }
@@ -1398,6 +1411,7 @@ cudaError_t launch_quantize_nv_fused(const QuantizeParams& p, float* ts_out, con
   qp.cols = (uint32_t)p.cols;
   qp.g4 = (uint32_t)((p.cols / 16 + 3) / 4);
   qp.seed = p.seed;
+  qp.keys = philox_keys(p.seed);
   qp.ts = nullptr;
   qp.ts_copy_out = nullptr;
   qp.codes = reinterpret_cast<uint32_t*>(p.codes);
@@ -1461,6 +1475,7 @@ cudaError_t launch_quantize(const QuantizeParams& p, int num_sms, cudaStream_t s
     qp.cols = (uint32_t)p.cols;
     qp.g4 = (uint32_t)((p.cols / bs + 3) / 4);
     qp.seed = p.seed;
+    qp.keys = philox_keys(p.seed);
     qp.ts = p.ts;
     qp.ts_copy_out = p.ts_copy_out;
     qp.codes = reinterpret_cast<uint32_t*>(p.codes);
@@ -1486,6 +1501,7 @@ cudaError_t launch_quantize(const QuantizeParams& p, int num_sms, cudaStream_t s
   qp.G = (uint32_t)(p.rows / bs);
   qp.g4 = (qp.G + 3u) / 4u;
   qp.seed = p.seed;
+  qp.keys = philox_keys(p.seed);
   qp.ts = p.ts;
   qp.ts_copy_out = p.ts_copy_out;
   qp.codes = p.codes;
@@ -1527,6 +1543,7 @@ cudaError_t launch_quantize_2d(const QuantizeParams& p, uint8_t* codes_t, uint8_
   qp.C = (uint32_t)p.cols;
   qp.ld = p.ld;
   qp.seed = p.seed;
+  qp.keys = philox_keys(p.seed);
   qp.ts = p.ts;
   qp.ts_copy_out = p.ts_copy_out;
   qp.codes = p.codes;
