@@ -61,17 +61,24 @@ __device__ __forceinline__ uint32_t mad_u32(uint32_t a, uint32_t b, uint32_t c) 
 // is 2 (m - 127) + floor(s) for s = |v| / step (exact).  floor(s) comes from one
 // round-toward-zero addition of 2^23 (the sum's last significand bits are the
 // integer part), p is the exact remainder, and codes past 6 (|v| >= 6, where s
-// reaches 3 on the top binade) clamp to 7.
+// reaches 3 on the top binade) clamp to 7.  The exponent is handled in place
+// (eb = m << 23): 1/step has the bits 0x7F800000 - eb and 2m = eb >> 22; the
+// shifts and the negation run as multiply-adds.
+__device__ __forceinline__ uint32_t mad_hi_u32(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("mad.hi.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
 __device__ __forceinline__ uint32_t e2m1_sr(float v, uint32_t r) {
   const uint32_t vb = __float_as_uint(v);
-  const uint32_t m = min(max((vb >> 23) & 0xFFu, 127u), 129u);
-  const float inv_step = __uint_as_float(mad_u32(m, 0xFF800000u, 0x7F800000u));   // (255 - m) << 23
+  const uint32_t eb = min(max(vb & 0x7F800000u, 0x3F800000u), 0x40800000u);
+  const float inv_step = __uint_as_float(mad_u32(eb, 0xFFFFFFFFu, 0x7F800000u));
   const float s = __fmul_rn(fabsf(v), inv_step);
   const float t = __fadd_rz(s, 8388608.0f);                        // 2^23 + floor(s)
   const float p = __fsub_rn(s, __fsub_rn(t, 8388608.0f));          // exact fractional part
   const uint32_t thr = __float2uint_ru(__fmul_rn(p, 4294967296.0f));   // < 2^32 since p < 1
-  const uint32_t code = min(mad_u32(m, 2u, __float_as_uint(t)) - (0x4B000000u + 254u) + (r < thr ? 1u : 0u), 7u);
-  return code | ((vb >> 28) & 8u);
+  const uint32_t code = min(mad_hi_u32(eb, 1024u, __float_as_uint(t)) - (0x4B000000u + 254u) + (r < thr ? 1u : 0u), 7u);
+  return code | (mad_hi_u32(vb, 16u, 0u) & 8u);
 }
 
 // Eight 4-bit codes, element i in nibble i, packed with multiply-adds.

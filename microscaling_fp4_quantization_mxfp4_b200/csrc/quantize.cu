@@ -1106,13 +1106,6 @@ struct DeqParams {
   void* out;
 };
 
-// E2M1 values of both nibbles of every code byte (low nibble first): a 2 KB
-// shared-memory table, so dequantizing 8 codes is 4 table loads.
-__device__ __forceinline__ void fill_pair_table(float2* pairs) {
-  for (int b = threadIdx.x; b < 256; b += blockDim.x)
-    pairs[b] = make_float2(e2m1_value((uint32_t)b & 0xFu), e2m1_value((uint32_t)b >> 4));
-}
-
 // Address of the scale byte of a chunk (8 codes) in either scale layout.
 template <int FMT, bool SFMMA>
 __device__ __forceinline__ const uint8_t* deq_scale_ptr(const DeqParams& p, uint32_t chunk) {
@@ -1124,24 +1117,44 @@ __device__ __forceinline__ const uint8_t* deq_scale_ptr(const DeqParams& p, uint
   return p.scales + chunk / LPB;
 }
 
+// Eight E2M1 codes (element i in nibble i of w) -> their values as four f16 pairs, element 2k in
+// the low half of h[k].
+__device__ __forceinline__ void e2m1x8_to_f16x2(uint32_t w, uint32_t (&h)[4]) {
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+      : "=r"(h[0]), "=r"(h[1]), "=r"(h[2]), "=r"(h[3])
+      : "r"(w));
+}
+
+// One chunk of 8 codes to fp32 (or bf16) values.  NV: fp32(fp32(G[c] * sb) * s_t), where the
+// product G[c] * sb (at most 6 significant bits, in [2^-10, 2688] or zero) is exact in f16.
+// MX: G[c] * 2^E in fp32.
 template <int FMT, bool BF16>
 __device__ __forceinline__ void dequantize_chunk_to(const DeqParams& p, uint32_t byte, uint32_t slot, uint32_t w,
-                                                    float s_t, const float2* pairs) {
+                                                    float s_t) {
+  uint32_t h[4];
+  e2m1x8_to_f16x2(w, h);
   float y[8];
-#pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    const float2 g = pairs[(w >> (8 * k)) & 0xFFu];
-    y[2 * k] = g.x;
-    y[2 * k + 1] = g.y;
-  }
   if (FMT == FMT_MX) {
     const float sc = mx_scale_value(byte);
 #pragma unroll
-    for (int i = 0; i < 8; ++i) y[i] = __fmul_rn(y[i], sc);
+    for (int k = 0; k < 4; ++k) {
+      const float2 g = __half22float2(*reinterpret_cast<const __half2*>(&h[k]));
+      y[2 * k] = __fmul_rn(g.x, sc);
+      y[2 * k + 1] = __fmul_rn(g.y, sc);
+    }
   } else {
-    const float sb = e4m3_value(byte);
+    const __half2 sb = __float2half2_rn(e4m3_value(byte));
 #pragma unroll
-    for (int i = 0; i < 8; ++i) y[i] = __fmul_rn(__fmul_rn(y[i], sb), s_t);
+    for (int k = 0; k < 4; ++k) {
+      const float2 g = __half22float2(__hmul2(*reinterpret_cast<const __half2*>(&h[k]), sb));
+      y[2 * k] = __fmul_rn(g.x, s_t);
+      y[2 * k + 1] = __fmul_rn(g.y, s_t);
+    }
   }
   if (BF16) {
     uint32_t o[4];
@@ -1173,9 +1186,7 @@ __global__ void __launch_bounds__(kDeqThreads) dequantize_stream_kernel(DeqParam
   constexpr int kOut = BF16 ? 16 : 32;                   // output bytes per chunk
   constexpr int kTileBytes = kDeqTileChunks * kOut;
   extern __shared__ __align__(128) uint8_t stage_buf[];
-  __shared__ float2 pairs[256];
   pdl_trigger();
-  fill_pair_table(pairs);
   pdl_wait();
   const float s_t = FMT == FMT_NV ? *p.ts : 1.0f;
   const uint32_t ntiles = (p.nchunks + kDeqTileChunks - 1) / kDeqTileChunks;
@@ -1219,7 +1230,7 @@ __global__ void __launch_bounds__(kDeqThreads) dequantize_stream_kernel(DeqParam
     for (int k = 0; k < 2; ++k) {
       const uint32_t local = threadIdx.x + k * kDeqThreads;
       const uint32_t c = i * kDeqTileChunks + local;
-      if (c < p.nchunks) dequantize_chunk_to<FMT, BF16>(q, sb[k], local, w[k], s_t, pairs);
+      if (c < p.nchunks) dequantize_chunk_to<FMT, BF16>(q, sb[k], local, w[k], s_t);
     }
     fence_async_smem();
     __syncthreads();
