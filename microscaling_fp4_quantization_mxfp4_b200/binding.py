@@ -46,8 +46,11 @@ def _check(status: int, where: str) -> None:
 
 
 def _stream(stream) -> int:
-    s = stream if stream is not None else torch.cuda.current_stream()
-    return s.cuda_stream
+    """cudaStream_t of `stream`, or of the current device's current stream (read as a raw handle,
+    without building a Stream object)."""
+    if stream is not None:
+        return stream.cuda_stream
+    return torch._C._cuda_getCurrentRawStream(torch._C._cuda_getDevice())
 
 
 def _ptr(t: Optional[torch.Tensor]):
