@@ -30,7 +30,8 @@ Salmon et al. SC'11, Sylvester Hadamard) and each module says which.
 
 Modules: `formats` (E2M1/E4M3/E8M0), `philox`, `quantize` (MX/NV, RTN/SR,
 axis 0/1, packing, dequantize; fmt "nvfp4_4o6" via `four_over_six`),
-`quantize2d` (square-tile 2-D blocks),
+`quantize2d` (square-tile 2-D blocks), `mse_grid` (MSE-searched NVFP4 scales,
+fmt "mxfp4_gs": MXFP4 with the MSE-fitted clip threshold),
 `hadamard`, `layout` (tensor-core scale-factor layout), `gemm` (fp64 reference
 and error bound).
 """
@@ -42,6 +43,7 @@ from .quantize import quantize, quantize_values, dequantize, pack_nibbles, unpac
 from .layout import sf_to_mma, sf_from_mma, sf_mma_bytes
 from .gemm import gemm_ref, gemm_ref_rows, gemm_ref_cols, deq_for_gemm
 from .quantize2d import quantize_2d
+from .mse_grid import quantize_mse
 
 __all__ = [
     "E2M1_GRID", "e2m1_decode", "e2m1_rtn", "e2m1_sr", "e4m3_decode", "e4m3_rne_sat",

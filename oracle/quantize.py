@@ -69,13 +69,18 @@ def nv_tensor_scale(x32: np.ndarray) -> np.float32:
 
 
 def _quantize_rows(xw: np.ndarray, idxw: np.ndarray, fmt: str, bs: int, rnd: str, seed: int,
-                   s_t: np.float32):
-    """Quantize every row of xw (fp32 [n, L], L % bs == 0) in contiguous bs-blocks."""
+                   s_t: np.float32, mx_clip=None):
+    """Quantize every row of xw (fp32 [n, L], L % bs == 0) in contiguous bs-blocks.  mx_clip: the
+    MXFP4 exponent's clip threshold (`mse_grid` reading 6), None for the OCP rule."""
     n, L = xw.shape
     xb = xw.reshape(n, L // bs, bs)
     amax_b = np.max(np.abs(xb), axis=2).astype(np.float32)                 # [n, G]
     if fmt == "mxfp4":
-        E = mx_scale_exponent(amax_b)
+        if mx_clip is None:
+            E = mx_scale_exponent(amax_b)
+        else:
+            from .mse_grid import mx_scale_exponent_clip
+            E = mx_scale_exponent_clip(amax_b, mx_clip)
         scale_bytes = (E + 127).astype(np.uint8)
         S = np.ldexp(np.float64(1.0), E)                                      # exact powers of two
         v = (xb.astype(np.float64) / S[..., None]).astype(np.float32)        # exact quotient, rounded to fp32
@@ -104,9 +109,15 @@ def quantize_values(x32, fmt: str = "mxfp4", block: int | None = None, axis: int
     The Philox index of element (r, c) is idx_base + r * idx_cols + c (idx_cols
     defaults to cols), so a row slice of a larger tensor can be quantized with
     its global indices.  For NVFP4 without `tensor_scale`, s_t comes from x32.
-    fmt "nvfp4_4o6" is NVFP4 with four-over-six block scales (`four_over_six`).
+    fmt "nvfp4_4o6" is NVFP4 with four-over-six block scales (`four_over_six`); fmt "mxfp4_gs" is
+    MXFP4 whose block exponents use the MSE-fitted clip threshold (`mse_grid`, readings 6-7).
     """
     four_six = fmt == "nvfp4_4o6"
+    mx_clip = None
+    if fmt == "mxfp4_gs":
+        from .mse_grid import MX_GRID_CLIP
+        mx_clip = MX_GRID_CLIP
+        fmt = "mxfp4"
     fmt = "nvfp4" if four_six else fmt
     bs = block or FMT_BLOCK[fmt]
     if (fmt, bs) not in (("mxfp4", 32), ("nvfp4", 16)):
@@ -127,7 +138,7 @@ def quantize_values(x32, fmt: str = "mxfp4", block: int | None = None, axis: int
         codes, scales = quantize_rows_46(np.ascontiguousarray(xw), np.ascontiguousarray(idxw), rnd, seed, s_t)
     else:
         codes, scales = _quantize_rows(np.ascontiguousarray(xw), np.ascontiguousarray(idxw),
-                                       fmt, bs, rnd, seed, s_t)
+                                       fmt, bs, rnd, seed, s_t, mx_clip)
     return {"codes": pack_nibbles(codes), "scales": scales, "tensor_scale": s_t}
 
 
