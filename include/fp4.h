@@ -86,6 +86,15 @@ enum { FP4_MXFP4 = 0, FP4_NVFP4 = 1 };              /* fp4_format    */
  * keep max->6).  Accepted by fp4_quantize and fp4_hadamard_quantize with block
  * 16; their outputs are plain NVFP4 (dequantize and GEMM with FP4_NVFP4). */
 enum { FP4_NVFP4_4O6 = 2 };
+/* Quantizer-only format: MXFP4 codes and E8M0 scales whose block exponent is
+ * the smallest one whose grid reaches 7.25 * 2^E >= amax_b instead of the OCP
+ * rule floor(log2 amax_b) - 2 (which clips up to 8 * 2^E): the MSE-fitted fixed
+ * grid scale for MXFP4 with Hadamard rotations (summary post of "Bridging the
+ * Gap Between Promise and Performance for Microscaling FP4 Quantization",
+ * MR-GPTQ list item 1; 7.25 minimises the RTN squared error of rotated Gaussian
+ * data over a 1/16 grid of [6, 8]).  Accepted by fp4_quantize and
+ * fp4_hadamard_quantize with block 32; outputs are plain MXFP4. */
+enum { FP4_MXFP4_GS = 3 };
 enum { FP4_RTN = 0, FP4_SR = 1 };                   /* fp4_round     */
 enum { FP4_SF_ROWMAJOR = 0, FP4_SF_MMA = 1 };       /* fp4_sf_layout */
 enum { FP4_OUT_F32 = 0, FP4_OUT_BF16 = 1 };         /* fp4_dtype     */
@@ -98,7 +107,8 @@ enum { FP4_OUT_F32 = 0, FP4_OUT_BF16 = 1 };         /* fp4_dtype     */
  *
  *   x          bf16 [rows, cols], row stride `ld` elements (ld >= cols).
  *              16-byte aligned; cols and ld multiples of 8.
- *   fmt,block  (FP4_MXFP4, 32), (FP4_NVFP4, 16) or (FP4_NVFP4_4O6, 16).
+ *   fmt,block  (FP4_MXFP4, 32), (FP4_NVFP4, 16), (FP4_NVFP4_4O6, 16) or
+ *              (FP4_MXFP4_GS, 32).
  *   axis       1: blocks along cols (cols % block == 0);
  *              0: blocks along rows (rows % block == 0), output transposed.
  *   rnd, seed  FP4_RTN, or FP4_SR with the 64-bit Philox key `seed`.
@@ -153,6 +163,36 @@ fp4_status fp4_quantize_2d(const void* x, int64_t rows, int64_t cols, int64_t ld
                            const float* tensor_scale_in, float* tensor_scale_out,
                            uint8_t* codes, uint8_t* scales, uint8_t* codes_t, uint8_t* scales_t,
                            int sf_layout, void* stream);
+
+/*
+ * fp4_quantize_mse -- NVFP4 quantization with MSE-searched scales (summary
+ * post of "Bridging the Gap Between Promise and Performance for Microscaling
+ * FP4 Quantization", MR-GPTQ list item 1: the grid is fitted to the data by
+ * optimizing it alternately per block and per tensor).
+ *   Block step (tensor scale s fixed): each 16-element block takes, among its
+ *   standard E4M3 byte b6 and the eight bytes below and above it (within
+ *   1..126), the one whose round-to-nearest result has the least squared error
+ *   (fp64, terms in element order; ties to the byte met first in the order
+ *   b6, b6-1, b6+1, b6-2, ...); a block with b6 = 0 keeps 0.
+ *   Tensor step: s becomes the best of fp32(s * (1 + k/64)), k = -8..8, each
+ *   scored after its own block step by sum over blocks of
+ *   floor(err_b * 2^(80 - 2 floor(log2 amax))) (an exact integer sum; ties to
+ *   the smallest |k|, then k < 0).
+ *   Schedule: s = amax / 2688, `iters` tensor steps (0..8), then a block step
+ *   whose bytes quantize the codes with `rnd` (FP4_SR: Philox as fp4_quantize).
+ *   fmt, block FP4_NVFP4, 16 (FP4_MXFP4: FP4_ERR_UNSUPPORTED).  Blocks run
+ *              along cols (axis 1); cols % 16 == 0; x finite.
+ *   x, rows, cols, ld, seed, codes, scales, sf_layout  as fp4_quantize axis 1.
+ *   tensor_scale_out  device fp32, required: receives the searched s_t.
+ * Outputs are plain NVFP4 (dequantize and GEMM with FP4_NVFP4).  Launches an
+ * amax pass, `iters` tensor steps and the final quantize kernel; uses the
+ * library's per-device scratch, so calls on one device must not run
+ * concurrently on different streams.
+ */
+fp4_status fp4_quantize_mse(const void* x, int64_t rows, int64_t cols, int64_t ld,
+                            int fmt, int block, int rnd, uint64_t seed, int iters,
+                            float* tensor_scale_out, uint8_t* codes, uint8_t* scales,
+                            int sf_layout, void* stream);
 
 /*
  * fp4_dequantize -- codes + scales (+ s_t) back to floating point

@@ -15,6 +15,7 @@ PROTOTYPES = {
                                      _int, _int, _vp, _vp]),
     "fp4_quantize_2d": (_int, [_vp, _i64, _i64, _i64, _int, _int, _int, _u64, _vp, _vp, _vp, _vp, _vp, _vp,
                                _int, _vp]),
+    "fp4_quantize_mse": (_int, [_vp, _i64, _i64, _i64, _int, _int, _int, _u64, _int, _vp, _vp, _vp, _int, _vp]),
     "fp4_dequantize": (_int, [_vp, _vp, _vp, _i64, _i64, _int, _int, _int, _vp, _int, _vp]),
     "fp4_gemm": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _int, _int, _vp, _i64, _int, _vp]),
     "fp4_amax": (_int, [_vp, _i64, _i64, _i64, _vp, _vp]),

@@ -14,17 +14,18 @@ import torch
 
 from . import _lib
 
-MXFP4, NVFP4, NVFP4_4O6 = 0, 1, 2
+MXFP4, NVFP4, NVFP4_4O6, MXFP4_GS = 0, 1, 2, 3
 RTN, SR = 0, 1
 SF_ROWMAJOR, SF_MMA = 0, 1
 OUT_F32, OUT_BF16 = 0, 1
 
-_FMT = {"mxfp4": MXFP4, "nvfp4": NVFP4, "nvfp4_4o6": NVFP4_4O6, MXFP4: MXFP4, NVFP4: NVFP4, NVFP4_4O6: NVFP4_4O6}
+_FMT = {"mxfp4": MXFP4, "nvfp4": NVFP4, "nvfp4_4o6": NVFP4_4O6, "mxfp4_gs": MXFP4_GS,
+        MXFP4: MXFP4, NVFP4: NVFP4, NVFP4_4O6: NVFP4_4O6, MXFP4_GS: MXFP4_GS}
 _RND = {"rtn": RTN, "sr": SR, RTN: RTN, SR: SR}
 _SF = {"rowmajor": SF_ROWMAJOR, "mma": SF_MMA, SF_ROWMAJOR: SF_ROWMAJOR, SF_MMA: SF_MMA}
 _OUT = {"f32": OUT_F32, "bf16": OUT_BF16, torch.float32: OUT_F32, torch.bfloat16: OUT_BF16,
         OUT_F32: OUT_F32, OUT_BF16: OUT_BF16}
-BLOCK = {MXFP4: 32, NVFP4: 16, NVFP4_4O6: 16}
+BLOCK = {MXFP4: 32, NVFP4: 16, NVFP4_4O6: 16, MXFP4_GS: 32}
 
 
 class Fp4Error(RuntimeError):
@@ -150,6 +151,20 @@ def fp4_quantize_2d(x: torch.Tensor, fmt="nvfp4", rnd="rtn", seed: int = 0,
     _check(st, "fp4_quantize_2d")
     ts = ts_out if f == NVFP4 else None
     return Fp4Quantized(codes, scales, ts), (Fp4Quantized(codes_t, scales_t, ts) if transposed else None)
+
+
+def fp4_quantize_mse(x: torch.Tensor, rnd="rtn", seed: int = 0, iters: int = 1, sf_layout="rowmajor", *,
+                     codes=None, scales=None, tensor_scale_out=None, stream=None) -> Fp4Quantized:
+    """NVFP4 quantization along rows with MSE-searched block and tensor scales (see fp4_quantize_mse in
+    include/fp4.h); outputs are plain NVFP4."""
+    _bf16_matrix(x)
+    r, sf = _RND[rnd], _SF[sf_layout]
+    codes, scales, ts_out = _alloc_quant_outputs(x, NVFP4, 1, sf, codes, scales, tensor_scale_out)
+    st = _lib.load().fp4_quantize_mse(
+        x.data_ptr(), x.shape[0], x.shape[1], x.stride(0), NVFP4, 16, r, seed & (2 ** 64 - 1), iters,
+        ts_out.data_ptr(), codes.data_ptr(), scales.data_ptr(), sf, _stream(stream))
+    _check(st, "fp4_quantize_mse")
+    return Fp4Quantized(codes, scales, ts_out)
 
 
 def fp4_dequantize(codes: torch.Tensor, scales: torch.Tensor, tensor_scale=None, fmt="mxfp4",

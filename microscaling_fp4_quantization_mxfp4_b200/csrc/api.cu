@@ -54,6 +54,14 @@ fp4_status device_state(DeviceState** out) {
     d.scratch.error = d.scratch.counter + 1;
     d.scratch.grid_arrive = d.scratch.counter + 2;
     d.scratch.grid_depart = d.scratch.counter + 3;
+    // MSE-searched quantization: its amax, its tensor step's per-CTA sums and completion ticket
+    void* mse = nullptr;
+    const size_t mse_bytes = sizeof(unsigned long long) * 2 * 17 * kMaxMseCtas + 256;
+    if (cudaMalloc(&mse, mse_bytes) != cudaSuccess) return FP4_ERR_CUDA;
+    if (cudaMemset(mse, 0, mse_bytes) != cudaSuccess) return FP4_ERR_CUDA;
+    d.scratch.mse_partials = static_cast<unsigned long long*>(mse);
+    d.scratch.mse_amax = reinterpret_cast<float*>(d.scratch.mse_partials + 2 * 17 * kMaxMseCtas);
+    d.scratch.mse_ticket = reinterpret_cast<unsigned*>(d.scratch.mse_amax + 4);
     d.num_sms = sms;
     d.ready = true;
   }
@@ -110,6 +118,12 @@ fp4_status quantize_impl(const void* x, int64_t rows, int64_t cols, int64_t ld, 
                          int rnd, uint64_t seed, const float* ts_in, float* ts_out, uint8_t* codes, uint8_t* scales,
                          int sf_layout, int had, float* rotated, cudaStream_t st) {
   int four_six = 0;
+  uint32_t mx_thr = 0x800000u;       // OCP exponent rule
+  if (fmt == FP4_MXFP4_GS) {         // MXFP4 codes and scales under the MSE-fitted clip threshold
+    if (block != 32) return FP4_ERR_UNSUPPORTED;
+    fmt = FP4_MXFP4;
+    mx_thr = 0x680000u;              // T = 7.25: T/4 = 1 + 0x680000 / 2^23
+  }
   if (fmt == FP4_NVFP4_4O6) {        // NVFP4 codes and scales with four-over-six block scales
     if (block != 16) return FP4_ERR_UNSUPPORTED;
     fmt = FP4_NVFP4;
@@ -160,6 +174,7 @@ fp4_status quantize_impl(const void* x, int64_t rows, int64_t cols, int64_t ld, 
   p.rotated = rotated;
   p.error = d->scratch.error;
   p.four_six = four_six;
+  p.mx_thr = mx_thr;
   size_t fused_smem = 0;
   uint32_t fused_tiles = 0;
   if (fmt == FP4_NVFP4 && ts_in == nullptr && axis == 1 && ld == cols && !single_pass_disabled() &&
@@ -258,6 +273,46 @@ fp4_status fp4_quantize_2d(const void* x, int64_t rows, int64_t cols, int64_t ld
     }
   }
   return from_cuda(launch_quantize_2d(p, codes_t, scales_t, d->num_sms, st));
+}
+
+fp4_status fp4_quantize_mse(const void* x, int64_t rows, int64_t cols, int64_t ld, int fmt, int block, int rnd,
+                            uint64_t seed, int iters, float* tensor_scale_out, uint8_t* codes, uint8_t* scales,
+                            int sf_layout, void* stream) {
+  if (fmt != FP4_NVFP4) return fmt == FP4_MXFP4 ? FP4_ERR_UNSUPPORTED : FP4_ERR_ARG;
+  if (block != 16) return FP4_ERR_UNSUPPORTED;
+  fp4_status s = check_input(x, rows, cols, ld);
+  if (s != FP4_OK) return s;
+  if (rnd != FP4_RTN && rnd != FP4_SR) return FP4_ERR_ARG;
+  if (iters < 0 || iters > 8) return FP4_ERR_ARG;
+  if (sf_layout != FP4_SF_ROWMAJOR && sf_layout != FP4_SF_MMA) return FP4_ERR_ARG;
+  if (codes == nullptr || scales == nullptr || tensor_scale_out == nullptr) return FP4_ERR_ARG;
+  if (cols % 16 != 0) return FP4_ERR_SHAPE;
+  if (!aligned16(codes)) return FP4_ERR_ALIGN;
+  DeviceState* d = nullptr;
+  if ((s = device_state(&d)) != FP4_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int64_t g = cols / 16;
+  if (sf_layout == FP4_SF_MMA && (rows % 128 != 0 || g % 4 != 0) &&
+      cudaMemsetAsync(scales, 0, (size_t)(round_up(rows, 128) * round_up(g, 4)), st) != cudaSuccess)
+    return FP4_ERR_CUDA;
+  QuantizeParams p;
+  p.x = x;
+  p.rows = rows;
+  p.cols = cols;
+  p.ld = ld;
+  p.fmt = FMT_NV;
+  p.axis = 1;
+  p.rnd = rnd == FP4_RTN ? RND_RTN : RND_SR;
+  p.seed = seed;
+  p.codes = codes;
+  p.scales = scales;
+  p.sf_mma = sf_layout == FP4_SF_MMA;
+  p.had = 0;
+  p.rotated = nullptr;
+  p.error = d->scratch.error;
+  p.ts = nullptr;
+  p.ts_copy_out = nullptr;
+  return from_cuda(launch_quantize_mse(p, tensor_scale_out, iters, d->scratch, d->num_sms, st));
 }
 
 fp4_status fp4_dequantize(const uint8_t* codes, const uint8_t* scales, const float* tensor_scale, int64_t rows,

@@ -6,6 +6,7 @@
 // Way", Abstract; "Bridging the Gap ...", Abstract -- but print no encodings).
 #pragma once
 
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -155,6 +156,19 @@ __device__ __forceinline__ u32x4 philox4x32_10(uint32_t c0, uint32_t c1, const P
   return {c0, c1, c2, c3};
 }
 
+// Philox4x32-10 key schedule of a 64-bit seed: round i uses (lo + i * 0x9E3779B9, hi + i * 0xBB67AE85).
+inline PhiloxKeys philox_keys(unsigned long long seed) {
+  PhiloxKeys ks;
+  uint32_t k0 = (uint32_t)seed, k1 = (uint32_t)(seed >> 32);
+  for (int i = 0; i < 10; ++i) {
+    ks.k[2 * i] = k0;
+    ks.k[2 * i + 1] = k1;
+    k0 += 0x9E3779B9u;
+    k1 += 0xBB67AE85u;
+  }
+  return ks;
+}
+
 // Random words for 8 consecutive elements starting at linear index idx0
 // (idx0 % 8 == 0): two counters, words in index order.
 __device__ __forceinline__ void philox_words8(unsigned long long idx0, unsigned long long seed,
@@ -183,6 +197,18 @@ __device__ __forceinline__ uint32_t mx_scale_byte(float amax) {
   const int f = (int)((__float_as_uint(amax) >> 23) & 0xFFu);
   return (uint32_t)max(f - 2, 0);
 }
+// The same exponent under a clip threshold T in (4, 8]: E = floor(log2 amax) - 2, plus one when
+// amax > T * 2^(floor(log2 amax) - 2), i.e. when amax's significand field exceeds
+// thr = (T/4 - 1) * 2^23.  thr = 2^23 never triggers (T = 8, the rule above).
+__device__ __forceinline__ uint32_t mx_scale_byte_clip(float amax, uint32_t thr) {
+  const uint32_t b = __float_as_uint(amax);
+  const int f = (int)((b >> 23) & 0xFFu);
+  return (uint32_t)max(f - 2 + ((b & 0x7FFFFFu) > thr ? 1 : 0), 0);
+}
+// Significand threshold of the MSE-fitted clip T = 7.25 (T/4 = 1.8125 = 1 + 0x680000 / 2^23),
+// and of the OCP rule (T = 8).
+constexpr uint32_t kMxClipFitted = 0x680000u;
+constexpr uint32_t kMxClipOcp = 0x800000u;
 // 2^(127 - byte) = 1 / 2^E as an exact fp32 (byte <= 252 for finite bf16 input).
 __device__ __forceinline__ float mx_inv_scale(uint32_t byte) {
   return __uint_as_float((254u - byte) << 23);
@@ -248,6 +274,51 @@ __device__ __forceinline__ uint32_t e2m1x2_rn(float a, float b) {
       : "=r"(out)
       : "f"(a), "f"(b));
   return out;
+}
+
+// ------------------------------------------------------ NVFP4 blocks -----
+// Whether a block may divide by its scale S with div_by_recip (exact IEEE quotients) instead of
+// __fdiv_rn.  Both need y = RN(1/S) usable (S in [2^-125, 2^20], y != 0) and quotients below
+// 2^64.  Stochastic rounding uses the exact quotient of every element, so it also needs every
+// |x| >= 2^-103 (or 0), where the residuals are exact.  Round-to-nearest only needs the codes:
+// with S >= 2^-100 an element below 2^-103 has |x/S| < 2^-3, and div_by_recip keeps such a
+// quotient below 0.13 with the sign of x, so it rounds to a signed zero code exactly like the
+// correctly rounded quotient, while every larger element is divided exactly; that saves the
+// per-element test.  RND: 0 round-to-nearest, 1 stochastic rounding.
+template <int RND, int E>
+__device__ __forceinline__ bool nv_fast_division(const float (&x)[E], float am, float S, float y) {
+  if (y == 0.0f || !(__fmul_rn(am, y) < 0x1p64f)) return false;
+  if (RND == 0) return S >= 0x1p-100f;
+  uint32_t kmin = 0xFFFFFFFFu;
+#pragma unroll
+  for (int i = 0; i < E; ++i) kmin = min(kmin, tiny_key(x[i]));
+  return kmin >= kTinyKeyMin;
+}
+
+// Quotients q = x / S of one NVFP4 block under the divisor S = sy.x (sy.y = RN(1/S)): div_by_recip
+// when the block passes nv_fast_division's test for this rounding, IEEE division otherwise.  q may
+// alias x.
+template <int RND, int E>
+__device__ __forceinline__ void nv_divide_block(const float (&x)[E], float am, float2 sy, float (&q)[E]) {
+  if (nv_fast_division<RND, E>(x, am, sy.x, sy.y)) {
+#pragma unroll
+    for (int i = 0; i < E; ++i) q[i] = div_by_recip(x[i], sy.x, sy.y);
+  } else {                                       // rare: tiny operands or scales
+#pragma unroll
+    for (int i = 0; i < E; ++i) q[i] = __fdiv_rn(x[i], sy.x);
+  }
+}
+
+// Round-to-nearest dequantization of two quotients: fp32(fp32(G[c] * sbv) * s_t) for each, where
+// c is the E2M1 code of the quotient and g holds the block scale sbv in both halves.  G[c] * sbv
+// has at most 6 significant bits and lies in [2^-10, 2688], so the f16 product is exact.
+__device__ __forceinline__ float2 nv_rtn_dequant2(float q0, float q1, __half2 g, float s_t) {
+  uint32_t h;
+  asm("{\n\t.reg .b8 c;\n\tcvt.rn.satfinite.e2m1x2.f32 c, %2, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, c;\n\t}"
+      : "=r"(h)
+      : "f"(q0), "f"(q1));
+  const float2 v = __half22float2(__hmul2(*reinterpret_cast<const __half2*>(&h), g));
+  return make_float2(__fmul_rn(v.x, s_t), __fmul_rn(v.y, s_t));
 }
 
 // -------------------------------------------------- scale-factor offsets ----

@@ -64,8 +64,12 @@ struct Scratch {
   unsigned* error;      // device error word set by bounded waits
   unsigned* grid_arrive;  // arrivals at the single-pass NVFP4 quantizer's grid barrier (self-resetting)
   unsigned* grid_depart;  // departures from it; the last CTA out zeroes both
+  float* mse_amax;        // MSE-searched quantization: the tensor amax
+  unsigned long long* mse_partials;  // its tensor step: [kMaxMseCtas][17][2] per-CTA 128-bit sums
+  unsigned* mse_ticket;   // its tensor step's CTA completion counter (self-resetting)
 };
 constexpr int kMaxAmaxBlocks = 2048;
+constexpr int kMaxMseCtas = 1024;
 
 // Unsigned 32-bit division by a runtime constant (round-up multiplier method,
 // Hacker's Delight ch. 10): q = (umulhi(n, mul) + n) >> shift for n < 2^32.
@@ -88,6 +92,7 @@ struct QuantizeParams {
   float* rotated;         // optional fp32 dump of the rotated input
   unsigned* error;        // device error word
   int four_six = 0;       // NVFP4: four-over-six block scales
+  uint32_t mx_thr = 0x800000u;  // MXFP4 exponent clip threshold as a significand field (0x800000: OCP)
 };
 
 // amax pass: mode 0 writes max|x| (after rotation when had > 0) to `out`,
@@ -108,6 +113,10 @@ cudaError_t launch_quantize_2d(const QuantizeParams& p, uint8_t* codes_t, uint8_
 bool fused_nv_fits(int64_t rows, int64_t cols, int num_sms, size_t* smem, uint32_t* tiles_per_cta);
 cudaError_t launch_quantize_nv_fused(const QuantizeParams& p, float* ts_out, const Scratch& s, int num_sms,
                                      cudaStream_t st);
+// NVFP4 quantization (axis 1, block 16) with MSE-searched scales: amax pass, `iters` tensor-scale
+// steps, then the per-block byte search and the codes (RTN or SR per q.rnd).  Writes s_t to ts_out.
+cudaError_t launch_quantize_mse(const QuantizeParams& q, float* ts_out, int iters, const Scratch& s, int num_sms,
+                                cudaStream_t st);
 cudaError_t launch_dequantize(const uint8_t* codes, const uint8_t* scales, const float* ts, int64_t rows,
                               int64_t cols, int fmt, int sf_mma, void* out, int out_bf16, int num_sms,
                               cudaStream_t st);

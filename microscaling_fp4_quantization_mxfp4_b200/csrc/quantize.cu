@@ -147,6 +147,7 @@ struct QRowParams {
   uint32_t g4;           // padded k-groups / 4 (tensor-core scale layout)
   unsigned long long seed;
   PhiloxKeys keys;      // the seed's Philox key schedule
+  uint32_t mx_thr;      // MXFP4 exponent clip threshold (significand field; kMxClipOcp: the OCP rule)
   const float* ts;
   float* ts_copy_out;
   uint32_t* codes;       // [rows, cols/8] 32-bit words of 8 nibbles
@@ -171,50 +172,6 @@ struct BlockShape {
   static constexpr int E = FMT == FMT_MX ? 32 : 16;   // elements per block
   static constexpr int V = E / 8;                      // uint4 per block
 };
-
-// Whether a block may divide by its scale S with div_by_recip (exact IEEE quotients) instead of
-// __fdiv_rn.  Both need y = RN(1/S) usable (S in [2^-125, 2^20], y != 0) and quotients below
-// 2^64.  Stochastic rounding uses the exact quotient of every element, so it also needs every
-// |x| >= 2^-103 (or 0), where the residuals are exact.  Round-to-nearest only needs the codes:
-// with S >= 2^-100 an element below 2^-103 has |x/S| < 2^-3, and div_by_recip keeps such a
-// quotient below 0.13 with the sign of x, so it rounds to a signed zero code exactly like the
-// correctly rounded quotient, while every larger element is divided exactly; that saves the
-// per-element test.
-template <int RND, int E>
-__device__ __forceinline__ bool nv_fast_division(const float (&x)[E], float am, float S, float y) {
-  if (y == 0.0f || !(__fmul_rn(am, y) < 0x1p64f)) return false;
-  if (RND == RND_RTN) return S >= 0x1p-100f;
-  uint32_t kmin = 0xFFFFFFFFu;
-#pragma unroll
-  for (int i = 0; i < E; ++i) kmin = min(kmin, tiny_key(x[i]));
-  return kmin >= kTinyKeyMin;
-}
-
-// Quotients q = x / S of one NVFP4 block under the divisor S = sy.x (sy.y = RN(1/S)): div_by_recip
-// when the block passes nv_fast_division's test for this rounding, IEEE division otherwise.  q may
-// alias x.
-template <int RND, int E>
-__device__ __forceinline__ void nv_divide_block(const float (&x)[E], float am, float2 sy, float (&q)[E]) {
-  if (nv_fast_division<RND, E>(x, am, sy.x, sy.y)) {
-#pragma unroll
-    for (int i = 0; i < E; ++i) q[i] = div_by_recip(x[i], sy.x, sy.y);
-  } else {                                       // rare: tiny operands or scales
-#pragma unroll
-    for (int i = 0; i < E; ++i) q[i] = __fdiv_rn(x[i], sy.x);
-  }
-}
-
-// Round-to-nearest dequantization of two quotients: fp32(fp32(G[c] * sbv) * s_t) for each, where
-// c is the E2M1 code of the quotient and g holds the block scale sbv in both halves.  G[c] * sbv
-// has at most 6 significant bits and lies in [2^-10, 2688], so the f16 product is exact.
-__device__ __forceinline__ float2 nv_rtn_dequant2(float q0, float q1, __half2 g, float s_t) {
-  uint32_t h;
-  asm("{\n\t.reg .b8 c;\n\tcvt.rn.satfinite.e2m1x2.f32 c, %2, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, c;\n\t}"
-      : "=r"(h)
-      : "f"(q0), "f"(q1));
-  const float2 v = __half22float2(__hmul2(*reinterpret_cast<const __half2*>(&h), g));
-  return make_float2(__fmul_rn(v.x, s_t), __fmul_rn(v.y, s_t));
-}
 
 // Four-over-six ("Four Over Six", Abstract): of the standard scale byte byte6 (block max -> 6) and
 // the max -> 4 byte, the block takes the one whose round-to-nearest result has the lower squared
@@ -312,7 +269,7 @@ __device__ __forceinline__ void quantize_block(const QRowParams& p, const uint4 
   uint32_t byte;
   bool zero;
   if (FMT == FMT_MX) {
-    byte = mx_scale_byte(am);
+    byte = mx_scale_byte_clip(am, p.mx_thr);
     const float inv = mx_inv_scale(byte);
 #pragma unroll
     for (int i = 0; i < E; ++i) x[i] = __fmul_rn(x[i], inv);          // exact power-of-two scaling
@@ -793,6 +750,7 @@ struct QColParams {
   uint32_t G, g4;        // k-groups per output row (R / block) and padded/4
   unsigned long long seed;
   PhiloxKeys keys;      // the seed's Philox key schedule
+  uint32_t mx_thr;      // MXFP4 exponent clip threshold (significand field; kMxClipOcp: the OCP rule)
   const float* ts;
   float* ts_copy_out;
   uint8_t* codes;
@@ -852,7 +810,7 @@ __global__ void __launch_bounds__(256, 2) quantize_cols_kernel(QColParams p) {
       float inv = 1.0f, S = 1.0f, y = 1.0f;
       bool fast = true;
       if (FMT == FMT_MX) {
-        byte = mx_scale_byte(am);
+        byte = mx_scale_byte_clip(am, p.mx_thr);
         inv = mx_inv_scale(byte);
         zero = (am == 0.0f);
       } else {
@@ -944,6 +902,7 @@ struct Q2Params {
   int64_t ld;
   unsigned long long seed;
   PhiloxKeys keys;      // the seed's Philox key schedule
+  uint32_t mx_thr;      // MXFP4 exponent clip threshold (significand field; kMxClipOcp: the OCP rule)
   const float* ts;
   float* ts_copy_out;
   uint8_t* codes;        // [R, C/2]
@@ -1000,7 +959,7 @@ __global__ void __launch_bounds__(256) quantize_2d_kernel(Q2Params p) {
     uint32_t byte;
     bool zero;
     if (FMT == FMT_MX) {
-      byte = mx_scale_byte(am);
+      byte = mx_scale_byte_clip(am, p.mx_thr);
       const float inv = mx_inv_scale(byte);
 #pragma unroll
       for (int i = 0; i < BS; ++i) x[i] = __fmul_rn(x[i], inv);
@@ -1322,19 +1281,6 @@ cudaError_t launch_amax_fixed_grid(const void* x, int64_t rows, int64_t cols, in
   return launch_kernel(amax_kernel<0>, dim3(grid), dim3(256), 0, st, false, 1u, ap);
 }
 
-// Philox4x32-10 key schedule of a 64-bit seed: round i uses (lo + i * 0x9E3779B9, hi + i * 0xBB67AE85).
-static PhiloxKeys philox_keys(unsigned long long seed) {
-  PhiloxKeys ks;
-  uint32_t k0 = (uint32_t)seed, k1 = (uint32_t)(seed >> 32);
-  for (int i = 0; i < 10; ++i) {
-    ks.k[2 * i] = k0;
-    ks.k[2 * i + 1] = k1;
-    k0 += 0x9E3779B9u;
-    k1 += 0xBB67AE85u;
-  }
-  return ks;
-}
-
 cudaError_t launch_nv_tensor_scale(const float* amax, float* out, cudaStream_t st) {
   return launch_kernel(nv_tensor_scale_kernel, dim3(1), dim3(1), 0, st, false, 1u, amax, out);
 }
@@ -1423,6 +1369,7 @@ cudaError_t launch_quantize_nv_fused(const QuantizeParams& p, float* ts_out, con
   qp.g4 = (uint32_t)((p.cols / 16 + 3) / 4);
   qp.seed = p.seed;
   qp.keys = philox_keys(p.seed);
+  qp.mx_thr = p.mx_thr;
   qp.ts = nullptr;
   qp.ts_copy_out = nullptr;
   qp.codes = reinterpret_cast<uint32_t*>(p.codes);
@@ -1487,6 +1434,7 @@ cudaError_t launch_quantize(const QuantizeParams& p, int num_sms, cudaStream_t s
     qp.g4 = (uint32_t)((p.cols / bs + 3) / 4);
     qp.seed = p.seed;
     qp.keys = philox_keys(p.seed);
+    qp.mx_thr = p.mx_thr;
     qp.ts = p.ts;
     qp.ts_copy_out = p.ts_copy_out;
     qp.codes = reinterpret_cast<uint32_t*>(p.codes);
@@ -1513,6 +1461,7 @@ cudaError_t launch_quantize(const QuantizeParams& p, int num_sms, cudaStream_t s
   qp.g4 = (qp.G + 3u) / 4u;
   qp.seed = p.seed;
   qp.keys = philox_keys(p.seed);
+  qp.mx_thr = p.mx_thr;
   qp.ts = p.ts;
   qp.ts_copy_out = p.ts_copy_out;
   qp.codes = p.codes;
@@ -1555,6 +1504,7 @@ cudaError_t launch_quantize_2d(const QuantizeParams& p, uint8_t* codes_t, uint8_
   qp.ld = p.ld;
   qp.seed = p.seed;
   qp.keys = philox_keys(p.seed);
+  qp.mx_thr = p.mx_thr;
   qp.ts = p.ts;
   qp.ts_copy_out = p.ts_copy_out;
   qp.codes = p.codes;

@@ -102,3 +102,12 @@ def test_other_entry_points_reject_before_launch(lib):
     assert lib.fp4_hadamard_quantize(FAKE, 4, 64, 64, 2, 16, 1, 0, 0, None, FAKE, FAKE, FAKE, 0, 16, None, None) == -4
     assert lib.fp4_dequantize(FAKE, FAKE, FAKE, 4, 64, 2, 16, 0, FAKE, 0, None) == -1
     assert lib.fp4_gemm(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 4, 64, 2, 16, FAKE, 4, 0, None) == -1
+    # MXFP4 with the fitted clip threshold (fmt 3): block 32 only, quantizer entry points only
+    assert lib.fp4_quantize(FAKE, 4, 64, 64, 3, 16, 1, 0, 0, None, None, FAKE, FAKE, 0, None) == -4
+    assert lib.fp4_quantize_2d(FAKE, 64, 64, 64, 3, 32, 0, 0, None, None, FAKE, FAKE, None, None, 0, None) == -1
+    # fp4_quantize_mse: NVFP4 block 16 only, iters in [0, 8], s_t out required, cols % 16
+    assert lib.fp4_quantize_mse(FAKE, 4, 64, 64, 0, 32, 0, 0, 1, FAKE, FAKE, FAKE, 0, None) == -4
+    assert lib.fp4_quantize_mse(FAKE, 4, 64, 64, 1, 16, 0, 0, 9, FAKE, FAKE, FAKE, 0, None) == -1
+    assert lib.fp4_quantize_mse(FAKE, 4, 64, 64, 1, 16, 0, 0, 1, None, FAKE, FAKE, 0, None) == -1
+    assert lib.fp4_quantize_mse(FAKE, 4, 40, 40, 1, 16, 0, 0, 1, FAKE, FAKE, FAKE, 0, None) == -2
+    assert lib.fp4_quantize_mse(FAKE, 4, 64, 64, 1, 16, 2, 0, 1, FAKE, FAKE, FAKE, 0, None) == -1

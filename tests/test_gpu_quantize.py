@@ -434,3 +434,101 @@ def test_four_over_six_ties_and_extreme_magnitudes(rnd):
         q = F.fp4_quantize(dev_bf16(xe), fmt="nvfp4_4o6", rnd=rnd, seed=6)
         _four_six_check(q, xe, 1, rnd, 6, "rowmajor")
     F.fp4_check_device_errors()
+
+
+# ------------------------------------------------------------ MSE-fitted grid scales ---
+
+@pytest.mark.parametrize("axis", [1, 0])
+@pytest.mark.parametrize("rnd", ["rtn", "sr"])
+def test_quantize_mxfp4_clip_threshold(axis, rnd):
+    """MXFP4 with the MSE-fitted exponent clip threshold 7.25: codes and scales bit-exact, and the
+    threshold changes some block exponents against the OCP rule."""
+    rows, cols = 96, 256
+    xb = mixed_input(rows, cols, 501 + axis, "mxfp4")
+    q = F.fp4_quantize(dev_bf16(xb), fmt="mxfp4_gs", axis=axis, rnd=rnd, seed=5, sf_layout="mma")
+    ref = O.quantize(xb, fmt="mxfp4_gs", axis=axis, rnd=rnd, seed=5)
+    _check_against_oracle(q, ref, "mxfp4", axis, rows, cols, "mma")
+    assert np.any(ref["scales"] != O.quantize(xb, fmt="mxfp4", axis=axis, rnd=rnd, seed=5)["scales"])
+    F.fp4_check_device_errors()
+
+
+def test_hadamard_quantize_mxfp4_clip_threshold():
+    """The fixed grid scale is meant for MXFP4 behind block-Hadamard rotations: the quantizer applied
+    to the kernel's own rotated values is bit-exact (as for the other Hadamard parity tests)."""
+    rows, cols = 64, 1024
+    g = np.random.default_rng(77)
+    from workloads import bf16_bits
+    x = g.standard_normal((rows, cols)).astype(np.float32)
+    x[:, g.choice(cols, 10, replace=False)] *= 50.0
+    xb = bf16_bits(x)
+    rot = torch.empty((rows, cols), dtype=torch.float32, device="cuda")
+    q = F.fp4_hadamard_quantize(dev_bf16(xb), 128, fmt="mxfp4_gs", rotated_out=rot)
+    ref = O.quantize_values(host_f32(rot), fmt="mxfp4_gs")
+    np.testing.assert_array_equal(host_u8(q.codes), ref["codes"])
+    np.testing.assert_array_equal(host_u8(q.scales), ref["scales"])
+    F.fp4_check_device_errors()
+
+
+@pytest.mark.parametrize("shape, iters, rnd, sf", [
+    ((64, 256), 0, "rtn", "rowmajor"), ((64, 256), 0, "sr", "mma"), ((64, 256), 2, "rtn", "mma"),
+    ((200, 384), 1, "sr", "rowmajor"), ((200, 384), 1, "rtn", "mma"), ((7, 64), 1, "rtn", "rowmajor"),
+    ((129, 1024), 1, "sr", "mma")])
+def test_quantize_mse(shape, iters, rnd, sf):
+    """NVFP4 with MSE-searched block and tensor scales: codes, scales and s_t bit-exact."""
+    rows, cols = shape
+    xb = student_t_bf16_(shape, 40 + rows)
+    q = F.fp4_quantize_mse(dev_bf16(xb), rnd=rnd, seed=11, iters=iters, sf_layout=sf)
+    ref = O.quantize_mse(xb, rnd=rnd, seed=11, iters=iters)
+    _check_against_oracle(q, ref, "nvfp4", 1, rows, cols, sf)
+    F.fp4_check_device_errors()
+
+
+def student_t_bf16_(shape, seed):
+    from workloads import student_t_bf16
+    return student_t_bf16(shape, 3.0, 0.1, seed, 0)
+
+
+def test_quantize_mse_strided_and_tied_blocks():
+    """Strided rows (ld > cols) and blocks whose candidates tie exactly -- constant magnitudes exact
+    under several bytes, a block exact on a non-standard grid, zero and tiny blocks -- which the
+    kernel settles with exact fp64 errors in tie-break order."""
+    from workloads import bf16_bits
+    g = np.random.default_rng(9)
+    x = (g.standard_t(3, size=(32, 320)) * 0.1).astype(np.float32)
+    x[0, :16] = 0.65625                               # 2688 * 2^-12 (exact on the 6-grid)
+    x[1, :16] = np.float32(2.0 ** -6) * np.array([0, .5, 1, 1.5, 2, 3, 4, 4, -.5, -1, -2, -3, 1.5, .5, 3, -4])
+    x[2, :32] = np.where(g.random(32) < 0.5, -1.0, 1.0) * np.float32(0.125)   # +-c: exact under several bytes
+    x[3, :16] = 0.0
+    x[4, :16] = np.float32(1e-30)
+    xb = bf16_bits(x)
+    xt = dev_bf16(xb)[:, :256]
+    q = F.fp4_quantize_mse(xt, rnd="rtn", iters=1, sf_layout="mma")
+    ref = O.quantize_mse(np.ascontiguousarray(xb[:, :256]), rnd="rtn", iters=1)
+    _check_against_oracle(q, ref, "nvfp4", 1, 32, 256, "mma")
+    F.fp4_check_device_errors()
+
+
+def test_quantize_mse_full_size_properties():
+    """W[1024, 1024] ~ N(0, 0.02) with one tensor step (multi-CTA objective, grid-stride blocks):
+    the searched s_t is one of the 17 candidates of amax/2688, its exact objective is no larger than
+    that of amax/2688 itself, and 64 sampled rows carry the oracle's bytes and codes under it."""
+    from oracle import mse_grid as M
+    from workloads import normal_bf16
+    xb = normal_bf16((1024, 1024), 0.02, 42, 0)
+    q = F.fp4_quantize_mse(dev_bf16(xb), iters=1)
+    x32 = bf16_to_f32(xb)
+    s0 = O.nv_tensor_scale(x32)
+    s1 = host_f32(q.tensor_scale)[0]
+    assert s1 in set(M.tensor_candidates(s0).tolist())
+    x16 = x32.reshape(-1, 16)
+    P = M.objective_exponent(np.float32(np.max(np.abs(x32))))
+    assert M.tensor_objective(x16, M.block_step(x16, s1), s1, P) <= M.tensor_objective(x16, M.block_step(x16, s0), s0, P)
+    codes, scales = host_u8(q.codes), host_u8(q.scales)
+    for r in np.sort(np.random.default_rng(3).choice(1024, 64, replace=False)):
+        sb = M.block_step(x32[r].reshape(-1, 16), np.float32(s1))
+        np.testing.assert_array_equal(scales[r], sb)
+        S = (O.e4m3_decode(sb).astype(np.float32) * np.float32(s1)).astype(np.float32)
+        v = (x32[r].reshape(-1, 16) / S[:, None]).astype(np.float32)
+        c = np.where((sb == 0)[:, None], np.uint8(0), O.e2m1_rtn(v))
+        np.testing.assert_array_equal(codes[r], O.pack_nibbles(c.reshape(1, -1))[0])
+    F.fp4_check_device_errors()
