@@ -13,10 +13,10 @@
 //     the reduction is parallelised.
 // The schedule is s = amax / 2688, `iters` tensor steps, then a block step whose bytes quantize
 // the codes (RTN or Philox SR).  One thread owns one block.  Each candidate byte is first scored
-// in fp32 (exact quotients, dequantized values, one fma per element; a score is within 18u of the
-// exact error, relatively, plus 16 * 2^-150); only candidates within 2^-16 (+2^-120) of the best
-// score are then scored exactly in fp64, so the fp64 argmin is found without evaluating every
-// candidate in fp64.  Inputs are finite bf16.
+// in fp32 from quotients by the reciprocal (a multiply instead of a correctly rounded division);
+// only candidates that the screen's error bound cannot rule out are scored exactly (exact
+// quotients, fp64 errors), so the fp64 argmin is found without evaluating every candidate in fp64.
+// Inputs are finite bf16.
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -82,21 +82,32 @@ __device__ __forceinline__ void load_block(const MseParams& p, uint32_t blk, flo
   }
 }
 
-// fp32 score of byte b: exact round-to-nearest codes, dequantized, squares summed with fma.
-__device__ __forceinline__ float score32(const float (&x)[16], float am, uint32_t b, float s, const float2* tab) {
-  float q[16];
-  nv_divide_block<0, 16>(x, am, tab[b], q);
-  const __half2 g = __float2half2_rn(e4m3_value(b));
+// RTN grid points (signed E2M1 values) of two scaled values.
+__device__ __forceinline__ float2 e2m1_rtn_value2(float q0, float q1) {
+  uint32_t h;
+  asm("{\n\t.reg .b8 c;\n\tcvt.rn.satfinite.e2m1x2.f32 c, %2, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, c;\n\t}"
+      : "=r"(h)
+      : "f"(q0), "f"(q1));
+  return __half22float2(*reinterpret_cast<const __half2*>(&h));
+}
+
+// fp32 screen of the byte with divisor sy.x = S and sy.y = RN(1/S): quotients q = x * RN(1/S) (not
+// correctly rounded), their round-to-nearest grid points G(q), and S^2 * sum (q - G(q))^2.  The
+// squared distance to the nearest grid point is 1-Lipschitz in q, so against the exact error each
+// element is off by at most ~16.5u x^2 (u = 2^-24; q within 2u of x/S, the method's own quotient
+// and dequantized value within 6u), and the fp32 sums add 20u relatively.
+__device__ __forceinline__ float screen32(const float (&x)[16], float2 sy) {
   float f = 0.0f;
 #pragma unroll
   for (int i = 0; i < 16; i += 2) {
-    const float2 d = nv_rtn_dequant2(q[i], q[i + 1], g, s);
-    float e = __fsub_rn(x[i], d.x);
+    const float q0 = __fmul_rn(x[i], sy.y), q1 = __fmul_rn(x[i + 1], sy.y);
+    const float2 g = e2m1_rtn_value2(q0, q1);
+    float e = __fsub_rn(q0, g.x);
     f = __fmaf_rn(e, e, f);
-    e = __fsub_rn(x[i + 1], d.y);
+    e = __fsub_rn(q1, g.y);
     f = __fmaf_rn(e, e, f);
   }
-  return f;
+  return __fmul_rn(f, __fmul_rn(sy.x, sy.x));
 }
 
 // Exact error of byte b (0: the block dequantizes to 0): fp64 terms in element order.
@@ -130,22 +141,32 @@ __device__ __forceinline__ uint32_t block_byte(const float (&x)[16], float am, f
     if (want_err) *err = score64(x, am, 0u, s, tab);
     return 0u;
   }
+  // fp32 screen of every candidate (NaN marks a byte whose quotients the screen cannot bound:
+  // unusable reciprocal or huge quotients; it always goes to the exact stage)
+  float x2 = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) x2 = __fmaf_rn(x[i], x[i], x2);
   float f[kCands];
   float m = __int_as_float(0x7F800000);
 #pragma unroll
   for (int j = 0; j < kCands; ++j) {
     const int b = b6 + cand_offset(j);
-    f[j] = (b >= 1 && b <= 126) ? score32(x, am, (uint32_t)b, s, tab) : __int_as_float(0x7F800000);
-    m = fminf(m, f[j]);
+    float v = __int_as_float(0x7F800000);
+    if (b >= 1 && b <= 126) {
+      const float2 sy = tab[b];
+      v = (sy.y != 0.0f && __fmul_rn(am, sy.y) < 0x1p64f) ? screen32(x, sy) : __int_as_float(0x7FC00000);
+    }
+    f[j] = v;
+    m = fminf(m, v);
   }
-  // candidates whose exact error may be the least: not above the best score by more than
-  // 2^-16 of it plus 2^-120 (twice the fp32 scores' error bound, with room; an infinite or NaN best
-  // score keeps every candidate)
-  const float tol = __fmaf_rn(m, 0x1p-16f, 0x1p-120f);
+  // candidates whose exact error may be the least: a screen score exceeds the best one by more
+  // than 2^-16 (sum x^2 + both scores) + 2^-120 -- eight times the two scores' error bounds --
+  // only if its exact error is larger too; an infinite best score keeps every candidate
   int count = 0, first = 0;
 #pragma unroll
   for (int j = kCands - 1; j >= 0; --j) {
     const int b = b6 + cand_offset(j);
+    const float tol = __fmaf_rn(__fadd_rn(x2, __fadd_rn(m, f[j])), 0x1p-16f, 0x1p-120f);
     if (b >= 1 && b <= 126 && !(__fsub_rn(f[j], m) > tol)) {
       ++count;
       first = j;
@@ -166,7 +187,7 @@ __device__ __forceinline__ uint32_t block_byte(const float (&x)[16], float am, f
     float fj = 0.0f;
 #pragma unroll
     for (int t = 0; t < kCands; ++t) fj = (t == j) ? f[t] : fj;
-    if (__fsub_rn(fj, m) > tol) continue;
+    if (__fsub_rn(fj, m) > __fmaf_rn(__fadd_rn(x2, __fadd_rn(m, fj)), 0x1p-16f, 0x1p-120f)) continue;
     const double e = score64(x, am, (uint32_t)b, s, tab);
     if (!have || e < be) {
       be = e;
