@@ -362,6 +362,92 @@ class Nvfp2dWeight(Workload):
         return 512, f"512 of {self.rows} rows per step (global tensor scale), NumPy 1 thread"
 
 
+class NvfpMseWeight(Workload):
+    """NVFP4 quantization of a Llama MLP weight W[11008, 4096] ~ N(0, 0.02) with MSE-searched scales:
+    one tensor step (17 tensor scales, each with a 17-byte block step) and the final block step, RTN.
+    Bound by instruction issue, so its roofline counts candidate evaluations (one element quantized,
+    dequantized and its squared error accumulated under one candidate scale)."""
+
+    name = "nvfp4_mse_weight_11008x4096"
+    rows, cols = 11008, 4096
+    iters = 1
+    n_inputs = 2
+    launches_per_step = 3        # amax, tensor step, block step + codes
+    unit = "GB/s"
+    evals_per_element = 17 * 17 * 1 + 17       # tensor step(s) + final block step
+    instr_per_eval = 5           # quotient multiply, 1/2 E2M1 conversion, 1/2 back + widen, subtract, fma
+
+    def __init__(self, torch, F):
+        self.t, self.F = torch, F
+        n = self.rows * self.cols
+        self.n = n
+        self.step_bytes = n * (2 + 0.5 + 1 / 16)
+
+    def _bits(self):
+        from workloads import normal_bf16
+        return normal_bf16((self.rows, self.cols), 0.02, 12, 0)
+
+    def setup(self, device):
+        t = self.t
+        self.host_in = _pinned_bf16(t, self._bits())
+        self.x = [self.host_in.to(device).clone() for _ in range(self.n_inputs)]
+        self.dev_in = t.empty_like(self.x[0])
+        self.q = self.F.fp4_quantize_mse(self.x[0], iters=self.iters, sf_layout="mma")
+        self.timers = {"quantize_mse": KernelTimer(t)}
+
+    def single_kernel(self):
+        return ("quantize_mse",)
+
+    def family_bound(self, key):
+        return "alu"
+
+    def alu_peak(self, sms):
+        return sms * 128 * 1.965e9 / self.instr_per_eval, self.instr_per_eval
+
+    def step(self, i, timed=False, x=None):
+        x = self.x[i % self.n_inputs] if x is None else x
+        fn = lambda: self.F.fp4_quantize_mse(x, iters=self.iters, sf_layout="mma", codes=self.q.codes,
+                                             scales=self.q.scales, tensor_scale_out=self.q.tensor_scale)
+        return self.timers["quantize_mse"].around(fn) if timed else fn()
+
+    def outputs(self):
+        return [self.q.codes, self.q.scales, self.q.tensor_scale]
+
+    def e2e_step(self, host_outs):
+        self.dev_in.copy_(self.host_in, non_blocking=True)
+        self.step(0, x=self.dev_in)
+        for h, o in zip(host_outs, self.outputs()):
+            h.copy_(o, non_blocking=True)
+        return (self.host_in.numel() * 2, sum(o.numel() * o.element_size() for o in self.outputs()))
+
+    def family_work(self, key):
+        return self.n * self.evals_per_element
+
+    def value_from_ms(self, ms_per_step, n_ranks):
+        return self.step_bytes * n_ranks / (ms_per_step * 1e-3) / 1e9
+
+    def config(self):
+        return {"workload": self.name, "shape": [self.rows, self.cols], "format": "nvfp4", "block": 16,
+                "distribution": "normal(0, 0.02)", "seed": 12, "rounding": "rtn", "tensor_steps": self.iters,
+                "sf_layout": "mma", "algorithmic_bytes_per_step": self.step_bytes,
+                "candidate_evaluations_per_step": self.n * self.evals_per_element,
+                "l2": f"{self.n_inputs} rotating weight copies (180 MB)"}
+
+    def oracle_setup(self):
+        self.host_bits = self._bits()
+
+    def oracle_step(self, rows):
+        import oracle as O
+        O.quantize_mse(self.host_bits[:rows], iters=self.iters)
+        return rows * self.cols * (2 + 0.5 + 1 / 16)
+
+    def cpu_sample(self):
+        return 32, f"32 of {self.rows} rows searched on their own (tensor scale of the sample), NumPy (1 thread)"
+
+    def reference_sample(self):
+        return 8, f"8 of {self.rows} rows per step searched on their own, NumPy 1 thread"
+
+
 def _dev_bf16(torch, bits, device):
     return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(device)
 
@@ -765,8 +851,8 @@ class MxLinear128(GemmWorkload):
         return 128, "the whole workload: quantize X and W, fp64 GEMM (NumPy)"
 
 
-WORKLOADS = {W.name: W for W in (NvfpStudentT, NvfpStudentT46, Nvfp2dWeight, HadamardMxGemm, VitLinears,
-                                  LlamaNvfp4, MxLinear128)}
+WORKLOADS = {W.name: W for W in (NvfpStudentT, NvfpStudentT46, Nvfp2dWeight, NvfpMseWeight, HadamardMxGemm,
+                                  VitLinears, LlamaNvfp4, MxLinear128)}
 
 
 # ------------------------------------------------------------------ arms ---
@@ -882,6 +968,15 @@ def run_fp4(args):
                     "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": _load_traffic(W.name, dom),
                     "peak_source": peaks["source"] + " (bf16 burst x 4)",
                     "frac_of_sustained_peak": round(achieved / (4.0 * peaks["bf16_tflops_sustained"]), 4)}
+    elif W.family_bound(dom) == "alu":
+        # instruction-issue bound: work in candidate evaluations, peak = SMs x 4 sub-partitions x 32
+        # lanes x max SM clock / instructions per evaluation (see the workload's alu_peak)
+        sms = torch.cuda.get_device_properties(device).multi_processor_count
+        peak, per_eval = W.alu_peak(sms)
+        achieved = W.family_work(dom) / (dom_ms * 1e-3) / 1e9
+        roofline = {"kernel": dom, "bound": "alu", "achieved": round(achieved, 1), "peak": round(peak / 1e9, 1),
+                    "unit": "Geval/s", "frac": round(achieved * 1e9 / peak, 4), "traffic": _load_traffic(W.name, dom),
+                    "peak_source": f"derived: {sms} SMs x 128 lanes x 1965 MHz / {per_eval} instructions per evaluation"}
     else:
         achieved = W.family_work(dom) / (dom_ms * 1e-3) / 1e9
         roofline = {"kernel": dom, "bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
@@ -892,6 +987,8 @@ def run_fp4(args):
         work = W.family_work(k)
         if W.family_bound(k) == "tensor":
             per_family[k] = {"us_per_step": round(ms * 1e3, 2), "tflops": round(work / (ms * 1e-3) / 1e12, 1)}
+        elif W.family_bound(k) == "alu":
+            per_family[k] = {"us_per_step": round(ms * 1e3, 2), "geval_s": round(work / (ms * 1e-3) / 1e9, 1)}
         else:
             per_family[k] = {"us_per_step": round(ms * 1e3, 2), "gbs": round(work / (ms * 1e-3) / 1e9, 1)}
     roofline["per_kernel"] = per_family
