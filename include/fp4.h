@@ -227,6 +227,32 @@ fp4_status fp4_gemm(const uint8_t* a, const uint8_t* a_sf, const float* a_ts,
                     void* y, int64_t ldy, int y_dtype, void* stream);
 
 /*
+ * fp4_gemm_quantize -- the block-scaled FP4 GEMM whose epilogue emits the next
+ * layer's FP4 operand instead of Y ("Bridging the Gap", Abstract: FP4 kernels
+ * with the activations' transforms computed online, here applied across
+ * layers): Y = alpha * A . B^T as fp4_gemm computes it (fp32 accumulation,
+ * the fp32 value fp4_gemm would store), quantized along its rows -- the next
+ * GEMM's contraction axis -- with fp4_quantize's arithmetic, and never written.
+ *   a .. fmt, block   as fp4_gemm (operands).
+ *   out_fmt, out_block  (FP4_MXFP4, 32), (FP4_MXFP4_GS, 32) or (FP4_NVFP4, 16).
+ *   rnd, seed   FP4_RTN, or FP4_SR with Philox words of Y's row-major element
+ *               index (as fp4_quantize of a materialised Y[M, N]).
+ *   out_tensor_scale  NVFP4 output: device fp32 s_t to quantize under (required;
+ *               the amax of Y is not known until the GEMM ends, e.g. the
+ *               previous step's scale); ignored for MXFP4.
+ *   out_codes  uint8 [M, N/2], 16-byte aligned; out_scales in out_sf_layout
+ *              (FP4_SF_MMA feeds the next fp4_gemm directly).
+ * N must be a multiple of 32, K of 64.  Runs the single-SM or SM-pair GEMM
+ * kernels (never the split-K clusters).
+ */
+fp4_status fp4_gemm_quantize(const uint8_t* a, const uint8_t* a_sf, const float* a_ts,
+                             const uint8_t* b, const uint8_t* b_sf, const float* b_ts,
+                             int64_t M, int64_t N, int64_t K, int fmt, int block,
+                             int out_fmt, int out_block, int rnd, uint64_t seed,
+                             const float* out_tensor_scale, uint8_t* out_codes,
+                             uint8_t* out_scales, int out_sf_layout, void* stream);
+
+/*
  * fp4_amax -- max |x| over a bf16 matrix into one device fp32 (the first
  * pass of NVFP4's per-tensor scale, "FP4 All the Way", Abstract).  Used when
  * a tensor is sharded and the maxima are combined across ranks before

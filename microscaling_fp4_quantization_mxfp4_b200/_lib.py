@@ -18,6 +18,8 @@ PROTOTYPES = {
     "fp4_quantize_mse": (_int, [_vp, _i64, _i64, _i64, _int, _int, _int, _u64, _int, _vp, _vp, _vp, _int, _vp]),
     "fp4_dequantize": (_int, [_vp, _vp, _vp, _i64, _i64, _int, _int, _int, _vp, _int, _vp]),
     "fp4_gemm": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _int, _int, _vp, _i64, _int, _vp]),
+    "fp4_gemm_quantize": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _int, _int, _int, _int, _int, _u64,
+                                 _vp, _vp, _vp, _int, _vp]),
     "fp4_amax": (_int, [_vp, _i64, _i64, _i64, _vp, _vp]),
     "fp4_amax_noalloc": (_int, [_vp, _i64, _i64, _i64, _vp, _vp]),
     "fp4_nv_tensor_scale": (_int, [_vp, _vp, _vp]),

@@ -202,6 +202,33 @@ def fp4_gemm(a_codes: torch.Tensor, a_scales: torch.Tensor, b_codes: torch.Tenso
     return out
 
 
+def fp4_gemm_quantize(a_codes: torch.Tensor, a_scales: torch.Tensor, b_codes: torch.Tensor, b_scales: torch.Tensor,
+                      fmt="mxfp4", a_tensor_scale=None, b_tensor_scale=None, out_fmt="mxfp4", rnd="rtn", seed: int = 0,
+                      out_tensor_scale: Optional[torch.Tensor] = None, out_sf_layout="mma", *, codes=None, scales=None,
+                      stream=None) -> Fp4Quantized:
+    """Y = alpha * A . B^T quantized along its rows in the GEMM epilogue (see fp4_gemm_quantize in
+    include/fp4.h): the next layer's FP4 operand, Y itself never written."""
+    for t, n in ((a_codes, "a_codes"), (b_codes, "b_codes"), (a_scales, "a_scales"), (b_scales, "b_scales")):
+        _need_cuda(t, n)
+    f, of, r, sf = _FMT[fmt], _FMT[out_fmt], _RND[rnd], _SF[out_sf_layout]
+    M, kb = a_codes.shape
+    N, kb2 = b_codes.shape
+    if kb != kb2:
+        raise ValueError("A and B must have the same K")
+    if codes is None:
+        codes = torch.empty((M, N // 2), dtype=torch.uint8, device=a_codes.device)
+    if scales is None:
+        nbytes = fp4_scales_bytes(M, N, BLOCK[of], 1, sf)
+        shape = (M, N // BLOCK[of]) if sf == SF_ROWMAJOR else (nbytes,)
+        scales = torch.empty(shape, dtype=torch.uint8, device=a_codes.device)
+    st = _lib.load().fp4_gemm_quantize(
+        a_codes.data_ptr(), a_scales.data_ptr(), _ptr(a_tensor_scale), b_codes.data_ptr(), b_scales.data_ptr(),
+        _ptr(b_tensor_scale), M, N, 2 * kb, f, BLOCK[f], of, BLOCK[of], r, seed & (2 ** 64 - 1),
+        _ptr(out_tensor_scale), codes.data_ptr(), scales.data_ptr(), sf, _stream(stream))
+    _check(st, "fp4_gemm_quantize")
+    return Fp4Quantized(codes, scales, out_tensor_scale if of == NVFP4 else None)
+
+
 def fp4_amax(x: torch.Tensor, *, out=None, stream=None) -> torch.Tensor:
     """max |x| of a bf16 matrix as a device fp32 [1]."""
     _bf16_matrix(x)

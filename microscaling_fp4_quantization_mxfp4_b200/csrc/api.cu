@@ -369,6 +369,70 @@ fp4_status fp4_gemm(const uint8_t* a, const uint8_t* a_sf, const float* a_ts, co
   return from_cuda(e);
 }
 
+fp4_status fp4_gemm_quantize(const uint8_t* a, const uint8_t* a_sf, const float* a_ts, const uint8_t* b,
+                             const uint8_t* b_sf, const float* b_ts, int64_t M, int64_t N, int64_t K, int fmt,
+                             int block, int out_fmt, int out_block, int rnd, uint64_t seed, const float* out_tensor_scale,
+                             uint8_t* out_codes, uint8_t* out_scales, int out_sf_layout, void* stream) {
+  fp4_status s = check_format(fmt, block);
+  if (s != FP4_OK) return s;
+  uint32_t mx_thr = 0x800000u;
+  int q_out = 0;
+  if (out_fmt == FP4_MXFP4 || out_fmt == FP4_MXFP4_GS) {
+    if (out_block != 32) return FP4_ERR_UNSUPPORTED;
+    q_out = 1;
+    if (out_fmt == FP4_MXFP4_GS) mx_thr = 0x680000u;
+  } else if (out_fmt == FP4_NVFP4) {
+    if (out_block != 16) return FP4_ERR_UNSUPPORTED;
+    if (out_tensor_scale == nullptr) return FP4_ERR_ARG;
+    q_out = 2;
+  } else {
+    return FP4_ERR_ARG;
+  }
+  if (a == nullptr || a_sf == nullptr || b == nullptr || b_sf == nullptr) return FP4_ERR_ARG;
+  if (out_codes == nullptr || out_scales == nullptr) return FP4_ERR_ARG;
+  if (fmt == FP4_NVFP4 && (a_ts == nullptr || b_ts == nullptr)) return FP4_ERR_ARG;
+  if (rnd != FP4_RTN && rnd != FP4_SR) return FP4_ERR_ARG;
+  if (out_sf_layout != FP4_SF_ROWMAJOR && out_sf_layout != FP4_SF_MMA) return FP4_ERR_ARG;
+  if (M <= 0 || N <= 0 || K <= 0) return FP4_ERR_ARG;
+  if (K % 64 != 0 || N % 32 != 0) return FP4_ERR_SHAPE;
+  if (M >= (int64_t)1 << 31 || N >= (int64_t)1 << 31 || K >= (int64_t)1 << 31) return FP4_ERR_SHAPE;
+  if (!aligned16(a) || !aligned16(b) || !aligned16(a_sf) || !aligned16(b_sf) || !aligned16(out_codes))
+    return FP4_ERR_ALIGN;
+  DeviceState* d = nullptr;
+  if ((s = device_state(&d)) != FP4_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int64_t g = N / out_block;
+  if (out_sf_layout == FP4_SF_MMA && (M % 128 != 0 || g % 4 != 0) &&
+      cudaMemsetAsync(out_scales, 0, (size_t)(round_up(M, 128) * round_up(g, 4)), st) != cudaSuccess)
+    return FP4_ERR_CUDA;
+  GemmParams p;
+  p.a = a;
+  p.a_sf = a_sf;
+  p.a_ts = a_ts;
+  p.b = b;
+  p.b_sf = b_sf;
+  p.b_ts = b_ts;
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.fmt = fmt == FP4_MXFP4 ? FMT_MX : FMT_NV;
+  p.y = nullptr;
+  p.ldy = N;
+  p.y_bf16 = 0;
+  p.error = d->scratch.error;
+  p.q_out = q_out;
+  p.q_codes = out_codes;
+  p.q_scales = out_scales;
+  p.q_ts = out_tensor_scale;
+  p.q_sf_mma = out_sf_layout == FP4_SF_MMA;
+  p.q_rnd = rnd == FP4_SR;
+  p.q_seed = seed;
+  p.q_mx_thr = mx_thr;
+  cudaError_t e = launch_gemm(p, d->num_sms, st);
+  if (e == cudaErrorNotSupported) return FP4_ERR_UNSUPPORTED;
+  return from_cuda(e);
+}
+
 fp4_status fp4_amax(const void* x, int64_t rows, int64_t cols, int64_t ld, float* amax_out, void* stream) {
   fp4_status s = check_input(x, rows, cols, ld);
   if (s != FP4_OK) return s;

@@ -134,6 +134,16 @@ struct GemmParams {
   int64_t ldy;
   int y_bf16;
   unsigned* error;
+  // fused quantization of Y along its rows instead of storing it: 0 (store Y), 1 (MXFP4 codes),
+  // 2 (NVFP4 codes under the tensor scale q_ts)
+  int q_out = 0;
+  uint8_t* q_codes = nullptr;
+  uint8_t* q_scales = nullptr;
+  const float* q_ts = nullptr;
+  int q_sf_mma = 0;
+  int q_rnd = 0;
+  uint64_t q_seed = 0;
+  uint32_t q_mx_thr = 0x800000u;
 };
 // Returns cudaErrorNotSupported if the driver entry point for tensor maps is missing.
 cudaError_t launch_gemm(const GemmParams& p, int num_sms, cudaStream_t st);

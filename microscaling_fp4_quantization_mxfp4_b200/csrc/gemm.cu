@@ -42,6 +42,7 @@
 #include <algorithm>
 #include <mutex>
 
+#include "fp4_device.cuh"
 #include "fp4_internal.h"
 
 namespace fp4lib {
@@ -302,7 +303,79 @@ struct KernelArgs {
   int vec_store;          // output rows 16-byte aligned: 128-bit stores
   int tma_store;          // bf16 output through shared memory and TMA stores (tensor map valid)
   unsigned* error;
+  // fused quantization of Y along its rows (kernels with QO != 0): codes [M, N/2], scale bytes in
+  // the row-major or tensor-core layout, NVFP4 tensor scale (QO = 2), rounding, MX clip threshold
+  uint8_t* q_codes;
+  uint8_t* q_scales;
+  const float* q_ts;
+  int q_sf_mma, q_g4, q_rnd;
+  uint32_t q_mx_thr;
+  fp4dev::PhiloxKeys q_keys;
 };
+
+// Byte offset of the scale of (row m, group g) of the quantized Y.
+__device__ __forceinline__ long long q_sf_offset(const KernelArgs& p, int m, int g, int groups) {
+  return p.q_sf_mma ? fp4dev::sf_mma_offset(m, g, p.q_g4) : (long long)m * groups + g;
+}
+
+// Eight codes of scaled values v[0..7] with RTN or SR (Philox word of element idx0 + i, idx0 % 8 == 0).
+__device__ __forceinline__ uint32_t q_codes8(const KernelArgs& p, const float* v, unsigned long long idx0) {
+  if (!p.q_rnd) return fp4dev::e2m1x4_rn(v[0], v[1], v[2], v[3], v[4], v[5], v[6], v[7]);
+  const unsigned long long j = idx0 >> 2;
+  const fp4dev::u32x4 a = fp4dev::philox4x32_10((uint32_t)j, (uint32_t)(j >> 32), p.q_keys);
+  const fp4dev::u32x4 b = fp4dev::philox4x32_10((uint32_t)(j + 1), (uint32_t)((j + 1) >> 32), p.q_keys);
+  const uint32_t n[8] = {fp4dev::e2m1_sr(v[0], a.x), fp4dev::e2m1_sr(v[1], a.y), fp4dev::e2m1_sr(v[2], a.z),
+                         fp4dev::e2m1_sr(v[3], a.w), fp4dev::e2m1_sr(v[4], b.x), fp4dev::e2m1_sr(v[5], b.y),
+                         fp4dev::e2m1_sr(v[6], b.z), fp4dev::e2m1_sr(v[7], b.w)};
+  return fp4dev::pack8_nibbles(n);
+}
+
+// Fused output quantization of one thread's 32 accumulator columns n0 .. n0+31 of row m
+// (rc: fp32 bit patterns, overwritten): y = alpha * acc is the value the fp32 output would hold;
+// blocks run along the row (the next GEMM's contraction axis) with the quantizers' arithmetic --
+// QO = 1: one MXFP4 block of 32 (E8M0 exponent with clip threshold q_mx_thr); QO = 2: two NVFP4
+// blocks of 16 under the given tensor scale st (y_st = RN(1/st), st_ok = recip_usable(st)).
+template <int QO>
+__device__ __forceinline__ void epi_quantize32(const KernelArgs& p, uint32_t (&rc)[32], float alpha, float st,
+                                               float y_st, bool st_ok, int m, int n0) {
+  float v[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __fmul_rn(__uint_as_float(rc[i]), alpha);
+  const unsigned long long idx0 = (unsigned long long)m * (unsigned)p.N + (unsigned)n0;
+  uint32_t w[4];
+  if (QO == 1) {
+    float am = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) am = fmaxf(am, fabsf(v[i]));
+    const uint32_t byte = fp4dev::mx_scale_byte_clip(am, p.q_mx_thr);
+    const float inv = fp4dev::mx_inv_scale(byte);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __fmul_rn(v[i], inv);           // exact power-of-two scaling
+#pragma unroll
+    for (int k = 0; k < 4; ++k) w[k] = am == 0.0f ? 0u : q_codes8(p, v + 8 * k, idx0 + 8 * k);
+    p.q_scales[q_sf_offset(p, m, n0 / 32, p.N / 32)] = (uint8_t)byte;
+  } else {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      float x[16];
+      float am = 0.0f;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        x[i] = v[16 * h + i];
+        am = fmaxf(am, fabsf(x[i]));
+      }
+      const uint32_t byte = fp4dev::e4m3_rn_sat(fp4dev::nv_scale_arg(am, st, y_st, st_ok));
+      const float S = byte == 0u ? 1.0f : __fmul_rn(fp4dev::e4m3_value(byte), st);
+      const float2 sy = make_float2(S, fp4dev::recip_usable(S) ? __frcp_rn(S) : 0.0f);
+      if (p.q_rnd) fp4dev::nv_divide_block<1, 16>(x, am, sy, x);
+      else fp4dev::nv_divide_block<0, 16>(x, am, sy, x);
+#pragma unroll
+      for (int k = 0; k < 2; ++k) w[2 * h + k] = byte == 0u ? 0u : q_codes8(p, x + 8 * k, idx0 + 16 * h + 8 * k);
+      p.q_scales[q_sf_offset(p, m, n0 / 16 + h, p.N / 16)] = (uint8_t)byte;
+    }
+  }
+  *reinterpret_cast<uint4*>(p.q_codes + (size_t)m * (unsigned)(p.N / 2) + n0 / 2) = make_uint4(w[0], w[1], w[2], w[3]);
+}
 
 __device__ __forceinline__ void tile_coords(int t, int num_m, int num_n, int& mt, int& nt) {
   constexpr int kGroup = 8;
@@ -314,7 +387,7 @@ __device__ __forceinline__ void tile_coords(int t, int num_m, int num_n, int& mt
   nt = local / gsize;
 }
 
-template <int BN, int FMT, bool BF16>
+template <int BN, int FMT, bool BF16, int QO = 0>
 __global__ void __launch_bounds__(Cfg<BN, FMT>::kThreads, 1)
     fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                     const __grid_constant__ CUtensorMap tmap_y, KernelArgs p) {
@@ -552,6 +625,9 @@ __global__ void __launch_bounds__(Cfg<BN, FMT>::kThreads, 1)
     const int col0 = ((warp - 2) / 4) * 128;
     const int row_in_tile = q * 32 + lane;
     const float alpha = FMT == FMT_NV ? __fmul_rn(*p.a_ts, *p.b_ts) : 1.0f;
+    const float q_st = QO == 2 ? *p.q_ts : 1.0f;
+    const float q_yst = __frcp_rn(q_st);
+    const bool q_stok = fp4dev::recip_usable(q_st);
     int local = 0;
     for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++local) {
       int mt, nt;
@@ -574,6 +650,18 @@ __global__ void __launch_bounds__(Cfg<BN, FMT>::kThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&tempty[acc]));
+      if (QO != 0) {
+        const int m = mt * BM + row_in_tile;
+        if (m < p.M) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const int n0 = nt * BN + col0 + 32 * c;
+            if (n0 >= p.N) break;
+            epi_quantize32<QO>(p, r[c], alpha, q_st, q_yst, q_stok, m, n0);
+          }
+        }
+        continue;
+      }
       if (BF16 && p.tma_store) {
         epi_store_bf16_tma(&tmap_y, sEpi + (warp - 2) * kEpiStage, r, alpha, nt * BN + col0, mt * BM + q * 32, p.M,
                            p.N, lane);
@@ -731,7 +819,7 @@ __device__ __forceinline__ void tc_mma_pair(uint32_t d, uint64_t adesc, uint64_t
   }
 }
 
-template <int BN, int FMT, bool BF16>
+template <int BN, int FMT, bool BF16, int QO = 0>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg2<BN, FMT>::kThreads, 1)
     fp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                          const __grid_constant__ CUtensorMap tmap_sfa, const __grid_constant__ CUtensorMap tmap_sfb,
@@ -941,6 +1029,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg2<BN, FMT>::kThre
     const int col0 = ((warp - 2) / 4) * 128;
     const int row_in_tile = (int)rank * 128 + q * 32 + lane;
     const float alpha = FMT == FMT_NV ? __fmul_rn(*p.a_ts, *p.b_ts) : 1.0f;
+    const float q_st = QO == 2 ? *p.q_ts : 1.0f;
+    const float q_yst = __frcp_rn(q_st);
+    const bool q_stok = fp4dev::recip_usable(q_st);
     int local = 0;
     for (int t = cluster; t < num_tiles; t += nclusters, ++local) {
       int mt, nt;
@@ -965,6 +1056,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg2<BN, FMT>::kThre
       __syncwarp();
       if (lane == 0) mbar_arrive_remote(tempty_leader);
       const int m = mt * 256 + row_in_tile;
+      if (QO != 0) {
+        if (m < p.M) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const int n0 = nt * BN + col0 + 32 * c;
+            if (n0 >= p.N) break;
+            epi_quantize32<QO>(p, r[c], alpha, q_st, q_yst, q_stok, m, n0);
+          }
+        }
+        continue;
+      }
       if (m < p.M) {
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
@@ -1390,11 +1492,24 @@ bool make_y_map(CUtensorMap* map, const GemmParams& gp) {
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int BN, int FMT, bool BF16>
+// The fused-quantization fields of the kernel arguments.
+void fill_quant_args(KernelArgs& ka, const GemmParams& gp) {
+  ka.q_codes = gp.q_codes;
+  ka.q_scales = gp.q_scales;
+  ka.q_ts = gp.q_ts;
+  ka.q_sf_mma = gp.q_sf_mma;
+  const int64_t bs = gp.q_out == 1 ? 32 : 16;
+  ka.q_g4 = (int)((gp.N / bs + 3) / 4);
+  ka.q_rnd = gp.q_rnd;
+  ka.q_mx_thr = gp.q_mx_thr;
+  ka.q_keys = fp4dev::philox_keys(gp.q_seed);
+}
+
+template <int BN, int FMT, bool BF16, int QO = 0>
 cudaError_t run_pair(const GemmParams& gp, int num_sms, cudaStream_t st) {
   using C = pair::Cfg2<BN, FMT>;
   static_assert(C::kStages >= 2, "shared memory too small for two stages");
-  auto kernel = pair::fp4_gemm_pair_kernel<BN, FMT, BF16>;
+  auto kernel = pair::fp4_gemm_pair_kernel<BN, FMT, BF16, QO>;
   static const cudaError_t attr =
       cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (attr != cudaSuccess) return attr;
@@ -1424,6 +1539,7 @@ cudaError_t run_pair(const GemmParams& gp, int num_sms, cudaStream_t st) {
     ka.vec_store = ((gp.ldy * esz) % 16 == 0 && (reinterpret_cast<uintptr_t>(gp.y) & 15u) == 0) ? 1 : 0;
   }
   ka.tma_store = 0;
+  fill_quant_args(ka, gp);
   const int tiles = ka.num_m * ka.num_n;
   int clusters = num_sms / 2;
   if (tiles < clusters) clusters = tiles;
@@ -1431,11 +1547,11 @@ cudaError_t run_pair(const GemmParams& gp, int num_sms, cudaStream_t st) {
                        ka);
 }
 
-template <int BN, int FMT, bool BF16>
+template <int BN, int FMT, bool BF16, int QO = 0>
 cudaError_t run(const GemmParams& gp, int num_sms, cudaStream_t st) {
   using C = Cfg<BN, FMT>;
   static_assert(C::kStages >= 2, "shared memory too small for two stages");
-  static const cudaError_t attr = cudaFuncSetAttribute(fp4_gemm_kernel<BN, FMT, BF16>,
+  static const cudaError_t attr = cudaFuncSetAttribute(fp4_gemm_kernel<BN, FMT, BF16, QO>,
                                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (attr != cudaSuccess) return attr;
   CUtensorMap ta, tb;
@@ -1461,11 +1577,12 @@ cudaError_t run(const GemmParams& gp, int num_sms, cudaStream_t st) {
   }
   CUtensorMap ty;
   memset(&ty, 0, sizeof(ty));
-  ka.tma_store = make_y_map(&ty, gp) ? 1 : 0;
+  ka.tma_store = QO == 0 && make_y_map(&ty, gp) ? 1 : 0;
+  fill_quant_args(ka, gp);
   const int tiles = ka.num_m * ka.num_n;
   const int grid = tiles < num_sms ? tiles : num_sms;
-  return launch_kernel(fp4_gemm_kernel<BN, FMT, BF16>, dim3(grid), dim3(C::kThreads), C::kSmemBytes, st, false, 1u,
-                       ta, tb, ty, ka);
+  return launch_kernel(fp4_gemm_kernel<BN, FMT, BF16, QO>, dim3(grid), dim3(C::kThreads), C::kSmemBytes, st, false,
+                       1u, ta, tb, ty, ka);
 }
 
 // Clusters of `split` CTAs of this kernel that the device can hold at once (0 if unknown).
@@ -1560,6 +1677,18 @@ static cudaError_t dispatch_pair(const GemmParams& p, int num_sms, cudaStream_t 
   return p.y_bf16 ? run_pair<BN, FMT_NV, true>(p, num_sms, st) : run_pair<BN, FMT_NV, false>(p, num_sms, st);
 }
 
+// Fused-quantization variants: the pair or single-SM kernel by the same rule as launch_gemm,
+// never split-K (its cross-CTA reduction would need its own quantizing epilogue).
+template <int QO>
+static cudaError_t dispatch_quant(const GemmParams& p, bool pair_tiles, int bn, int num_sms, cudaStream_t st) {
+  if (pair_tiles)
+    return p.fmt == FMT_MX ? run_pair<256, FMT_MX, false, QO>(p, num_sms, st)
+                           : run_pair<256, FMT_NV, false, QO>(p, num_sms, st);
+  if (bn == 256)
+    return p.fmt == FMT_MX ? run<256, FMT_MX, false, QO>(p, num_sms, st) : run<256, FMT_NV, false, QO>(p, num_sms, st);
+  return p.fmt == FMT_MX ? run<128, FMT_MX, false, QO>(p, num_sms, st) : run<128, FMT_NV, false, QO>(p, num_sms, st);
+}
+
 cudaError_t launch_gemm(const GemmParams& p, int num_sms, cudaStream_t st) {
   // Tuning overrides: FP4_GEMM_BN=128|256 (tile width), FP4_GEMM_PAIR=0|1 (SM-pair kernel off/forced).
   static const int forced_bn = [] {
@@ -1578,6 +1707,12 @@ cudaError_t launch_gemm(const GemmParams& p, int num_sms, cudaStream_t st) {
   const int pair_bn = forced_bn ? forced_bn : 256;
   const bool pair_auto = p.K >= 2048 && p.M >= 256 && p.N >= 256 &&
                          ((p.M + 255) / 256) * ((p.N + pair_bn - 1) / pair_bn) >= num_sms / 2;
+  if (p.q_out != 0) {
+    const bool pair_tiles = pair_mode != 0 && p.K % 256 == 0 && (pair_mode == 1 || pair_auto) && pair_bn == 256;
+    const int qbn = forced_bn ? forced_bn : (p.N >= 256 ? 256 : 128);
+    return p.q_out == 1 ? dispatch_quant<1>(p, pair_tiles, qbn, num_sms, st)
+                        : dispatch_quant<2>(p, pair_tiles, qbn, num_sms, st);
+  }
   if (pair_mode != 0 && p.K % 256 == 0 && (pair_mode == 1 || pair_auto))
     return pair_bn == 256 ? dispatch_pair<256>(p, num_sms, st) : dispatch_pair<128>(p, num_sms, st);
   const int bn = forced_bn ? forced_bn : (p.N >= 256 ? 256 : 128);

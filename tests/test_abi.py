@@ -111,3 +111,14 @@ def test_other_entry_points_reject_before_launch(lib):
     assert lib.fp4_quantize_mse(FAKE, 4, 64, 64, 1, 16, 0, 0, 1, None, FAKE, FAKE, 0, None) == -1
     assert lib.fp4_quantize_mse(FAKE, 4, 40, 40, 1, 16, 0, 0, 1, FAKE, FAKE, FAKE, 0, None) == -2
     assert lib.fp4_quantize_mse(FAKE, 4, 64, 64, 1, 16, 2, 0, 1, FAKE, FAKE, FAKE, 0, None) == -1
+    # fp4_gemm_quantize: N % 32, NV output needs a tensor scale, output (format, block) pairs
+    assert lib.fp4_gemm_quantize(FAKE, FAKE, None, FAKE, FAKE, None, 4, 48, 64, 0, 32, 0, 32, 0, 0, None, FAKE, FAKE,
+                                 1, None) == -2
+    assert lib.fp4_gemm_quantize(FAKE, FAKE, None, FAKE, FAKE, None, 4, 64, 64, 0, 32, 1, 16, 0, 0, None, FAKE, FAKE,
+                                 1, None) == -1
+    assert lib.fp4_gemm_quantize(FAKE, FAKE, None, FAKE, FAKE, None, 4, 64, 64, 0, 32, 0, 16, 0, 0, None, FAKE, FAKE,
+                                 1, None) == -4
+    assert lib.fp4_gemm_quantize(FAKE, FAKE, None, FAKE, FAKE, None, 4, 64, 64, 0, 32, 2, 16, 0, 0, FAKE, FAKE, FAKE,
+                                 1, None) == -1
+    assert lib.fp4_gemm_quantize(FAKE, FAKE, None, FAKE, FAKE, None, 4, 64, 64, 0, 32, 0, 32, 0, 0, None, FAKE + 8,
+                                 FAKE, 1, None) == -3
