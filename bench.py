@@ -556,6 +556,87 @@ class HadamardMxGemm(GemmWorkload):
         return 16, "b = 128: rotate+quantize 16 rows of X and their fp64 GEMM against 256 rows of W (NumPy)"
 
 
+class FusedMxLinear(GemmWorkload):
+    """One MXFP4 linear of an FP4 pipeline: Y = X W^T with X[8192,4096] ~ N(0,1) and W[11008,4096] ~
+    N(0,0.02) as resident MXFP4 operands, whose epilogue quantizes Y (RTN, MXFP4) into the next
+    layer's codes and tensor-core-layout scales; Y itself is never written."""
+
+    name = "mxfp4_fused_linear_8192x11008x4096"
+    M, N, K = 8192, 11008, 4096
+    launches_per_step = 1
+
+    def __init__(self, torch, F):
+        self.t, self.F = torch, F
+        self.step_flops = 2.0 * self.M * self.N * self.K
+
+    def setup(self, device):
+        from workloads import normal_bf16
+        t, F = self.t, self.F
+        xb, wb = normal_bf16((self.M, self.K), 1.0, 13, 0), normal_bf16((self.N, self.K), 0.02, 13, 1)
+        self.host_in = (_pinned_bf16(t, xb), _pinned_bf16(t, wb))
+        self.dev_in = tuple(t.empty_like(h, device=device) for h in self.host_in)
+        self.qx = F.fp4_quantize(self.host_in[0].to(device), fmt="mxfp4", sf_layout="mma")
+        self.qw = F.fp4_quantize(self.host_in[1].to(device), fmt="mxfp4", sf_layout="mma")
+        self.codes = t.empty((self.M, self.N // 2), dtype=t.uint8, device=device)
+        self.scales = t.empty((F.fp4_scales_bytes(self.M, self.N, 32, 1, "mma"),), dtype=t.uint8, device=device)
+        self.outs = [self.codes, self.scales]
+        self.timers = {"gemm_quantize": KernelTimer(t), "quantize": KernelTimer(t)}
+
+    def single_kernel(self):
+        return ("gemm_quantize",)
+
+    def family_bound(self, key):
+        return "tensor" if key == "gemm_quantize" else "hbm"
+
+    def step(self, i, timed=False, q=None):
+        F = self.F
+        qx, qw = (self.qx, self.qw) if q is None else q
+        fn = lambda: F.fp4_gemm_quantize(qx.codes, qx.scales, qw.codes, qw.scales, fmt="mxfp4", out_fmt="mxfp4",
+                                         codes=self.codes, scales=self.scales)
+        return self.timers["gemm_quantize"].around(fn) if timed else fn()
+
+    def e2e_step(self, host_outs):
+        # end to end: bf16 X and W from pinned host memory, both quantized, the fused linear, codes
+        # and scales back
+        F = self.F
+        for h, d in zip(self.host_in, self.dev_in):
+            d.copy_(h, non_blocking=True)
+        qx = F.fp4_quantize(self.dev_in[0], fmt="mxfp4", sf_layout="mma", codes=self.qx.codes, scales=self.qx.scales)
+        qw = F.fp4_quantize(self.dev_in[1], fmt="mxfp4", sf_layout="mma", codes=self.qw.codes, scales=self.qw.scales)
+        self.step(0, q=(qx, qw))
+        for h, o in zip(host_outs, self.outs):
+            h.copy_(o, non_blocking=True)
+        return (sum(h.numel() * 2 for h in self.host_in), sum(o.numel() for o in self.outs))
+
+    def family_work(self, key):
+        return self.step_flops
+
+    def config(self):
+        return {"workload": self.name, "M": self.M, "N": self.N, "K": self.K, "format": "mxfp4", "block": 32,
+                "activations": "N(0,1), seed 13", "weights": "N(0,0.02), quantized offline (untimed)",
+                "out": "MXFP4 codes + scales of Y (RTN, tensor-core layout), Y not written",
+                "gemm_flops_per_step": self.step_flops, "l2": "operands 69 MB + 48 MB of output codes per step"}
+
+    def oracle_setup(self):
+        from workloads import normal_bf16
+        import oracle as O
+        self.xb = normal_bf16((self.M, self.K), 1.0, 13, 0)
+        self.ow = O.quantize(normal_bf16((self.N, self.K), 0.02, 13, 1)[:1024], fmt="mxfp4")
+
+    def oracle_step(self, rows):
+        import oracle as O
+        qx = O.quantize(self.xb[:rows], fmt="mxfp4")
+        y, _ = O.gemm_ref(qx, self.ow, "mxfp4")
+        O.quantize_values(y.astype(np.float32), fmt="mxfp4")
+        return 2.0 * rows * 1024 * self.K
+
+    def cpu_sample(self):
+        return 8192, "all 8192 rows of X: quantize, fp64 GEMM against 1024 rows of W, quantize the product (NumPy)"
+
+    def reference_sample(self):
+        return 64, "64 rows of X: quantize, fp64 GEMM against 1024 rows of W, quantize the product (NumPy)"
+
+
 class VitLinears(GemmWorkload):
     """ViT-B/16 training linears at M = 256*197 = 50432: per layer (qkv, fc1, fc2) the forward
     (RTN), dgrad and wgrad GEMMs, each operand quantized to MXFP4 along its own contraction axis
@@ -852,7 +933,7 @@ class MxLinear128(GemmWorkload):
 
 
 WORKLOADS = {W.name: W for W in (NvfpStudentT, NvfpStudentT46, Nvfp2dWeight, NvfpMseWeight, HadamardMxGemm,
-                                  VitLinears, LlamaNvfp4, MxLinear128)}
+                                  FusedMxLinear, VitLinears, LlamaNvfp4, MxLinear128)}
 
 
 # ------------------------------------------------------------------ arms ---

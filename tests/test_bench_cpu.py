@@ -21,7 +21,8 @@ def _run(*args):
 
 
 @pytest.mark.parametrize("workload", ["mx_linear_128x512", "nvfp4_student_t_4096", "nvfp4_4o6_student_t_4096",
-                                      "nvfp4_2d_weight_11008x4096", "nvfp4_mse_weight_11008x4096"])
+                                      "nvfp4_2d_weight_11008x4096", "nvfp4_mse_weight_11008x4096",
+                                      "mxfp4_fused_linear_8192x11008x4096"])
 def test_reference_arm_line(workload):
     d = _run("--impl", "reference", "--workload", workload, "--steps", "1", "--warmup", "3")
     for k in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better", "scaling",
