@@ -146,13 +146,15 @@ class Workload:
 
 
 class NvfpStudentT(Workload):
-    """NVFP4 quantize (RTN, then Philox SR) + fp32 dequantize of 0.1*Student-t(3), 4096x4096."""
+    """NVFP4 quantize + fp32 dequantize of 0.1*Student-t(3), 4096x4096, once with RTN and once with
+    Philox SR: each one fp4_quantize_dequantize launch (codes, scales and dequantized values)."""
 
     name = "nvfp4_student_t_4096"
     fmt = "nvfp4"                # the quantizer's format ("nvfp4_4o6": four-over-six block scales)
+    fused_deq = True             # quantize and dequantize in one launch (fp4_quantize_dequantize)
     rows = cols = 4096
     n_inputs = 4                 # rotating input copies: 128 MB of inputs, each step writes ~146 MB
-    launches_per_step = 4        # single-pass amax+quantize RTN, dequantize, quantize SR, dequantize
+    launches_per_step = 2        # single-pass amax + quantize + dequantize (RTN), quantize + dequantize (SR)
     unit = "GB/s"
 
     def __init__(self, torch, F):
@@ -160,10 +162,11 @@ class NvfpStudentT(Workload):
         n = self.rows * self.cols
         self.n = n
         # algorithmic HBM bytes per element: quantize = 2 (bf16 in) + 0.5 (codes) + 1/16 (E4M3 scales);
-        # dequantize = 0.5 + 1/16 in + 4 (fp32) out.  The tensor amax needs x once more, which the
-        # method can serve from L2 (32 MB < 126 MB), so it adds no algorithmic bytes.
+        # dequantize = 4 (fp32) out, plus 0.5 + 1/16 in when it is a separate pass over the codes.
+        # The tensor amax needs x once more, which the method can serve from L2 (32 MB < 126 MB),
+        # so it adds no algorithmic bytes.
         self.q_bytes = n * (2 + 0.5 + 1 / 16)
-        self.d_bytes = n * (0.5 + 1 / 16 + 4)
+        self.d_bytes = n * (4 if self.fused_deq else 0.5 + 1 / 16 + 4)
         self.step_bytes = 2 * self.q_bytes + 2 * self.d_bytes
 
     def setup(self, device):
@@ -180,11 +183,15 @@ class NvfpStudentT(Workload):
         self.deq = [t.empty((self.rows, self.cols), dtype=t.float32, device=device) for _ in range(2)]
         # "amax+quantize_rtn" covers the single-pass amax+quantize kernel (two kernels when the
         # tensor does not fit the single pass); the others time exactly one kernel per launch.
-        self.timers = {k: KernelTimer(t) for k in ("amax+quantize_rtn", "quantize_sr", "dequantize")}
+        keys = ("amax+quantize_dequantize_rtn", "quantize_dequantize_sr") if self.fused_deq else \
+            ("amax+quantize_rtn", "quantize_sr", "dequantize")
+        self.timers = {k: KernelTimer(t) for k in keys}
         self.host_in = t.from_numpy(bits.view(np.int16)).view(t.bfloat16).pin_memory()
         self.dev_in = t.empty_like(self.x[0])
 
     def single_kernel(self):
+        if self.fused_deq:
+            return ("amax+quantize_dequantize_rtn", "quantize_dequantize_sr")
         return ("quantize_sr", "dequantize")
 
     def step(self, i, timed=False, x=None):
@@ -194,6 +201,15 @@ class NvfpStudentT(Workload):
 
         def run(key, fn):
             return T[key].around(fn) if T is not None else fn()
+
+        if self.fused_deq:
+            run("amax+quantize_dequantize_rtn", lambda: F.fp4_quantize_dequantize(
+                x, fmt=self.fmt, rnd="rtn", codes=self.codes[0], scales=self.scales[0], tensor_scale_out=self.ts,
+                out=self.deq[0]))
+            run("quantize_dequantize_sr", lambda: F.fp4_quantize_dequantize(
+                x, fmt=self.fmt, rnd="sr", seed=1, tensor_scale_in=self.ts, codes=self.codes[1],
+                scales=self.scales[1], tensor_scale_out=self.ts_sr, out=self.deq[1]))
+            return
 
         # RTN: tensor amax + quantize (one entry point), then dequantize
         run("amax+quantize_rtn", lambda: F.fp4_quantize(x, fmt=self.fmt, rnd="rtn", codes=self.codes[0],
@@ -221,8 +237,9 @@ class NvfpStudentT(Workload):
 
     def family_work(self, key):
         """Algorithmic work per step of a kernel family (bytes here)."""
-        return {"amax+quantize_rtn": self.q_bytes, "quantize_sr": self.q_bytes,
-                "dequantize": 2 * self.d_bytes}[key]
+        return {"amax+quantize_rtn": self.q_bytes, "quantize_sr": self.q_bytes, "dequantize": 2 * self.d_bytes,
+                "amax+quantize_dequantize_rtn": self.q_bytes + self.d_bytes,
+                "quantize_dequantize_sr": self.q_bytes + self.d_bytes}[key]
 
     def value_from_ms(self, ms_per_step, n_ranks):
         return self.step_bytes * n_ranks / (ms_per_step * 1e-3) / 1e9
@@ -230,7 +247,8 @@ class NvfpStudentT(Workload):
     def config(self):
         return {"workload": self.name, "shape": [self.rows, self.cols], "format": self.fmt, "block": 16,
                 "distribution": "0.1*student_t(3)", "seed": 1, "rounding": ["rtn", "sr(philox4x32-10, seed 1)"],
-                "dequantize": "f32", "algorithmic_bytes_per_step": self.step_bytes,
+                "dequantize": "f32, in the quantizing launch" if self.fused_deq else "f32, separate launch",
+                "algorithmic_bytes_per_step": self.step_bytes,
                 "l2": f"{self.n_inputs} rotating input copies (128 MB) and ~146 MB written per step"}
 
     # ---- CPU oracle on the same workload ----
@@ -247,7 +265,7 @@ class NvfpStudentT(Workload):
         O.dequantize(r["codes"], r["scales"], fmt="nvfp4", tensor_scale=s_t)
         r = O.quantize_values(x32, fmt=self.fmt, rnd="sr", seed=1, tensor_scale=s_t)
         O.dequantize(r["codes"], r["scales"], fmt="nvfp4", tensor_scale=s_t)
-        return rows * self.cols * (2 * (2 + 0.5 + 1 / 16) + 2 * (0.5 + 1 / 16 + 4))
+        return rows * self.cols * self.step_bytes / self.n
 
     def cpu_sample(self):
         return self.rows, f"one full step ({self.rows}x{self.cols}) on the host, NumPy elementwise (1 thread)"
@@ -262,6 +280,8 @@ class NvfpStudentT46(NvfpStudentT):
 
     name = "nvfp4_4o6_student_t_4096"
     fmt = "nvfp4_4o6"
+    fused_deq = False            # four-over-six quantizes, then a separate dequantize launch
+    launches_per_step = 4
 
     def cpu_sample(self):
         return 512, f"512 of {self.rows} rows (global tensor scale), NumPy elementwise (1 thread)"

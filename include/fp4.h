@@ -141,6 +141,22 @@ fp4_status fp4_hadamard_quantize(const void* x, int64_t rows, int64_t cols, int6
                                  int had_block, float* rotated_out, void* stream);
 
 /*
+ * fp4_quantize_dequantize -- fp4_quantize along axis 1 that also writes the
+ * dequantized values ("FP4 All the Way", Abstract: the E2M1 values times their
+ * block scale), as fp4_dequantize would compute them from the codes just
+ * written, without re-reading the codes: one launch for quantize + dequantize.
+ *   x .. sf_layout  as fp4_quantize with axis = 1 (fmt FP4_MXFP4, FP4_MXFP4_GS
+ *              or FP4_NVFP4; FP4_NVFP4_4O6 is not supported here).
+ *   out        fp32 or bf16 (out_dtype) [rows, cols], row stride cols,
+ *              16-byte aligned.
+ */
+fp4_status fp4_quantize_dequantize(const void* x, int64_t rows, int64_t cols, int64_t ld,
+                                   int fmt, int block, int rnd, uint64_t seed,
+                                   const float* tensor_scale_in, float* tensor_scale_out,
+                                   uint8_t* codes, uint8_t* scales, int sf_layout,
+                                   void* out, int out_dtype, void* stream);
+
+/*
  * fp4_quantize_2d -- square-tile block quantization of a matrix
  * ("Pretraining Large Language Models with NVFP4", Abstract: a two-dimensional
  * quantization gives weights one consistent representation in the forward and

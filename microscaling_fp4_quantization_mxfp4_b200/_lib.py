@@ -13,6 +13,8 @@ PROTOTYPES = {
     "fp4_quantize": (_int, [_vp, _i64, _i64, _i64, _int, _int, _int, _int, _u64, _vp, _vp, _vp, _vp, _int, _vp]),
     "fp4_hadamard_quantize": (_int, [_vp, _i64, _i64, _i64, _int, _int, _int, _int, _u64, _vp, _vp, _vp, _vp,
                                      _int, _int, _vp, _vp]),
+    "fp4_quantize_dequantize": (_int, [_vp, _i64, _i64, _i64, _int, _int, _int, _u64, _vp, _vp, _vp, _vp, _int, _vp,
+                                       _int, _vp]),
     "fp4_quantize_2d": (_int, [_vp, _i64, _i64, _i64, _int, _int, _int, _u64, _vp, _vp, _vp, _vp, _vp, _vp,
                                _int, _vp]),
     "fp4_quantize_mse": (_int, [_vp, _i64, _i64, _i64, _int, _int, _int, _u64, _int, _vp, _vp, _vp, _int, _vp]),

@@ -131,6 +131,24 @@ def fp4_hadamard_quantize(x: torch.Tensor, had_block: int, fmt="mxfp4", axis: in
     return Fp4Quantized(codes, scales, ts_out if f in (NVFP4, NVFP4_4O6) else None)
 
 
+def fp4_quantize_dequantize(x: torch.Tensor, fmt="nvfp4", rnd="rtn", seed: int = 0,
+                            tensor_scale_in: Optional[torch.Tensor] = None, sf_layout="rowmajor", out_dtype="f32", *,
+                            codes=None, scales=None, tensor_scale_out=None, out=None, stream=None):
+    """fp4_quantize along rows plus the dequantized values in the same launch (see include/fp4.h).
+    Returns (Fp4Quantized, dequantized tensor)."""
+    _bf16_matrix(x)
+    f, r, sf, od = _FMT[fmt], _RND[rnd], _SF[sf_layout], _OUT[out_dtype]
+    codes, scales, ts_out = _alloc_quant_outputs(x, f, 1, sf, codes, scales, tensor_scale_out)
+    if out is None:
+        out = torch.empty(x.shape, dtype=torch.float32 if od == OUT_F32 else torch.bfloat16, device=x.device)
+    st = _lib.load().fp4_quantize_dequantize(
+        x.data_ptr(), x.shape[0], x.shape[1], x.stride(0), f, BLOCK[f], r, seed & (2 ** 64 - 1),
+        _ptr(tensor_scale_in), _ptr(ts_out), codes.data_ptr(), scales.data_ptr(), sf, out.data_ptr(), od,
+        _stream(stream))
+    _check(st, "fp4_quantize_dequantize")
+    return Fp4Quantized(codes, scales, ts_out if f in (NVFP4, NVFP4_4O6) else None), out
+
+
 def fp4_quantize_2d(x: torch.Tensor, fmt="nvfp4", rnd="rtn", seed: int = 0,
                     tensor_scale_in: Optional[torch.Tensor] = None, sf_layout="rowmajor", transposed: bool = True,
                     *, codes=None, scales=None, codes_t=None, scales_t=None, tensor_scale_out=None,

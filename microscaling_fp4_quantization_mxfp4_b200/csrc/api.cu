@@ -116,7 +116,8 @@ fp4_status check_input(const void* x, int64_t rows, int64_t cols, int64_t ld) {
 
 fp4_status quantize_impl(const void* x, int64_t rows, int64_t cols, int64_t ld, int fmt, int block, int axis,
                          int rnd, uint64_t seed, const float* ts_in, float* ts_out, uint8_t* codes, uint8_t* scales,
-                         int sf_layout, int had, float* rotated, cudaStream_t st) {
+                         int sf_layout, int had, float* rotated, cudaStream_t st, void* deq = nullptr,
+                         int deq_mode = 0) {
   int four_six = 0;
   uint32_t mx_thr = 0x800000u;       // OCP exponent rule
   if (fmt == FP4_MXFP4_GS) {         // MXFP4 codes and scales under the MSE-fitted clip threshold
@@ -141,6 +142,11 @@ fp4_status quantize_impl(const void* x, int64_t rows, int64_t cols, int64_t ld, 
   const int64_t orows = axis == 1 ? rows : cols;
   if (qlen % block != 0) return FP4_ERR_SHAPE;
   if (!aligned16(codes)) return FP4_ERR_ALIGN;
+  if (deq_mode != 0) {
+    if (deq == nullptr) return FP4_ERR_ARG;
+    if (axis != 1 || four_six || had != 0) return FP4_ERR_UNSUPPORTED;
+    if (!aligned16(deq)) return FP4_ERR_ALIGN;
+  }
   if (had != 0) {
     if (had != 16 && had != 32 && had != 64 && had != 128) return FP4_ERR_ARG;
     if (axis != 1 || four_six) return FP4_ERR_UNSUPPORTED;
@@ -175,6 +181,8 @@ fp4_status quantize_impl(const void* x, int64_t rows, int64_t cols, int64_t ld, 
   p.error = d->scratch.error;
   p.four_six = four_six;
   p.mx_thr = mx_thr;
+  p.deq = deq;
+  p.deq_mode = deq_mode;
   size_t fused_smem = 0;
   uint32_t fused_tiles = 0;
   if (fmt == FP4_NVFP4 && ts_in == nullptr && axis == 1 && ld == cols && !single_pass_disabled() &&
@@ -217,6 +225,17 @@ fp4_status fp4_hadamard_quantize(const void* x, int64_t rows, int64_t cols, int6
   if (had_block == 0) return FP4_ERR_ARG;
   return quantize_impl(x, rows, cols, ld, fmt, block, axis, rnd, seed, tensor_scale_in, tensor_scale_out, codes,
                        scales, sf_layout, had_block, rotated_out, static_cast<cudaStream_t>(stream));
+}
+
+fp4_status fp4_quantize_dequantize(const void* x, int64_t rows, int64_t cols, int64_t ld, int fmt, int block,
+                                   int rnd, uint64_t seed, const float* tensor_scale_in, float* tensor_scale_out,
+                                   uint8_t* codes, uint8_t* scales, int sf_layout, void* out, int out_dtype,
+                                   void* stream) {
+  if (out_dtype != FP4_OUT_F32 && out_dtype != FP4_OUT_BF16) return FP4_ERR_ARG;
+  if (out == nullptr) return FP4_ERR_ARG;
+  return quantize_impl(x, rows, cols, ld, fmt, block, 1, rnd, seed, tensor_scale_in, tensor_scale_out, codes, scales,
+                       sf_layout, 0, nullptr, static_cast<cudaStream_t>(stream), out,
+                       out_dtype == FP4_OUT_F32 ? 1 : 2);
 }
 
 fp4_status fp4_quantize_2d(const void* x, int64_t rows, int64_t cols, int64_t ld, int fmt, int block, int rnd,

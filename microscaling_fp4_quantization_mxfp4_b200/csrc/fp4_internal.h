@@ -93,6 +93,8 @@ struct QuantizeParams {
   unsigned* error;        // device error word
   int four_six = 0;       // NVFP4: four-over-six block scales
   uint32_t mx_thr = 0x800000u;  // MXFP4 exponent clip threshold as a significand field (0x800000: OCP)
+  void* deq = nullptr;    // axis 1: also write the dequantized values [rows, cols] here
+  int deq_mode = 0;       // 0: no, 1: fp32, 2: bf16
 };
 
 // amax pass: mode 0 writes max|x| (after rotation when had > 0) to `out`,

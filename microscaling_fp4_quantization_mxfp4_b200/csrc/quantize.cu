@@ -154,6 +154,7 @@ struct QRowParams {
   uint8_t* scales;
   float* rotated;
   unsigned* error;       // device error word (streaming kernels: bit 2 = a ring wait expired)
+  void* deq;             // DQ kernels: the dequantized values [rows, cols] (fp32, or bf16 for DQ = 2)
 };
 
 
@@ -243,7 +244,64 @@ __device__ __forceinline__ uint32_t nv_four_over_six(float (&x)[E], float am, ui
   return pick4 ? byte4 : byte6;
 }
 
-template <int FMT, int RND, int HAD, bool SFMMA>
+// Dequantized values of one block's packed codes w (E/8 words) under scale byte `byte`, as
+// fp4_dequantize computes them (NVFP4: fp32(fp32(G[c] * sb) * s_t) with the exact f16 product;
+// MXFP4: G[c] * 2^E), stored at element blk * E of the row-major output: fp32 (DQ = 1) or bf16
+// (DQ = 2, round to nearest even).
+template <int FMT, int DQ>
+__device__ __forceinline__ void dequant_block_out(const QRowParams& p, const uint32_t* w, uint32_t byte, uint32_t blk,
+                                                  float s_t) {
+  constexpr int E = BlockShape<FMT>::E;
+  float y[E];
+  const __half2 sb = __float2half2_rn(FMT == FMT_MX ? 1.0f : e4m3_value(byte));
+  const float sc = FMT == FMT_MX ? mx_scale_value(byte) : s_t;
+#pragma unroll
+  for (int k = 0; k < E / 8; ++k) {
+    uint32_t h[4];
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\tmov.b32 {b0, b1, b2, b3}, %4;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %0, b0;\n\tcvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %2, b2;\n\tcvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+        : "=r"(h[0]), "=r"(h[1]), "=r"(h[2]), "=r"(h[3])
+        : "r"(w[k]));
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const __half2 hv = *reinterpret_cast<const __half2*>(&h[i]);
+      const float2 g = __half22float2(FMT == FMT_MX ? hv : __hmul2(hv, sb));
+      y[8 * k + 2 * i] = __fmul_rn(g.x, sc);
+      y[8 * k + 2 * i + 1] = __fmul_rn(g.y, sc);
+    }
+  }
+  // 32-byte stores (one whole L2 sector per lane) when the output base allows them: a block's
+  // values start at a multiple of 32 bytes.  16-byte stores from neighbouring lanes 64 bytes
+  // apart would each half-fill a sector.
+  const bool wide = (reinterpret_cast<uintptr_t>(p.deq) & 31u) == 0;
+  uint32_t o32[DQ == 1 ? E : E / 2];
+  if (DQ == 1) {
+#pragma unroll
+    for (int i = 0; i < E; ++i) o32[i] = __float_as_uint(y[i]);
+  } else {
+#pragma unroll
+    for (int i = 0; i < E / 2; ++i)
+      o32[i] = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(y[2 * i])) |
+               ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(y[2 * i + 1])) << 16);
+  }
+  constexpr int W = DQ == 1 ? E : E / 2;                   // 32-bit words of the block's output
+  uint32_t* o = static_cast<uint32_t*>(p.deq) + (size_t)blk * W;
+  if (wide) {
+#pragma unroll
+    for (int k = 0; k < W / 8; ++k)
+      asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(o + 8 * k), "r"(o32[8 * k]),
+                   "r"(o32[8 * k + 1]), "r"(o32[8 * k + 2]), "r"(o32[8 * k + 3]), "r"(o32[8 * k + 4]),
+                   "r"(o32[8 * k + 5]), "r"(o32[8 * k + 6]), "r"(o32[8 * k + 7])
+                   : "memory");
+  } else {
+#pragma unroll
+    for (int k = 0; k < W / 4; ++k)
+      reinterpret_cast<uint4*>(o)[k] = make_uint4(o32[4 * k], o32[4 * k + 1], o32[4 * k + 2], o32[4 * k + 3]);
+  }
+}
+
+template <int FMT, int RND, int HAD, bool SFMMA, int DQ = 0>
 __device__ __forceinline__ void quantize_block(const QRowParams& p, const uint4 (&v)[BlockShape<FMT>::V], uint32_t blk,
                                                bool valid, int lane, const NvConsts& nv) {
   constexpr int E = BlockShape<FMT>::E, V = BlockShape<FMT>::V;
@@ -303,11 +361,16 @@ __device__ __forceinline__ void quantize_block(const QRowParams& p, const uint4 
     }
   }
   if (!valid) return;
-  if (FMT == FMT_MX) {
-    reinterpret_cast<uint4*>(p.codes)[blk] = zero ? make_uint4(0u, 0u, 0u, 0u) : make_uint4(w[0], w[1], w[2], w[3]);
-  } else {
-    reinterpret_cast<uint2*>(p.codes)[blk] = zero ? make_uint2(0u, 0u) : make_uint2(w[0], w[1]);
+  if (zero) {
+#pragma unroll
+    for (int k = 0; k < E / 8; ++k) w[k] = 0u;
   }
+  if (FMT == FMT_MX) {
+    reinterpret_cast<uint4*>(p.codes)[blk] = make_uint4(w[0], w[1], w[2], w[3]);
+  } else {
+    reinterpret_cast<uint2*>(p.codes)[blk] = make_uint2(w[0], w[1]);
+  }
+  if (DQ != 0) dequant_block_out<FMT, DQ>(p, w, byte, blk, nv.s_t);
   if (SFMMA) {
     const uint32_t row = fdiv(blk, p.bpr);
     p.scales[sf_mma_offset(row, blk - row * p.bpr.d, p.g4)] = (uint8_t)byte;
@@ -317,7 +380,7 @@ __device__ __forceinline__ void quantize_block(const QRowParams& p, const uint4 
 }
 
 // Strided inputs (ld != cols): one thread per scale block, loads straight from global memory.
-template <int FMT, int RND, int HAD, bool SFMMA>
+template <int FMT, int RND, int HAD, bool SFMMA, int DQ = 0>
 __global__ void __launch_bounds__(256) quantize_rows_kernel(QRowParams p) {
   pdl_trigger();
   constexpr int V = BlockShape<FMT>::V;
@@ -348,7 +411,7 @@ __global__ void __launch_bounds__(256) quantize_rows_kernel(QRowParams p) {
 #pragma unroll
       for (int k = 0; k < V; ++k) v[k] = ld_stream(src + 8 * k);
     }
-    quantize_block<FMT, RND, HAD, SFMMA>(p, v, blk, valid, lane, nv);
+    quantize_block<FMT, RND, HAD, SFMMA, DQ>(p, v, blk, valid, lane, nv);
   }
 }
 
@@ -441,7 +504,7 @@ __device__ void stream_produce(const StreamRing& r, const uint16_t* x, uint32_t 
   }
 }
 
-template <int FMT, int RND, int HAD, bool SFMMA>
+template <int FMT, int RND, int HAD, bool SFMMA, int DQ = 0>
 __global__ void __launch_bounds__(StreamWarps<FMT, RND>::kThreads, 1) quantize_stream_kernel(QRowParams p) {
   constexpr int kStreamWarps = StreamWarps<FMT, RND>::kWarps;
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -485,7 +548,7 @@ __global__ void __launch_bounds__(StreamWarps<FMT, RND>::kThreads, 1) quantize_s
       uint4 v[V];
 #pragma unroll
       for (int k = 0; k < V; ++k) v[k] = valid ? src[lb * V + k] : make_uint4(0u, 0u, 0u, 0u);
-      quantize_block<FMT, RND, HAD, SFMMA>(p, v, c0 / V + lb, valid, lane, nv);
+      quantize_block<FMT, RND, HAD, SFMMA, DQ>(p, v, c0 / V + lb, valid, lane, nv);
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(smem_addr(&r.empty[stage]));
@@ -593,7 +656,7 @@ struct FusedWarps {
 constexpr int kFusedMaxSmem = 227 * 1024 - 2048;          // staged slice; room left for the static data
 constexpr int kFusedPieces = 8;                           // bulk copies (and mbarriers) per slice
 
-template <int FMT, int RND, int HAD, bool SFMMA>
+template <int FMT, int RND, int HAD, bool SFMMA, int DQ = 0>
 __global__ void __launch_bounds__(FusedWarps<FMT>::kThreads, 1) nv_quantize_fused_kernel(FusedParams fp) {
   constexpr int kFusedWarps = FusedWarps<FMT>::kWarps;
   extern __shared__ __align__(1024) uint4 slice[];
@@ -709,7 +772,7 @@ __global__ void __launch_bounds__(FusedWarps<FMT>::kThreads, 1) nv_quantize_fuse
     uint4 v[2];
     v[0] = valid ? slice[lb * 2u] : make_uint4(0u, 0u, 0u, 0u);
     v[1] = valid ? slice[lb * 2u + 1u] : make_uint4(0u, 0u, 0u, 0u);
-    quantize_block<FMT, RND, HAD, SFMMA>(p, v, c_begin / 2u + lb, valid, lane, nv);
+    quantize_block<FMT, RND, HAD, SFMMA, DQ>(p, v, c_begin / 2u + lb, valid, lane, nv);
   }
 }
 
@@ -1285,9 +1348,9 @@ cudaError_t launch_nv_tensor_scale(const float* amax, float* out, cudaStream_t s
   return launch_kernel(nv_tensor_scale_kernel, dim3(1), dim3(1), 0, st, false, 1u, amax, out);
 }
 
-template <int FMT, int RND, int HAD, bool SFMMA>
+template <int FMT, int RND, int HAD, bool SFMMA, int DQ = 0>
 static cudaError_t rows_stream_launch(const QRowParams& qp, int num_sms, cudaStream_t st) {
-  auto kernel = quantize_stream_kernel<FMT, RND, HAD, SFMMA>;
+  auto kernel = quantize_stream_kernel<FMT, RND, HAD, SFMMA, DQ>;
   static const cudaError_t attr =
       cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kStreamSmem);
   if (attr != cudaSuccess) return attr;
@@ -1297,20 +1360,28 @@ static cudaError_t rows_stream_launch(const QRowParams& qp, int num_sms, cudaStr
   return launch_kernel(kernel, dim3(grid), dim3(StreamWarps<FMT, RND>::kThreads), kStreamSmem, st, false, 1u, qp);
 }
 
-template <int FMT, int RND, int HAD, bool SFMMA>
+template <int FMT, int RND, int HAD, bool SFMMA, int DQ = 0>
 static cudaError_t rows_launch(const QRowParams& qp, int num_sms, cudaStream_t st) {
-  if (qp.contig) return rows_stream_launch<FMT, RND, HAD, SFMMA>(qp, num_sms, st);
-  static int occ = resident_ctas(quantize_rows_kernel<FMT, RND, HAD, SFMMA>, 256);
+  if (qp.contig) return rows_stream_launch<FMT, RND, HAD, SFMMA, DQ>(qp, num_sms, st);
+  static int occ = resident_ctas(quantize_rows_kernel<FMT, RND, HAD, SFMMA, DQ>, 256);
   const uint32_t nunits = (qp.nblocks + 31u) / 32u;
   uint32_t want = (nunits + 7u) / 8u;
   uint32_t grid = (uint32_t)num_sms * (uint32_t)occ;
   if (want < grid) grid = want > 0 ? want : 1;
-  return launch_kernel(quantize_rows_kernel<FMT, RND, HAD, SFMMA>, dim3(grid), dim3(256), 0, st, false, 1u, qp);
+  return launch_kernel(quantize_rows_kernel<FMT, RND, HAD, SFMMA, DQ>, dim3(grid), dim3(256), 0, st, false, 1u, qp);
 }
 
 template <int FMT, int RND, int HAD>
 static cudaError_t rows_dispatch_sf(const QRowParams& qp, bool sfmma, int num_sms, cudaStream_t st) {
   return sfmma ? rows_launch<FMT, RND, HAD, true>(qp, num_sms, st) : rows_launch<FMT, RND, HAD, false>(qp, num_sms, st);
+}
+
+// Quantize + dequantize variants (no rotation): dq 1 = fp32 values, 2 = bf16.
+template <int FMT, int RND>
+static cudaError_t rows_dispatch_dq(const QRowParams& qp, int dq, bool sfmma, int num_sms, cudaStream_t st) {
+  if (dq == 1)
+    return sfmma ? rows_launch<FMT, RND, 0, true, 1>(qp, num_sms, st) : rows_launch<FMT, RND, 0, false, 1>(qp, num_sms, st);
+  return sfmma ? rows_launch<FMT, RND, 0, true, 2>(qp, num_sms, st) : rows_launch<FMT, RND, 0, false, 2>(qp, num_sms, st);
 }
 
 template <int FMT, int RND>
@@ -1325,9 +1396,9 @@ static cudaError_t rows_dispatch_had(const QRowParams& qp, int had, bool sfmma, 
   }
 }
 
-template <int FMT, int RND, int HAD, bool SFMMA>
+template <int FMT, int RND, int HAD, bool SFMMA, int DQ = 0>
 static cudaError_t fused_launch(const FusedParams& fp, uint32_t grid, size_t smem, cudaStream_t st) {
-  auto kernel = nv_quantize_fused_kernel<FMT, RND, HAD, SFMMA>;
+  auto kernel = nv_quantize_fused_kernel<FMT, RND, HAD, SFMMA, DQ>;
   static const cudaError_t attr =
       cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kFusedMaxSmem);
   if (attr != cudaSuccess) return attr;
@@ -1376,6 +1447,7 @@ cudaError_t launch_quantize_nv_fused(const QuantizeParams& p, float* ts_out, con
   qp.scales = p.scales;
   qp.rotated = p.rotated;
   qp.error = s.error;
+  qp.deq = p.deq;
   fp.ts_out = ts_out;
   fp.partials = s.partials;
   fp.arrive = s.grid_arrive;
@@ -1386,9 +1458,22 @@ cudaError_t launch_quantize_nv_fused(const QuantizeParams& p, float* ts_out, con
   const uint32_t grid = (uint32_t)((ntiles + per - 1) / per);
   const bool sfmma = p.sf_mma != 0;
   if (p.four_six) {
-    if (p.had != 0) return cudaErrorInvalidValue;
+    if (p.had != 0 || p.deq_mode != 0) return cudaErrorInvalidValue;
     return p.rnd == RND_RTN ? fused_dispatch_sf<RND_RTN, 0, FMT_NV46>(fp, sfmma, grid, smem, st)
                             : fused_dispatch_sf<RND_SR, 0, FMT_NV46>(fp, sfmma, grid, smem, st);
+  }
+  if (p.deq_mode != 0) {
+    if (p.had != 0) return cudaErrorInvalidValue;
+    fp.q.deq = p.deq;
+#define FP4_FUSED_DQ(R, D) \
+    return sfmma ? fused_launch<FMT_NV, R, 0, true, D>(fp, grid, smem, st) : fused_launch<FMT_NV, R, 0, false, D>(fp, grid, smem, st)
+    if (p.rnd == RND_RTN) {
+      if (p.deq_mode == 1) FP4_FUSED_DQ(RND_RTN, 1);
+      FP4_FUSED_DQ(RND_RTN, 2);
+    }
+    if (p.deq_mode == 1) FP4_FUSED_DQ(RND_SR, 1);
+    FP4_FUSED_DQ(RND_SR, 2);
+#undef FP4_FUSED_DQ
   }
 #define FP4_FUSED_HAD(H)                                                                               \
   return p.rnd == RND_RTN ? fused_dispatch_sf<RND_RTN, H>(fp, sfmma, grid, smem, st)                  \
@@ -1441,6 +1526,15 @@ cudaError_t launch_quantize(const QuantizeParams& p, int num_sms, cudaStream_t s
     qp.scales = p.scales;
     qp.rotated = p.rotated;
     qp.error = p.error;
+    qp.deq = p.deq;
+    if (p.deq_mode != 0) {
+      if (p.had != 0 || p.four_six) return cudaErrorInvalidValue;
+      if (p.fmt == FMT_MX)
+        return p.rnd == RND_RTN ? rows_dispatch_dq<FMT_MX, RND_RTN>(qp, p.deq_mode, sfmma, num_sms, st)
+                                : rows_dispatch_dq<FMT_MX, RND_SR>(qp, p.deq_mode, sfmma, num_sms, st);
+      return p.rnd == RND_RTN ? rows_dispatch_dq<FMT_NV, RND_RTN>(qp, p.deq_mode, sfmma, num_sms, st)
+                              : rows_dispatch_dq<FMT_NV, RND_SR>(qp, p.deq_mode, sfmma, num_sms, st);
+    }
     if (p.fmt == FMT_MX)
       return p.rnd == RND_RTN ? rows_dispatch_had<FMT_MX, RND_RTN>(qp, p.had, sfmma, num_sms, st)
                               : rows_dispatch_had<FMT_MX, RND_SR>(qp, p.had, sfmma, num_sms, st);

@@ -122,3 +122,9 @@ def test_other_entry_points_reject_before_launch(lib):
                                  1, None) == -1
     assert lib.fp4_gemm_quantize(FAKE, FAKE, None, FAKE, FAKE, None, 4, 64, 64, 0, 32, 0, 32, 0, 0, None, FAKE + 8,
                                  FAKE, 1, None) == -3
+    # fp4_quantize_dequantize: output required, dtype, no four-over-six, aligned output
+    assert lib.fp4_quantize_dequantize(FAKE, 4, 64, 64, 0, 32, 0, 0, None, None, FAKE, FAKE, 0, None, 0, None) == -1
+    assert lib.fp4_quantize_dequantize(FAKE, 4, 64, 64, 0, 32, 0, 0, None, None, FAKE, FAKE, 0, FAKE, 5, None) == -1
+    assert lib.fp4_quantize_dequantize(FAKE, 4, 64, 64, 2, 16, 0, 0, None, FAKE, FAKE, FAKE, 0, FAKE, 0, None) == -4
+    assert lib.fp4_quantize_dequantize(FAKE, 4, 64, 64, 0, 32, 0, 0, None, None, FAKE, FAKE, 0, FAKE + 4, 0,
+                                       None) == -3

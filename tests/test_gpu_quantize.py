@@ -532,3 +532,73 @@ def test_quantize_mse_full_size_properties():
         c = np.where((sb == 0)[:, None], np.uint8(0), O.e2m1_rtn(v))
         np.testing.assert_array_equal(codes[r], O.pack_nibbles(c.reshape(1, -1))[0])
     F.fp4_check_device_errors()
+
+
+# ------------------------------------------------------------- quantize + dequantize ---
+
+@pytest.mark.parametrize("out", ["f32", "bf16"])
+@pytest.mark.parametrize("sf", ["rowmajor", "mma"])
+@pytest.mark.parametrize("rnd", ["rtn", "sr"])
+@pytest.mark.parametrize("fmt, shape, given_ts, strided", [
+    ("nvfp4", (200, 384), False, False),        # single-pass amax + quantize kernel
+    ("nvfp4", (129, 1024), True, False),        # streaming kernel under a caller's s_t
+    ("nvfp4", (64, 256), False, True),          # strided rows (ld > cols): amax pass + rows kernel
+    ("mxfp4", (96, 512), False, False),
+    ("mxfp4_gs", (33, 1056), False, True)])
+def test_quantize_dequantize(fmt, shape, given_ts, strided, rnd, sf, out):
+    """One launch writes codes, scales and the dequantized values: codes and scales bit-exact
+    against the oracle's quantize, values bit-exact against the oracle's dequantize of them."""
+    rows, cols = shape
+    xfull = mixed_input(rows, cols + (64 if strided else 0), rows + cols, "mxfp4" if fmt != "nvfp4" else "nvfp4")
+    xb = np.ascontiguousarray(xfull[:, :cols])
+    x = dev_bf16(xfull)[:, :cols] if strided else dev_bf16(xb)
+    ts = None
+    kw = {}
+    if given_ts:
+        ts = np.float32(O.nv_tensor_scale(bf16_to_f32(xb)) * np.float32(0.75))
+        kw["tensor_scale_in"] = torch.tensor([ts], dtype=torch.float32, device="cuda")
+    q, y = F.fp4_quantize_dequantize(x, fmt=fmt, rnd=rnd, seed=21, sf_layout=sf, out_dtype=out, **kw)
+    ref = O.quantize(xb, fmt=fmt, rnd=rnd, seed=21, tensor_scale=ts)
+    _check_against_oracle(q, ref, "nvfp4" if fmt == "nvfp4" else "mxfp4", 1, rows, cols, sf)
+    base = "nvfp4" if fmt == "nvfp4" else "mxfp4"
+    want = O.dequantize(ref["codes"], ref["scales"], fmt=base, tensor_scale=ref["tensor_scale"], out=out)
+    if out == "f32":
+        np.testing.assert_array_equal(host_f32(y).view(np.uint32), want.view(np.uint32))
+    else:
+        np.testing.assert_array_equal(host_bf16_bits(y), want)
+    F.fp4_check_device_errors()
+
+
+def test_quantize_dequantize_two_pass_large_tensor():
+    """A 64 MiB tensor (amax pass, then the streaming kernel): 64 sampled rows bit-exact."""
+    from workloads import student_t_bf16
+    xb = student_t_bf16((8192, 4096), 3.0, 0.1, 7, 1)
+    q, y = F.fp4_quantize_dequantize(dev_bf16(xb), fmt="nvfp4", rnd="sr", seed=4)
+    x32 = bf16_to_f32(xb)
+    s_t = O.nv_tensor_scale(x32)
+    assert host_f32(q.tensor_scale)[0] == s_t
+    codes, scales, yv = host_u8(q.codes), host_u8(q.scales), host_f32(y)
+    for r in np.sort(np.random.default_rng(5).choice(8192, 64, replace=False)):
+        ref = O.quantize_values(x32[r:r + 1], fmt="nvfp4", rnd="sr", seed=4, tensor_scale=s_t, idx_base=int(r) * 4096)
+        np.testing.assert_array_equal(codes[r:r + 1], ref["codes"])
+        np.testing.assert_array_equal(scales[r:r + 1], ref["scales"])
+        want = O.dequantize(ref["codes"], ref["scales"], fmt="nvfp4", tensor_scale=s_t)
+        np.testing.assert_array_equal(yv[r:r + 1].view(np.uint32), want.view(np.uint32))
+    F.fp4_check_device_errors()
+
+
+@pytest.mark.parametrize("out", ["f32", "bf16"])
+def test_quantize_dequantize_output_16_byte_aligned(out):
+    """An output 16- but not 32-byte aligned takes the 16-byte stores: same values."""
+    rows, cols = 64, 512
+    xb = mixed_input(rows, cols, 77, "nvfp4")
+    dt = torch.float32 if out == "f32" else torch.bfloat16
+    shift = 4 if out == "f32" else 8                      # 16 bytes
+    buf = torch.empty(rows * cols + shift, dtype=dt, device="cuda")
+    y = buf[shift:].view(rows, cols)
+    q, _ = F.fp4_quantize_dequantize(dev_bf16(xb), fmt="nvfp4", rnd="sr", seed=3, out_dtype=out, out=y)
+    ref = O.quantize(xb, fmt="nvfp4", rnd="sr", seed=3)
+    want = O.dequantize(ref["codes"], ref["scales"], fmt="nvfp4", tensor_scale=ref["tensor_scale"], out=out)
+    got = host_f32(y).view(np.uint32) if out == "f32" else host_bf16_bits(y)
+    np.testing.assert_array_equal(got, want.view(np.uint32) if out == "f32" else want)
+    F.fp4_check_device_errors()
