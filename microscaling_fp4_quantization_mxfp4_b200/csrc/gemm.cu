@@ -300,7 +300,7 @@ struct KernelArgs {
   int M, N, K;
   int num_m, num_n;
   int g4;                 // padded k-groups / 4 of both scale tensors
-  int vec_store;          // output rows 16-byte aligned: 128-bit stores
+  int vec_store;          // output rows 16-byte aligned: 128-bit stores (2: 32-byte aligned, 256-bit stores)
   int tma_store;          // bf16 output through shared memory and TMA stores (tensor map valid)
   unsigned* error;
   // fused quantization of Y along its rows (kernels with QO != 0): codes [M, N/2], scale bytes in
@@ -312,6 +312,13 @@ struct KernelArgs {
   uint32_t q_mx_thr;
   fp4dev::PhiloxKeys q_keys;
 };
+
+// One 32-byte store (a whole L2 sector) of eight 32-bit words; dst 32-byte aligned.
+__device__ __forceinline__ void st_global_v8(void* dst, const uint32_t (&w)[8]) {
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(dst), "r"(w[0]), "r"(w[1]), "r"(w[2]),
+               "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
+               : "memory");
+}
 
 // Byte offset of the scale of (row m, group g) of the quantized Y.
 __device__ __forceinline__ long long q_sf_offset(const KernelArgs& p, int m, int g, int groups) {
@@ -675,7 +682,20 @@ __global__ void __launch_bounds__(Cfg<BN, FMT>::kThreads, 1)
           if (n0 >= p.N) break;
           if (BF16) {
             __nv_bfloat16* yr = reinterpret_cast<__nv_bfloat16*>(p.y) + (size_t)m * p.ldy + n0;
-            if (p.vec_store && n0 + 32 <= p.N) {
+            if (p.vec_store == 2 && n0 + 32 <= p.N) {
+#pragma unroll
+              for (int v = 0; v < 2; ++v) {
+                uint32_t w[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                  const float lo = __fmul_rn(__uint_as_float(r[c][16 * v + 2 * i]), alpha);
+                  const float hi = __fmul_rn(__uint_as_float(r[c][16 * v + 2 * i + 1]), alpha);
+                  w[i] = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(lo)) |
+                         ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(hi)) << 16);
+                }
+                st_global_v8(yr + 16 * v, w);
+              }
+            } else if (p.vec_store && n0 + 32 <= p.N) {
 #pragma unroll
               for (int v = 0; v < 4; ++v) {
                 uint32_t w[4];
@@ -695,7 +715,15 @@ __global__ void __launch_bounds__(Cfg<BN, FMT>::kThreads, 1)
             }
           } else {
             float* yr = reinterpret_cast<float*>(p.y) + (size_t)m * p.ldy + n0;
-            if (p.vec_store && n0 + 32 <= p.N) {
+            if (p.vec_store == 2 && n0 + 32 <= p.N) {
+#pragma unroll
+              for (int v = 0; v < 4; ++v) {
+                uint32_t w[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) w[i] = __float_as_uint(__fmul_rn(__uint_as_float(r[c][8 * v + i]), alpha));
+                st_global_v8(yr + 8 * v, w);
+              }
+            } else if (p.vec_store && n0 + 32 <= p.N) {
 #pragma unroll
               for (int v = 0; v < 8; ++v)
                 reinterpret_cast<float4*>(yr)[v] = make_float4(
@@ -1074,7 +1102,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg2<BN, FMT>::kThre
           if (n0 >= p.N) break;
           if (BF16) {
             __nv_bfloat16* yr = reinterpret_cast<__nv_bfloat16*>(p.y) + (size_t)m * p.ldy + n0;
-            if (p.vec_store && n0 + 32 <= p.N) {
+            if (p.vec_store == 2 && n0 + 32 <= p.N) {
+#pragma unroll
+              for (int v = 0; v < 2; ++v) {
+                uint32_t w[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                  const float lo = __fmul_rn(__uint_as_float(r[c][16 * v + 2 * i]), alpha);
+                  const float hi = __fmul_rn(__uint_as_float(r[c][16 * v + 2 * i + 1]), alpha);
+                  w[i] = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(lo)) |
+                         ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(hi)) << 16);
+                }
+                st_global_v8(yr + 16 * v, w);
+              }
+            } else if (p.vec_store && n0 + 32 <= p.N) {
 #pragma unroll
               for (int v = 0; v < 4; ++v) {
                 uint32_t w[4];
@@ -1094,7 +1135,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg2<BN, FMT>::kThre
             }
           } else {
             float* yr = reinterpret_cast<float*>(p.y) + (size_t)m * p.ldy + n0;
-            if (p.vec_store && n0 + 32 <= p.N) {
+            if (p.vec_store == 2 && n0 + 32 <= p.N) {
+#pragma unroll
+              for (int v = 0; v < 4; ++v) {
+                uint32_t w[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) w[i] = __float_as_uint(__fmul_rn(__uint_as_float(r[c][8 * v + i]), alpha));
+                st_global_v8(yr + 8 * v, w);
+              }
+            } else if (p.vec_store && n0 + 32 <= p.N) {
 #pragma unroll
               for (int v = 0; v < 8; ++v)
                 reinterpret_cast<float4*>(yr)[v] = make_float4(
@@ -1536,7 +1585,9 @@ cudaError_t run_pair(const GemmParams& gp, int num_sms, cudaStream_t st) {
   ka.error = gp.error;
   {
     const int64_t esz = gp.y_bf16 ? 2 : 4;
-    ka.vec_store = ((gp.ldy * esz) % 16 == 0 && (reinterpret_cast<uintptr_t>(gp.y) & 15u) == 0) ? 1 : 0;
+    ka.vec_store = ((gp.ldy * esz) % 32 == 0 && (reinterpret_cast<uintptr_t>(gp.y) & 31u) == 0)   ? 2
+                   : ((gp.ldy * esz) % 16 == 0 && (reinterpret_cast<uintptr_t>(gp.y) & 15u) == 0) ? 1
+                                                                                                   : 0;
   }
   ka.tma_store = 0;
   fill_quant_args(ka, gp);
@@ -1573,7 +1624,9 @@ cudaError_t run(const GemmParams& gp, int num_sms, cudaStream_t st) {
   ka.error = gp.error;
   {
     const int64_t esz = gp.y_bf16 ? 2 : 4;
-    ka.vec_store = ((gp.ldy * esz) % 16 == 0 && (reinterpret_cast<uintptr_t>(gp.y) & 15u) == 0) ? 1 : 0;
+    ka.vec_store = ((gp.ldy * esz) % 32 == 0 && (reinterpret_cast<uintptr_t>(gp.y) & 31u) == 0)   ? 2
+                   : ((gp.ldy * esz) % 16 == 0 && (reinterpret_cast<uintptr_t>(gp.y) & 15u) == 0) ? 1
+                                                                                                   : 0;
   }
   CUtensorMap ty;
   memset(&ty, 0, sizeof(ty));
@@ -1641,7 +1694,9 @@ cudaError_t run_splitk(const GemmParams& gp, int split, cudaStream_t st) {
   ka.error = gp.error;
   {
     const int64_t esz = gp.y_bf16 ? 2 : 4;
-    ka.vec_store = ((gp.ldy * esz) % 16 == 0 && (reinterpret_cast<uintptr_t>(gp.y) & 15u) == 0) ? 1 : 0;
+    ka.vec_store = ((gp.ldy * esz) % 32 == 0 && (reinterpret_cast<uintptr_t>(gp.y) & 31u) == 0)   ? 2
+                   : ((gp.ldy * esz) % 16 == 0 && (reinterpret_cast<uintptr_t>(gp.y) & 15u) == 0) ? 1
+                                                                                                   : 0;
   }
   ka.tma_store = 0;
   return launch_kernel(kernel, dim3((unsigned)(ka.num_m * ka.num_n * split)), dim3(C::kThreads), C::kSmemBytes, st,
