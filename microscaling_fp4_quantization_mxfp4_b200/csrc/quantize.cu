@@ -954,12 +954,18 @@ __global__ void __launch_bounds__(256, 2) quantize_cols_kernel(QColParams p) {
 // element is scaled and rounded once, and its code goes both to W's codes
 // (packed along rows, [R, C/2]) and, when asked, to W^T's codes (packed along
 // W's columns, [C, R/2]), each row or column segment carrying the tile's
-// scale byte.  A CTA stages a (4 x block) x 64 bf16 tile in shared memory;
-// `block` consecutive threads own one square tile, one row segment each: the
-// tile amax is a shuffle reduction over them, and the row segment is quantized
-// like a 1-D block (same Philox indices).  The codes are parked in shared
-// memory one per byte; then one thread per tile row writes W's 32 code bytes
-// of that row and one thread per tile column packs and writes W^T's.
+// scale byte.  A CTA takes (4 x block) x 64 tiles of W; thread t owns the row
+// segment (row t % (4 block), block columns of segment t / (4 block)), so the
+// `block` rows of a square tile sit on consecutive lanes: the tile amax is a
+// shuffle reduction, and each row segment is quantized like a 1-D block (same
+// Philox indices).  Tiles arrive in shared memory by coalesced 16-byte async
+// copies (8 lanes per 128-byte row; the next tile's in flight while the
+// current one is processed), their 16-byte chunks XOR-swizzled by row so that
+// the lanes' row-segment reads are conflict-free.  W's codes
+// leave as the packed words of each row; W^T's come from 8 x 8 nibble
+// transposes across groups of 8 lanes (three shuffle stages), and both are
+// gathered in shared memory so that one thread writes a whole output row
+// segment (32 bytes of W, 32 or 64 bytes of W^T) with sector-wide stores.
 struct Q2Params {
   const uint16_t* x;
   uint32_t R, C;
@@ -976,19 +982,59 @@ struct Q2Params {
   uint32_t g4, g4_t;     // padded groups / 4 of the two scale tensors (tensor-core layout)
 };
 
+// Transpose of the 8 x 8 nibble matrix held by the 8 lanes of an aligned lane group (lane j: row
+// j, nibble i = column i): on return lane i holds column i (nibble j = row j).  Every lane of the
+// warp must call it.
+__device__ __forceinline__ uint32_t nibble_transpose8(uint32_t v, int lane) {
+  uint32_t o = __shfl_xor_sync(0xFFFFFFFFu, v, 4);
+  v = (lane & 4) ? ((v & 0xFFFF0000u) | (o >> 16)) : ((v & 0x0000FFFFu) | (o << 16));
+  o = __shfl_xor_sync(0xFFFFFFFFu, v, 2);
+  v = (lane & 2) ? ((v & 0xFF00FF00u) | ((o & 0xFF00FF00u) >> 8)) : ((v & 0x00FF00FFu) | ((o & 0x00FF00FFu) << 8));
+  o = __shfl_xor_sync(0xFFFFFFFFu, v, 1);
+  v = (lane & 1) ? ((v & 0xF0F0F0F0u) | ((o & 0xF0F0F0F0u) >> 4)) : ((v & 0x0F0F0F0Fu) | ((o & 0x0F0F0F0Fu) << 4));
+  return v;
+}
+
+// N bytes of words (N = 32 or 64) to dst, of which the first n (a multiple of 8) are written:
+// 32-byte stores (mode 32: dst 32-byte aligned and n == N), 16-byte (mode 16) or 8-byte stores.
+template <int N>
+__device__ __forceinline__ void store_segment(uint8_t* dst, const uint32_t (&w)[N / 4], uint32_t n, int mode) {
+  if (n == N && mode == 32) {
+#pragma unroll
+    for (int k = 0; k < N / 32; ++k)
+      asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(dst + 32 * k), "r"(w[8 * k]),
+                   "r"(w[8 * k + 1]), "r"(w[8 * k + 2]), "r"(w[8 * k + 3]), "r"(w[8 * k + 4]), "r"(w[8 * k + 5]),
+                   "r"(w[8 * k + 6]), "r"(w[8 * k + 7])
+                   : "memory");
+  } else if (n == N && mode == 16) {
+#pragma unroll
+    for (int k = 0; k < N / 16; ++k)
+      reinterpret_cast<uint4*>(dst)[k] = make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
+  } else {
+#pragma unroll
+    for (int k = 0; k < N / 8; ++k)
+      if (8u * k < n) reinterpret_cast<uint2*>(dst)[k] = make_uint2(w[2 * k], w[2 * k + 1]);
+  }
+}
+
 template <int FMT, int RND, bool SFMMA>
 __global__ void __launch_bounds__(256) quantize_2d_kernel(Q2Params p) {
   pdl_trigger();
   constexpr int BS = FMT == FMT_MX ? 32 : 16;
   constexpr int TR = 4 * BS, TC = 64;                     // CTA tile: (4 x block) rows x 64 columns
-  constexpr int SPR = TC / BS;                            // square tiles across the CTA tile
-  __shared__ __align__(16) uint16_t tile[TR][TC + 8];     // 144-byte rows: 16-byte loads of 16 rows hit 2-way
-  __shared__ __align__(16) uint8_t code_sm[TR][TC + 4];    // 68-byte rows
-  __shared__ uint8_t tile_byte[4][SPR];
+  constexpr int SEGS = TC / BS;                           // row segments (square tiles) across the CTA tile
+  constexpr int V = BS / 8;                               // 16-byte chunks (and code words) per segment
+  constexpr int RG = TR / 8;                              // 8-row groups
+  constexpr int ROWW = TC / 8 + 1;                        // W words per row (+1: conflict-free parking)
+  constexpr int COLW = RG + 4;                             // W^T words per column (+4: 16-byte rows, no conflicts)
+  __shared__ __align__(16) uint4 xin[2][TR * 8];       // two input tiles: row r, chunk j at r * 8 + (j ^ r % 8)
+  __shared__ uint32_t code_row[TR * ROWW];
+  __shared__ __align__(16) uint32_t code_col[TC * COLW];
+  __shared__ uint8_t sc_row[TR][SEGS];
+  __shared__ uint8_t sc_col[TC][4];
   __shared__ float2 tab[128];
-  const int tid = threadIdx.x;
-  const int sq = tid / BS, rr = tid % BS;                 // square tile of the thread, its row in it
-  const int sq_r = sq / SPR, sq_c = sq % SPR;
+  const int tid = threadIdx.x, lane = tid & 31;
+  const int row = tid % TR, seg = tid / TR;
   pdl_wait();
   float s_t = 1.0f, y_st = 1.0f;
   bool st_ok = true;
@@ -996,25 +1042,54 @@ __global__ void __launch_bounds__(256) quantize_2d_kernel(Q2Params p) {
     s_t = *p.ts;
     y_st = __frcp_rn(s_t);
     st_ok = recip_usable(s_t);
-    nv_fill_scale_table(tab, s_t);                        // visible after the tile loop's first barrier
+    nv_fill_scale_table(tab, s_t);
     if (p.ts_copy_out != nullptr && blockIdx.x == 0 && tid == 0) *p.ts_copy_out = s_t;
   }
+  __syncthreads();                                        // the scale table is read by the first tile
+  // store widths of the two outputs (rows of W's codes are C/2 bytes apart, of W^T's R/2)
+  auto mode_of = [](const void* base, uint32_t pitch) {
+    const uintptr_t a = reinterpret_cast<uintptr_t>(base);
+    return (a % 32 == 0 && pitch % 32 == 0) ? 32 : (a % 16 == 0 && pitch % 16 == 0) ? 16 : 8;
+  };
+  const int mode_w = mode_of(p.codes, p.C / 2);
+  const int mode_t = p.codes_t != nullptr ? mode_of(p.codes_t, p.R / 2) : 8;
   const uint32_t tiles_r = (p.R + TR - 1) / TR, tiles_c = (p.C + TC - 1) / TC;
-  for (uint32_t t = blockIdx.x; t < tiles_r * tiles_c; t += gridDim.x) {
-    const uint32_t r0 = (t / tiles_c) * TR, c0 = (t % tiles_c) * TC;
-    __syncthreads();                                      // the previous tile's shared data is consumed
-    for (int i = tid; i < TR * (TC / 8); i += 256) {
-      const int row = i / (TC / 8), ch = i % (TC / 8);
-      const uint32_t gr = r0 + row, gc = c0 + ch * 8;
-      uint4 v = make_uint4(0u, 0u, 0u, 0u);
-      if (gr < p.R && gc < p.C) v = ld_stream(p.x + (int64_t)gr * p.ld + gc);
-      *reinterpret_cast<uint4*>(&tile[row][ch * 8]) = v;
+  const uint32_t ntiles = tiles_r * tiles_c;
+  // async copies of tile t into buffer b: thread i moves chunks i, i + 256, ... (row q / 8,
+  // chunk q % 8); chunks outside the matrix are zero-filled
+  auto issue = [&](uint32_t t, int b) {
+    if (t < ntiles) {
+      const uint32_t r0 = (t / tiles_c) * TR, c0 = (t % tiles_c) * TC;
+#pragma unroll
+      for (int q = tid; q < TR * 8; q += 256) {
+        const uint32_t r = (uint32_t)q / 8u, j = (uint32_t)q % 8u;
+        const uint32_t gr = r0 + r, gc = c0 + 8u * j;
+        const uint32_t dst = smem_addr(&xin[b][r * 8 + (j ^ (r % 8u))]);
+        const bool in = gr < p.R && gc < p.C;
+        const uint16_t* src = in ? p.x + (int64_t)gr * p.ld + gc : p.x;
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(in ? 16 : 0)
+                     : "memory");
+      }
     }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  };
+  issue(blockIdx.x, 0);
+  int buf = 0;
+  for (uint32_t t = blockIdx.x; t < ntiles; t += gridDim.x, buf ^= 1) {
+    issue(t + gridDim.x, buf ^ 1);                        // in flight while this tile is processed
+    asm volatile("cp.async.wait_group 1;" ::: "memory");  // this tile's copies have landed
     __syncthreads();
-    const uint32_t row = r0 + sq_r * BS + rr, col = c0 + sq_c * BS;   // this thread's row segment
+    const uint32_t r0 = (t / tiles_c) * TR, c0 = (t % tiles_c) * TC;
+    const uint32_t grow = r0 + row, gcol = c0 + seg * BS;
     float x[BS];
 #pragma unroll
-    for (int i = 0; i < BS; ++i) x[i] = __uint_as_float((uint32_t)tile[sq_r * BS + rr][sq_c * BS + i] << 16);
+    for (int k = 0; k < V; ++k) {
+      const uint32_t j = (uint32_t)(seg * V + k);
+      float t8[8];
+      unpack8(xin[buf][row * 8 + (j ^ ((uint32_t)row % 8u))], t8);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) x[8 * k + i] = t8[i];
+    }
     float am = 0.0f;
 #pragma unroll
     for (int i = 0; i < BS; ++i) am = fmaxf(am, fabsf(x[i]));
@@ -1031,25 +1106,18 @@ __global__ void __launch_bounds__(256) quantize_2d_kernel(Q2Params p) {
     } else {
       byte = e4m3_rn_sat(nv_scale_arg(am, s_t, y_st, st_ok));
       zero = (byte == 0u);
-      const float2 sy = tab[byte];
-      if (nv_fast_division<RND, BS>(x, am, sy.x, sy.y)) {
-#pragma unroll
-        for (int i = 0; i < BS; ++i) x[i] = div_by_recip(x[i], sy.x, sy.y);
-      } else {
-#pragma unroll
-        for (int i = 0; i < BS; ++i) x[i] = __fdiv_rn(x[i], sy.x);
-      }
+      nv_divide_block<RND, BS>(x, am, tab[byte], x);
     }
-    uint32_t w[BS / 8];
+    uint32_t w[V];
     if (RND == RND_RTN) {
 #pragma unroll
-      for (int k = 0; k < BS / 8; ++k)
+      for (int k = 0; k < V; ++k)
         w[k] = e2m1x4_rn(x[8 * k], x[8 * k + 1], x[8 * k + 2], x[8 * k + 3], x[8 * k + 4], x[8 * k + 5], x[8 * k + 6],
                          x[8 * k + 7]);
     } else {
-      const unsigned long long j0 = ((unsigned long long)row * p.C + col) >> 2;   // col % 4 == 0
+      const unsigned long long j0 = ((unsigned long long)grow * p.C + gcol) >> 2;   // gcol % 4 == 0
 #pragma unroll
-      for (int k = 0; k < BS / 8; ++k) {
+      for (int k = 0; k < V; ++k) {
         const unsigned long long j = j0 + 2u * k;
         const u32x4 a = philox4x32_10((uint32_t)j, (uint32_t)(j >> 32), p.keys);
         const u32x4 b = philox4x32_10((uint32_t)(j + 1), (uint32_t)((j + 1) >> 32), p.keys);
@@ -1061,61 +1129,61 @@ __global__ void __launch_bounds__(256) quantize_2d_kernel(Q2Params p) {
     }
     if (zero) {
 #pragma unroll
-      for (int k = 0; k < BS / 8; ++k) w[k] = 0u;
+      for (int k = 0; k < V; ++k) w[k] = 0u;
     }
-    // park the codes one per byte (row rr of the square tile) and the tile's scale byte
+    uint32_t wt[V];
 #pragma unroll
-    for (int k = 0; k < BS / 8; ++k)
+    for (int k = 0; k < V; ++k) wt[k] = nibble_transpose8(w[k], lane);   // column 8k + lane % 8, 8 rows
+    __syncthreads();                                      // the previous tile's write-out read its data
 #pragma unroll
-      for (int i = 0; i < 8; ++i) code_sm[sq_r * BS + rr][sq_c * BS + 8 * k + i] = (uint8_t)((w[k] >> (4 * i)) & 0xFu);
-    if (rr == 0) tile_byte[sq_r][sq_c] = (uint8_t)byte;
+    for (int k = 0; k < V; ++k) {
+      code_row[row * ROWW + seg * V + k] = w[k];
+      code_col[(seg * BS + 8 * k + (lane & 7)) * COLW + row / 8] = wt[k];
+    }
+    sc_col[seg * BS + row % BS][row / BS] = (uint8_t)byte;
+    sc_row[row][seg] = (uint8_t)byte;
     __syncthreads();
-    // write-out: one thread per tile row (W, 32 code bytes per row) and, when asked, one per tile
-    // column (W^T, TR/2 code bytes per column): whole sectors instead of 8-byte pieces
-    const uint32_t vcols = min((uint32_t)TC, p.C > c0 ? p.C - c0 : 0u);      // multiple of the block
+    const uint32_t vcols = min((uint32_t)TC, p.C > c0 ? p.C - c0 : 0u);      // multiples of the block
     const uint32_t vrows = min((uint32_t)TR, p.R > r0 ? p.R - r0 : 0u);
     if (tid < TR) {
       const uint32_t lr = (uint32_t)tid;
       if (lr < vrows) {
-        uint8_t* dst = p.codes + (size_t)(r0 + lr) * (p.C / 2) + c0 / 2;
-        for (uint32_t c = 0; c < vcols; c += 16) {                              // 8 bytes per 16 codes
-          uint32_t lo = 0u, hi = 0u;
+        uint32_t o[8];
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            lo |= (uint32_t)code_sm[lr][c + i] << (4 * i);
-            hi |= (uint32_t)code_sm[lr][c + 8 + i] << (4 * i);
-          }
-          *reinterpret_cast<uint2*>(dst + c / 2) = make_uint2(lo, hi);
-        }
-        for (uint32_t c = 0; c < vcols; c += BS) {
-          const uint8_t b = tile_byte[lr / BS][c / BS];
-          const uint32_t g = (c0 + c) / BS;
-          if (SFMMA) p.scales[sf_mma_offset(r0 + lr, g, p.g4)] = b;
-          else p.scales[(size_t)(r0 + lr) * (p.C / BS) + g] = b;
+        for (int k = 0; k < 8; ++k) o[k] = code_row[lr * ROWW + k];
+        store_segment<32>(p.codes + (size_t)(r0 + lr) * (p.C / 2) + c0 / 2, o, vcols / 2, mode_w);
+#pragma unroll
+        for (int g = 0; g < SEGS; ++g) {
+          if ((uint32_t)(g * BS) >= vcols) break;
+          const uint32_t gg = c0 / BS + g;
+          if (SFMMA) p.scales[sf_mma_offset(r0 + lr, gg, p.g4)] = sc_row[lr][g];
+          else p.scales[(size_t)(r0 + lr) * (p.C / BS) + gg] = sc_row[lr][g];
         }
       }
     } else if (p.codes_t != nullptr && tid < TR + TC) {
       const uint32_t lc = (uint32_t)(tid - TR);
       if (lc < vcols) {
-        uint8_t* dst = p.codes_t + (size_t)(c0 + lc) * (p.R / 2) + r0 / 2;
-        for (uint32_t r = 0; r < vrows; r += 16) {
-          uint32_t lo = 0u, hi = 0u;
+        uint32_t o[RG];
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            lo |= (uint32_t)code_sm[r + i][lc] << (4 * i);
-            hi |= (uint32_t)code_sm[r + 8 + i][lc] << (4 * i);
-          }
-          *reinterpret_cast<uint2*>(dst + r / 2) = make_uint2(lo, hi);
+        for (int k = 0; k < RG / 4; ++k) {
+          const uint4 q = *reinterpret_cast<const uint4*>(&code_col[lc * COLW + 4 * k]);
+          o[4 * k] = q.x;
+          o[4 * k + 1] = q.y;
+          o[4 * k + 2] = q.z;
+          o[4 * k + 3] = q.w;
         }
-        for (uint32_t r = 0; r < vrows; r += BS) {
-          const uint8_t b = tile_byte[r / BS][lc / BS];
-          const uint32_t g = (r0 + r) / BS;
-          if (SFMMA) p.scales_t[sf_mma_offset(c0 + lc, g, p.g4_t)] = b;
-          else p.scales_t[(size_t)(c0 + lc) * (p.R / BS) + g] = b;
+        store_segment<TR / 2>(p.codes_t + (size_t)(c0 + lc) * (p.R / 2) + r0 / 2, o, vrows / 2, mode_t);
+#pragma unroll
+        for (int a = 0; a < 4; ++a) {
+          if ((uint32_t)(a * BS) >= vrows) break;
+          const uint32_t gg = r0 / BS + a;
+          if (SFMMA) p.scales_t[sf_mma_offset(c0 + lc, gg, p.g4_t)] = sc_col[lc][a];
+          else p.scales_t[(size_t)(c0 + lc) * (p.R / BS) + gg] = sc_col[lc][a];
         }
       }
     }
   }
+  asm volatile("cp.async.wait_group 0;" ::: "memory");   // no copy outlives the CTA
 }
 
 // ============================================================ dequantize ===
