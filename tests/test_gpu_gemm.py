@@ -78,6 +78,24 @@ def test_gemm_shapes(mnk, fmt):
     F.fp4_check_device_errors()
 
 
+@pytest.mark.parametrize("fmt", ["mxfp4", "nvfp4"])
+def test_pair_tiles_ragged_edges(fmt):
+    """2400 x 1900 x 2048: enough 256 x 256 tiles for the SM-pair kernel, with the last row tile's
+    second 128-row half and the last column tile's second 128-row scale block outside the operands
+    (their boxes read the tensor map's zero fill)."""
+    M, N, K = 2400, 1900, 2048
+    g = np.random.default_rng(77)
+    from workloads import bf16_bits
+    a = bf16_bits(g.standard_normal((M, K)).astype(np.float32))
+    b = bf16_bits((g.standard_normal((N, K)) * 0.02).astype(np.float32))
+    qa, qb = _gpu_quant(dev_bf16(a), fmt), _gpu_quant(dev_bf16(b), fmt)
+    y32 = F.fp4_gemm(qa.codes, qa.scales, qb.codes, qb.scales, fmt=fmt, a_tensor_scale=qa.tensor_scale,
+                     b_tensor_scale=qb.tensor_scale, out_dtype="f32")
+    yr, bd = O.gemm_ref(_as_oracle(qa, fmt, M, K), _as_oracle(qb, fmt, N, K), fmt)
+    _check(host_f32(y32), yr, bd)
+    F.fp4_check_device_errors()
+
+
 def test_gemm_strided_output():
     M, N, K = 64, 96, 256
     g = np.random.default_rng(1)
