@@ -69,7 +69,8 @@ extern "C" {
 typedef int fp4_status;
 enum {
   FP4_OK = 0,
-  FP4_ERR_ARG = -1,          /* null pointer, bad enum value, negative size       */
+  FP4_ERR_ARG = -1,          /* null pointer, bad enum value, size not positive
+                                (empty tensors are rejected, nothing launched)    */
   FP4_ERR_SHAPE = -2,        /* size not a multiple of what the format needs     */
   FP4_ERR_ALIGN = -3,        /* pointer or leading dimension misaligned          */
   FP4_ERR_UNSUPPORTED = -4,  /* (format, block) or option combination not built  */

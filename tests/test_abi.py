@@ -128,3 +128,30 @@ def test_other_entry_points_reject_before_launch(lib):
     assert lib.fp4_quantize_dequantize(FAKE, 4, 64, 64, 2, 16, 0, 0, None, FAKE, FAKE, FAKE, 0, FAKE, 0, None) == -4
     assert lib.fp4_quantize_dequantize(FAKE, 4, 64, 64, 0, 32, 0, 0, None, None, FAKE, FAKE, 0, FAKE + 4, 0,
                                        None) == -3
+
+
+@pytest.mark.parametrize("rows, cols", [(0, 64), (64, 0), (0, 0), (-1, 64)])
+def test_empty_and_negative_shapes_rejected(lib, rows, cols):
+    """Zero-sized (and negative) tensors are argument errors at every entry point, returned before
+    any CUDA call; the size helpers report 0 bytes for them."""
+    assert lib.fp4_quantize(FAKE, rows, cols, max(cols, 1), 0, 32, 1, 0, 0, None, None, FAKE, FAKE, 0, None) == -1
+    assert lib.fp4_quantize(FAKE, rows, cols, max(cols, 1), 1, 16, 1, 0, 0, None, FAKE, FAKE, FAKE, 0, None) == -1
+    assert lib.fp4_hadamard_quantize(FAKE, rows, cols, max(cols, 1), 0, 32, 1, 0, 0, None, None, FAKE, FAKE, 0, 32,
+                                     None, None) == -1
+    assert lib.fp4_quantize_dequantize(FAKE, rows, cols, max(cols, 1), 0, 32, 0, 0, None, None, FAKE, FAKE, 0, FAKE,
+                                       0, None) == -1
+    assert lib.fp4_quantize_2d(FAKE, rows, cols, max(cols, 1), 0, 32, 0, 0, None, None, FAKE, FAKE, None, None, 0,
+                               None) == -1
+    assert lib.fp4_quantize_mse(FAKE, rows, cols, max(cols, 1), 1, 16, 0, 0, 1, FAKE, FAKE, FAKE, 0, None) == -1
+    assert lib.fp4_dequantize(FAKE, FAKE, None, rows, cols, 0, 32, 0, FAKE, 0, None) == -1
+    assert lib.fp4_amax(FAKE, rows, cols, max(cols, 1), FAKE, None) == -1
+    assert lib.fp4_codes_bytes(rows, cols) == 0
+    assert lib.fp4_scales_bytes(rows, cols, 32, 1, 0) == 0
+
+
+@pytest.mark.parametrize("mnk", [(0, 64, 64), (64, 0, 64), (64, 64, 0), (-128, 64, 64)])
+def test_empty_gemm_rejected(lib, mnk):
+    M, N, K = mnk
+    assert lib.fp4_gemm(FAKE, FAKE, None, FAKE, FAKE, None, M, N, K, 0, 32, FAKE, max(N, 1), 0, None) == -1
+    assert lib.fp4_gemm_quantize(FAKE, FAKE, None, FAKE, FAKE, None, M, N, K, 0, 32, 0, 32, 0, 0, None, FAKE, FAKE, 0,
+                                 None) == -1
