@@ -778,24 +778,25 @@ __global__ void __launch_bounds__(FusedWarps<FMT>::kThreads, 1) nv_quantize_fuse
 }
 
 // ======================================================== axis-0 quantize ===
-// 4 x 4 transpose of 32-bit words across the four lanes of a quad: on entry
-// lane q holds row q (w[0..3]); on return t[s] is word q of row s.  In round
-// k lane q reads from lane s = (q + k) & 3, which sends its word (s - k) & 3,
-// that is word q.  Every lane of the warp must call it.
+// 4 x 4 transpose of 32-bit words across the four lanes of a quad: on entry lane q holds row q
+// (w[0..3], one word per column); on return t[s] is word q of row s.  Two butterfly stages: with
+// lane q ^ 1 swap the two words of the columns whose bit 0 differs from q's, then with lane q ^ 2
+// the two (of four held) whose bit 1 differs; lane q then holds column q of rows q, q ^ 1, q ^ 2,
+// q ^ 3, which two conditional swaps put in row order.  Every lane of the warp must call it.
 __device__ __forceinline__ void quad_transpose4(const uint32_t (&w)[4], uint32_t (&t)[4], int lane) {
-  const int q = lane & 3;
-  t[0] = t[1] = t[2] = t[3] = 0u;
-#pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    const int si = (q - k) & 3;
-    const uint32_t send = si == 0 ? w[0] : (si == 1 ? w[1] : (si == 2 ? w[2] : w[3]));
-    const uint32_t recv = __shfl_sync(0xFFFFFFFFu, send, (lane & ~3) | ((q + k) & 3));
-    const int row = (q + k) & 3;
-    t[0] = row == 0 ? recv : t[0];
-    t[1] = row == 1 ? recv : t[1];
-    t[2] = row == 2 ? recv : t[2];
-    t[3] = row == 3 ? recv : t[3];
-  }
+  const bool b0 = (lane & 1) != 0, b1 = (lane & 2) != 0;
+  const uint32_t o0 = b0 ? w[1] : w[0], o1 = b0 ? w[3] : w[2];            // own columns with bit 0 = q0
+  const uint32_t r0 = __shfl_xor_sync(0xFFFFFFFFu, b0 ? w[0] : w[1], 1);  // row q ^ 1, columns q0, 2 + q0
+  const uint32_t r1 = __shfl_xor_sync(0xFFFFFFFFu, b0 ? w[2] : w[3], 1);
+  const uint32_t a0 = b1 ? o1 : o0, a1 = b1 ? r1 : r0;                     // column q of rows q, q ^ 1
+  const uint32_t a2 = __shfl_xor_sync(0xFFFFFFFFu, b1 ? o0 : o1, 2);      // column q of row q ^ 2
+  const uint32_t a3 = __shfl_xor_sync(0xFFFFFFFFu, b1 ? r0 : r1, 2);      // column q of row q ^ 3
+  // t[s] = a[s ^ q]
+  const uint32_t u0 = b0 ? a1 : a0, u1 = b0 ? a0 : a1, u2 = b0 ? a3 : a2, u3 = b0 ? a2 : a3;
+  t[0] = b1 ? u2 : u0;
+  t[1] = b1 ? u3 : u1;
+  t[2] = b1 ? u0 : u2;
+  t[3] = b1 ? u1 : u3;
 }
 
 // Blocks run down the columns of x[R, C]; the output is written transposed
@@ -822,7 +823,7 @@ struct QColParams {
 };
 
 template <int FMT, int RND, bool SFMMA>
-__global__ void __launch_bounds__(256, 2) quantize_cols_kernel(QColParams p) {
+__global__ void __launch_bounds__(256, (RND == RND_SR && FMT != FMT_NV46) ? 3 : 2) quantize_cols_kernel(QColParams p) {
   pdl_trigger();
   __shared__ __align__(16) uint16_t tile[128][64];
   __shared__ float2 tab[128];
