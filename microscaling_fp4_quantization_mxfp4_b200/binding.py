@@ -70,14 +70,20 @@ def _bf16_matrix(x: torch.Tensor, name: str = "x") -> None:
 
 
 def fp4_codes_bytes(rows: int, cols: int) -> int:
+    """Bytes of packed codes for a [rows, cols] tensor (two E2M1 codes per byte); 0 for an empty
+    or odd-sized tensor."""
     return _lib.load().fp4_codes_bytes(rows, cols)
 
 
 def fp4_scales_bytes(rows: int, cols: int, block: int, axis: int, sf_layout="rowmajor") -> int:
+    """Bytes of block scales for a [rows, cols] tensor quantized along `axis` in `block`-element
+    blocks: one byte per block row-major, or the tensor-core layout padded to 128 rows x 4 block
+    columns ("mma"); 0 for an invalid shape."""
     return _lib.load().fp4_scales_bytes(rows, cols, block, axis, _SF[sf_layout])
 
 
 def fp4_status_string(status: int) -> str:
+    """Short message for an fp4_status code (e.g. "invalid argument" for FP4_ERR_ARG)."""
     return _lib.load().fp4_status_string(status).decode()
 
 
