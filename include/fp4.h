@@ -292,11 +292,18 @@ fp4_status fp4_amax(const void* x, int64_t rows, int64_t cols, int64_t ld,
  *   the process exits.  One CTA covers 8192 elements, so inputs are limited to
  *   rows * cols <= 2^26 (67,108,864) elements; larger inputs return
  *   FP4_ERR_SHAPE.  Other requirements and errors as fp4_amax.
- *   The first call on each device looks up the array's device address
- *   (cudaGetSymbolAddress) with that device current; make that first call
- *   before any stream capture.  Every call resets the counter, and all calls
- *   share the one array: calls that overlap on the GPU (e.g. on two streams)
- *   race, so the caller must serialize them.
+ *   Set-up: the first call on each device (and the first after that device's
+ *   context was destroyed and created again, e.g. by cudaDeviceReset), made
+ *   with that device current, loads the library's amax kernel and looks up
+ *   the array's device address (cudaGetSymbolAddress).  Under CUDA's lazy
+ *   module loading this is where the kernel's code and the array first take
+ *   device memory, so the first call can fail with FP4_ERR_CUDA when no device
+ *   memory is left.  Make it early, as a warm-up (e.g. on a tiny tensor): before
+ *   a caching allocator takes all free memory, outside any allocator callback
+ *   and before any stream capture.  Later calls take no device memory.
+ *   Every call resets the counter, and all calls share the one array: calls
+ *   that overlap on the GPU (e.g. on two streams) race, so the caller must
+ *   serialize them (one stream, or events between the streams).
  */
 fp4_status fp4_amax_noalloc(const void* x, int64_t rows, int64_t cols, int64_t ld,
                             float* amax_out, void* stream);

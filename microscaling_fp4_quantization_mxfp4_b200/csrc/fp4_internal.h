@@ -104,6 +104,9 @@ cudaError_t launch_amax(const void* x, int64_t rows, int64_t cols, int64_t ld, i
 // amax pass (mode 0) with a caller-chosen grid; scratch must hold `grid` partials.
 cudaError_t launch_amax_fixed_grid(const void* x, int64_t rows, int64_t cols, int64_t ld, float* out,
                                    const Scratch& s, uint32_t grid, cudaStream_t st);
+// Loads launch_amax_fixed_grid's kernel onto the current device now (under lazy module loading it
+// would otherwise load, and take device memory, at its first launch).
+cudaError_t load_amax_fixed_grid_kernel();
 cudaError_t launch_nv_tensor_scale(const float* amax, float* out, cudaStream_t st);
 cudaError_t launch_quantize(const QuantizeParams& p, int num_sms, cudaStream_t st);
 // Square-tile (2-D) quantize along axis 1 (codes/scales) and, when codes_t is not null, the same

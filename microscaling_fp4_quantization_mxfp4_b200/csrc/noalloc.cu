@@ -8,7 +8,9 @@
 // code running inside an allocator callback, where calling back into the CUDA
 // allocator is not allowed.  For them this entry point keeps its scratch in a
 // fixed array compiled into the library instead.
+#include <cuda.h>
 #include <cuda_runtime.h>
+#include <cudaTypedefs.h>
 #include <stdint.h>
 
 #include <mutex>
@@ -30,21 +32,63 @@ constexpr size_t kScratchBytes = kCounterOffset + 256;      // 33,024 bytes in t
 static __device__ __align__(256) unsigned char fp4_noalloc_scratch[kScratchBytes];
 
 constexpr int kMaxDevices = 64;
-std::mutex g_mutex;
-void* g_scratch[kMaxDevices] = {};
 
-// Device address of the array on the current device, looked up once per
-// device (the host-side symbol is only a stand-in and must never reach a kernel).
+// Per-device set-up, keyed by the identifier of the context it was done in: a
+// context that was destroyed and created again (cudaDeviceReset) may hold the
+// array at another address, so a new context repeats the set-up.
+struct Setup {
+  unsigned long long ctx_id = 0;   // 0: not done (context identifiers start at 1)
+  void* scratch = nullptr;
+};
+
+std::mutex g_mutex;
+Setup g_setup[kMaxDevices];
+PFN_cuCtxGetCurrent_v4000 g_ctx_current = nullptr;
+PFN_cuCtxGetId_v12000 g_ctx_id = nullptr;
+std::once_flag g_entry_once;
+
+// Identifier of the calling thread's current context, or 0 when it cannot be read.
+unsigned long long current_context_id() {
+  std::call_once(g_entry_once, [] {
+    void* f0 = nullptr;
+    void* f1 = nullptr;
+    cudaDriverEntryPointQueryResult q0, q1;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f0, cudaEnableDefault, &q0) == cudaSuccess &&
+        q0 == cudaDriverEntryPointSuccess &&
+        cudaGetDriverEntryPoint("cuCtxGetId", &f1, cudaEnableDefault, &q1) == cudaSuccess &&
+        q1 == cudaDriverEntryPointSuccess) {
+      g_ctx_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(f0);
+      g_ctx_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(f1);
+    }
+  });
+  if (g_ctx_current == nullptr || g_ctx_id == nullptr) return 0;
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (g_ctx_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return 0;
+  if (g_ctx_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
+
+// Device address of the array on the current device.  The set-up, done once per device and
+// context with that device current, loads the amax kernel and looks up the array's address
+// (cudaGetSymbolAddress also loads this file's device code).  Under lazy module loading these two
+// steps are where the library's code and the array first take device memory; later calls take
+// none.  The host-side symbol is only a stand-in and must never reach a kernel.
 fp4_status scratch_address(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FP4_ERR_CUDA;
   std::lock_guard<std::mutex> lock(g_mutex);
-  if (g_scratch[dev] == nullptr) {
+  Setup& s = g_setup[dev];
+  unsigned long long id = current_context_id();
+  if (id == 0 || s.ctx_id != id || s.scratch == nullptr) {
+    if (fp4lib::load_amax_fixed_grid_kernel() != cudaSuccess) return FP4_ERR_CUDA;
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, fp4_noalloc_scratch) != cudaSuccess || p == nullptr) return FP4_ERR_CUDA;
-    g_scratch[dev] = p;
+    if (id == 0) id = current_context_id();   // the runtime calls above made the context current
+    s.scratch = p;
+    s.ctx_id = id;                             // stays 0 (set-up on every call) if ids are unreadable
   }
-  *out = g_scratch[dev];
+  *out = s.scratch;
   return FP4_OK;
 }
 

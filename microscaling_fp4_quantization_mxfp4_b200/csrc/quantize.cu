@@ -1477,6 +1477,11 @@ cudaError_t launch_amax_fixed_grid(const void* x, int64_t rows, int64_t cols, in
   return launch_kernel(amax_kernel<0>, dim3(grid), dim3(256), 0, st, false, 1u, ap);
 }
 
+cudaError_t load_amax_fixed_grid_kernel() {
+  cudaFuncAttributes a;
+  return cudaFuncGetAttributes(&a, amax_kernel<0>);
+}
+
 cudaError_t launch_nv_tensor_scale(const float* amax, float* out, cudaStream_t st) {
   return launch_kernel(nv_tensor_scale_kernel, dim3(1), dim3(1), 0, st, false, 1u, amax, out);
 }
