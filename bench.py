@@ -89,11 +89,15 @@ class ClockSampler:
             except subprocess.TimeoutExpired:
                 self.proc.kill()
 
-    def summary(self):
+    def summary(self, t_start=None, t_end=None):
+        """Median SM clock, max clock and active throttle reasons over the samples taken inside
+        [t_start, t_end] (default: the main timed window); the nearest sample if none fell inside."""
+        t_start = self.t_start if t_start is None else t_start
+        t_end = self.t_end if t_end is None else t_end
         if not self.samples:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
-        inside = [s for t, s in self.samples if self.t_start <= t <= self.t_end]
-        used = inside if inside else [min(self.samples, key=lambda ts: abs(ts[0] - self.t_end))[1]]
+        inside = [s for t, s in self.samples if t_start <= t <= t_end]
+        used = inside if inside else [min(self.samples, key=lambda ts: abs(ts[0] - t_end))[1]]
         sm = [float(s[0]) for s in used if s[0].replace(".", "").isdigit()]
         mx = [float(s[1]) for s in used if s[1].replace(".", "").isdigit()]
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
@@ -156,6 +160,7 @@ class NvfpStudentT(Workload):
     n_inputs = 4                 # rotating input copies: 128 MB of inputs, each step writes ~146 MB
     launches_per_step = 2        # single-pass amax + quantize + dequantize (RTN), quantize + dequantize (SR)
     unit = "GB/s"
+    gemm_companion = True        # the line also carries the GEMM half of the metric (b = 128 Hadamard GEMM)
 
     def __init__(self, torch, F):
         self.t, self.F = torch, F
@@ -241,6 +246,14 @@ class NvfpStudentT(Workload):
                 "amax+quantize_dequantize_rtn": self.q_bytes + self.d_bytes,
                 "quantize_dequantize_sr": self.q_bytes + self.d_bytes}[key]
 
+    def family_launches(self, key):
+        """Launches of a kernel family per step."""
+        return 2 if key == "dequantize" else 1
+
+    def family_elements(self, key):
+        """Elements a kernel family processes per step (each launch covers the whole tensor)."""
+        return self.n * self.family_launches(key)
+
     def value_from_ms(self, ms_per_step, n_ranks):
         return self.step_bytes * n_ranks / (ms_per_step * 1e-3) / 1e9
 
@@ -282,6 +295,7 @@ class NvfpStudentT46(NvfpStudentT):
     fmt = "nvfp4_4o6"
     fused_deq = False            # four-over-six quantizes, then a separate dequantize launch
     launches_per_step = 4
+    gemm_companion = False
 
     def cpu_sample(self):
         return 512, f"512 of {self.rows} rows (global tensor scale), NumPy elementwise (1 thread)"
@@ -574,6 +588,21 @@ class HadamardMxGemm(GemmWorkload):
 
     def reference_sample(self):
         return 16, "b = 128: rotate+quantize 16 rows of X and their fp64 GEMM against 256 rows of W (NumPy)"
+
+
+class HadamardMxGemm128(HadamardMxGemm):
+    """The Hadamard workload at one block size, b = 128: one rotate+quantize of X[8192,4096] and one
+    GEMM against W[11008,4096] per step.  The default workload's line carries it as the GEMM half of
+    the metric."""
+
+    name = "hadamard_mxfp4_gemm_8192x11008x4096_b128"
+    blocks = (128,)
+    launches_per_step = 2
+
+    def release(self):
+        for a in ("x", "qw", "codes", "scales", "outs", "host_in", "dev_in"):
+            if hasattr(self, a):
+                delattr(self, a)
 
 
 class FusedMxLinear(GemmWorkload):
@@ -953,7 +982,7 @@ class MxLinear128(GemmWorkload):
 
 
 WORKLOADS = {W.name: W for W in (NvfpStudentT, NvfpStudentT46, Nvfp2dWeight, NvfpMseWeight, HadamardMxGemm,
-                                  FusedMxLinear, VitLinears, LlamaNvfp4, MxLinear128)}
+                                  HadamardMxGemm128, FusedMxLinear, VitLinears, LlamaNvfp4, MxLinear128)}
 
 
 # ------------------------------------------------------------------ arms ---
@@ -1001,61 +1030,44 @@ def _nv_single_pass(rows, cols, num_sms):
     return per * 512 <= 227 * 1024 - 2048
 
 
-def run_fp4(args):
-    import torch
-    import microscaling_fp4_quantization_mxfp4_b200 as F
-    from microscaling_fp4_quantization_mxfp4_b200 import _lib
-    _lib.load()                                  # fail loudly when the CUDA library is missing
-    ws, rank, local, pg = _dist_setup(torch)
-    if not torch.cuda.is_available():
-        raise RuntimeError("bench.py needs a CUDA device")
-    device = torch.device("cuda", local)
-    W = WORKLOADS[args.workload](torch, F)
-    W.setup(device)
-    if isinstance(W, LlamaNvfp4):
-        sms = torch.cuda.get_device_properties(device).multi_processor_count
-        W.launches_per_step = sum(1 + (1 if _nv_single_pass(m, k, sms) else 2) for k, n, m in W.cases)
-
-    for i in range(args.warmup):
-        W.step(i)
-    F.fp4_check_device_errors()
-
-    sampler = ClockSampler(_smi_id(torch, local))
-    sampler.start()
-    time.sleep(0.3)                              # let the sampler produce its first line
+def _timed_steps(W, steps, torch, pg):
+    """K steps bracketed by a barrier + synchronize on both sides; returns (ms per step, max over
+    ranks; host window of the timed region)."""
     _barrier(torch, pg)
-    sampler.t_start = time.time()
+    t0 = time.time()
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     start.record()
-    for i in range(args.steps):
+    for i in range(steps):
         # bracketed workloads run the steps bare: events between kernels would serialize their
         # launches (no programmatic dependent launch overlap) and add ~3 us each
         W.step(i, timed=not W.bracket)
     end.record()
     torch.cuda.synchronize()
-    sampler.t_end = time.time()
+    t1 = time.time()
     _barrier(torch, pg)
-    sampler.stop()
-    F.fp4_check_device_errors()
     local_ms = start.elapsed_time(end) if W.bracket else W.timed_ms_total()
-    ms_total = _max_over_ranks(torch, pg, local_ms)
-    ms_step = ms_total / args.steps
-    value = W.value_from_ms(ms_step, ws)
+    return _max_over_ranks(torch, pg, local_ms) / steps, (t0, t1)
 
-    # per-kernel attribution: for bracketed workloads a second pass of the same steps with CUDA
-    # events around every launch (its per-launch durations include the event-serialized launch
-    # gaps, so the kernels' rates below are conservative against the headline pass)
-    attr_steps = args.steps
+
+def _attribution(W, steps, torch, pg, F):
+    """Per-family device time per step.  For bracketed workloads a second pass of the same steps with
+    CUDA events around every launch (its per-launch durations include the event-serialized launch
+    gaps, so the kernels' rates are conservative against the headline pass)."""
+    attr_steps = steps
     if W.bracket:
-        attr_steps = max(3, min(args.steps, 1000))
+        attr_steps = max(3, min(steps, 1000))
         _barrier(torch, pg)
         for i in range(attr_steps):
             W.step(i, timed=True)
         torch.cuda.synchronize()
         F.fp4_check_device_errors()
-
-    # dominant kernel: the single-kernel family with the largest share of device time
     fam_ms = {k: sum(a.elapsed_time(b) for a, b in tm.pairs) / attr_steps for k, tm in W.timers.items() if tm.pairs}
+    return attr_steps, fam_ms
+
+
+def _roofline(W, fam_ms, attr_steps, torch, pg, device):
+    """Roofline of the dominant single-kernel family (largest share of device time) and the rates of
+    every family."""
     dom = max((k for k in fam_ms if k in W.single_kernel()), key=lambda k: fam_ms[k])
     dom_ms = _max_over_ranks(torch, pg, fam_ms[dom])
     peaks = _peaks()
@@ -1083,6 +1095,18 @@ def run_fp4(args):
         roofline = {"kernel": dom, "bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
                     "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
                     "traffic": _load_traffic(W.name, dom), "peak_source": peaks["source"]}
+    l2w = _load_counter(W.name, dom, "l2_write_bytes_per_launch")
+    if l2w is not None:
+        # DRAM writes of a launch miss what is still in L2 when it ends; the bytes the SMs wrote
+        # to L2 confirm the written side instead
+        rd = _load_counter(W.name, dom, "dram_read_bytes_per_launch")
+        roofline["traffic_l2_writes"] = l2w
+        if rd is not None:
+            alg = W.family_work(dom) / (W.family_launches(dom) if hasattr(W, "family_launches") else 1)
+            roofline["traffic_read_plus_l2_writes_over_algorithmic"] = round((rd + l2w) / alg, 4)
+    issue = _issue_roofline(W, dom, dom_ms, torch, device)
+    if issue is not None:
+        roofline["issue"] = issue
     per_family = {}
     for k, ms in fam_ms.items():
         work = W.family_work(k)
@@ -1094,6 +1118,81 @@ def run_fp4(args):
             per_family[k] = {"us_per_step": round(ms * 1e3, 2), "gbs": round(work / (ms * 1e-3) / 1e9, 1)}
     roofline["per_kernel"] = per_family
     roofline["attribution_steps"] = attr_steps
+    return roofline
+
+
+def _issue_roofline(W, dom, dom_ms, torch, device):
+    """Instruction-issue roofline of the dominant kernel when ncu counted its instructions
+    (profiles/traffic.json: warp instructions executed per launch, from the same capture as its DRAM
+    bytes): achieved issue rate = counted warp instructions per step / device time; peak = SMs x 4
+    sub-partitions x 1 warp instruction per cycle x max SM clock."""
+    inst = _load_counter(W.name, dom, "warp_inst_per_launch")
+    if inst is None:
+        return None
+    launches = W.family_launches(dom) if hasattr(W, "family_launches") else 1
+    sms = torch.cuda.get_device_properties(device).multi_processor_count
+    peak = sms * 4 * 1965e6
+    achieved = inst * launches / (dom_ms * 1e-3)
+    elems = W.family_elements(dom) if hasattr(W, "family_elements") else None
+    out = {"bound": "alu", "achieved": round(achieved / 1e9, 1), "peak": round(peak / 1e9, 1),
+           "unit": "G warp instructions/s", "frac": round(achieved / peak, 4),
+           "peak_source": f"derived: {sms} SMs x 4 schedulers x 1 warp instruction per cycle x 1965 MHz",
+           "warp_inst_per_launch": inst}
+    if elems:
+        out["thread_inst_per_element"] = round(inst * 32 * launches / elems, 2)
+    return out
+
+
+def _run_companion(args, torch, F, device, pg, sampler):
+    """The block-scaled GEMM half of the metric, measured in the same process as the default
+    workload: rotate + quantize X[8192, 4096] with b = 128, then the MXFP4 GEMM against the offline
+    W[11008, 4096] with bf16 output, timed under the same clock sampler."""
+    W = HadamardMxGemm128(torch, F)
+    W.setup(device)
+    for i in range(max(3, min(args.warmup, 10))):
+        W.step(i)
+    F.fp4_check_device_errors()
+    steps = max(3, min(args.steps, 300))
+    ms_step, window = _timed_steps(W, steps, torch, pg)
+    F.fp4_check_device_errors()
+    attr_steps, fam_ms = _attribution(W, steps, torch, pg, F)
+    roofline = _roofline(W, fam_ms, attr_steps, torch, pg, device)
+    out = {"workload": W.name, "metric": "block-scaled FP4 GEMM TFLOP/s (GEMM flops / step time incl. rotate+quantize)",
+           "value": round(W.value_from_ms(ms_step, 1), 1), "unit": W.unit, "steps": steps,
+           "ms_per_step": round(ms_step, 5), "config": W.config(), "roofline": roofline,
+           "gpu_launches": W.launches_per_step * steps, "window": window}
+    W.release()
+    return out
+
+
+def run_fp4(args):
+    import torch
+    import microscaling_fp4_quantization_mxfp4_b200 as F
+    from microscaling_fp4_quantization_mxfp4_b200 import _lib
+    _lib.load()                                  # fail loudly when the CUDA library is missing
+    ws, rank, local, pg = _dist_setup(torch)
+    if not torch.cuda.is_available():
+        raise RuntimeError("bench.py needs a CUDA device")
+    device = torch.device("cuda", local)
+    W = WORKLOADS[args.workload](torch, F)
+    W.setup(device)
+    if isinstance(W, LlamaNvfp4):
+        sms = torch.cuda.get_device_properties(device).multi_processor_count
+        W.launches_per_step = sum(1 + (1 if _nv_single_pass(m, k, sms) else 2) for k, n, m in W.cases)
+
+    for i in range(args.warmup):
+        W.step(i)
+    F.fp4_check_device_errors()
+
+    sampler = ClockSampler(_smi_id(torch, local))
+    sampler.start()
+    time.sleep(0.3)                              # let the sampler produce its first line
+    ms_step, window = _timed_steps(W, args.steps, torch, pg)
+    sampler.t_start, sampler.t_end = window
+    F.fp4_check_device_errors()
+    value = W.value_from_ms(ms_step, ws)
+    attr_steps, fam_ms = _attribution(W, args.steps, torch, pg, F)
+    roofline = _roofline(W, fam_ms, attr_steps, torch, pg, device)
     cases = W.cases_summary(args.steps) if hasattr(W, "cases_summary") else None
 
     # end to end through the public API with host buffers: pinned H2D of the step's inputs, the
@@ -1114,10 +1213,18 @@ def run_fp4(args):
     e2e = {"value": round(W.value_from_ms(e2e_ms, ws), 2), "unit": W.unit, "ms_per_step": round(e2e_ms, 4),
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
+    companion = None
+    if getattr(W, "gemm_companion", False) and not args.no_gemm:
+        companion = _run_companion(args, torch, F, device, pg, sampler)
+        time.sleep(0.25)                         # the sampler's last line inside the window
+    sampler.stop()
+    clocks = sampler.summary()
+    if companion is not None:
+        companion["clocks"] = sampler.summary(*companion.pop("window"))
+
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         cpu = _cpu_baseline(W)
-    clocks = sampler.summary()
     if pg is not None:
         pg.destroy_process_group()
     if rank != 0:
@@ -1132,6 +1239,8 @@ def run_fp4(args):
     }
     if cases is not None:
         line["cases"] = cases
+    if companion is not None:
+        line["gemm"] = companion
     print(json.dumps(line), flush=True)
 
 
@@ -1153,9 +1262,9 @@ def _sources_hash(files):
     return h.hexdigest()[:16]
 
 
-def _load_traffic(workload, kernel):
-    """DRAM bytes (read + write) per launch of `kernel` from the committed ncu capture
-    (profiles/traffic.json), or None when none exists or the kernel's sources changed since."""
+def _load_counter(workload, kernel, key):
+    """A per-launch ncu figure of `kernel` from the committed captures (profiles/traffic.json), or
+    None when none exists or the kernel's sources changed since."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
@@ -1163,7 +1272,12 @@ def _load_traffic(workload, kernel):
         d = json.load(f).get(workload, {}).get(kernel)
     if not d or d.get("sources_sha256_16") != _sources_hash(d.get("sources", [])):
         return None
-    return d["dram_bytes_per_launch"]
+    return d.get(key)
+
+
+def _load_traffic(workload, kernel):
+    """DRAM bytes (read + write) per launch of `kernel` from the committed ncu capture."""
+    return _load_counter(workload, kernel, "dram_bytes_per_launch")
 
 
 def _scale_work(W, work, seconds):
@@ -1225,6 +1339,8 @@ def main():
     ap.add_argument("--impl", default="fp4", choices=["fp4", "reference"])
     ap.add_argument("--workload", default=NvfpStudentT.name, choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-gemm", action="store_true",
+                    help="skip the GEMM measurement that the default workload's line carries")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

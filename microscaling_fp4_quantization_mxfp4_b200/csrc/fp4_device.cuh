@@ -56,30 +56,22 @@ __device__ __forceinline__ uint32_t mad_u32(uint32_t a, uint32_t b, uint32_t c) 
 // Stochastic rounding of one scaled value with a 32-bit random word; returns
 // the 4-bit code with the sign in bit 3.  lo <= |v| < hi adjacent grid points,
 // p = (|v| - lo) / (hi - lo) (exact in fp32), round up iff r < ceil(p * 2^32);
-// |v| >= 6 gives 6; sign kept.
-// On [0,2), [2,4), [4,8) the grid step is 0.5, 1, 2 = 2^(m-128) with m the
-// biased exponent of |v| clamped to [127, 129], and the lower grid point's code
-// is 2 (m - 127) + floor(s) for s = |v| / step (exact).  floor(s) comes from one
-// round-toward-zero addition of 2^23 (the sum's last significand bits are the
-// integer part), p is the exact remainder, and codes past 6 (|v| >= 6, where s
-// reaches 3 on the top binade) clamp to 7.  The exponent is handled in place
-// (eb = m << 23): 1/step has the bits 0x7F800000 - eb and 2m = eb >> 22; the
-// shifts and the negation run as multiply-adds.
-__device__ __forceinline__ uint32_t mad_hi_u32(uint32_t a, uint32_t b, uint32_t c) {
-  uint32_t d;
-  asm("mad.hi.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
-  return d;
-}
+// |v| >= 6 gives 6; sign kept.  With a = min(|v|, 6):
+//  * a >= 1: the grid step is a quarter of a's binade, so p * 2^32 = f * 2^10 for
+//    the low 22 significand bits f of a, and "r < f * 2^10" is "(r >> 10) < f",
+//    i.e. the carry out of f + ((~r) >> 10) into bit 22.  The sum, shifted right by
+//    22, is the binade and top significand bit of the rounded value, which are its
+//    code plus 252: (A + 2^22 - 1 - (r >> 10) - 252 * 2^22) >> 22 for A = bits(a)
+//    (codes 2 .. 7; 6 has f = 0 and never rounds up).
+//  * a < 1: the step is 0.5, so with C = ceil(a * 2^33) (a * 2^33 is exact, below
+//    2^33), floor(2a) = C >> 32 is the lower point's code (0 or 1) and C mod 2^32 =
+//    ceil(p * 2^32) the threshold: code = (C >> 32) + (r < C mod 2^32).
 __device__ __forceinline__ uint32_t e2m1_sr(float v, uint32_t r) {
-  const uint32_t vb = __float_as_uint(v);
-  const uint32_t eb = min(max(vb & 0x7F800000u, 0x3F800000u), 0x40800000u);
-  const float inv_step = __uint_as_float(mad_u32(eb, 0xFFFFFFFFu, 0x7F800000u));
-  const float s = __fmul_rn(fabsf(v), inv_step);
-  const float t = __fadd_rz(s, 8388608.0f);                        // 2^23 + floor(s)
-  const float p = __fsub_rn(s, __fsub_rn(t, 8388608.0f));          // exact fractional part
-  const uint32_t thr = __float2uint_ru(__fmul_rn(p, 4294967296.0f));   // < 2^32 since p < 1
-  const uint32_t code = min(mad_hi_u32(eb, 1024u, __float_as_uint(t)) - (0x4B000000u + 254u) + (r < thr ? 1u : 0u), 7u);
-  return code | (mad_hi_u32(vb, 16u, 0u) & 8u);
+  const float a = fminf(fabsf(v), 6.0f);
+  const uint32_t big = (__float_as_uint(a) + (0x003FFFFFu - 0x3F000000u) - (r >> 10)) >> 22;
+  const unsigned long long c = __float2ull_ru(__fmul_rn(a, 0x1p33f));
+  const uint32_t small = (uint32_t)(c >> 32) + (r < (uint32_t)c ? 1u : 0u);
+  return (a < 1.0f ? small : big) | ((__float_as_uint(v) >> 28) & 8u);
 }
 
 // Eight 4-bit codes, element i in nibble i, packed with multiply-adds.
@@ -108,6 +100,22 @@ __device__ __forceinline__ float div_by_recip(float x, float S, float y) {
   q = __fmaf_rn(r, y, q);
   r = -__fmaf_rn(q, S, -x);
   return __fmaf_rn(r, y, q);
+}
+// x / S rounded to nearest-even through fp64: q = RN32(x * yd) with yd = RN64(1/S).
+// For any fp32 x (at most 24 significant bits) and fp32 S > 0 this is the IEEE
+// fp32 quotient whenever that quotient is normal: x / S cannot lie exactly on a
+// rounding midpoint of fp32 (the midpoint's 25-bit odd significand would have to
+// divide x's), and when it is not on one it is at least 2^-49 (relative) away
+// from every midpoint (the residual x - m * S is a nonzero multiple of
+// m's and S's last-place product), while x * yd in fp64 is within 2^-52 of x / S.
+// Quotients below 2^-126 may round differently only at subnormal midpoints; the
+// quantizers use such a quotient only through its E2M1 code (RTN: a signed zero
+// either way) or its threshold ceil(|q| * 2^33) (1 for every nonzero |q| below
+// 2^-33), and its zero-ness agrees: the one tie that decides it, x / S = 2^-150,
+// gives RN64(a * RN64(1/a)) <= 1 (a the significand), which rounds to 0 as the
+// IEEE division's tie-to-even does.  So the codes are those of IEEE division.
+__device__ __forceinline__ float div_by_recip64(float x, double yd) {
+  return __double2float_rn(__dmul_rn((double)x, yd));
 }
 // Running minimum over a block of 2*|x| - 2 as an unsigned integer (zeros wrap
 // to the top): the block passes div_by_recip's |x| >= 2^-103 test iff the
@@ -249,6 +257,14 @@ __device__ __forceinline__ float nv_scale_arg4(float am, float s_t, float y_st, 
   return ok ? t : __fdiv_rn(d4, s_t);
 }
 
+// Four-over-six candidate t4 = RN(RN(amax_b / 4) / s_t) through the fp64 reciprocal of s_t (exact
+// when amax_b / 4 is normal; smaller non-zero maxima take the IEEE division).
+__device__ __forceinline__ float nv_scale_arg4_64(float am, float s_t, double yd_st) {
+  const float d4 = __fmul_rn(am, 0.25f);
+  if (am != 0.0f && am < 0x1p-120f) return __fdiv_rn(d4, s_t);
+  return div_by_recip64(d4, yd_st);
+}
+
 // Per-CTA table of the element divisor S = RN(e4m3(b) * s_t) and RN(1/S) for
 // every E4M3 byte b (b = 0 is the zero scale; its entry is unused).  A scale
 // whose reciprocal is out of the fast path's range gets y = 0, which makes
@@ -258,6 +274,32 @@ __device__ __forceinline__ void nv_fill_scale_table(float2* tab, float s_t) {
     const float S = (b == 0 || b == 127) ? 1.0f : __fmul_rn(e4m3_value((uint32_t)b), s_t);
     tab[b] = make_float2(S, recip_usable(S) ? __frcp_rn(S) : 0.0f);
   }
+}
+
+// Per-CTA table of RN64(1 / S) for S = RN32(e4m3(b) * s_t) and every E4M3 byte b (b = 0 and the
+// NaN byte 127 get 0: their blocks' codes are zeroed or never produced).
+__device__ __forceinline__ void nv_fill_recip64_table(double* tabd, float s_t) {
+  for (int b = threadIdx.x; b < 128; b += blockDim.x) {
+    const float S = (b == 0 || b == 127) ? 0.0f : __fmul_rn(e4m3_value((uint32_t)b), s_t);
+    tabd[b] = S > 0.0f ? __drcp_rn((double)S) : 0.0;
+  }
+}
+
+// Quotients q = x / S of one NVFP4 block through the fp64 reciprocal yd = RN64(1/S)
+// (div_by_recip64); q may alias x.
+template <int E>
+__device__ __forceinline__ void nv_divide_block64(const float (&x)[E], double yd, float (&q)[E]) {
+#pragma unroll
+  for (int i = 0; i < E; ++i) q[i] = div_by_recip64(x[i], yd);
+}
+
+// NVFP4 block-scale argument t = RN(RN(amax_b / 6) / s_t) through fp64 reciprocals (yd_st =
+// RN64(1/s_t)): both quotients are exact when amax_b / 6 is a normal fp32 (amax_b >= 2^-120 here);
+// a subnormal t has E4M3 byte 0 either way.  Smaller non-zero maxima take the IEEE divisions.
+__device__ __forceinline__ float nv_scale_arg64(float am, float s_t, double yd_st) {
+  if (am != 0.0f && am < 0x1p-120f) return __fdiv_rn(__fdiv_rn(am, 6.0f), s_t);
+  const float d6 = div_by_recip64(am, 0x1.5555555555555p-3);      // RN64(1/6)
+  return div_by_recip64(d6, yd_st);
 }
 
 // -------------------------------------------------------- E2M1 decoding -----
@@ -347,11 +389,13 @@ __device__ __forceinline__ void hadamard_rotate(float (&x)[8], int lane) {
   }
 #pragma unroll
   for (int ld = 1; ld < HB / 8; ld <<= 1) {
-    const bool upper = (lane & ld) != 0;
+    // upper lanes take p - x, lower ones x + p: one multiply-add by -1 or +1 (exact negation,
+    // a single rounding, so the same value as the subtraction or addition)
+    const float sgn = (lane & ld) != 0 ? -1.0f : 1.0f;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       const float p = __shfl_xor_sync(0xFFFFFFFFu, x[i], ld);
-      x[i] = upper ? __fsub_rn(p, x[i]) : __fadd_rn(x[i], p);
+      x[i] = __fmaf_rn(x[i], sgn, p);
     }
   }
   const float s = HB == 16 ? 0.25f : HB == 32 ? 0.17677669529663687f : HB == 64 ? 0.125f : 0.08838834764831845f;
@@ -380,11 +424,11 @@ __device__ __forceinline__ void hadamard_rotate_block(float (&x)[E], int lane) {
   }
 #pragma unroll
   for (int ld = 1; ld < HB / E; ld <<= 1) {
-    const bool upper = (lane & ld) != 0;
+    const float sgn = (lane & ld) != 0 ? -1.0f : 1.0f;     // p - x or x + p, as in hadamard_rotate
 #pragma unroll
     for (int i = 0; i < E; ++i) {
       const float p = __shfl_xor_sync(0xFFFFFFFFu, x[i], ld);
-      x[i] = upper ? __fsub_rn(p, x[i]) : __fadd_rn(x[i], p);
+      x[i] = __fmaf_rn(x[i], sgn, p);
     }
   }
   const float s = HB == 16 ? 0.25f : HB == 32 ? 0.17677669529663687f : HB == 64 ? 0.125f : 0.08838834764831845f;

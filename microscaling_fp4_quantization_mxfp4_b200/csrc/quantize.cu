@@ -161,14 +161,24 @@ struct QRowParams {
 
 // Per-thread NVFP4 constants: the tensor scale, its reciprocal and the (S, 1/S) table.
 struct NvConsts {
-  float s_t, y_st;
-  bool st_ok;
-  const float2* tab;
+  float s_t;
+  double yd_st;          // RN64(1 / s_t)
+  const double* tabd;    // RN64(1 / S) for every E4M3 byte
 };
+
+// The per-CTA NVFP4 constants under tensor scale s_t: fills the reciprocal table (every thread of
+// the CTA takes part; visible after the caller's next __syncthreads).
+__device__ __forceinline__ NvConsts nv_consts(float s_t, double* tabd) {
+  nv_fill_recip64_table(tabd, s_t);
+  return NvConsts{s_t, __drcp_rn((double)s_t), tabd};
+}
 
 // One thread quantizes one whole scale block of E = 32 (MX) or 16 (NV)
 // elements held as E/8 uint4: the block maximum, the scale and every division
 // are computed once per block, with E independent element computations.
+// (Splitting an MXFP4 block over a lane pair, 16 elements a thread at 31 warps,
+// measured slower: 52.8 vs 48.5 us for SR and 17.8 vs 16.3 us for RTN at
+// 8192 x 4096, since the per-block work is then done twice.)
 template <int FMT>
 struct BlockShape {
   static constexpr int E = FMT == FMT_MX ? 32 : 16;   // elements per block
@@ -188,15 +198,15 @@ struct BlockShape {
 // square at most 52).  A screen gap above 2^-17 of the sums plus 2^-120 therefore decides the
 // fp64 comparison; anything closer (near-ties, non-finite or tiny sums) takes the fp64 sums.
 template <int RND, int E>
-__device__ __forceinline__ uint32_t nv_four_over_six(float (&x)[E], float am, uint32_t byte6, float s_t,
-                                                     float y_st, bool st_ok, const float2* tab) {
+__device__ __forceinline__ uint32_t nv_four_over_six(float (&x)[E], float am, uint32_t byte6, const NvConsts& nv) {
+  const float s_t = nv.s_t;
   float q6[E];
-  nv_divide_block<RND, E>(x, am, tab[byte6], q6);
-  const uint32_t byte4 = e4m3_rn_sat(nv_scale_arg4(am, s_t, y_st, st_ok));
+  nv_divide_block64<E>(x, nv.tabd[byte6], q6);
+  const uint32_t byte4 = e4m3_rn_sat(nv_scale_arg4_64(am, s_t, nv.yd_st));
   bool pick4 = false;
   if (byte4 != byte6 && byte4 != 0u) {
     float q4[E];
-    nv_divide_block<RND, E>(x, am, tab[byte4], q4);
+    nv_divide_block64<E>(x, nv.tabd[byte4], q4);
     const __half2 g6 = __float2half2_rn(e4m3_value(byte6)), g4 = __float2half2_rn(e4m3_value(byte4));
     float f6 = 0.0f, f4 = 0.0f;
 #pragma unroll
@@ -334,11 +344,11 @@ __device__ __forceinline__ void quantize_block(const QRowParams& p, const uint4 
     for (int i = 0; i < E; ++i) x[i] = __fmul_rn(x[i], inv);          // exact power-of-two scaling
     zero = (am == 0.0f);
   } else {
-    byte = e4m3_rn_sat(nv_scale_arg(am, nv.s_t, nv.y_st, nv.st_ok));
+    byte = e4m3_rn_sat(nv_scale_arg64(am, nv.s_t, nv.yd_st));
     if (FMT == FMT_NV46) {
-      byte = nv_four_over_six<RND, E>(x, am, byte, nv.s_t, nv.y_st, nv.st_ok, nv.tab);
+      byte = nv_four_over_six<RND, E>(x, am, byte, nv);
     } else {
-      nv_divide_block<RND, E>(x, am, nv.tab[byte], x);
+      nv_divide_block64<E>(x, nv.tabd[byte], x);
     }
     zero = (byte == 0u);
   }
@@ -385,15 +395,12 @@ template <int FMT, int RND, int HAD, bool SFMMA, int DQ = 0>
 __global__ void __launch_bounds__(256) quantize_rows_kernel(QRowParams p) {
   pdl_trigger();
   constexpr int V = BlockShape<FMT>::V;
-  __shared__ float2 tab[128];
+  __shared__ double tabd[128];
   const int lane = threadIdx.x & 31;
   pdl_wait();
-  NvConsts nv{1.0f, 1.0f, true, tab};
+  NvConsts nv{1.0f, 1.0, tabd};
   if (FMT != FMT_MX) {
-    nv.s_t = *p.ts;
-    nv.y_st = __frcp_rn(nv.s_t);
-    nv.st_ok = recip_usable(nv.s_t);
-    nv_fill_scale_table(tab, nv.s_t);
+    nv = nv_consts(*p.ts, tabd);
     if (p.ts_copy_out != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *p.ts_copy_out = nv.s_t;
     __syncthreads();
   }
@@ -509,18 +516,15 @@ template <int FMT, int RND, int HAD, bool SFMMA, int DQ = 0>
 __global__ void __launch_bounds__(StreamWarps<FMT, RND>::kThreads, 1) quantize_stream_kernel(QRowParams p) {
   constexpr int kStreamWarps = StreamWarps<FMT, RND>::kWarps;
   extern __shared__ __align__(1024) uint8_t smem[];
-  __shared__ float2 tab[128];
+  __shared__ double tabd[128];
   pdl_trigger();
   const StreamRing r = stream_ring(smem);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   stream_ring_init(r, kStreamWarps);
   pdl_wait();
-  NvConsts nv{1.0f, 1.0f, true, tab};
+  NvConsts nv{1.0f, 1.0, tabd};
   if (FMT != FMT_MX) {
-    nv.s_t = *p.ts;
-    nv.y_st = __frcp_rn(nv.s_t);
-    nv.st_ok = recip_usable(nv.s_t);
-    nv_fill_scale_table(tab, nv.s_t);
+    nv = nv_consts(*p.ts, tabd);
     if (p.ts_copy_out != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *p.ts_copy_out = nv.s_t;
   }
   __syncthreads();
@@ -661,7 +665,7 @@ template <int FMT, int RND, int HAD, bool SFMMA, int DQ = 0>
 __global__ void __launch_bounds__(FusedWarps<FMT>::kThreads, 1) nv_quantize_fused_kernel(FusedParams fp) {
   constexpr int kFusedWarps = FusedWarps<FMT>::kWarps;
   extern __shared__ __align__(1024) uint4 slice[];
-  __shared__ float2 tab[128];
+  __shared__ double tabd[128];
   __shared__ float red[kFusedWarps];
   __shared__ float s_t_shared;
   __shared__ __align__(8) uint64_t piece_bar[kFusedPieces];
@@ -761,8 +765,7 @@ __global__ void __launch_bounds__(FusedWarps<FMT>::kThreads, 1) nv_quantize_fuse
     }
   }
   __syncthreads();
-  NvConsts nv{s_t_shared, __frcp_rn(s_t_shared), recip_usable(s_t_shared), tab};
-  nv_fill_scale_table(tab, nv.s_t);
+  const NvConsts nv = nv_consts(s_t_shared, tabd);
   __syncthreads();
   if (warp == 0) return;
 
@@ -826,18 +829,14 @@ template <int FMT, int RND, bool SFMMA>
 __global__ void __launch_bounds__(256, (RND == RND_SR && FMT != FMT_NV46) ? 3 : 2) quantize_cols_kernel(QColParams p) {
   pdl_trigger();
   __shared__ __align__(16) uint16_t tile[128][64];
-  __shared__ float2 tab[128];
+  __shared__ double tabd[128];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   pdl_wait();
   const uint32_t tiles_r = (p.R + 127u) / 128u, tiles_c = (p.C + 63u) / 64u;
-  float s_t = 1.0f, y_st = 1.0f;
-  bool st_ok = true;
+  NvConsts nv{1.0f, 1.0, tabd};
   if (FMT != FMT_MX) {
-    s_t = *p.ts;
-    y_st = __frcp_rn(s_t);
-    st_ok = recip_usable(s_t);
-    nv_fill_scale_table(tab, s_t);          // visible after the first __syncthreads of the tile loop
-    if (p.ts_copy_out != nullptr && blockIdx.x == 0 && tid == 0) *p.ts_copy_out = s_t;
+    nv = nv_consts(*p.ts, tabd);            // visible after the first __syncthreads of the tile loop
+    if (p.ts_copy_out != nullptr && blockIdx.x == 0 && tid == 0) *p.ts_copy_out = nv.s_t;
   }
   for (uint32_t t = blockIdx.x; t < tiles_r * tiles_c; t += gridDim.x) {
     const uint32_t tc = t / tiles_r, tr = t - tc * tiles_r;
@@ -872,26 +871,23 @@ __global__ void __launch_bounds__(256, (RND == RND_SR && FMT != FMT_NV46) ? 3 : 
       for (int i = 0; i < BS; ++i) am = fmaxf(am, fabsf(xv[b * BS + i]));
       uint32_t byte;
       bool zero;
-      float inv = 1.0f, S = 1.0f, y = 1.0f;
-      bool fast = true;
+      float inv = 1.0f;
+      double yd = 1.0;
       if (FMT == FMT_MX) {
         byte = mx_scale_byte_clip(am, p.mx_thr);
         inv = mx_inv_scale(byte);
         zero = (am == 0.0f);
       } else {
-        float xb[BS];
-#pragma unroll
-        for (int i = 0; i < BS; ++i) xb[i] = xv[b * BS + i];
-        byte = e4m3_rn_sat(nv_scale_arg(am, s_t, y_st, st_ok));
+        byte = e4m3_rn_sat(nv_scale_arg64(am, nv.s_t, nv.yd_st));
         if (FMT == FMT_NV46) {
-          byte = nv_four_over_six<RND, BS>(xb, am, byte, s_t, y_st, st_ok, tab);
+          float xb[BS];
+#pragma unroll
+          for (int i = 0; i < BS; ++i) xb[i] = xv[b * BS + i];
+          byte = nv_four_over_six<RND, BS>(xb, am, byte, nv);
 #pragma unroll
           for (int i = 0; i < BS; ++i) xv[b * BS + i] = xb[i];     // quotients under the chosen scale
         } else {
-          const float2 sy = tab[byte];
-          S = sy.x;
-          y = sy.y;
-          fast = nv_fast_division<RND, BS>(xb, am, S, y);
+          yd = nv.tabd[byte];
         }
         zero = (byte == 0u);
       }
@@ -906,7 +902,7 @@ __global__ void __launch_bounds__(256, (RND == RND_SR && FMT != FMT_NV46) ? 3 : 
           } else if (FMT == FMT_NV46) {
             v8[i] = xi;
           } else {
-            v8[i] = fast ? div_by_recip(xi, S, y) : __fdiv_rn(xi, S);
+            v8[i] = div_by_recip64(xi, yd);
           }
         }
         uint32_t packed;
@@ -1033,18 +1029,14 @@ __global__ void __launch_bounds__(256) quantize_2d_kernel(Q2Params p) {
   __shared__ __align__(16) uint32_t code_col[TC * COLW];
   __shared__ uint8_t sc_row[TR][SEGS];
   __shared__ uint8_t sc_col[TC][4];
-  __shared__ float2 tab[128];
+  __shared__ double tabd[128];
   const int tid = threadIdx.x, lane = tid & 31;
   const int row = tid % TR, seg = tid / TR;
   pdl_wait();
-  float s_t = 1.0f, y_st = 1.0f;
-  bool st_ok = true;
+  NvConsts nv{1.0f, 1.0, tabd};
   if (FMT != FMT_MX) {
-    s_t = *p.ts;
-    y_st = __frcp_rn(s_t);
-    st_ok = recip_usable(s_t);
-    nv_fill_scale_table(tab, s_t);
-    if (p.ts_copy_out != nullptr && blockIdx.x == 0 && tid == 0) *p.ts_copy_out = s_t;
+    nv = nv_consts(*p.ts, tabd);
+    if (p.ts_copy_out != nullptr && blockIdx.x == 0 && tid == 0) *p.ts_copy_out = nv.s_t;
   }
   __syncthreads();                                        // the scale table is read by the first tile
   // store widths of the two outputs (rows of W's codes are C/2 bytes apart, of W^T's R/2)
@@ -1105,9 +1097,9 @@ __global__ void __launch_bounds__(256) quantize_2d_kernel(Q2Params p) {
       for (int i = 0; i < BS; ++i) x[i] = __fmul_rn(x[i], inv);
       zero = (am == 0.0f);
     } else {
-      byte = e4m3_rn_sat(nv_scale_arg(am, s_t, y_st, st_ok));
+      byte = e4m3_rn_sat(nv_scale_arg64(am, nv.s_t, nv.yd_st));
       zero = (byte == 0u);
-      nv_divide_block<RND, BS>(x, am, tab[byte], x);
+      nv_divide_block64<BS>(x, nv.tabd[byte], x);
     }
     uint32_t w[V];
     if (RND == RND_RTN) {
