@@ -250,6 +250,20 @@ class NvfpStudentT(Workload):
         """Launches of a kernel family per step."""
         return 2 if key == "dequantize" else 1
 
+    def solo_calls(self):
+        """Each kernel family's launch alone (for _solo_times): key -> (call(i), launches per step)."""
+        if not self.fused_deq:
+            return None
+        F = self.F
+        return {
+            "amax+quantize_dequantize_rtn": (lambda i: F.fp4_quantize_dequantize(
+                self.x[i % self.n_inputs], fmt=self.fmt, rnd="rtn", codes=self.codes[0], scales=self.scales[0],
+                tensor_scale_out=self.ts, out=self.deq[0]), 1),
+            "quantize_dequantize_sr": (lambda i: F.fp4_quantize_dequantize(
+                self.x[i % self.n_inputs], fmt=self.fmt, rnd="sr", seed=1, tensor_scale_in=self.ts,
+                codes=self.codes[1], scales=self.scales[1], tensor_scale_out=self.ts_sr, out=self.deq[1]), 1),
+        }
+
     def family_elements(self, key):
         """Elements a kernel family processes per step (each launch covers the whole tensor)."""
         return self.n * self.family_launches(key)
@@ -539,6 +553,25 @@ class HadamardMxGemm(GemmWorkload):
     def single_kernel(self):
         return ("rotate_quantize", "gemm")
 
+    def solo_calls(self):
+        """Each family alone (for _solo_times): rotate+quantize over three input copies (192 MB, past
+        L2), the GEMMs writing their 180 MB outputs; every block size in turn."""
+        F, nb = self.F, len(self.blocks)
+        if not hasattr(self, "x_copies"):
+            self.x_copies = [self.x] + [self.x.clone() for _ in range(2)]
+
+        def rq(i):
+            b = self.blocks[i % nb]
+            F.fp4_hadamard_quantize(self.x_copies[i % 3], b, fmt="mxfp4", sf_layout="mma", codes=self.codes,
+                                    scales=self.scales)
+
+        def gm(i):
+            qw = self.qw[self.blocks[i % nb]]
+            F.fp4_gemm(self.codes, self.scales, qw.codes, qw.scales, fmt="mxfp4", out_dtype="bf16",
+                       out=self.outs[i % nb])
+
+        return {"rotate_quantize": (rq, nb), "gemm": (gm, nb)}
+
     def step(self, i, timed=False, x=None):
         F = self.F
         x = self.x if x is None else x
@@ -569,7 +602,7 @@ class HadamardMxGemm(GemmWorkload):
                 "hadamard_blocks": list(self.blocks), "activations": "N(0,1), 41 of 4096 channels x50, seed 2",
                 "weights": "N(0,0.02), rotated and quantized offline (untimed)", "out": "bf16",
                 "gemm_flops_per_step": self.step_flops,
-                "l2": "inputs + 4 x 180 MB bf16 outputs per step exceed L2"}
+                "l2": f"inputs + {len(self.blocks)} x 180 MB bf16 outputs per step exceed L2"}
 
     def oracle_setup(self):
         from workloads import hadamard_acts, hadamard_weights
@@ -600,7 +633,7 @@ class HadamardMxGemm128(HadamardMxGemm):
     launches_per_step = 2
 
     def release(self):
-        for a in ("x", "qw", "codes", "scales", "outs", "host_in", "dev_in"):
+        for a in ("x", "x_copies", "qw", "codes", "scales", "outs", "host_in", "dev_in"):
             if hasattr(self, a):
                 delattr(self, a)
 
@@ -880,7 +913,9 @@ class LlamaNvfp4(GemmWorkload):
         out = {}
         for (k, n, m), ct in zip(self.cases, self.case_timers):
             ms = float(np.mean([a.elapsed_time(b) for a, b in ct.pairs]))
-            out[f"K{k}_N{n}_M{m}"] = {"us": round(ms * 1e3, 2), "tflops": round(2.0 * m * n * k / (ms * 1e-3) / 1e12, 1)}
+            wgb = n * k * (0.5 + 1 / 16) / (ms * 1e-3) / 1e9          # weight codes + E4M3 scales streamed
+            out[f"K{k}_N{n}_M{m}"] = {"us": round(ms * 1e3, 2), "tflops": round(2.0 * m * n * k / (ms * 1e-3) / 1e12, 1),
+                                      "weight_gbs": round(wgb, 1)}
         return out
 
     def config(self):
@@ -1065,9 +1100,38 @@ def _attribution(W, steps, torch, pg, F):
     return attr_steps, fam_ms
 
 
-def _roofline(W, fam_ms, attr_steps, torch, pg, device):
+def _solo_times(W, steps, torch, pg):
+    """Per-step device time of each kernel family timed alone: its launches back to back (inputs
+    rotating past L2 as in the step), bracketed by one CUDA event pair, after warm-up.  Unlike events
+    around every launch of the step, this keeps programmatic dependent launch overlapping each
+    launch's setup with the previous one's tail, as in the timed step; None if the workload has no
+    per-family calls."""
+    calls = W.solo_calls() if hasattr(W, "solo_calls") else None
+    if not calls:
+        return None
+    n = max(3, min(steps, 200))
+    out = {}
+    for key, (fn, launches) in calls.items():
+        for i in range(3):
+            fn(i)
+        _barrier(torch, pg)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for i in range(n):
+            fn(i)
+        b.record()
+        torch.cuda.synchronize()
+        out[key] = a.elapsed_time(b) / n * launches
+    return out
+
+
+def _roofline(W, fam_ms, attr_steps, torch, pg, device, solo_ms=None):
     """Roofline of the dominant single-kernel family (largest share of device time) and the rates of
-    every family."""
+    every family.  With solo_ms (per-family times from _solo_times) those set the rates; the
+    in-step event times are kept beside them."""
+    events_ms = fam_ms
+    if solo_ms:
+        fam_ms = {k: solo_ms.get(k, v) for k, v in fam_ms.items()}
     dom = max((k for k in fam_ms if k in W.single_kernel()), key=lambda k: fam_ms[k])
     dom_ms = _max_over_ranks(torch, pg, fam_ms[dom])
     peaks = _peaks()
@@ -1116,6 +1180,11 @@ def _roofline(W, fam_ms, attr_steps, torch, pg, device):
             per_family[k] = {"us_per_step": round(ms * 1e3, 2), "geval_s": round(work / (ms * 1e-3) / 1e9, 1)}
         else:
             per_family[k] = {"us_per_step": round(ms * 1e3, 2), "gbs": round(work / (ms * 1e-3) / 1e9, 1)}
+    if solo_ms:
+        for k in per_family:
+            per_family[k]["us_per_step_events_in_step"] = round(events_ms[k] * 1e3, 2)
+        roofline["timing"] = ("per-kernel times: each family's launches alone, back to back, one CUDA event pair; "
+                              "us_per_step_events_in_step: events around every launch of the step")
     roofline["per_kernel"] = per_family
     roofline["attribution_steps"] = attr_steps
     return roofline
@@ -1156,7 +1225,9 @@ def _run_companion(args, torch, F, device, pg, sampler):
     ms_step, window = _timed_steps(W, steps, torch, pg)
     F.fp4_check_device_errors()
     attr_steps, fam_ms = _attribution(W, steps, torch, pg, F)
-    roofline = _roofline(W, fam_ms, attr_steps, torch, pg, device)
+    solo = _solo_times(W, steps, torch, pg)
+    F.fp4_check_device_errors()
+    roofline = _roofline(W, fam_ms, attr_steps, torch, pg, device, solo)
     out = {"workload": W.name, "metric": "block-scaled FP4 GEMM TFLOP/s (GEMM flops / step time incl. rotate+quantize)",
            "value": round(W.value_from_ms(ms_step, 1), 1), "unit": W.unit, "steps": steps,
            "ms_per_step": round(ms_step, 5), "config": W.config(), "roofline": roofline,
@@ -1192,7 +1263,9 @@ def run_fp4(args):
     F.fp4_check_device_errors()
     value = W.value_from_ms(ms_step, ws)
     attr_steps, fam_ms = _attribution(W, args.steps, torch, pg, F)
-    roofline = _roofline(W, fam_ms, attr_steps, torch, pg, device)
+    solo = _solo_times(W, args.steps, torch, pg)
+    F.fp4_check_device_errors()
+    roofline = _roofline(W, fam_ms, attr_steps, torch, pg, device, solo)
     cases = W.cases_summary(args.steps) if hasattr(W, "cases_summary") else None
 
     # end to end through the public API with host buffers: pinned H2D of the step's inputs, the

@@ -73,25 +73,7 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 }  // namespace
 
-// FP4_PDL=0 launches without programmatic dependent launch (for debugging and comparison).
-bool fp4lib::pdl_enabled() {
-  static const bool on = [] {
-    const char* e = getenv("FP4_PDL");
-    return !(e != nullptr && e[0] == '0');
-  }();
-  return on;
-}
-
 namespace {
-
-// FP4_SINGLE_PASS=0 forces the two-pass NVFP4 path (amax kernel, then quantize); for testing.
-bool single_pass_disabled() {
-  static const bool off = [] {
-    const char* e = getenv("FP4_SINGLE_PASS");
-    return e != nullptr && e[0] == '0';
-  }();
-  return off;
-}
 
 fp4_status check_format(int fmt, int block) {
   if (fmt == FP4_MXFP4 && block == 32) return FP4_OK;
@@ -159,8 +141,8 @@ fp4_status quantize_impl(const void* x, int64_t rows, int64_t cols, int64_t ld, 
     fprintf(stderr, "[fp4] quantize rows=%lld cols=%lld ld=%lld fmt=%d axis=%d rnd=%d had=%d sf=%d\n",
             (long long)rows, (long long)cols, (long long)ld, fmt, axis, rnd, had, sf_layout);
   const int64_t groups = qlen / block;
-  if (sf_layout == FP4_SF_MMA && (orows % 128 != 0 || groups % 4 != 0)) {
-    // padding bytes of the tensor-core layout must read as scale 0
+  if (sf_layout == FP4_SF_MMA && axis == 0 && (orows % 128 != 0 || groups % 4 != 0)) {
+    // padding bytes of the tensor-core layout must read as scale 0 (the axis-1 kernels write them)
     if (cudaMemsetAsync(scales, 0, (size_t)(round_up(orows, 128) * round_up(groups, 4)), st) != cudaSuccess)
       return FP4_ERR_CUDA;
   }
@@ -185,7 +167,7 @@ fp4_status quantize_impl(const void* x, int64_t rows, int64_t cols, int64_t ld, 
   p.deq_mode = deq_mode;
   size_t fused_smem = 0;
   uint32_t fused_tiles = 0;
-  if (fmt == FP4_NVFP4 && ts_in == nullptr && axis == 1 && ld == cols && !single_pass_disabled() &&
+  if (fmt == FP4_NVFP4 && ts_in == nullptr && axis == 1 && ld == cols &&
       fused_nv_fits(rows, cols, d->num_sms, &fused_smem, &fused_tiles)) {
     // one HBM read: amax and quantize in a single cooperative launch
     return from_cuda(launch_quantize_nv_fused(p, ts_out, d->scratch, d->num_sms, st));

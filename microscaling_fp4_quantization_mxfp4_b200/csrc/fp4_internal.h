@@ -8,7 +8,7 @@
 namespace fp4lib {
 
 // Programmatic dependent launch.  Every kernel of the library is launched with programmatic
-// stream serialization (unless FP4_PDL=0), so its CTAs may be scheduled -- and run their
+// stream serialization, so its CTAs may be scheduled -- and run their
 // shared-memory, barrier and tensor-memory setup -- while the previous kernel in the stream
 // drains.  Each kernel calls pdl_wait() before its first global-memory access (that returns once
 // the previous grid has completed and its writes are visible) and pdl_trigger() at entry, so that
@@ -17,7 +17,6 @@ namespace fp4lib {
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 #endif
-bool pdl_enabled();
 
 // cudaLaunchKernelEx with the programmatic-serialization attribute, plus optional cooperative
 // launch and cluster width.
@@ -31,11 +30,9 @@ cudaError_t launch_kernel(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_
   cfg.stream = st;
   cudaLaunchAttribute at[3];
   unsigned n = 0;
-  if (pdl_enabled()) {
-    at[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    at[n].val.programmaticStreamSerializationAllowed = 1;
-    ++n;
-  }
+  at[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[n].val.programmaticStreamSerializationAllowed = 1;
+  ++n;
   if (cooperative) {
     at[n].id = cudaLaunchAttributeCooperative;
     at[n].val.cooperative = 1;

@@ -1482,6 +1482,340 @@ __global__ void __launch_bounds__(Cfg<BN, FMT, false>::kThreads, 1)
 
 }  // namespace splitk
 
+// ============================== swap-AB split-K (at most 128 activation rows) ===
+// Weight streaming for small M (decode steps and short batches).  The tensor cores compute
+// Y^T = W . X^T: 128 rows of the weights W fill the MMA's M dimension and the M <= 128 activation
+// rows are its N (BNT = 16, 32, 64 or 128 columns, the block-scaled MMA taking any multiple of 8
+// from 8 to 256), so no tensor-core work or shared memory is spent on padding rows of X and each
+// stage carries a full 16 KB of W.  Each 128-row weight tile is a cluster of `split` CTAs that
+// divide its k-tiles, so every SM streams a disjoint slice of W once.  The roles are the single-SM
+// kernel's (TMA producer, scale copier, MMA thread); the four epilogue warps park the fp32 partial
+// Y^T tile transposed (one shared-memory row per activation row) in the idle stage ring, and after a
+// cluster barrier every CTA sums one slice of it across the cluster through distributed shared
+// memory, in rank order (deterministic), scales by alpha and stores rows of Y.  Both cluster
+// barriers are reached on every path, errors included.
+namespace swapab {
+
+template <int BNT, int FMT>
+struct CfgS {
+  static constexpr int kApk = FmtTraits<FMT>::kAtomsPerKTile;
+  static constexpr int kThreads = 224;                   // producer, MMA, 4 epilogue warps, scale copier
+  static constexpr int kSfWarp = 6;
+  static constexpr int kWBytes = 128 * BK_BYTES;         // 16 KB of weights per stage
+  static constexpr int kXBytes = BNT * BK_BYTES;
+  static constexpr int kSfBytes = kApk * 512;            // one 128-row scale block per operand
+  static constexpr int kStageBytes = kWBytes + kXBytes + 2 * kSfBytes;
+  static constexpr int kStages = kSmemRing / kStageBytes > 8 ? 8 : kSmemRing / kStageBytes;
+  static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + 1024;
+  static constexpr int kPStride = 128 + 4;               // floats per parked row (one activation row)
+  static constexpr int kPartBytes = BNT * kPStride * 4;
+  static constexpr uint32_t kSfBase = 128;               // scale buffers after the <= 128-column accumulator
+  // Twelve 32-column scale buffers (weights' then activations' atoms, <= 16 columns each): a k-tile's
+  // MMAs are short here, so the copier may run up to 12 k-tiles ahead of them instead of 4; with 4
+  // the copy -> MMA -> release round trip, not the weight stream, set the pace.
+  static constexpr uint32_t kSfBufs = 12;
+  static constexpr uint32_t kSfCols = 32;
+  static_assert(kSfBase + kSfBufs * kSfCols <= kTmemCols, "tensor memory budget");
+  static_assert(kPartBytes <= kStages * kStageBytes, "partial tile must fit in the stage ring");
+  static_assert(BNT == 16 || BNT == 32 || BNT == 64 || BNT == 128, "activation tile");
+};
+
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+
+template <int BNT, int FMT, bool BF16>
+__global__ void __launch_bounds__(CfgS<BNT, FMT>::kThreads, 1)
+    fp4_gemm_swap_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
+                         KernelArgs p, int split) {
+  pdl_trigger();
+  using C = CfgS<BNT, FMT>;
+  constexpr int S = C::kStages;
+  constexpr int APK = C::kApk;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sW = smem;
+  uint8_t* sX = sW + S * C::kWBytes;
+  uint8_t* sSFW = sX + S * C::kXBytes;
+  uint8_t* sSFX = sSFW + S * C::kSfBytes;
+  float* part = reinterpret_cast<float*>(smem);               // reuses the ring after the last MMA
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sSFX + S * C::kSfBytes);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + S;
+  uint64_t* tfull = bars + 2 * S;
+  uint64_t* drain = bars + 2 * S + 1;
+  uint64_t* sfdrain = bars + 2 * S + 2;
+  uint64_t* sf_full = bars + 2 * S + 3;
+  uint64_t* sf_empty = sf_full + C::kSfBufs;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sf_empty + C::kSfBufs);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = split > 1 ? pair::cluster_rank() : 0u;
+  const int nt = (int)(blockIdx.x / (uint32_t)split);           // 128-row weight tile
+  const int nkb = (p.K + BK - 1) / BK;
+  const int kb0 = (int)((int64_t)nkb * rank / split), kb1 = (int)((int64_t)nkb * (rank + 1) / split);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(smem_u32(&full[s]), 1);
+      mbar_init(smem_u32(&empty[s]), 1);
+    }
+    mbar_init(smem_u32(tfull), 1);
+    mbar_init(smem_u32(drain), 1);
+    mbar_init(smem_u32(sfdrain), 1);
+    for (uint32_t b = 0; b < C::kSfBufs; ++b) {
+      mbar_init(smem_u32(&sf_full[b]), 1);
+      mbar_init(smem_u32(&sf_empty[b]), 1);
+    }
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  pdl_wait();                               // the previous kernel's outputs (our operands) are complete
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer --
+    if (lane == 0) {
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_w)) : "memory");
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_x)) : "memory");
+      int stage = 0;
+      uint32_t phase = 0, issued = 0, issued_parity = 0;
+      bool ok = true;
+      for (int kb = kb0; kb < kb1; ++kb) {
+        if (!wait_spin(smem_u32(&empty[stage]), phase ^ 1u, abort_flag)) {
+          raise_abort(abort_flag, p.error);
+          ok = false;
+          break;
+        }
+        const int kvalid = min(BK, p.K - kb * BK);
+        const int atoms = (kvalid / FmtTraits<FMT>::kBlock + 3) / 4;
+        const uint32_t fb = smem_u32(&full[stage]);
+        mbar_expect_tx(fb, (uint32_t)(C::kWBytes + C::kXBytes + 2 * atoms * 512));
+        tma_load_2d(smem_u32(sW + stage * C::kWBytes), &tmap_w, kb * BK_BYTES, nt * 128, fb);
+        tma_load_2d(smem_u32(sX + stage * C::kXBytes), &tmap_x, kb * BK_BYTES, 0, fb);
+        bulk_load(smem_u32(sSFW + stage * C::kSfBytes), p.b_sf + ((size_t)nt * p.g4 + (size_t)kb * APK) * 512,
+                  (uint32_t)atoms * 512u, fb);
+        bulk_load(smem_u32(sSFX + stage * C::kSfBytes), p.a_sf + (size_t)kb * APK * 512, (uint32_t)atoms * 512u, fb);
+        issued |= 1u << stage;
+        issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
+        if (++stage == S) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      if (!ok) {
+        for (int s = 0; s < S; ++s)
+          if (issued & (1u << s)) {
+            volatile int never = 0;
+            wait_bounded(smem_u32(&full[s]), (issued_parity >> s) & 1u, &never);
+          }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer --
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true, any_mma = false;
+      for (int kb = kb0; kb < kb1; ++kb) {
+        const uint32_t n = (uint32_t)(kb - kb0), b = n % C::kSfBufs, use_b = n / C::kSfBufs;
+        if (!wait_spin(smem_u32(&sf_full[b]), use_b & 1u, abort_flag) ||
+            !wait_spin(smem_u32(&full[stage]), phase, abort_flag)) {
+          raise_abort(abort_flag, p.error);
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const int kvalid = min(BK, p.K - kb * BK);
+        const uint32_t sfw_col = C::kSfBase + b * C::kSfCols;
+        const uint32_t sfx_col = sfw_col + 16u;
+        const uint64_t wdesc = desc_sw128(smem_u32(sW + stage * C::kWBytes));
+        const uint64_t xdesc = desc_sw128(smem_u32(sX + stage * C::kXBytes));
+        const int nmma = kvalid / 64;
+        for (int j = 0; j < nmma; ++j) {
+          const uint32_t chunk = FMT == FMT_MX ? (uint32_t)(j >> 1) : (uint32_t)j;
+          const uint32_t sf_id = FMT == FMT_MX ? (uint32_t)((j & 1) * 2) : 0u;
+          const uint32_t idesc = idesc_base<BNT, FMT>() | (sf_id << 29) | (sf_id << 4);
+          tc_mma<FMT>(tmem, wdesc + (uint64_t)(2 * j), xdesc + (uint64_t)(2 * j), idesc, tmem + sfw_col + 4u * chunk,
+                      tmem + sfx_col + 4u * chunk, (kb > kb0 || j > 0) ? 1u : 0u);
+          any_mma = true;
+        }
+        tc_commit(smem_u32(&empty[stage]));
+        tc_commit(smem_u32(&sf_empty[b]));
+        if (++stage == S) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      if (ok) {
+        tc_commit(smem_u32(tfull));
+      } else if (any_mma) {
+        tc_commit(smem_u32(drain));
+        volatile int never = 0;
+        wait_bounded(smem_u32(drain), 0u, &never);
+      }
+    }
+    __syncwarp();
+  } else if (warp == C::kSfWarp) {
+    // ------------------------------------------------------ scale copier --
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true, any_cp = false;
+      for (int kb = kb0; kb < kb1; ++kb) {
+        const uint32_t n = (uint32_t)(kb - kb0), b = n % C::kSfBufs, use_b = n / C::kSfBufs;
+        if (!wait_spin(smem_u32(&full[stage]), phase, abort_flag) ||
+            !wait_spin(smem_u32(&sf_empty[b]), (use_b & 1u) ^ 1u, abort_flag)) {
+          raise_abort(abort_flag, p.error);
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const int kvalid = min(BK, p.K - kb * BK);
+        const int atoms = (kvalid / FmtTraits<FMT>::kBlock + 3) / 4;
+        const uint32_t sfw_col = C::kSfBase + b * C::kSfCols;
+        const uint32_t sfx_col = sfw_col + 16u;
+        for (int i = 0; i < atoms; ++i) {
+          tc_cp_sf(tmem + sfw_col + 4u * i, desc_sf(smem_u32(sSFW + stage * C::kSfBytes + i * 512)));
+          tc_cp_sf(tmem + sfx_col + 4u * i, desc_sf(smem_u32(sSFX + stage * C::kSfBytes + i * 512)));
+        }
+        tc_commit(smem_u32(&sf_full[b]));
+        any_cp = true;
+        if (++stage == S) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      if (!ok && any_cp) {
+        tc_commit(smem_u32(sfdrain));
+        volatile int never = 0;
+        wait_bounded(smem_u32(sfdrain), 0u, &never);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------- partial Y^T tile, parked transposed --
+    // warp w reads tensor-memory lanes 32*(w%4) .. +31 (weight rows) and all BNT columns
+    // (activation rows); activation row m of the partial goes to shared-memory row m.
+    const int q = warp & 3;
+    int ok = 1;
+    if (lane == 0) ok = wait_bounded(smem_u32(tfull), 0u, abort_flag) ? 1 : 0;
+    ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+    if (!ok) {
+      if (lane == 0) raise_abort(abort_flag, p.error);
+    } else {
+      tc_fence_after();
+      const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16);
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // ring bytes last touched by the async proxy
+      float* col = part + q * 32 + lane;
+      if (BNT == 16) {
+        uint32_t r[16];
+        tmem_ld16(tbase, r);
+        asm volatile("tcgen05.wait::ld.sync.aligned;" : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]),
+                     "+r"(r[5]), "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]),
+                     "+r"(r[13]), "+r"(r[14]), "+r"(r[15])::"memory");
+#pragma unroll
+        for (int m = 0; m < 16; ++m) col[m * C::kPStride] = __uint_as_float(r[m]);
+      } else {
+#pragma unroll
+        for (int c = 0; c < BNT / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld32(tbase + (uint32_t)(32 * c), r);
+          asm volatile("tcgen05.wait::ld.sync.aligned;"
+                       : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                         "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]),
+                         "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]),
+                         "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]),
+                         "+r"(r[29]), "+r"(r[30]), "+r"(r[31])::"memory");
+#pragma unroll
+          for (int i = 0; i < 32; ++i) col[(32 * c + i) * C::kPStride] = __uint_as_float(r[i]);
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (split > 1) pair::cluster_sync_all();  // every CTA's partial tile is in its shared memory
+
+  // ------------------------------------------- reduce one slice across ranks --
+  {
+    const int nvalid = min(128, p.N - nt * 128);                  // weight rows of this tile
+    const int c4n = (nvalid + 3) / 4;                              // float4 groups per activation row
+    const int items = p.M * c4n;
+    const int i0 = (int)((int64_t)items * rank / split), i1 = (int)((int64_t)items * (rank + 1) / split);
+    const float alpha = FMT == FMT_NV ? __fmul_rn(*p.a_ts, *p.b_ts) : 1.0f;
+    const uint32_t part_base = smem_u32(part);
+    for (int it = i0 + (int)threadIdx.x; it < i1; it += (int)blockDim.x) {
+      const int m = it / c4n, c4 = it - m * c4n;
+      const uint32_t addr = part_base + (uint32_t)((m * C::kPStride + 4 * c4) * 4);
+      float4 v[splitk::kMaxSplit];                               // all remote loads in flight at once
+      if (split == 1) {
+        v[0] = *reinterpret_cast<const float4*>(part + m * C::kPStride + 4 * c4);
+      } else {
+#pragma unroll
+        for (int s = 0; s < splitk::kMaxSplit; ++s)
+          if (s < split) v[s] = splitk::ld_cluster_f4(pair::map_rank(addr, (uint32_t)s));
+      }
+      float4 acc = v[0];
+#pragma unroll
+      for (int s = 1; s < splitk::kMaxSplit; ++s)
+        if (s < split) {
+          acc.x = __fadd_rn(acc.x, v[s].x);
+          acc.y = __fadd_rn(acc.y, v[s].y);
+          acc.z = __fadd_rn(acc.z, v[s].z);
+          acc.w = __fadd_rn(acc.w, v[s].w);
+        }
+      const float y4[4] = {__fmul_rn(acc.x, alpha), __fmul_rn(acc.y, alpha), __fmul_rn(acc.z, alpha),
+                           __fmul_rn(acc.w, alpha)};
+      const int n0 = nt * 128 + 4 * c4;
+      if (BF16) {
+        __nv_bfloat16* yr = reinterpret_cast<__nv_bfloat16*>(p.y) + (size_t)m * p.ldy + n0;
+        if (p.vec_store && n0 + 4 <= p.N) {
+          const uint32_t lo = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(y4[0])) |
+                              ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(y4[1])) << 16);
+          const uint32_t hi = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(y4[2])) |
+                              ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(y4[3])) << 16);
+          *reinterpret_cast<uint2*>(yr) = make_uint2(lo, hi);
+        } else {
+          for (int i = 0; i < 4; ++i)
+            if (n0 + i < p.N) yr[i] = __float2bfloat16_rn(y4[i]);
+        }
+      } else {
+        float* yr = reinterpret_cast<float*>(p.y) + (size_t)m * p.ldy + n0;
+        if (p.vec_store && n0 + 4 <= p.N) {
+          *reinterpret_cast<float4*>(yr) = make_float4(y4[0], y4[1], y4[2], y4[3]);
+        } else {
+          for (int i = 0; i < 4; ++i)
+            if (n0 + i < p.N) yr[i] = y4[i];
+        }
+      }
+    }
+  }
+  if (split > 1) pair::cluster_sync_all();  // no CTA leaves while a peer may still read its partial
+  tc_fence_after();
+  if (warp == 1) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
+  }
+}
+
+}  // namespace swapab
+
 
 // ------------------------------------------------------------------ host ---
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
@@ -1703,6 +2037,51 @@ cudaError_t run_splitk(const GemmParams& gp, int split, cudaStream_t st) {
                        false, (unsigned)split, ta, tb, ka, split);
 }
 
+// Swap-AB launch: the weights gp.b stream through the MMA's M dimension in 128-row tiles, the
+// M <= BNT activation rows gp.a are its N; `split` CTAs (a cluster when > 1) share a tile's k-tiles.
+template <int BNT, int FMT, bool BF16>
+cudaError_t run_swap(const GemmParams& gp, int split, cudaStream_t st) {
+  using C = swapab::CfgS<BNT, FMT>;
+  auto kernel = swapab::fp4_gemm_swap_kernel<BNT, FMT, BF16>;
+  static const cudaError_t attr = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                       C::kSmemBytes);
+  if (attr != cudaSuccess) return attr;
+  CUtensorMap tw, tx;
+  if (!make_code_map(&tw, gp.b, gp.N, gp.K / 2, 128)) return cudaErrorNotSupported;
+  if (!make_code_map(&tx, gp.a, gp.M, gp.K / 2, BNT)) return cudaErrorNotSupported;
+  KernelArgs ka;
+  ka.a_sf = gp.a_sf;
+  ka.b_sf = gp.b_sf;
+  ka.a_ts = gp.a_ts;
+  ka.b_ts = gp.b_ts;
+  ka.y = gp.y;
+  ka.ldy = gp.ldy;
+  ka.M = (int)gp.M;
+  ka.N = (int)gp.N;
+  ka.K = (int)gp.K;
+  ka.num_m = 1;
+  ka.num_n = (int)((gp.N + 127) / 128);
+  ka.g4 = (int)((gp.K / FmtTraits<FMT>::kBlock + 3) / 4);
+  ka.error = gp.error;
+  {
+    const int64_t esz = gp.y_bf16 ? 2 : 4;
+    ka.vec_store = ((gp.ldy * esz) % 32 == 0 && (reinterpret_cast<uintptr_t>(gp.y) & 31u) == 0)   ? 2
+                   : ((gp.ldy * esz) % 16 == 0 && (reinterpret_cast<uintptr_t>(gp.y) & 15u) == 0) ? 1
+                                                                                                   : 0;
+  }
+  ka.tma_store = 0;
+  return launch_kernel(kernel, dim3((unsigned)(ka.num_n * split)), dim3(C::kThreads), C::kSmemBytes, st, false,
+                       (unsigned)split, tw, tx, ka, split);
+}
+
+template <int FMT, bool BF16>
+cudaError_t dispatch_swap_bnt(const GemmParams& gp, int split, cudaStream_t st) {
+  if (gp.M <= 16) return run_swap<16, FMT, BF16>(gp, split, st);
+  if (gp.M <= 32) return run_swap<32, FMT, BF16>(gp, split, st);
+  if (gp.M <= 64) return run_swap<64, FMT, BF16>(gp, split, st);
+  return run_swap<128, FMT, BF16>(gp, split, st);
+}
+
 }  // namespace
 
 template <int BN>
@@ -1745,44 +2124,38 @@ static cudaError_t dispatch_quant(const GemmParams& p, bool pair_tiles, int bn, 
 }
 
 cudaError_t launch_gemm(const GemmParams& p, int num_sms, cudaStream_t st) {
-  // Tuning overrides: FP4_GEMM_BN=128|256 (tile width), FP4_GEMM_PAIR=0|1 (SM-pair kernel off/forced).
-  static const int forced_bn = [] {
-    const char* e = getenv("FP4_GEMM_BN");
-    const int v = e ? atoi(e) : 0;
-    return v == 128 || v == 256 ? v : 0;
-  }();
-  static const int pair_mode = [] {
-    const char* e = getenv("FP4_GEMM_PAIR");
-    return e == nullptr ? -1 : (e[0] == '0' ? 0 : 1);
-  }();
   // SM-pair 256 x 256 tiles when K is a multiple of 256 (every scale box then stays inside its row
   // block), long enough (>= 2048) for the single accumulator's epilogue to hide behind the mainloop,
   // and the problem has enough tiles to occupy the SM pairs.  Shorter K runs on single-SM 128 x 256
-  // tiles (measured faster at K = 768).  256 x 128 pair tiles are only used when forced.
-  const int pair_bn = forced_bn ? forced_bn : 256;
-  const bool pair_auto = p.K >= 2048 && p.M >= 256 && p.N >= 256 &&
-                         ((p.M + 255) / 256) * ((p.N + pair_bn - 1) / pair_bn) >= num_sms / 2;
-  if (p.q_out != 0) {
-    const bool pair_tiles = pair_mode != 0 && p.K % 256 == 0 && (pair_mode == 1 || pair_auto) && pair_bn == 256;
-    const int qbn = forced_bn ? forced_bn : (p.N >= 256 ? 256 : 128);
-    return p.q_out == 1 ? dispatch_quant<1>(p, pair_tiles, qbn, num_sms, st)
-                        : dispatch_quant<2>(p, pair_tiles, qbn, num_sms, st);
+  // tiles (measured faster at K = 768), N < 256 on 128 x 128 tiles.
+  const bool pair_tiles = p.K % 256 == 0 && p.K >= 2048 && p.M >= 256 && p.N >= 256 &&
+                          ((p.M + 255) / 256) * ((p.N + 255) / 256) >= num_sms / 2;
+  const int bn = p.N >= 256 ? 256 : 128;
+  if (p.q_out != 0)
+    return p.q_out == 1 ? dispatch_quant<1>(p, pair_tiles, bn, num_sms, st)
+                        : dispatch_quant<2>(p, pair_tiles, bn, num_sms, st);
+  const int64_t wtiles = (p.N + 127) / 128, nkb_s = (p.K + BK - 1) / BK;
+  if (p.M <= 128 && 2 * wtiles <= num_sms && nkb_s >= 2) {
+    // at most 128 activation rows and at most half as many 128-row weight tiles as SMs: swap-AB
+    // weight streaming, each tile's k-tiles split over a cluster of 2 to 8 CTAs so that about one
+    // CTA runs per SM.  (Both small-M kernels are bound by the tensor-memory scale copies, eight
+    // 512-byte atoms per k-tile here; with a single CTA per tile, N > 9472 on 148 SMs, the
+    // 128 x 256 split-K tiles below measured faster.)
+    int64_t split = std::min<int64_t>(std::min<int64_t>(num_sms / wtiles, splitk::kMaxSplit), nkb_s);
+    if (p.fmt == FMT_MX)
+      return p.y_bf16 ? dispatch_swap_bnt<FMT_MX, true>(p, (int)split, st)
+                      : dispatch_swap_bnt<FMT_MX, false>(p, (int)split, st);
+    return p.y_bf16 ? dispatch_swap_bnt<FMT_NV, true>(p, (int)split, st)
+                    : dispatch_swap_bnt<FMT_NV, false>(p, (int)split, st);
   }
-  if (pair_mode != 0 && p.K % 256 == 0 && (pair_mode == 1 || pair_auto))
-    return pair_bn == 256 ? dispatch_pair<256>(p, num_sms, st) : dispatch_pair<128>(p, num_sms, st);
-  const int bn = forced_bn ? forced_bn : (p.N >= 256 ? 256 : 128);
-  // Too few output tiles to fill the SMs (small M): split each tile's k-range over a cluster of up
-  // to 8 CTAs, as many as keep the launch within one CTA per SM.  FP4_GEMM_SPLIT=1 turns it off.
-  static const int split_mode = [] {
-    const char* e = getenv("FP4_GEMM_SPLIT");
-    return e == nullptr ? -1 : atoi(e);
-  }();
+  if (pair_tiles) return dispatch_pair<256>(p, num_sms, st);
+  // Too few output tiles to fill the SMs: split each tile's k-range over a cluster of up to 8 CTAs,
+  // as many as keep the launch within one CTA per SM.
   const int64_t tiles = ((p.M + BM - 1) / BM) * ((p.N + bn - 1) / bn);
   const int64_t nkb = (p.K + BK - 1) / BK;
   int64_t split = tiles > 0 ? num_sms / tiles : 1;
   if (split > splitk::kMaxSplit) split = splitk::kMaxSplit;
   if (split > nkb) split = nkb;
-  if (split_mode >= 1) split = std::min<int64_t>(std::min<int64_t>(split_mode, splitk::kMaxSplit), nkb);
   // every cluster must be resident at once: shrink the clusters until the device holds them all
   // (clusters of 8 x 220 KB CTAs need 8 free SMs in one GPC)
   while (split >= 2 &&

@@ -156,7 +156,32 @@ struct QRowParams {
   float* rotated;
   unsigned* error;       // device error word (streaming kernels: bit 2 = a ring wait expired)
   void* deq;             // DQ kernels: the dequantized values [rows, cols] (fp32, or bf16 for DQ = 2)
+  uint32_t sf_rows;      // tensor-core scale layout: valid rows and scale groups per row, whose padding
+  uint32_t sf_groups;    // bytes (rows up to 128, groups up to 4 g4) the kernel writes as 0
 };
+
+// Zero bytes of the tensor-core scale layout's padding (rows sf_rows .. multiple of 128, groups
+// sf_groups .. 4 g4), dealt over the grid's threads `t` of `nt`; the valid bytes are the
+// quantizer's.  Replaces a separate memset launch ahead of the quantizer.
+__device__ __forceinline__ void sf_pad_zero(const QRowParams& p, uint32_t t, uint32_t nt) {
+  const uint32_t gp = 4u * p.g4;                                   // padded groups per row
+  const uint32_t rpad = ((p.sf_rows + 127u) & ~127u) - p.sf_rows;   // padding rows
+  const uint32_t gpad = gp - p.sf_groups;                          // padding groups of valid rows
+  const unsigned long long n_rows = (unsigned long long)rpad * gp;
+  const unsigned long long n_all = n_rows + (unsigned long long)p.sf_rows * gpad;
+  for (unsigned long long i = t; i < n_all; i += nt) {
+    uint32_t r, g;
+    if (i < n_rows) {
+      r = p.sf_rows + (uint32_t)(i / gp);
+      g = (uint32_t)(i % gp);
+    } else {
+      const unsigned long long j = i - n_rows;
+      r = (uint32_t)(j / gpad);
+      g = p.sf_groups + (uint32_t)(j % gpad);
+    }
+    p.scales[sf_mma_offset(r, g, p.g4)] = 0u;
+  }
+}
 
 
 // Per-thread NVFP4 constants: the tensor scale, its reciprocal and the (S, 1/S) table.
@@ -398,6 +423,7 @@ __global__ void __launch_bounds__(256) quantize_rows_kernel(QRowParams p) {
   __shared__ double tabd[128];
   const int lane = threadIdx.x & 31;
   pdl_wait();
+  if (SFMMA) sf_pad_zero(p, blockIdx.x * blockDim.x + threadIdx.x, gridDim.x * blockDim.x);
   NvConsts nv{1.0f, 1.0, tabd};
   if (FMT != FMT_MX) {
     nv = nv_consts(*p.ts, tabd);
@@ -522,6 +548,7 @@ __global__ void __launch_bounds__(StreamWarps<FMT, RND>::kThreads, 1) quantize_s
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   stream_ring_init(r, kStreamWarps);
   pdl_wait();
+  if (SFMMA) sf_pad_zero(p, blockIdx.x * blockDim.x + threadIdx.x, gridDim.x * blockDim.x);
   NvConsts nv{1.0f, 1.0, tabd};
   if (FMT != FMT_MX) {
     nv = nv_consts(*p.ts, tabd);
@@ -684,6 +711,7 @@ __global__ void __launch_bounds__(FusedWarps<FMT>::kThreads, 1) nv_quantize_fuse
     mbar_init_fence();
   }
   pdl_wait();
+  if (SFMMA) sf_pad_zero(p, blockIdx.x * blockDim.x + threadIdx.x, gridDim.x * blockDim.x);
   __syncthreads();
   // phase 1: the slice lands in shared memory as kFusedPieces bulk copies; consumers reduce the
   // amax (of the rotated values when HAD > 0) of each piece as soon as it arrives
@@ -1578,6 +1606,8 @@ cudaError_t launch_quantize_nv_fused(const QuantizeParams& p, float* ts_out, con
   qp.rotated = p.rotated;
   qp.error = s.error;
   qp.deq = p.deq;
+  qp.sf_rows = (uint32_t)p.rows;
+  qp.sf_groups = (uint32_t)(p.cols / 16);
   fp.ts_out = ts_out;
   fp.partials = s.partials;
   fp.arrive = s.grid_arrive;
@@ -1657,6 +1687,8 @@ cudaError_t launch_quantize(const QuantizeParams& p, int num_sms, cudaStream_t s
     qp.rotated = p.rotated;
     qp.error = p.error;
     qp.deq = p.deq;
+    qp.sf_rows = (uint32_t)p.rows;
+    qp.sf_groups = (uint32_t)(p.cols / bs);
     if (p.deq_mode != 0) {
       if (p.had != 0 || p.four_six) return cudaErrorInvalidValue;
       if (p.fmt == FMT_MX)
@@ -1742,22 +1774,13 @@ cudaError_t launch_quantize_2d(const QuantizeParams& p, uint8_t* codes_t, uint8_
                          : q2d_dispatch<FMT_NV>(qp, p.rnd, sfmma, num_sms, st);
 }
 
-// FP4_DEQ_STAGED=1 selects the shared-memory-staged dequantize kernel (tuning override).
-static bool deq_staged() {
-  static const bool on = [] {
-    const char* e = getenv("FP4_DEQ_STAGED");
-    return e != nullptr && e[0] == '1';
-  }();
-  return on;
-}
-
 // Direct stores, except for fp32 outputs well beyond L2 (> 96 MB), which stream to HBM faster
 // through the staging ring and bulk stores (measured: 8192^2 fp32 53.6 us staged, 58.7 us direct;
 // 8192^2 bf16 with tensor-core-layout scales 41.4 us staged, 35.2 us direct).
 template <int FMT, bool SFMMA, bool BF16>
 static cudaError_t deq_launch(const DeqParams& dp, int num_sms, cudaStream_t st) {
   const bool big_f32 = !BF16 && (uint64_t)dp.nchunks * 32u > 96ull * 1024 * 1024;
-  if (!deq_staged() && !big_f32) {
+  if (!big_f32) {
     auto direct = dequantize_direct_kernel<FMT, SFMMA, BF16>;
     static const int occ_d = resident_ctas(direct, 256);
     const uint32_t want = (dp.nchunks + 256u * kDeqDirectUnroll - 1) / (256u * kDeqDirectUnroll);

@@ -78,6 +78,40 @@ def test_gemm_shapes(mnk, fmt):
     F.fp4_check_device_errors()
 
 
+SMALL_M = [1, 3, 16, 17, 32, 33, 64, 65, 127, 128]
+SMALL_NK = [(128, 4096), (300, 320), (4100, 1024)]
+
+
+@pytest.mark.parametrize("fmt", ["mxfp4", "nvfp4"])
+@pytest.mark.parametrize("nk", SMALL_NK)
+@pytest.mark.parametrize("M", SMALL_M)
+def test_gemm_small_m_weight_streaming(M, nk, fmt):
+    """At most 128 activation rows: the weights stream through the MMA's M dimension in 128-row
+    tiles with the activations as its N (16, 32, 64 or 128 columns), k-tiles split over a cluster.
+    Ragged M inside each activation tile width, a ragged last weight tile (N = 300, 4100), a k-tail
+    (K = 320: one 256-wide k-tile and one of 64), a single weight tile split eight ways (N = 128);
+    fp32 output against the fp64 oracle, bf16 within one ulp of it, and a strided output."""
+    N, K = nk
+    g = np.random.default_rng(M * 131 + N + K)
+    from workloads import bf16_bits
+    a = bf16_bits(g.standard_normal((M, K)).astype(np.float32))
+    b = bf16_bits((g.standard_normal((N, K)) * 0.02).astype(np.float32))
+    qa, qb = _gpu_quant(dev_bf16(a), fmt), _gpu_quant(dev_bf16(b), fmt)
+    kw = dict(fmt=fmt, a_tensor_scale=qa.tensor_scale, b_tensor_scale=qb.tensor_scale)
+    y32 = F.fp4_gemm(qa.codes, qa.scales, qb.codes, qb.scales, out_dtype="f32", **kw)
+    y16 = F.fp4_gemm(qa.codes, qa.scales, qb.codes, qb.scales, out_dtype="bf16", **kw)
+    big = torch.full((M, N + 36), 7.0, dtype=torch.float32, device="cuda")
+    F.fp4_gemm(qa.codes, qa.scales, qb.codes, qb.scales, out_dtype="f32", out=big[:, :N], **kw)
+    yr, bd = O.gemm_ref(_as_oracle(qa, fmt, M, K), _as_oracle(qb, fmt, N, K), fmt)
+    got = host_f32(y32)
+    _check(got, yr, bd)
+    _bf16_ulp_check(y16, got)
+    out = host_f32(big)
+    np.testing.assert_array_equal(out[:, :N].view(np.uint32), got.view(np.uint32))
+    assert np.all(out[:, N:] == 7.0)            # nothing written past N
+    F.fp4_check_device_errors()
+
+
 @pytest.mark.parametrize("fmt", ["mxfp4", "nvfp4"])
 def test_pair_tiles_ragged_edges(fmt):
     """2400 x 1900 x 2048: enough 256 x 256 tiles for the SM-pair kernel, with the last row tile's
