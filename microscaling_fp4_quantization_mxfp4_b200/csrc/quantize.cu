@@ -337,9 +337,23 @@ __device__ __forceinline__ void dequant_block_out(const QRowParams& p, const uin
   }
 }
 
+// Chunk order of a block as the shared-memory streaming kernels load it: register k holds the
+// block's 16-byte chunk k ^ sw, with sw = bit 2 of the lane for NVFP4 (two chunks) and bits 1-2 for
+// MXFP4 (four chunks), so that the eight lanes of a quarter warp read eight distinct 16-byte bank
+// groups (in chunk order the 32- or 64-byte blocks of those lanes share banks: 2- or 4-way
+// conflicts).  quantize_block puts the codes (and dequantized values) back in chunk order before
+// they leave.  0 for four-over-six, which adds its error terms in element order, and under the
+// rotation, whose butterflies pair chunks by position.
+template <int FMT, int HAD>
+__device__ __forceinline__ uint32_t chunk_swap(int lane) {
+  if (HAD != 0) return 0u;
+  return FMT == FMT_NV ? (uint32_t)(lane >> 2) & 1u : FMT == FMT_MX ? (uint32_t)(lane >> 1) & 3u : 0u;
+}
+
+// v[k] holds the block's chunk k ^ sw (sw = chunk_swap or 0).
 template <int FMT, int RND, int HAD, bool SFMMA, int DQ = 0>
 __device__ __forceinline__ void quantize_block(const QRowParams& p, const uint4 (&v)[BlockShape<FMT>::V], uint32_t blk,
-                                               bool valid, int lane, const NvConsts& nv) {
+                                               bool valid, int lane, const NvConsts& nv, uint32_t sw = 0u) {
   constexpr int E = BlockShape<FMT>::E, V = BlockShape<FMT>::V;
   float x[E];
 #pragma unroll
@@ -387,13 +401,31 @@ __device__ __forceinline__ void quantize_block(const QRowParams& p, const uint4 
     const unsigned long long j0 = (unsigned long long)blk * (E / 4);     // Philox counter of element blk*E
 #pragma unroll
     for (int k = 0; k < E / 8; ++k) {
-      const unsigned long long j = j0 + 2u * k;
+      const unsigned long long j = j0 + 2u * ((uint32_t)k ^ sw);          // slot k holds chunk k ^ sw
       const u32x4 a = philox4x32_10((uint32_t)j, (uint32_t)(j >> 32), p.keys);
       const u32x4 b = philox4x32_10((uint32_t)(j + 1), (uint32_t)((j + 1) >> 32), p.keys);
       const float* xe = x + 8 * k;
       const uint32_t n[8] = {e2m1_sr(xe[0], a.x), e2m1_sr(xe[1], a.y), e2m1_sr(xe[2], a.z), e2m1_sr(xe[3], a.w),
                              e2m1_sr(xe[4], b.x), e2m1_sr(xe[5], b.y), e2m1_sr(xe[6], b.z), e2m1_sr(xe[7], b.w)};
       w[k] = pack8_nibbles(n);
+    }
+  }
+  if (FMT != FMT_NV46 && HAD == 0) {                     // back to chunk order: w[c] <- w[c ^ sw]
+    if (sw & 1u) {
+#pragma unroll
+      for (int k = 0; k < E / 8; k += 2) {
+        const uint32_t t = w[k];
+        w[k] = w[k + 1];
+        w[k + 1] = t;
+      }
+    }
+    if (E / 8 == 4 && (sw & 2u)) {
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        const uint32_t t = w[k];
+        w[k] = w[k + 2 < E / 8 ? k + 2 : k];
+        w[k + 2 < E / 8 ? k + 2 : k] = t;
+      }
     }
   }
   if (!valid) return;
@@ -578,9 +610,10 @@ __global__ void __launch_bounds__(StreamWarps<FMT, RND>::kThreads, 1) quantize_s
       const uint32_t lb = u * 32u + lane;                                    // block within the stage
       const bool valid = lb * V < n;
       uint4 v[V];
+      const uint32_t sw = chunk_swap<FMT, HAD>(lane);
 #pragma unroll
-      for (int k = 0; k < V; ++k) v[k] = valid ? src[lb * V + k] : make_uint4(0u, 0u, 0u, 0u);
-      quantize_block<FMT, RND, HAD, SFMMA, DQ>(p, v, c0 / V + lb, valid, lane, nv);
+      for (int k = 0; k < V; ++k) v[k] = valid ? src[lb * V + ((uint32_t)k ^ sw)] : make_uint4(0u, 0u, 0u, 0u);
+      quantize_block<FMT, RND, HAD, SFMMA, DQ>(p, v, c0 / V + lb, valid, lane, nv, sw);
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(smem_addr(&r.empty[stage]));
@@ -802,9 +835,10 @@ __global__ void __launch_bounds__(FusedWarps<FMT>::kThreads, 1) nv_quantize_fuse
     const uint32_t lb = u * 32u + lane;
     const bool valid = lb * 2u < nslice;
     uint4 v[2];
-    v[0] = valid ? slice[lb * 2u] : make_uint4(0u, 0u, 0u, 0u);
-    v[1] = valid ? slice[lb * 2u + 1u] : make_uint4(0u, 0u, 0u, 0u);
-    quantize_block<FMT, RND, HAD, SFMMA, DQ>(p, v, c_begin / 2u + lb, valid, lane, nv);
+    const uint32_t sw = chunk_swap<FMT, HAD>(lane);
+    v[0] = valid ? slice[lb * 2u + sw] : make_uint4(0u, 0u, 0u, 0u);
+    v[1] = valid ? slice[lb * 2u + (sw ^ 1u)] : make_uint4(0u, 0u, 0u, 0u);
+    quantize_block<FMT, RND, HAD, SFMMA, DQ>(p, v, c_begin / 2u + lb, valid, lane, nv, sw);
   }
 }
 
