@@ -408,27 +408,64 @@ __device__ __forceinline__ void hadamard_rotate(float (&x)[8], int lane) {
 // then across HB/E consecutive lanes.  The stages run in the same order
 // (distance 1, 2, 4, ...) with the same operand order as hadamard_rotate, so
 // both layouts give bit-identical fp32 results.
-template <int HB, int E>
-__device__ __forceinline__ void hadamard_rotate_block(float (&x)[E], int lane) {
+//
+// The block's 8-element chunks may sit in XOR order: register chunk k holding
+// chunk k ^ sw, with sw = (lane >> SWS) & SWM (the order in which the streaming
+// kernels read shared memory without bank conflicts; SWM = 0: plain order).
+// A stage at distance 8 or 16 then pairs the same two registers, but when the
+// matching bit of sw is set the lower element sits in the upper register, so
+// each register takes x[i] * s + x[j] with the sign s of that bit (an exact
+// sum or difference, one rounding: the values of the plain order).  A cross-lane
+// stage whose partner lane has the other sw (a lane bit inside the sw field)
+// exchanges the register of the flipped chunk, chosen at compile time.
+template <int HB, int E, int SWS = 0, int SWM = 0>
+__device__ __forceinline__ void hadamard_rotate_block(float (&x)[E], int lane, uint32_t sw = 0u) {
   constexpr int IN = HB < E ? HB : E;
 #pragma unroll
   for (int d = 1; d < IN; d <<= 1) {
+    if (d < 8 || SWM == 0) {
 #pragma unroll
-    for (int i = 0; i < E; ++i) {
-      if ((i & d) == 0) {
-        const float a = x[i], b = x[i + d];
-        x[i] = __fadd_rn(a, b);
-        x[i + d] = __fsub_rn(a, b);
+      for (int i = 0; i < E; ++i) {
+        if ((i & d) == 0) {
+          const float a = x[i], b = x[i + d];
+          x[i] = __fadd_rn(a, b);
+          x[i + d] = __fsub_rn(a, b);
+        }
+      }
+    } else {
+      const float sg = ((sw >> (d == 8 ? 0 : 1)) & 1u) != 0u ? -1.0f : 1.0f;
+#pragma unroll
+      for (int i = 0; i < E; ++i) {
+        if ((i & d) == 0) {
+          const float a = x[i], b = x[i + d];
+          x[i] = __fmaf_rn(a, sg, b);
+          x[i + d] = __fmaf_rn(b, -sg, a);
+        }
       }
     }
   }
 #pragma unroll
   for (int ld = 1; ld < HB / E; ld <<= 1) {
     const float sgn = (lane & ld) != 0 ? -1.0f : 1.0f;     // p - x or x + p, as in hadamard_rotate
+    const int flip = ((ld >> SWS) & SWM) << 3;             // chunk bits by which the partner's order differs
+    if (flip == 0) {
 #pragma unroll
-    for (int i = 0; i < E; ++i) {
-      const float p = __shfl_xor_sync(0xFFFFFFFFu, x[i], ld);
-      x[i] = __fmaf_rn(x[i], sgn, p);
+      for (int i = 0; i < E; ++i) {
+        const float p = __shfl_xor_sync(0xFFFFFFFFu, x[i], ld);
+        x[i] = __fmaf_rn(x[i], sgn, p);
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < E; ++i) {
+        if ((i & flip) == 0) {
+          const int j = i ^ flip;
+          const float a = x[i], b = x[j];
+          const float pa = __shfl_xor_sync(0xFFFFFFFFu, b, ld);   // the partner's element at i's position
+          const float pb = __shfl_xor_sync(0xFFFFFFFFu, a, ld);   // and at j's
+          x[i] = __fmaf_rn(a, sgn, pa);
+          x[j] = __fmaf_rn(b, sgn, pb);
+        }
+      }
     }
   }
   const float s = HB == 16 ? 0.25f : HB == 32 ? 0.17677669529663687f : HB == 64 ? 0.125f : 0.08838834764831845f;

@@ -337,21 +337,26 @@ __device__ __forceinline__ void dequant_block_out(const QRowParams& p, const uin
   }
 }
 
+// The lane bits that select a block's chunk order (chunk_swap): bit 2 for NVFP4, bits 1-2 for MXFP4.
+template <int FMT> constexpr int kSwShift = FMT == FMT_MX ? 1 : 2;
+template <int FMT> constexpr uint32_t kSwMask = FMT == FMT_MX ? 3u : FMT == FMT_NV ? 1u : 0u;
+
 // Chunk order of a block as the shared-memory streaming kernels load it: register k holds the
 // block's 16-byte chunk k ^ sw, with sw = bit 2 of the lane for NVFP4 (two chunks) and bits 1-2 for
 // MXFP4 (four chunks), so that the eight lanes of a quarter warp read eight distinct 16-byte bank
 // groups (in chunk order the 32- or 64-byte blocks of those lanes share banks: 2- or 4-way
 // conflicts).  quantize_block puts the codes (and dequantized values) back in chunk order before
-// they leave.  0 for four-over-six, which adds its error terms in element order, and under the
-// rotation, whose butterflies pair chunks by position.
+// they leave, and the rotation's butterflies follow the order (hadamard_rotate_block).  0 for
+// four-over-six, which adds its error terms in element order.
 template <int FMT, int HAD>
 __device__ __forceinline__ uint32_t chunk_swap(int lane) {
-  if (HAD != 0) return 0u;
-  return FMT == FMT_NV ? (uint32_t)(lane >> 2) & 1u : FMT == FMT_MX ? (uint32_t)(lane >> 1) & 3u : 0u;
+  return FMT == FMT_NV ? (uint32_t)(lane >> kSwShift<FMT>) & kSwMask<FMT>
+                       : FMT == FMT_MX ? (uint32_t)(lane >> kSwShift<FMT>) & kSwMask<FMT> : 0u;
 }
 
-// v[k] holds the block's chunk k ^ sw (sw = chunk_swap or 0).
-template <int FMT, int RND, int HAD, bool SFMMA, int DQ = 0>
+// v[k] holds the block's chunk k ^ sw: SWZ = true with sw = chunk_swap(lane) in the streaming
+// kernels (every lane's order set by its lane bits), SWZ = false and sw = 0 elsewhere.
+template <int FMT, int RND, int HAD, bool SFMMA, int DQ = 0, bool SWZ = false>
 __device__ __forceinline__ void quantize_block(const QRowParams& p, const uint4 (&v)[BlockShape<FMT>::V], uint32_t blk,
                                                bool valid, int lane, const NvConsts& nv, uint32_t sw = 0u) {
   constexpr int E = BlockShape<FMT>::E, V = BlockShape<FMT>::V;
@@ -364,11 +369,14 @@ __device__ __forceinline__ void quantize_block(const QRowParams& p, const uint4 
     for (int i = 0; i < 8; ++i) x[8 * k + i] = t8[i];
   }
   if (HAD) {
-    hadamard_rotate_block<HAD, E>(x, lane);
+    hadamard_rotate_block<HAD, E, kSwShift<FMT>, (SWZ ? (int)kSwMask<FMT> : 0)>(x, lane, sw);
     if (p.rotated != nullptr && valid) {
       float4* r = reinterpret_cast<float4*>(p.rotated + (size_t)blk * E);
 #pragma unroll
-      for (int k = 0; k < E / 4; ++k) r[k] = make_float4(x[4 * k], x[4 * k + 1], x[4 * k + 2], x[4 * k + 3]);
+      for (int k = 0; k < E / 4; ++k) {
+        const uint32_t q = (((uint32_t)(k >> 1) ^ sw) << 1) | (uint32_t)(k & 1);   // chunk k/2 is chunk k/2 ^ sw
+        r[q] = make_float4(x[4 * k], x[4 * k + 1], x[4 * k + 2], x[4 * k + 3]);
+      }
     }
   }
   float am = 0.0f;
@@ -410,7 +418,7 @@ __device__ __forceinline__ void quantize_block(const QRowParams& p, const uint4 
       w[k] = pack8_nibbles(n);
     }
   }
-  if (FMT != FMT_NV46 && HAD == 0) {                     // back to chunk order: w[c] <- w[c ^ sw]
+  if (FMT != FMT_NV46) {                                  // back to chunk order: w[c] <- w[c ^ sw]
     if (sw & 1u) {
 #pragma unroll
       for (int k = 0; k < E / 8; k += 2) {
@@ -613,7 +621,7 @@ __global__ void __launch_bounds__(StreamWarps<FMT, RND>::kThreads, 1) quantize_s
       const uint32_t sw = chunk_swap<FMT, HAD>(lane);
 #pragma unroll
       for (int k = 0; k < V; ++k) v[k] = valid ? src[lb * V + ((uint32_t)k ^ sw)] : make_uint4(0u, 0u, 0u, 0u);
-      quantize_block<FMT, RND, HAD, SFMMA, DQ>(p, v, c0 / V + lb, valid, lane, nv, sw);
+      quantize_block<FMT, RND, HAD, SFMMA, DQ, true>(p, v, c0 / V + lb, valid, lane, nv, sw);
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(smem_addr(&r.empty[stage]));
@@ -838,7 +846,7 @@ __global__ void __launch_bounds__(FusedWarps<FMT>::kThreads, 1) nv_quantize_fuse
     const uint32_t sw = chunk_swap<FMT, HAD>(lane);
     v[0] = valid ? slice[lb * 2u + sw] : make_uint4(0u, 0u, 0u, 0u);
     v[1] = valid ? slice[lb * 2u + (sw ^ 1u)] : make_uint4(0u, 0u, 0u, 0u);
-    quantize_block<FMT, RND, HAD, SFMMA, DQ>(p, v, c_begin / 2u + lb, valid, lane, nv, sw);
+    quantize_block<FMT, RND, HAD, SFMMA, DQ, true>(p, v, c_begin / 2u + lb, valid, lane, nv, sw);
   }
 }
 
