@@ -200,3 +200,35 @@ def test_hadamard_quantize_full_size_8192x4096(cfg3_acts, had, fmt, rnd):
                                       rnd, seed, s_k, s_o)
     assert near <= 64
     F.fp4_check_device_errors()
+
+
+@pytest.mark.parametrize("sf", ["rowmajor", "mma"])
+@pytest.mark.parametrize("had", HADS)
+def test_hadamard_mxfp4_rtn_without_rotation_dump(had, sf):
+    """The production call (no dump of the rotated values) gives the codes and scales of the call
+    with the dump, which the other tests pin to the oracle, over rows scaled from 2^-130 to 2^121
+    (subnormal quotients, block maxima at and above 2^125), for the streaming and the strided-row
+    kernels."""
+    rows, cols = 512, 1024
+    g = np.random.default_rng(500 + had)
+    x = g.standard_normal((rows, cols)).astype(np.float32)
+    x *= np.exp2(g.integers(-130, 122, size=(rows, 1))).astype(np.float32)
+    x[:8] = (g.standard_normal((8, cols)) * np.float32(2.0 ** 121)).astype(np.float32)   # maxima >= 2^125
+    x[8:16, ::5] *= np.float32(2.0 ** -40)                                                # tiny inside blocks
+    xb = bf16_bits(x)
+    assert np.all(np.isfinite(bf16_to_f32(xb)))
+    xd = dev_bf16(xb)
+    rot = torch.empty((rows, cols), dtype=torch.float32, device="cuda")
+    q_dump = F.fp4_hadamard_quantize(xd, had, fmt="mxfp4", sf_layout=sf, rotated_out=rot)
+    q_fold = F.fp4_hadamard_quantize(xd, had, fmt="mxfp4", sf_layout=sf)
+    np.testing.assert_array_equal(host_u8(q_fold.codes), host_u8(q_dump.codes))
+    np.testing.assert_array_equal(host_u8(q_fold.scales), host_u8(q_dump.scales))
+    ref = O.quantize_values(host_f32(rot), fmt="mxfp4")
+    np.testing.assert_array_equal(host_u8(q_fold.codes), ref["codes"])
+    # the strided-row kernel (ld > cols) folds the same way
+    wide = torch.zeros((rows, cols + 64), dtype=torch.bfloat16, device="cuda")
+    wide[:, :cols] = xd
+    q_strided = F.fp4_hadamard_quantize(wide[:, :cols], had, fmt="mxfp4", sf_layout=sf)
+    np.testing.assert_array_equal(host_u8(q_strided.codes), host_u8(q_dump.codes))
+    np.testing.assert_array_equal(host_u8(q_strided.scales), host_u8(q_dump.scales))
+    F.fp4_check_device_errors()
