@@ -126,6 +126,27 @@ fp4_status fp4_quantize(const void* x, int64_t rows, int64_t cols, int64_t ld,
                         uint8_t* codes, uint8_t* scales, int sf_layout, void* stream);
 
 /*
+ * fp4_quantize_shard -- fp4_quantize of a row shard: x holds rows
+ * [first_row, first_row + rows) of a larger [*, cols] tensor, and the result is
+ * those rows of the whole tensor's quantization ("FP4 All the Way", Abstract:
+ * FP4 training across many accelerators, with stochastic rounding in the
+ * backward pass).  Stochastic rounding draws the Philox words of the elements'
+ * row-major indices in the whole tensor, (first_row + r) * cols + c, so shards
+ * quantized on different devices concatenate to the unsharded codes bit for
+ * bit.  For NVFP4 pass the whole tensor's scale in tensor_scale_in (e.g. from a
+ * max all-reduce of the shards' fp4_amax and fp4_nv_tensor_scale); without it
+ * the shard's own amax sets s_t.
+ *   first_row  0 <= first_row < 2^40 (FP4_ERR_ARG otherwise); a multiple of the
+ *              block for axis = 0 (FP4_ERR_SHAPE otherwise), so the shard's blocks
+ *              are the tensor's.
+ *   others     as fp4_quantize (first_row = 0 is fp4_quantize).
+ */
+fp4_status fp4_quantize_shard(const void* x, int64_t rows, int64_t cols, int64_t ld, int64_t first_row,
+                              int fmt, int block, int axis, int rnd, uint64_t seed,
+                              const float* tensor_scale_in, float* tensor_scale_out,
+                              uint8_t* codes, uint8_t* scales, int sf_layout, void* stream);
+
+/*
  * fp4_hadamard_quantize -- fp4_quantize with a block-diagonal Hadamard
  * rotation applied along the quantization axis first ("Bridging the Gap",
  * Abstract: block-wise Hadamard computed online for the activations; its

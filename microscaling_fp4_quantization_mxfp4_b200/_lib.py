@@ -11,6 +11,8 @@ _i64, _u64, _int, _vp, _sz = ctypes.c_int64, ctypes.c_uint64, ctypes.c_int, ctyp
 # name -> (restype, argtypes); mirrors include/fp4.h
 PROTOTYPES = {
     "fp4_quantize": (_int, [_vp, _i64, _i64, _i64, _int, _int, _int, _int, _u64, _vp, _vp, _vp, _vp, _int, _vp]),
+    "fp4_quantize_shard": (_int, [_vp, _i64, _i64, _i64, _i64, _int, _int, _int, _int, _u64, _vp, _vp, _vp, _vp, _int,
+                                  _vp]),
     "fp4_hadamard_quantize": (_int, [_vp, _i64, _i64, _i64, _int, _int, _int, _int, _u64, _vp, _vp, _vp, _vp,
                                      _int, _int, _vp, _vp]),
     "fp4_quantize_dequantize": (_int, [_vp, _i64, _i64, _i64, _int, _int, _int, _u64, _vp, _vp, _vp, _vp, _int, _vp,

@@ -110,15 +110,24 @@ def _alloc_quant_outputs(x, fmt, axis, sf, codes, scales, ts_out):
 
 def fp4_quantize(x: torch.Tensor, fmt="mxfp4", axis: int = 1, rnd="rtn", seed: int = 0,
                  tensor_scale_in: Optional[torch.Tensor] = None, sf_layout="rowmajor", *,
-                 codes=None, scales=None, tensor_scale_out=None, stream=None) -> Fp4Quantized:
-    """Block-scaled FP4 quantization of a bf16 matrix (see fp4_quantize in include/fp4.h)."""
+                 codes=None, scales=None, tensor_scale_out=None, first_row: int = 0, stream=None) -> Fp4Quantized:
+    """Block-scaled FP4 quantization of a bf16 matrix (see fp4_quantize in include/fp4.h).  With
+    first_row > 0, x is a row shard of a larger tensor starting at that row (fp4_quantize_shard)."""
     _bf16_matrix(x)
     f, r, sf = _FMT[fmt], _RND[rnd], _SF[sf_layout]
     codes, scales, ts_out = _alloc_quant_outputs(x, f, axis, sf, codes, scales, tensor_scale_out)
-    st = _lib.load().fp4_quantize(
-        x.data_ptr(), x.shape[0], x.shape[1], x.stride(0), f, BLOCK[f], axis, r, seed & (2 ** 64 - 1),
-        _ptr(tensor_scale_in), _ptr(ts_out), codes.data_ptr(), scales.data_ptr(), sf, _stream(stream))
-    _check(st, "fp4_quantize")
+    lib = _lib.load()
+    if first_row:
+        st = lib.fp4_quantize_shard(
+            x.data_ptr(), x.shape[0], x.shape[1], x.stride(0), first_row, f, BLOCK[f], axis, r,
+            seed & (2 ** 64 - 1), _ptr(tensor_scale_in), _ptr(ts_out), codes.data_ptr(), scales.data_ptr(), sf,
+            _stream(stream))
+        _check(st, "fp4_quantize_shard")
+    else:
+        st = lib.fp4_quantize(
+            x.data_ptr(), x.shape[0], x.shape[1], x.stride(0), f, BLOCK[f], axis, r, seed & (2 ** 64 - 1),
+            _ptr(tensor_scale_in), _ptr(ts_out), codes.data_ptr(), scales.data_ptr(), sf, _stream(stream))
+        _check(st, "fp4_quantize")
     return Fp4Quantized(codes, scales, ts_out if f in (NVFP4, NVFP4_4O6) else None)
 
 

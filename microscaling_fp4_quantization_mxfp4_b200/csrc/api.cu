@@ -99,7 +99,7 @@ fp4_status check_input(const void* x, int64_t rows, int64_t cols, int64_t ld) {
 fp4_status quantize_impl(const void* x, int64_t rows, int64_t cols, int64_t ld, int fmt, int block, int axis,
                          int rnd, uint64_t seed, const float* ts_in, float* ts_out, uint8_t* codes, uint8_t* scales,
                          int sf_layout, int had, float* rotated, cudaStream_t st, void* deq = nullptr,
-                         int deq_mode = 0) {
+                         int deq_mode = 0, uint64_t idx_base = 0) {
   int four_six = 0;
   uint32_t mx_thr = 0x800000u;       // OCP exponent rule
   if (fmt == FP4_MXFP4_GS) {         // MXFP4 codes and scales under the MSE-fitted clip threshold
@@ -165,6 +165,7 @@ fp4_status quantize_impl(const void* x, int64_t rows, int64_t cols, int64_t ld, 
   p.mx_thr = mx_thr;
   p.deq = deq;
   p.deq_mode = deq_mode;
+  p.idx_base = idx_base;
   size_t fused_smem = 0;
   uint32_t fused_tiles = 0;
   if (fmt == FP4_NVFP4 && ts_in == nullptr && axis == 1 && ld == cols &&
@@ -198,6 +199,18 @@ fp4_status fp4_quantize(const void* x, int64_t rows, int64_t cols, int64_t ld, i
                         uint8_t* scales, int sf_layout, void* stream) {
   return quantize_impl(x, rows, cols, ld, fmt, block, axis, rnd, seed, tensor_scale_in, tensor_scale_out, codes,
                        scales, sf_layout, 0, nullptr, static_cast<cudaStream_t>(stream));
+}
+
+fp4_status fp4_quantize_shard(const void* x, int64_t rows, int64_t cols, int64_t ld, int64_t first_row, int fmt,
+                              int block, int axis, int rnd, uint64_t seed, const float* tensor_scale_in,
+                              float* tensor_scale_out, uint8_t* codes, uint8_t* scales, int sf_layout, void* stream) {
+  if (first_row < 0 || first_row >= ((int64_t)1 << 40)) return FP4_ERR_ARG;
+  const int blk = block > 0 ? block : 1;
+  if (axis == 0 && first_row % blk != 0) return FP4_ERR_SHAPE;     // the shard's blocks are the tensor's
+  if (cols > 0 && first_row > (((int64_t)1 << 62) / cols)) return FP4_ERR_SHAPE;
+  return quantize_impl(x, rows, cols, ld, fmt, block, axis, rnd, seed, tensor_scale_in, tensor_scale_out, codes,
+                       scales, sf_layout, 0, nullptr, static_cast<cudaStream_t>(stream), nullptr, 0,
+                       (uint64_t)first_row * (uint64_t)(cols > 0 ? cols : 0));
 }
 
 fp4_status fp4_hadamard_quantize(const void* x, int64_t rows, int64_t cols, int64_t ld, int fmt, int block, int axis,

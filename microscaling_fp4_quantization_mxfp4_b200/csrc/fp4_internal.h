@@ -92,6 +92,8 @@ struct QuantizeParams {
   uint32_t mx_thr = 0x800000u;  // MXFP4 exponent clip threshold as a significand field (0x800000: OCP)
   void* deq = nullptr;    // axis 1: also write the dequantized values [rows, cols] here
   int deq_mode = 0;       // 0: no, 1: fp32, 2: bf16
+  uint64_t idx_base = 0;  // row-major index of x's first element in the tensor it is a row shard of
+                          // (a multiple of 8; stochastic rounding draws the words of idx_base + index)
 };
 
 // amax pass: mode 0 writes max|x| (after rotation when had > 0) to `out`,

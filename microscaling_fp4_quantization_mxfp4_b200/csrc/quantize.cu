@@ -158,6 +158,7 @@ struct QRowParams {
   void* deq;             // DQ kernels: the dequantized values [rows, cols] (fp32, or bf16 for DQ = 2)
   uint32_t sf_rows;      // tensor-core scale layout: valid rows and scale groups per row, whose padding
   uint32_t sf_groups;    // bytes (rows up to 128, groups up to 4 g4) the kernel writes as 0
+  unsigned long long jbase;  // Philox counter of the first element (row shards: first_row * cols / 4)
 };
 
 // Zero bytes of the tensor-core scale layout's padding (rows sf_rows .. multiple of 128, groups
@@ -406,7 +407,7 @@ __device__ __forceinline__ void quantize_block(const QRowParams& p, const uint4 
       w[k] = e2m1x4_rn(x[8 * k], x[8 * k + 1], x[8 * k + 2], x[8 * k + 3], x[8 * k + 4], x[8 * k + 5], x[8 * k + 6],
                        x[8 * k + 7]);
   } else {
-    const unsigned long long j0 = (unsigned long long)blk * (E / 4);     // Philox counter of element blk*E
+    const unsigned long long j0 = p.jbase + (unsigned long long)blk * (E / 4);   // counter of element blk*E
 #pragma unroll
     for (int k = 0; k < E / 8; ++k) {
       const unsigned long long j = j0 + 2u * ((uint32_t)k ^ sw);          // slot k holds chunk k ^ sw
@@ -888,6 +889,7 @@ struct QColParams {
   uint32_t G, g4;        // k-groups per output row (R / block) and padded/4
   unsigned long long seed;
   PhiloxKeys keys;      // the seed's Philox key schedule
+  unsigned long long jbase;  // Philox counter of element (0, 0) (row shards: first_row * C / 4)
   uint32_t mx_thr;      // MXFP4 exponent clip threshold (significand field; kMxClipOcp: the OCP rule)
   const float* ts;
   float* ts_copy_out;
@@ -984,7 +986,7 @@ __global__ void __launch_bounds__(256, (RND == RND_SR && FMT != FMT_NV46) ? 3 : 
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
             const unsigned long long row = rb + w8 * 8 + 4 * h + (lane & 3);
-            const unsigned long long j = (row * p.C + (c & ~3u)) >> 2;
+            const unsigned long long j = p.jbase + ((row * p.C + (c & ~3u)) >> 2);
             const u32x4 ph = philox4x32_10((uint32_t)j, (uint32_t)(j >> 32), p.keys);
             const uint32_t w[4] = {ph.x, ph.y, ph.z, ph.w};
             uint32_t t[4];
@@ -1640,6 +1642,7 @@ cudaError_t launch_quantize_nv_fused(const QuantizeParams& p, float* ts_out, con
   qp.g4 = (uint32_t)((p.cols / 16 + 3) / 4);
   qp.seed = p.seed;
   qp.keys = philox_keys(p.seed);
+  qp.jbase = p.idx_base >> 2;
   qp.mx_thr = p.mx_thr;
   qp.ts = nullptr;
   qp.ts_copy_out = nullptr;
@@ -1721,6 +1724,7 @@ cudaError_t launch_quantize(const QuantizeParams& p, int num_sms, cudaStream_t s
     qp.g4 = (uint32_t)((p.cols / bs + 3) / 4);
     qp.seed = p.seed;
     qp.keys = philox_keys(p.seed);
+    qp.jbase = p.idx_base >> 2;
     qp.mx_thr = p.mx_thr;
     qp.ts = p.ts;
     qp.ts_copy_out = p.ts_copy_out;
@@ -1759,6 +1763,7 @@ cudaError_t launch_quantize(const QuantizeParams& p, int num_sms, cudaStream_t s
   qp.g4 = (qp.G + 3u) / 4u;
   qp.seed = p.seed;
   qp.keys = philox_keys(p.seed);
+  qp.jbase = p.idx_base >> 2;
   qp.mx_thr = p.mx_thr;
   qp.ts = p.ts;
   qp.ts_copy_out = p.ts_copy_out;

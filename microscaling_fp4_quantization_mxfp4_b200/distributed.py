@@ -45,11 +45,14 @@ def sharded_nvfp4_tensor_scale(x_shard: torch.Tensor, group=None, *,
     return (scale_fn or fp4_nv_tensor_scale)(amax)
 
 
-def sharded_nvfp4_quantize(x_shard: torch.Tensor, group=None, sf_layout="rowmajor", **kw):
-    """Round-to-nearest NVFP4 quantization of this rank's rows under the global tensor scale.
-
-    (Stochastic rounding keys Philox by the element index within the tensor the
-    kernel sees, so a sharded SR run draws different words than an unsharded one.)
-    """
-    ts = sharded_nvfp4_tensor_scale(x_shard, group)
-    return fp4_quantize(x_shard, fmt="nvfp4", rnd="rtn", tensor_scale_in=ts, sf_layout=sf_layout, **kw)
+def sharded_nvfp4_quantize(x_shard: torch.Tensor, first_row: int, group=None, rnd="rtn", seed: int = 0,
+                           sf_layout="rowmajor", *, amax_fn: Optional[Callable] = None,
+                           scale_fn: Optional[Callable] = None, quantize_fn: Optional[Callable] = None, **kw):
+    """NVFP4 quantization of this rank's rows [first_row, first_row + rows) under the global tensor
+    scale.  Stochastic rounding draws the Philox words of the whole tensor's element indices
+    (fp4_quantize_shard), so the ranks' codes concatenate to the unsharded tensor's, for either
+    rounding.  The *_fn parameters default to the CUDA entry points; they exist only so the host
+    logic can be exercised without a GPU."""
+    ts = sharded_nvfp4_tensor_scale(x_shard, group, amax_fn=amax_fn, scale_fn=scale_fn)
+    return (quantize_fn or fp4_quantize)(x_shard, fmt="nvfp4", rnd=rnd, seed=seed, tensor_scale_in=ts,
+                                         sf_layout=sf_layout, first_row=first_row, **kw)

@@ -96,6 +96,11 @@ def test_other_entry_points_reject_before_launch(lib):
     assert lib.fp4_quantize_2d(FAKE, 64, 64, 64, 0, 32, 0, 0, None, None, FAKE, FAKE, FAKE, None, 0, None) == -1
     assert lib.fp4_quantize_2d(FAKE, 64, 64, 64, 1, 16, 0, 0, None, None, FAKE, FAKE, None, None, 0, None) == -1
     assert lib.fp4_quantize_2d(FAKE, 64, 64, 64, 0, 32, 0, 0, None, None, FAKE + 4, FAKE, None, None, 0, None) == -3
+    # fp4_quantize_shard: negative first row, axis-0 shard not starting on a block, then fp4_quantize's checks
+    assert lib.fp4_quantize_shard(FAKE, 4, 64, 64, -16, 0, 32, 1, 0, 0, None, None, FAKE, FAKE, 0, None) == -1
+    assert lib.fp4_quantize_shard(FAKE, 64, 64, 64, 16, 0, 32, 0, 0, 0, None, None, FAKE, FAKE, 0, None) == -2
+    assert lib.fp4_quantize_shard(FAKE, 4, 64, 64, 8, 0, 16, 1, 0, 0, None, None, FAKE, FAKE, 0, None) == -4
+    assert lib.fp4_quantize_shard(FAKE + 2, 4, 64, 64, 8, 0, 32, 1, 0, 0, None, None, FAKE, FAKE, 0, None) == -3
     # four-over-six NVFP4 (fmt 2): block 16 only, needs s_t out, no Hadamard, quantizer entry points only
     assert lib.fp4_quantize(FAKE, 4, 64, 64, 2, 32, 1, 0, 0, None, None, FAKE, FAKE, 0, None) == -4
     assert lib.fp4_quantize(FAKE, 4, 64, 64, 2, 16, 1, 0, 0, None, None, FAKE, FAKE, 0, None) == -1

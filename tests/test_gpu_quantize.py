@@ -84,6 +84,47 @@ def test_sr_deterministic_and_seeded():
     assert not torch.equal(a.codes, c.codes)
 
 
+SHARD_CASES = [(1, (300, 384), [0, 1, 150, 299, 300]), (1, (2048, 4096), [0, 16, 1000, 2048]),
+               (0, (512, 200), [0, 64, 320, 512]), (0, (4096, 1024), [0, 2048, 4096])]
+
+
+@pytest.mark.parametrize("rnd", ["rtn", "sr"])
+@pytest.mark.parametrize("fmt", ["mxfp4", "nvfp4"])
+@pytest.mark.parametrize("axis, shape, cuts", SHARD_CASES)
+def test_row_shards_reproduce_the_whole(axis, shape, cuts, fmt, rnd):
+    """fp4_quantize_shard on each row shard (NVFP4 under the whole tensor's scale) gives the whole
+    tensor's codes and scales bit for bit; each shard also matches the oracle with its index base."""
+    rows, cols = shape
+    xb = mixed_input(rows, cols, rows + 3 * cols, fmt)
+    x = dev_bf16(xb)
+    whole = F.fp4_quantize(x, fmt=fmt, axis=axis, rnd=rnd, seed=0x5EED)
+    ts = whole.tensor_scale
+    for a, b in zip(cuts, cuts[1:]):
+        part = F.fp4_quantize(x[a:b], fmt=fmt, axis=axis, rnd=rnd, seed=0x5EED, tensor_scale_in=ts, first_row=a)
+        bs = 32 if fmt == "mxfp4" else 16
+        if axis == 1:
+            assert torch.equal(part.codes, whole.codes[a:b]) and torch.equal(part.scales, whole.scales[a:b])
+        else:
+            assert torch.equal(part.codes, whole.codes[:, a // 2:b // 2])
+            assert torch.equal(part.scales, whole.scales[:, a // bs:b // bs])
+    a, b = cuts[1], cuts[2]
+    s_t = None if ts is None else host_f32(ts)[0]
+    ref = O.quantize(np.ascontiguousarray(xb[a:b]), fmt=fmt, axis=axis, rnd=rnd, seed=0x5EED, tensor_scale=s_t,
+                     idx_base=a * cols)
+    part = F.fp4_quantize(x[a:b], fmt=fmt, axis=axis, rnd=rnd, seed=0x5EED, tensor_scale_in=ts, first_row=a)
+    _check_against_oracle(part, ref, fmt, axis, b - a, cols, "rowmajor")
+
+
+@pytest.mark.parametrize("fmt", ["mxfp4", "nvfp4"])
+def test_row_shard_far_into_a_tensor(fmt):
+    """A shard 2^24 rows into a 4096-column tensor: Philox counters above 2^32 (the high word)."""
+    xb = mixed_input(64, 4096, 17, fmt)
+    first = 1 << 24
+    q = F.fp4_quantize(dev_bf16(xb), fmt=fmt, rnd="sr", seed=99, first_row=first)
+    ref = O.quantize(xb, fmt=fmt, rnd="sr", seed=99, idx_base=first * 4096)
+    _check_against_oracle(q, ref, fmt, 1, 64, 4096, "rowmajor")
+
+
 def test_zero_tensor_nv():
     x = torch.zeros((16, 64), dtype=torch.bfloat16, device="cuda")
     q = F.fp4_quantize(x, fmt="nvfp4")

@@ -178,6 +178,30 @@ def test_sr_uses_input_index_for_axis0():
     np.testing.assert_array_equal(codes_of(r0), want)
 
 
+@pytest.mark.parametrize("axis", [0, 1])
+@pytest.mark.parametrize("fmt", ["mxfp4", "nvfp4"])
+def test_sr_row_shards_with_index_base_reproduce_the_whole(fmt, axis):
+    """A row shard quantized with idx_base = first_row * cols (and the whole tensor's s_t) draws the
+    whole tensor's Philox words, so the shards' codes and scales are the whole's, piece by piece."""
+    rng = np.random.default_rng(3)
+    x = bf16_to_f32(bf16_bits((rng.standard_t(3, size=(96, 64)) * 0.1).astype(np.float32)))
+    whole = O.quantize_values(x, fmt=fmt, axis=axis, rnd="sr", seed=5)
+    ts = whole["tensor_scale"]
+    cuts = [0, 32, 64, 96]
+    for a, b in zip(cuts, cuts[1:]):
+        part = O.quantize_values(x[a:b], fmt=fmt, axis=axis, rnd="sr", seed=5, tensor_scale=ts, idx_base=a * 64)
+        local = O.quantize_values(x[a:b], fmt=fmt, axis=axis, rnd="sr", seed=5, tensor_scale=ts)
+        if axis == 1:
+            np.testing.assert_array_equal(part["codes"], whole["codes"][a:b])
+            np.testing.assert_array_equal(part["scales"], whole["scales"][a:b])
+        else:
+            bs = 32 if fmt == "mxfp4" else 16
+            np.testing.assert_array_equal(part["codes"], whole["codes"][:, a // 2:b // 2])
+            np.testing.assert_array_equal(part["scales"], whole["scales"][:, a // bs:b // bs])
+        if a:
+            assert not np.array_equal(part["codes"], local["codes"])    # the index base matters
+
+
 @pytest.mark.parametrize("fmt", ["mxfp4", "nvfp4"])
 def test_axis0_is_axis1_of_transpose_rtn(fmt):
     rng = np.random.default_rng(2)
