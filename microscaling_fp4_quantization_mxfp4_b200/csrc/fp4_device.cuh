@@ -351,6 +351,35 @@ __device__ __forceinline__ void nv_divide_block(const float (&x)[E], float am, f
   }
 }
 
+// Round-to-nearest quotients of one NVFP4 block on packed fp32 pairs: div_by_recip's reciprocal
+// and two corrections, each pair instruction doing two elements (5 pair instructions for two
+// quotients, against 3 conversions and fp64 multiplies per quotient through div_by_recip64, 2 of
+// them conversions).  The residual is formed as S*q - x and its product with y subtracted, the
+// same values as div_by_recip's -(S*q - x) added (the sign of a zero dividend survives).  Under
+// nv_fast_division's round-to-nearest test (which has no per-element part) the codes are those of
+// IEEE division; blocks that fail it take __fdiv_rn.  sy = (S, RN(1/S)).
+template <int E>
+__device__ __forceinline__ void nv_divide_block_rtn2(float (&x)[E], float am, float2 sy) {
+  if (nv_fast_division<0, E>(x, am, sy.x, sy.y)) {
+    const float2 S2 = make_float2(sy.x, sy.x), y2 = make_float2(sy.y, sy.y), ny2 = make_float2(-sy.y, -sy.y);
+#pragma unroll
+    for (int i = 0; i < E / 2; ++i) {
+      const float2 xv = make_float2(x[2 * i], x[2 * i + 1]);
+      const float2 nx = make_float2(-xv.x, -xv.y);
+      float2 q = __fmul2_rn(xv, y2);
+      float2 t = __ffma2_rn(q, S2, nx);
+      q = __ffma2_rn(t, ny2, q);
+      t = __ffma2_rn(q, S2, nx);
+      q = __ffma2_rn(t, ny2, q);
+      x[2 * i] = q.x;
+      x[2 * i + 1] = q.y;
+    }
+  } else {                                       // rare: tiny or huge scales
+#pragma unroll
+    for (int i = 0; i < E; ++i) x[i] = __fdiv_rn(x[i], sy.x);
+  }
+}
+
 // Round-to-nearest dequantization of two quotients: fp32(fp32(G[c] * sbv) * s_t) for each, where
 // c is the E2M1 code of the quotient and g holds the block scale sbv in both halves.  G[c] * sbv
 // has at most 6 significant bits and lies in [2^-10, 2688], so the f16 product is exact.
@@ -360,7 +389,7 @@ __device__ __forceinline__ float2 nv_rtn_dequant2(float q0, float q1, __half2 g,
       : "=r"(h)
       : "f"(q0), "f"(q1));
   const float2 v = __half22float2(__hmul2(*reinterpret_cast<const __half2*>(&h), g));
-  return make_float2(__fmul_rn(v.x, s_t), __fmul_rn(v.y, s_t));
+  return __fmul2_rn(v, make_float2(s_t, s_t));
 }
 
 // -------------------------------------------------- scale-factor offsets ----
@@ -371,36 +400,88 @@ __device__ __forceinline__ long long sf_mma_offset(long long row, long long g, l
 }
 
 // ------------------------------------------------------ Hadamard (fp32) -----
-// In-register fast Walsh-Hadamard transform of a contiguous block of HB
-// elements held 8 per lane by HB/8 consecutive lanes (Sylvester order:
-// pairs (i, i + 2^s) -> (a + b, a - b)), then scaled by 1/sqrt(HB).
+// The butterflies run on packed fp32 pairs (the f32x2 add / multiply-add /
+// multiply of sm_100): each half of a pair operation is the IEEE fp32 operation
+// of that half alone, so a pair gives the values of the two scalar operations
+// it replaces in one instruction.  A thread's E values sit in E/2 pairs
+// (x[p], x[p + E/2]); a stage at a distance below E/2 combines two pairs, the
+// stage at distance E/2 the two halves of each pair.
+__device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
+__device__ __forceinline__ float2 splat2(float v) { return make_float2(v, v); }
+
 template <int HB>
-__device__ __forceinline__ void hadamard_rotate(float (&x)[8], int lane) {
+__device__ __forceinline__ float hadamard_norm() {
+  return HB == 16 ? 0.25f : HB == 32 ? 0.17677669529663687f : HB == 64 ? 0.125f : 0.08838834764831845f;
+}
+
+// One butterfly stage at distance d inside a thread's pairs P[E/2] (element e is
+// P[e % H].x for e < H, P[e - H].y otherwise, H = E/2): (a, b) -> (a + b, a - b),
+// or with a sign sg (chunk order, see hadamard_rotate_block) -> (a*sg + b, b*(-sg) + a).
+template <int E, bool SIGNED>
+__device__ __forceinline__ void butterfly_stage(float2 (&P)[E / 2], int d, float sg) {
+  constexpr int H = E / 2;
+  if (d < H) {
+    const float2 s2 = splat2(SIGNED ? sg : 1.0f), m2 = splat2(SIGNED ? -sg : -1.0f);
 #pragma unroll
-  for (int d = 1; d < 8; d <<= 1) {
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      if ((i & d) == 0) {
-        const float a = x[i], b = x[i + d];
-        x[i] = __fadd_rn(a, b);
-        x[i + d] = __fsub_rn(a, b);
+    for (int p = 0; p < H; ++p) {
+      if ((p & d) == 0) {
+        const float2 a = P[p], b = P[p + d];
+        P[p] = SIGNED ? fma2(a, s2, b) : add2(a, b);
+        P[p + d] = fma2(b, m2, a);                   // a - b: one rounding, as the subtraction
       }
     }
-  }
+  } else {
 #pragma unroll
-  for (int ld = 1; ld < HB / 8; ld <<= 1) {
-    // upper lanes take p - x, lower ones x + p: one multiply-add by -1 or +1 (exact negation,
-    // a single rounding, so the same value as the subtraction or addition)
-    const float sgn = (lane & ld) != 0 ? -1.0f : 1.0f;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const float p = __shfl_xor_sync(0xFFFFFFFFu, x[i], ld);
-      x[i] = __fmaf_rn(x[i], sgn, p);
+    for (int p = 0; p < H; ++p) {
+      const float a = P[p].x, b = P[p].y;
+      P[p].x = SIGNED ? __fmaf_rn(a, sg, b) : __fadd_rn(a, b);
+      P[p].y = SIGNED ? __fmaf_rn(b, -sg, a) : __fsub_rn(a, b);
     }
   }
-  const float s = HB == 16 ? 0.25f : HB == 32 ? 0.17677669529663687f : HB == 64 ? 0.125f : 0.08838834764831845f;
+}
+
+// A stage across lanes at lane distance ld: every element takes x * sgn + p,
+// p the partner lane's element at register position e ^ flip (upper lanes
+// p - x, lower ones x + p: a multiply-add by -1 or +1, exact negation, a single
+// rounding, so the same value as the subtraction or addition).
+template <int E>
+__device__ __forceinline__ void butterfly_lanes(float2 (&P)[E / 2], int lane, int ld, int flip) {
+  constexpr int H = E / 2;
+  const float2 s2 = splat2((lane & ld) != 0 ? -1.0f : 1.0f);
+  float2 Q[H];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) x[i] = __fmul_rn(x[i], s);
+  for (int p = 0; p < H; ++p) {
+    const int e0 = p ^ flip, e1 = (p + H) ^ flip;
+    const float v0 = e0 < H ? P[e0].x : P[e0 - H].y;
+    const float v1 = e1 < H ? P[e1].x : P[e1 - H].y;
+    Q[p] = make_float2(__shfl_xor_sync(0xFFFFFFFFu, v0, ld), __shfl_xor_sync(0xFFFFFFFFu, v1, ld));
+  }
+#pragma unroll
+  for (int p = 0; p < H; ++p) P[p] = fma2(P[p], s2, Q[p]);
+}
+
+// In-register fast Walsh-Hadamard transform of a contiguous block of HB
+// elements held 8 per lane by HB/8 consecutive lanes (Sylvester order:
+// pairs (i, i + 2^s) -> (a + b, a - b), distances 1, 2, 4, ... in turn), then
+// scaled by 1/sqrt(HB).
+template <int HB>
+__device__ __forceinline__ void hadamard_rotate(float (&x)[8], int lane) {
+  float2 P[4];
+#pragma unroll
+  for (int p = 0; p < 4; ++p) P[p] = make_float2(x[p], x[p + 4]);
+#pragma unroll
+  for (int d = 1; d < 8; d <<= 1) butterfly_stage<8, false>(P, d, 1.0f);
+#pragma unroll
+  for (int ld = 1; ld < HB / 8; ld <<= 1) butterfly_lanes<8>(P, lane, ld, 0);
+  const float2 s2 = splat2(hadamard_norm<HB>());
+#pragma unroll
+  for (int p = 0; p < 4; ++p) {
+    P[p] = mul2(P[p], s2);
+    x[p] = P[p].x;
+    x[p + 4] = P[p].y;
+  }
 }
 
 // Same transform with one thread holding E consecutive elements (E = 16 or
@@ -420,57 +501,27 @@ __device__ __forceinline__ void hadamard_rotate(float (&x)[8], int lane) {
 // exchanges the register of the flipped chunk, chosen at compile time.
 template <int HB, int E, int SWS = 0, int SWM = 0>
 __device__ __forceinline__ void hadamard_rotate_block(float (&x)[E], int lane, uint32_t sw = 0u) {
-  constexpr int IN = HB < E ? HB : E;
+  constexpr int IN = HB < E ? HB : E, H = E / 2;
+  float2 P[H];
+#pragma unroll
+  for (int p = 0; p < H; ++p) P[p] = make_float2(x[p], x[p + H]);
 #pragma unroll
   for (int d = 1; d < IN; d <<= 1) {
     if (d < 8 || SWM == 0) {
-#pragma unroll
-      for (int i = 0; i < E; ++i) {
-        if ((i & d) == 0) {
-          const float a = x[i], b = x[i + d];
-          x[i] = __fadd_rn(a, b);
-          x[i + d] = __fsub_rn(a, b);
-        }
-      }
+      butterfly_stage<E, false>(P, d, 1.0f);
     } else {
-      const float sg = ((sw >> (d == 8 ? 0 : 1)) & 1u) != 0u ? -1.0f : 1.0f;
-#pragma unroll
-      for (int i = 0; i < E; ++i) {
-        if ((i & d) == 0) {
-          const float a = x[i], b = x[i + d];
-          x[i] = __fmaf_rn(a, sg, b);
-          x[i + d] = __fmaf_rn(b, -sg, a);
-        }
-      }
+      butterfly_stage<E, true>(P, d, ((sw >> (d == 8 ? 0 : 1)) & 1u) != 0u ? -1.0f : 1.0f);
     }
   }
 #pragma unroll
-  for (int ld = 1; ld < HB / E; ld <<= 1) {
-    const float sgn = (lane & ld) != 0 ? -1.0f : 1.0f;     // p - x or x + p, as in hadamard_rotate
-    const int flip = ((ld >> SWS) & SWM) << 3;             // chunk bits by which the partner's order differs
-    if (flip == 0) {
+  for (int ld = 1; ld < HB / E; ld <<= 1) butterfly_lanes<E>(P, lane, ld, ((ld >> SWS) & SWM) << 3);
+  const float2 s2 = splat2(hadamard_norm<HB>());
 #pragma unroll
-      for (int i = 0; i < E; ++i) {
-        const float p = __shfl_xor_sync(0xFFFFFFFFu, x[i], ld);
-        x[i] = __fmaf_rn(x[i], sgn, p);
-      }
-    } else {
-#pragma unroll
-      for (int i = 0; i < E; ++i) {
-        if ((i & flip) == 0) {
-          const int j = i ^ flip;
-          const float a = x[i], b = x[j];
-          const float pa = __shfl_xor_sync(0xFFFFFFFFu, b, ld);   // the partner's element at i's position
-          const float pb = __shfl_xor_sync(0xFFFFFFFFu, a, ld);   // and at j's
-          x[i] = __fmaf_rn(a, sgn, pa);
-          x[j] = __fmaf_rn(b, sgn, pb);
-        }
-      }
-    }
+  for (int p = 0; p < H; ++p) {
+    P[p] = mul2(P[p], s2);
+    x[p] = P[p].x;
+    x[p + H] = P[p].y;
   }
-  const float s = HB == 16 ? 0.25f : HB == 32 ? 0.17677669529663687f : HB == 64 ? 0.125f : 0.08838834764831845f;
-#pragma unroll
-  for (int i = 0; i < E; ++i) x[i] = __fmul_rn(x[i], s);
 }
 
 // ------------------------------------------- bulk copies and mbarriers -----

@@ -189,15 +189,28 @@ __device__ __forceinline__ void sf_pad_zero(const QRowParams& p, uint32_t t, uin
 struct NvConsts {
   float s_t;
   double yd_st;          // RN64(1 / s_t)
-  const double* tabd;    // RN64(1 / S) for every E4M3 byte
+  const double* tabd;    // per E4M3 byte: RN64(1 / S), or (S, RN32(1 / S)) as a float2 (PAIRS)
 };
 
-// The per-CTA NVFP4 constants under tensor scale s_t: fills the reciprocal table (every thread of
-// the CTA takes part; visible after the caller's next __syncthreads).
+// The per-CTA NVFP4 constants under tensor scale s_t: fills the 1 KB divisor table (every thread
+// of the CTA takes part; visible after the caller's next __syncthreads).  PAIRS: the table holds
+// (S, RN32(1 / S)) pairs for nv_divide_block_rtn2 (round-to-nearest NVFP4 blocks in quantize_block,
+// measured faster: 28.8 -> 27.7 us for the single-pass 4096^2 quantize + dequantize), else the
+// fp64 reciprocals of div_by_recip64 (stochastic rounding, which needs every quotient exact without
+// a per-element range test, four-over-six, axis-0 and 2-D blocks).
+template <bool PAIRS = false>
 __device__ __forceinline__ NvConsts nv_consts(float s_t, double* tabd) {
-  nv_fill_recip64_table(tabd, s_t);
+  if (PAIRS) {
+    nv_fill_scale_table(reinterpret_cast<float2*>(tabd), s_t);
+  } else {
+    nv_fill_recip64_table(tabd, s_t);
+  }
   return NvConsts{s_t, __drcp_rn((double)s_t), tabd};
 }
+
+// Whether quantize_block divides with the pair table (see nv_consts).
+template <int FMT, int RND>
+constexpr bool kNvPairs = FMT == FMT_NV && RND == RND_RTN;
 
 // One thread quantizes one whole scale block of E = 32 (MX) or 16 (NV)
 // elements held as E/8 uint4: the block maximum, the scale and every division
@@ -304,8 +317,9 @@ __device__ __forceinline__ void dequant_block_out(const QRowParams& p, const uin
     for (int i = 0; i < 4; ++i) {
       const __half2 hv = *reinterpret_cast<const __half2*>(&h[i]);
       const float2 g = __half22float2(FMT == FMT_MX ? hv : __hmul2(hv, sb));
-      y[8 * k + 2 * i] = __fmul_rn(g.x, sc);
-      y[8 * k + 2 * i + 1] = __fmul_rn(g.y, sc);
+      const float2 r = mul2(g, splat2(sc));
+      y[8 * k + 2 * i] = r.x;
+      y[8 * k + 2 * i + 1] = r.y;
     }
   }
   // 32-byte stores (one whole L2 sector per lane) when the output base allows them: a block's
@@ -387,16 +401,24 @@ __device__ __forceinline__ void quantize_block(const QRowParams& p, const uint4 
   bool zero;
   if (FMT == FMT_MX) {
     byte = mx_scale_byte_clip(am, p.mx_thr);
-    const float inv = mx_inv_scale(byte);
+    const float2 inv = splat2(mx_inv_scale(byte));
 #pragma unroll
-    for (int i = 0; i < E; ++i) x[i] = __fmul_rn(x[i], inv);          // exact power-of-two scaling
+    for (int i = 0; i < E / 2; ++i) {                                   // exact power-of-two scaling
+      const float2 t = mul2(make_float2(x[i], x[i + E / 2]), inv);
+      x[i] = t.x;
+      x[i + E / 2] = t.y;
+    }
     zero = (am == 0.0f);
   } else {
     byte = e4m3_rn_sat(nv_scale_arg64(am, nv.s_t, nv.yd_st));
     if (FMT == FMT_NV46) {
       byte = nv_four_over_six<RND, E>(x, am, byte, nv);
     } else {
-      nv_divide_block64<E>(x, nv.tabd[byte], x);
+      if (kNvPairs<FMT, RND>) {
+        nv_divide_block_rtn2<E>(x, am, reinterpret_cast<const float2*>(nv.tabd)[byte]);
+      } else {
+        nv_divide_block64<E>(x, nv.tabd[byte], x);
+      }
     }
     zero = (byte == 0u);
   }
@@ -467,7 +489,7 @@ __global__ void __launch_bounds__(256) quantize_rows_kernel(QRowParams p) {
   if (SFMMA) sf_pad_zero(p, blockIdx.x * blockDim.x + threadIdx.x, gridDim.x * blockDim.x);
   NvConsts nv{1.0f, 1.0, tabd};
   if (FMT != FMT_MX) {
-    nv = nv_consts(*p.ts, tabd);
+    nv = nv_consts<kNvPairs<FMT, RND>>(*p.ts, tabd);
     if (p.ts_copy_out != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *p.ts_copy_out = nv.s_t;
     __syncthreads();
   }
@@ -501,7 +523,8 @@ constexpr int kStreamSmem = kStreamStages * kStreamChunks * 16 + 2 * kStreamStag
 // Consumer warps per CTA (measured): 31 for NVFP4 and the amax (with the
 // producer, the 1024-thread maximum, so at most 64 registers a thread, which
 // their 16-element blocks fit); 16 for MXFP4 round-to-nearest, with or
-// without rotation (31 warps ran 10-20 % slower); 15 for MXFP4 stochastic
+// without rotation (31 warps ran 10-20 % slower, 19 warps at the same 96
+// registers 5-6 % slower); 15 for MXFP4 stochastic
 // rounding, whose 32-element blocks with their eight Philox blocks want about
 // 124 registers; 15 for four-over-six NVFP4, whose second candidate scale and
 // fp64 error sums do not fit in 64 registers.  Units of a stage are dealt to
@@ -592,7 +615,7 @@ __global__ void __launch_bounds__(StreamWarps<FMT, RND>::kThreads, 1) quantize_s
   if (SFMMA) sf_pad_zero(p, blockIdx.x * blockDim.x + threadIdx.x, gridDim.x * blockDim.x);
   NvConsts nv{1.0f, 1.0, tabd};
   if (FMT != FMT_MX) {
-    nv = nv_consts(*p.ts, tabd);
+    nv = nv_consts<kNvPairs<FMT, RND>>(*p.ts, tabd);
     if (p.ts_copy_out != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *p.ts_copy_out = nv.s_t;
   }
   __syncthreads();
@@ -835,7 +858,7 @@ __global__ void __launch_bounds__(FusedWarps<FMT>::kThreads, 1) nv_quantize_fuse
     }
   }
   __syncthreads();
-  const NvConsts nv = nv_consts(s_t_shared, tabd);
+  const NvConsts nv = nv_consts<kNvPairs<FMT, RND>>(s_t_shared, tabd);
   __syncthreads();
   if (warp == 0) return;
 
@@ -1300,16 +1323,18 @@ __device__ __forceinline__ void dequantize_chunk_to(const DeqParams& p, uint32_t
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       const float2 g = __half22float2(*reinterpret_cast<const __half2*>(&h[k]));
-      y[2 * k] = __fmul_rn(g.x, sc);
-      y[2 * k + 1] = __fmul_rn(g.y, sc);
+      const float2 r = mul2(g, splat2(sc));
+      y[2 * k] = r.x;
+      y[2 * k + 1] = r.y;
     }
   } else {
     const __half2 sb = __float2half2_rn(e4m3_value(byte));
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       const float2 g = __half22float2(__hmul2(*reinterpret_cast<const __half2*>(&h[k]), sb));
-      y[2 * k] = __fmul_rn(g.x, s_t);
-      y[2 * k + 1] = __fmul_rn(g.y, s_t);
+      const float2 r = mul2(g, splat2(s_t));
+      y[2 * k] = r.x;
+      y[2 * k + 1] = r.y;
     }
   }
   if (BF16) {
@@ -1367,8 +1392,9 @@ __global__ void __launch_bounds__(256) dequantize_direct_kernel(DeqParams p) {
       for (int k = 0; k < 4; ++k) {
         const __half2 hv = *reinterpret_cast<const __half2*>(&h[k]);
         const float2 g = __half22float2(FMT == FMT_MX ? hv : __hmul2(hv, sb));
-        y[2 * k] = __fmul_rn(g.x, sc);
-        y[2 * k + 1] = __fmul_rn(g.y, sc);
+        const float2 r = mul2(g, splat2(sc));
+        y[2 * k] = r.x;
+        y[2 * k + 1] = r.y;
       }
       if (BF16) {
         uint32_t o[4];

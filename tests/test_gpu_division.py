@@ -1,6 +1,8 @@
 """GPU: the NVFP4 quantizer's scale division x / S (correctly rounded reciprocal
 plus two FMA corrections, IEEE fallback for tiny operands) is bit-identical to
-CUDA's IEEE division for every finite bf16 x over thousands of divisors S."""
+CUDA's IEEE division for every finite bf16 x over thousands of divisors S, and
+the packed-pair block form used for round-to-nearest gives IEEE quotients
+(tiny dividends: the same E2M1 codes) on blocks of every bf16 pattern."""
 import ctypes
 import os
 import subprocess
@@ -24,6 +26,7 @@ def checker(tmp_path_factory):
     subprocess.run(cmd, check=True, capture_output=True)
     lib = ctypes.CDLL(str(out))
     lib.div_check.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p]
+    lib.div_check_rtn2.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_uint, ctypes.c_void_p, ctypes.c_void_p]
     return lib
 
 
@@ -50,3 +53,17 @@ def test_scale_division_matches_ieee(checker):
     assert bad.item() == 0, f"{bad.item()} of {total} quotients differ from IEEE division"
     # the fallback is only for tiny operands and extreme scales; most quotients take the fast path
     assert slow.item() < 0.7 * total
+
+
+@pytest.mark.parametrize("stride", [1, 4099, 40961])
+def test_block_pair_division_rtn_matches_ieee(checker, stride):
+    S = torch.from_numpy(_divisors()).cuda()
+    bad = torch.zeros(1, dtype=torch.int64, device="cuda")
+    slow = torch.zeros(1, dtype=torch.int64, device="cuda")
+    for i in range(0, S.numel(), 1024):
+        chunk = S[i:i + 1024].contiguous()
+        assert checker.div_check_rtn2(chunk.data_ptr(), chunk.numel(), stride, bad.data_ptr(), slow.data_ptr()) == 0
+    assert bad.item() == 0, f"{bad.item()} block quotients differ from IEEE division"
+    # neighbouring patterns mostly take the fast path; mixed blocks hold huge elements whose
+    # quotients could overflow the corrections, so most of them fall back, but not all
+    assert slow.item() < (0.7 if stride == 1 else 0.99) * S.numel() * 4096
