@@ -11,7 +11,7 @@ import sys
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
-SOURCES = ["api.cu", "quantize.cu", "mse.cu", "gemm.cu", "noalloc.cu"]
+SOURCES = ["api.cu", "quantize.cu", "mse.cu", "gemm.cu", "gemv.cu", "noalloc.cu"]
 HEADERS = ["fp4_device.cuh", "fp4_internal.h"]
 LIB = os.path.join(PKG, "libfp4.so")
 OBJDIR = os.path.join(ROOT, "_build")

@@ -24,6 +24,20 @@ __device__ __forceinline__ void unpack8(const uint4& v, float (&x)[8]) {
 }
 
 // ------------------------------------------------------------ E2M1 codes ---
+// Eight E2M1 codes (element i in nibble i of w) -> their values as four f16 pairs, element 2k in
+// the low half of h[k].
+__device__ __forceinline__ void e2m1x8_to_f16x2(uint32_t w, uint32_t (&h)[4]) {
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+      : "=r"(h[0]), "=r"(h[1]), "=r"(h[2]), "=r"(h[3])
+      : "r"(w));
+}
+
+
 // Hardware conversion: round to nearest even, saturating to +-6, sign kept.
 // Element `a` lands in the low nibble, `b` in the high nibble.
 __device__ __forceinline__ uint32_t e2m1x4_rn(float a0, float b0, float a1, float b1,

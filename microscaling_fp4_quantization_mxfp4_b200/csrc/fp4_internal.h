@@ -152,4 +152,13 @@ struct GemmParams {
 // Returns cudaErrorNotSupported if the driver entry point for tensor maps is missing.
 cudaError_t launch_gemm(const GemmParams& p, int num_sms, cudaStream_t st);
 
+// CUDA-core GEMM for at most kGemvMaxM activation rows (gemv.cu): taken by launch_gemm when
+// gemv_applies (plain Y output, the converted activations fit kGemvMaxSmem of shared memory).
+// One row: measured faster than the tensor-core swap-AB kernel for every Llama-7B shape (NVFP4
+// 4096 x 4096: 7.0 -> 5.0 us, MXFP4 6.6 -> 4.1 us); two or more rows were not.
+constexpr int64_t kGemvMaxM = 1;
+constexpr size_t kGemvMaxSmem = 160 * 1024;
+bool gemv_applies(const GemmParams& p);
+cudaError_t launch_gemv(const GemmParams& p, int num_sms, cudaStream_t st);
+
 }  // namespace fp4lib

@@ -2134,6 +2134,8 @@ cudaError_t launch_gemm(const GemmParams& p, int num_sms, cudaStream_t st) {
   if (p.q_out != 0)
     return p.q_out == 1 ? dispatch_quant<1>(p, pair_tiles, bn, num_sms, st)
                         : dispatch_quant<2>(p, pair_tiles, bn, num_sms, st);
+  // at most kGemvMaxM activation rows: the weights stream through the CUDA cores (gemv.cu)
+  if (gemv_applies(p)) return launch_gemv(p, num_sms, st);
   const int64_t wtiles = (p.N + 127) / 128, nkb_s = (p.K + BK - 1) / BK;
   if (p.M <= 128 && 2 * wtiles <= num_sms && nkb_s >= 2) {
     // at most 128 activation rows and at most half as many 128-row weight tiles as SMs: swap-AB

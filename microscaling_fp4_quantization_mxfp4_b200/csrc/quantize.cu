@@ -1296,19 +1296,6 @@ __device__ __forceinline__ const uint8_t* deq_scale_ptr(const DeqParams& p, uint
   return p.scales + chunk / LPB;
 }
 
-// Eight E2M1 codes (element i in nibble i of w) -> their values as four f16 pairs, element 2k in
-// the low half of h[k].
-__device__ __forceinline__ void e2m1x8_to_f16x2(uint32_t w, uint32_t (&h)[4]) {
-  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
-      "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
-      "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
-      "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
-      "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
-      "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
-      : "=r"(h[0]), "=r"(h[1]), "=r"(h[2]), "=r"(h[3])
-      : "r"(w));
-}
-
 // One chunk of 8 codes to fp32 (or bf16) values.  NV: fp32(fp32(G[c] * sb) * s_t), where the
 // product G[c] * sb (at most 6 significant bits, in [2^-10, 2688] or zero) is exact in f16.
 // MX: G[c] * 2^E in fp32.

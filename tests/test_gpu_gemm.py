@@ -7,7 +7,7 @@ import torch
 
 import oracle as O
 import microscaling_fp4_quantization_mxfp4_b200 as F
-from gpu_utils import dev_bf16, host_f32, host_u8
+from gpu_utils import dev_bf16, host_f32, host_u8, mixed_input
 from workloads import (bf16_to_f32, hadamard_acts, hadamard_weights, llama_acts, llama_weights,
                        mx_linear_128x512, vit_layer, normal_bf16)
 
@@ -78,7 +78,7 @@ def test_gemm_shapes(mnk, fmt):
     F.fp4_check_device_errors()
 
 
-SMALL_M = [1, 3, 16, 17, 32, 33, 64, 65, 127, 128]
+SMALL_M = [1, 2, 3, 4, 5, 16, 17, 32, 33, 64, 65, 127, 128]
 SMALL_NK = [(128, 4096), (300, 320), (4100, 1024)]
 
 
@@ -109,6 +109,35 @@ def test_gemm_small_m_weight_streaming(M, nk, fmt):
     out = host_f32(big)
     np.testing.assert_array_equal(out[:, :N].view(np.uint32), got.view(np.uint32))
     assert np.all(out[:, N:] == 7.0)            # nothing written past N
+    F.fp4_check_device_errors()
+
+
+@pytest.mark.parametrize("fmt", ["mxfp4", "nvfp4"])
+@pytest.mark.parametrize("M, N, K", [(1, 4096, 4096), (1, 11008, 4096), (1, 4096, 11008), (1, 1000, 11008),
+                                     (1, 77, 64), (1, 1, 128)])
+def test_gemm_cuda_core_rows(M, N, K, fmt):
+    """One activation row runs on the CUDA cores (exact f16 block sums, fp32 across blocks): the
+    Llama-7B decode shapes, a ragged N, the shortest K, a single output; a heavy-tailed activation
+    row with a zero block; fp32 against the fp64 oracle (sampled columns for the large N), bf16
+    within one ulp, and a strided output."""
+    g = np.random.default_rng(M * 7 + N + K)
+    from workloads import bf16_bits
+    a = mixed_input(M, K, M + K, fmt)
+    b = bf16_bits((g.standard_t(4, (N, K)) * 0.02).astype(np.float32))
+    qa, qb = _gpu_quant(dev_bf16(a), fmt), _gpu_quant(dev_bf16(b), fmt)
+    kw = dict(fmt=fmt, a_tensor_scale=qa.tensor_scale, b_tensor_scale=qb.tensor_scale)
+    y32 = F.fp4_gemm(qa.codes, qa.scales, qb.codes, qb.scales, out_dtype="f32", **kw)
+    y16 = F.fp4_gemm(qa.codes, qa.scales, qb.codes, qb.scales, out_dtype="bf16", **kw)
+    big = torch.full((M, N + 20), 7.0, dtype=torch.float32, device="cuda")
+    F.fp4_gemm(qa.codes, qa.scales, qb.codes, qb.scales, out_dtype="f32", out=big[:, :N], **kw)
+    rows = np.arange(N) if N <= 1000 else np.sort(np.random.default_rng(1).choice(N, 1000, replace=False))
+    yr, bd = O.gemm_ref_cols(_as_oracle(qa, fmt, M, K), _as_oracle(qb, fmt, N, K), fmt, rows)
+    got = host_f32(y32)
+    _check(got[:, rows], yr, bd)
+    _bf16_ulp_check(y16, got)
+    out = host_f32(big)
+    np.testing.assert_array_equal(out[:, :N].view(np.uint32), got.view(np.uint32))
+    assert np.all(out[:, N:] == 7.0)
     F.fp4_check_device_errors()
 
 
