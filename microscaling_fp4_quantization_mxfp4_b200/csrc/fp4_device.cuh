@@ -365,16 +365,17 @@ __device__ __forceinline__ void nv_divide_block(const float (&x)[E], float am, f
   }
 }
 
-// Round-to-nearest quotients of one NVFP4 block on packed fp32 pairs: div_by_recip's reciprocal
-// and two corrections, each pair instruction doing two elements (5 pair instructions for two
-// quotients, against 3 conversions and fp64 multiplies per quotient through div_by_recip64, 2 of
-// them conversions).  The residual is formed as S*q - x and its product with y subtracted, the
-// same values as div_by_recip's -(S*q - x) added (the sign of a zero dividend survives).  Under
-// nv_fast_division's round-to-nearest test (which has no per-element part) the codes are those of
-// IEEE division; blocks that fail it take __fdiv_rn.  sy = (S, RN(1/S)).
-template <int E>
-__device__ __forceinline__ void nv_divide_block_rtn2(float (&x)[E], float am, float2 sy) {
-  if (nv_fast_division<0, E>(x, am, sy.x, sy.y)) {
+// Quotients of one NVFP4 block on packed fp32 pairs: div_by_recip's reciprocal and two
+// corrections, each pair instruction doing two elements (5 pair instructions for two quotients,
+// against 3 conversions and fp64 multiplies per quotient through div_by_recip64, 2 of them
+// conversions).  The residual is formed as S*q - x and its product with y subtracted, the same
+// values as div_by_recip's -(S*q - x) added (the sign of a zero dividend survives).  Under
+// nv_fast_division's test for the rounding RND (round-to-nearest: per block only; stochastic
+// rounding: also every |x| >= 2^-103) the quotients are those of IEEE division (tiny dividends
+// under round-to-nearest: the same codes); blocks that fail it take __fdiv_rn.  sy = (S, RN(1/S)).
+template <int RND, int E>
+__device__ __forceinline__ void nv_divide_block2(float (&x)[E], float am, float2 sy) {
+  if (nv_fast_division<RND, E>(x, am, sy.x, sy.y)) {
     const float2 S2 = make_float2(sy.x, sy.x), y2 = make_float2(sy.y, sy.y), ny2 = make_float2(-sy.y, -sy.y);
 #pragma unroll
     for (int i = 0; i < E / 2; ++i) {

@@ -194,10 +194,7 @@ struct NvConsts {
 
 // The per-CTA NVFP4 constants under tensor scale s_t: fills the 1 KB divisor table (every thread
 // of the CTA takes part; visible after the caller's next __syncthreads).  PAIRS: the table holds
-// (S, RN32(1 / S)) pairs for nv_divide_block_rtn2 (round-to-nearest NVFP4 blocks in quantize_block,
-// measured faster: 28.8 -> 27.7 us for the single-pass 4096^2 quantize + dequantize), else the
-// fp64 reciprocals of div_by_recip64 (stochastic rounding, which needs every quotient exact without
-// a per-element range test, four-over-six, axis-0 and 2-D blocks).
+// (S, RN32(1 / S)) pairs for nv_divide_block2, else the fp64 reciprocals of div_by_recip64.
 template <bool PAIRS = false>
 __device__ __forceinline__ NvConsts nv_consts(float s_t, double* tabd) {
   if (PAIRS) {
@@ -208,9 +205,13 @@ __device__ __forceinline__ NvConsts nv_consts(float s_t, double* tabd) {
   return NvConsts{s_t, __drcp_rn((double)s_t), tabd};
 }
 
-// Whether quantize_block divides with the pair table (see nv_consts).
-template <int FMT, int RND>
-constexpr bool kNvPairs = FMT == FMT_NV && RND == RND_RTN;
+// Whether quantize_block divides NVFP4 blocks with the pair table (nv_divide_block2), by measured
+// speed: round-to-nearest (single-pass 4096^2 quantize + dequantize 28.8 -> 27.7 us) and stochastic
+// rounding with the fused dequantize (36.6 -> 35.7 us).  Stochastic rounding alone, whose
+// per-element range test then costs more than the conversions it saves, keeps the fp64
+// reciprocals, as do four-over-six, axis-0 and 2-D blocks.
+template <int FMT, int RND, int DQ>
+constexpr bool kNvPairs = FMT == FMT_NV && (RND == RND_RTN || DQ != 0);
 
 // One thread quantizes one whole scale block of E = 32 (MX) or 16 (NV)
 // elements held as E/8 uint4: the block maximum, the scale and every division
@@ -414,8 +415,8 @@ __device__ __forceinline__ void quantize_block(const QRowParams& p, const uint4 
     if (FMT == FMT_NV46) {
       byte = nv_four_over_six<RND, E>(x, am, byte, nv);
     } else {
-      if (kNvPairs<FMT, RND>) {
-        nv_divide_block_rtn2<E>(x, am, reinterpret_cast<const float2*>(nv.tabd)[byte]);
+      if (kNvPairs<FMT, RND, DQ>) {
+        nv_divide_block2<RND, E>(x, am, reinterpret_cast<const float2*>(nv.tabd)[byte]);
       } else {
         nv_divide_block64<E>(x, nv.tabd[byte], x);
       }
@@ -489,7 +490,7 @@ __global__ void __launch_bounds__(256) quantize_rows_kernel(QRowParams p) {
   if (SFMMA) sf_pad_zero(p, blockIdx.x * blockDim.x + threadIdx.x, gridDim.x * blockDim.x);
   NvConsts nv{1.0f, 1.0, tabd};
   if (FMT != FMT_MX) {
-    nv = nv_consts<kNvPairs<FMT, RND>>(*p.ts, tabd);
+    nv = nv_consts<kNvPairs<FMT, RND, DQ>>(*p.ts, tabd);
     if (p.ts_copy_out != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *p.ts_copy_out = nv.s_t;
     __syncthreads();
   }
@@ -615,7 +616,7 @@ __global__ void __launch_bounds__(StreamWarps<FMT, RND>::kThreads, 1) quantize_s
   if (SFMMA) sf_pad_zero(p, blockIdx.x * blockDim.x + threadIdx.x, gridDim.x * blockDim.x);
   NvConsts nv{1.0f, 1.0, tabd};
   if (FMT != FMT_MX) {
-    nv = nv_consts<kNvPairs<FMT, RND>>(*p.ts, tabd);
+    nv = nv_consts<kNvPairs<FMT, RND, DQ>>(*p.ts, tabd);
     if (p.ts_copy_out != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *p.ts_copy_out = nv.s_t;
   }
   __syncthreads();
@@ -858,7 +859,7 @@ __global__ void __launch_bounds__(FusedWarps<FMT>::kThreads, 1) nv_quantize_fuse
     }
   }
   __syncthreads();
-  const NvConsts nv = nv_consts<kNvPairs<FMT, RND>>(s_t_shared, tabd);
+  const NvConsts nv = nv_consts<kNvPairs<FMT, RND, DQ>>(s_t_shared, tabd);
   __syncthreads();
   if (warp == 0) return;
 

@@ -2,7 +2,8 @@
 // (reciprocal + two FMA corrections, IEEE fallback) with CUDA's IEEE
 // division __fdiv_rn for every finite bf16 dividend and a list of divisors,
 // one element at a time (div_by_recip) and in 16-element blocks on packed
-// pairs (nv_divide_block_rtn2, round-to-nearest codes).
+// pairs (nv_divide_block2: bit-identical quotients under the stochastic-rounding test,
+// round-to-nearest codes under the round-to-nearest one).
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -39,8 +40,10 @@ __device__ __forceinline__ uint32_t rtn_code(float q) {
 // Blocks of 16 bf16 dividends: thread t takes patterns (t * 16 + i * stride) mod 2^16, i < 16
 // (stride 1: neighbours of one magnitude; a large odd stride: tiny and large elements mixed).
 // Quotients of elements with |x| >= 2^-103 (or 0) must equal IEEE division bit for bit; smaller
-// ones must give the same round-to-nearest E2M1 code.
-__global__ void div_check_rtn2_kernel(const float* scales, int n, uint32_t stride, unsigned long long* mismatches,
+// ones must give the same round-to-nearest E2M1 code (RND = 0), or, under the stochastic-rounding
+// test (RND = 1, which sends blocks with such elements to IEEE division), be equal too.
+template <int RND>
+__global__ void div_check_pair_kernel(const float* scales, int n, uint32_t stride, unsigned long long* mismatches,
                                       unsigned long long* fallbacks) {
   const int s_idx = blockIdx.y;
   if (s_idx >= n) return;
@@ -59,11 +62,11 @@ __global__ void div_check_rtn2_kernel(const float* scales, int n, uint32_t strid
       am = fmaxf(am, fabsf(x[i]));
     }
     if (!finite) continue;
-    if (!fp4dev::nv_fast_division<0, 16>(x, am, sy.x, sy.y)) ++slow;
-    fp4dev::nv_divide_block_rtn2<16>(q, am, sy);
+    if (!fp4dev::nv_fast_division<RND, 16>(x, am, sy.x, sy.y)) ++slow;
+    fp4dev::nv_divide_block2<RND, 16>(q, am, sy);
     for (int i = 0; i < 16; ++i) {
       const float ref = __fdiv_rn(x[i], S);
-      const bool exact = x[i] == 0.0f || fabsf(x[i]) >= 0x1p-103f;
+      const bool exact = RND == 1 || x[i] == 0.0f || fabsf(x[i]) >= 0x1p-103f;
       if (exact ? __float_as_uint(q[i]) != __float_as_uint(ref) : rtn_code(q[i]) != rtn_code(ref)) ++bad;
     }
   }
@@ -71,10 +74,14 @@ __global__ void div_check_rtn2_kernel(const float* scales, int n, uint32_t strid
   if (slow) atomicAdd(fallbacks, slow);
 }
 
-extern "C" int div_check_rtn2(const float* scales, int n, unsigned stride, unsigned long long* mismatches,
+extern "C" int div_check_pair(const float* scales, int n, unsigned stride, int rnd, unsigned long long* mismatches,
                               unsigned long long* fallbacks) {
   dim3 grid(16, n);
-  div_check_rtn2_kernel<<<grid, 256>>>(scales, n, stride, mismatches, fallbacks);
+  if (rnd) {
+    div_check_pair_kernel<1><<<grid, 256>>>(scales, n, stride, mismatches, fallbacks);
+  } else {
+    div_check_pair_kernel<0><<<grid, 256>>>(scales, n, stride, mismatches, fallbacks);
+  }
   return (int)cudaDeviceSynchronize();
 }
 

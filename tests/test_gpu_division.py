@@ -1,8 +1,8 @@
 """GPU: the NVFP4 quantizer's scale division x / S (correctly rounded reciprocal
 plus two FMA corrections, IEEE fallback for tiny operands) is bit-identical to
 CUDA's IEEE division for every finite bf16 x over thousands of divisors S, and
-the packed-pair block form used for round-to-nearest gives IEEE quotients
-(tiny dividends: the same E2M1 codes) on blocks of every bf16 pattern."""
+the packed-pair block form gives IEEE quotients (round-to-nearest, tiny
+dividends: the same E2M1 codes) on blocks of every bf16 pattern."""
 import ctypes
 import os
 import subprocess
@@ -26,7 +26,8 @@ def checker(tmp_path_factory):
     subprocess.run(cmd, check=True, capture_output=True)
     lib = ctypes.CDLL(str(out))
     lib.div_check.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p]
-    lib.div_check_rtn2.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_uint, ctypes.c_void_p, ctypes.c_void_p]
+    lib.div_check_pair.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_uint, ctypes.c_int, ctypes.c_void_p,
+                                   ctypes.c_void_p]
     return lib
 
 
@@ -55,15 +56,18 @@ def test_scale_division_matches_ieee(checker):
     assert slow.item() < 0.7 * total
 
 
+@pytest.mark.parametrize("rnd", [0, 1])
 @pytest.mark.parametrize("stride", [1, 4099, 40961])
-def test_block_pair_division_rtn_matches_ieee(checker, stride):
+def test_block_pair_division_matches_ieee(checker, stride, rnd):
     S = torch.from_numpy(_divisors()).cuda()
     bad = torch.zeros(1, dtype=torch.int64, device="cuda")
     slow = torch.zeros(1, dtype=torch.int64, device="cuda")
     for i in range(0, S.numel(), 1024):
         chunk = S[i:i + 1024].contiguous()
-        assert checker.div_check_rtn2(chunk.data_ptr(), chunk.numel(), stride, bad.data_ptr(), slow.data_ptr()) == 0
+        assert checker.div_check_pair(chunk.data_ptr(), chunk.numel(), stride, rnd, bad.data_ptr(),
+                                      slow.data_ptr()) == 0
     assert bad.item() == 0, f"{bad.item()} block quotients differ from IEEE division"
     # neighbouring patterns mostly take the fast path; mixed blocks hold huge elements whose
-    # quotients could overflow the corrections, so most of them fall back, but not all
-    assert slow.item() < (0.7 if stride == 1 else 0.99) * S.numel() * 4096
+    # quotients could overflow the corrections (or, under stochastic rounding, tiny elements), so
+    # most of them fall back, but not all
+    assert slow.item() < (0.7 if stride == 1 else 1.0) * S.numel() * 4096
