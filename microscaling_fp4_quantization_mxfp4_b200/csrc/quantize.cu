@@ -158,32 +158,36 @@ struct QRowParams {
   void* deq;             // DQ kernels: the dequantized values [rows, cols] (fp32, or bf16 for DQ = 2)
   uint32_t sf_rows;      // tensor-core scale layout: valid rows and scale groups per row, whose padding
   uint32_t sf_groups;    // bytes (rows up to 128, groups up to 4 g4) the kernel writes as 0
+  FastDiv g4d;           // division by g4
   unsigned long long jbase;  // Philox counter of the first element (row shards: first_row * cols / 4)
 };
 
-// Zero bytes of the tensor-core scale layout's padding (rows sf_rows .. multiple of 128, groups
-// sf_groups .. 4 g4), dealt over the grid's threads `t` of `nt`; the valid bytes are the
-// quantizer's.  Replaces a separate memset launch ahead of the quantizer.
+// Zero the tensor-core scale layout's padding (rows sf_rows .. multiple of 128, groups sf_groups ..
+// 4 g4), dealt over the grid's threads `t` of `nt`; the valid bytes are the quantizer's.  A padding
+// row's four groups 4j .. 4j + 3 are one aligned 32-bit word (one store each when the buffer is
+// 4-byte aligned); the groups past sf_groups of valid rows (fewer than 4) are single bytes.  32-bit
+// indices with the precomputed division by g4 (a 64-bit division per byte made the padding of a
+// one-row activation cost about 10 us on a single CTA).
 __device__ __forceinline__ void sf_pad_zero(const QRowParams& p, uint32_t t, uint32_t nt) {
-  const uint32_t gp = 4u * p.g4;                                   // padded groups per row
-  const uint32_t rpad = ((p.sf_rows + 127u) & ~127u) - p.sf_rows;   // padding rows
+  const uint32_t g4 = p.g4, gp = 4u * g4;
+  const uint32_t rpad = ((p.sf_rows + 127u) & ~127u) - p.sf_rows;  // padding rows
   const uint32_t gpad = gp - p.sf_groups;                          // padding groups of valid rows
-  const unsigned long long n_rows = (unsigned long long)rpad * gp;
-  const unsigned long long n_all = n_rows + (unsigned long long)p.sf_rows * gpad;
-  for (unsigned long long i = t; i < n_all; i += nt) {
-    uint32_t r, g;
-    if (i < n_rows) {
-      r = p.sf_rows + (uint32_t)(i / gp);
-      g = (uint32_t)(i % gp);
-    } else {
-      const unsigned long long j = i - n_rows;
-      r = (uint32_t)(j / gpad);
-      g = p.sf_groups + (uint32_t)(j % gpad);
+  if ((reinterpret_cast<uintptr_t>(p.scales) & 3u) == 0u) {
+    for (uint32_t i = t; i < rpad * g4; i += nt) {
+      const uint32_t k = fdiv(i, p.g4d), r = p.sf_rows + k, j = i - k * g4;
+      *reinterpret_cast<uint32_t*>(p.scales + sf_mma_offset(r, 4u * j, g4)) = 0u;
     }
-    p.scales[sf_mma_offset(r, g, p.g4)] = 0u;
+  } else {
+    for (uint32_t i = t; i < rpad * gp; i += nt) {
+      const uint32_t k = i / gp;
+      p.scales[sf_mma_offset(p.sf_rows + k, i - k * gp, g4)] = 0u;
+    }
+  }
+  for (uint32_t i = t; i < p.sf_rows * gpad; i += nt) {
+    const uint32_t r = i / gpad;
+    p.scales[sf_mma_offset(r, p.sf_groups + (i - r * gpad), g4)] = 0u;
   }
 }
-
 
 // Per-thread NVFP4 constants: the tensor scale, its reciprocal and the (S, 1/S) table.
 struct NvConsts {
@@ -525,7 +529,10 @@ constexpr int kStreamSmem = kStreamStages * kStreamChunks * 16 + 2 * kStreamStag
 // producer, the 1024-thread maximum, so at most 64 registers a thread, which
 // their 16-element blocks fit); 16 for MXFP4 round-to-nearest, with or
 // without rotation (31 warps ran 10-20 % slower, 19 warps at the same 96
-// registers 5-6 % slower); 15 for MXFP4 stochastic
+// registers 5-6 % slower; for rotations of 64 and 128 elements, two blocks a
+// thread on 15 warps, which keeps one or both cross-lane stages inside the
+// thread, measured slower too: 20.1 -> 22.9 and 22.0 -> 24.1 us at 8192 x 4096);
+// 15 for MXFP4 stochastic
 // rounding, whose 32-element blocks with their eight Philox blocks want about
 // 124 registers; 15 for four-over-six NVFP4, whose second candidate scale and
 // fp64 error sums do not fit in 64 registers.  Units of a stage are dealt to
@@ -733,7 +740,10 @@ __global__ void __launch_bounds__(32 * (kAmaxWarps + 1), 1) amax_stream_kernel(A
 // tensor fits in shared memory across the SMs (148 x ~227 KB on B200), one
 // cooperative launch reads it from HBM once: each CTA stages a contiguous run
 // of warp tiles in shared memory while reducing its amax, the CTAs meet at a
-// bounded grid barrier, and each quantizes its staged slice.
+// bounded grid barrier, and each quantizes its staged slice.  Small tensors
+// still take one 512-byte tile a CTA: a single CTA for a decode-sized
+// activation (1 x 4096, tensor-core scale layout) measured 6.7 against 4.8 us,
+// mostly the padding of the 128-row scale tiles written from one SM.
 struct FusedParams {
   QRowParams q;
   float* ts_out;          // s_t, written by CTA 0
@@ -1667,6 +1677,7 @@ cudaError_t launch_quantize_nv_fused(const QuantizeParams& p, float* ts_out, con
   qp.deq = p.deq;
   qp.sf_rows = (uint32_t)p.rows;
   qp.sf_groups = (uint32_t)(p.cols / 16);
+  qp.g4d = make_fastdiv(qp.g4 > 0u ? qp.g4 : 1u);
   fp.ts_out = ts_out;
   fp.partials = s.partials;
   fp.arrive = s.grid_arrive;
@@ -1749,6 +1760,7 @@ cudaError_t launch_quantize(const QuantizeParams& p, int num_sms, cudaStream_t s
     qp.deq = p.deq;
     qp.sf_rows = (uint32_t)p.rows;
     qp.sf_groups = (uint32_t)(p.cols / bs);
+    qp.g4d = make_fastdiv(qp.g4 > 0u ? qp.g4 : 1u);
     if (p.deq_mode != 0) {
       if (p.had != 0 || p.four_six) return cudaErrorInvalidValue;
       if (p.fmt == FMT_MX)

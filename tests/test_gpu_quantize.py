@@ -582,6 +582,7 @@ def test_quantize_mse_full_size_properties():
 @pytest.mark.parametrize("rnd", ["rtn", "sr"])
 @pytest.mark.parametrize("fmt, shape, given_ts, strided", [
     ("nvfp4", (200, 384), False, False),        # single-pass amax + quantize kernel
+    ("nvfp4", (3, 320), False, False),          # single-pass kernel, a partial tile
     ("nvfp4", (129, 1024), True, False),        # streaming kernel under a caller's s_t
     ("nvfp4", (64, 256), False, True),          # strided rows (ld > cols): amax pass + rows kernel
     ("mxfp4", (96, 512), False, False),
