@@ -1050,6 +1050,90 @@ __global__ void __launch_bounds__(256, (RND == RND_SR && FMT != FMT_NV46) ? 3 : 
   }
 }
 
+// MXFP4 stochastic rounding along axis 0 with four adjacent columns and eight rows a thread: the
+// four columns share one Philox4x32-10 evaluation per row (counter (row * C + c) / 4 for c a
+// multiple of 4, word c & 3), so every word is drawn where it is used, with no exchange between
+// lanes (the kernel above hands each lane its column's words through a quad transpose per four
+// rows).  A quad's lanes hold the four 8-row slices of the same four columns, one 32-row block
+// each: a two-stage shuffle gives the blocks' maxima, and one quad transpose of the packed codes
+// (one 32-bit word per column and slice) lets lane q store column q's 16 bytes of codes.  The
+// 128 x 64 bf16 tile's 16-byte chunks sit XOR-ed with bit 3 of the row moved to chunk bit 2, so
+// that the four 8-row slices of a warp's 8-byte reads fall in two bank halves.
+template <bool SFMMA>
+__global__ void __launch_bounds__(256, 3) quantize_cols_mx_sr_kernel(QColParams p) {
+  pdl_trigger();
+  __shared__ __align__(16) uint16_t tile[128][64];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int half = warp & 1, seg = warp >> 1, cgi = lane >> 2, rgi = lane & 3;
+  pdl_wait();
+  const uint32_t tiles_r = (p.R + 127u) / 128u, tiles_c = (p.C + 63u) / 64u;
+  for (uint32_t t = blockIdx.x; t < tiles_r * tiles_c; t += gridDim.x) {
+    const uint32_t tc = t / tiles_r, tr = t - tc * tiles_r;
+    const uint32_t r0 = tr * 128u, c0 = tc * 64u;
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int idx = tid + 256 * i, row = idx >> 3, ch = idx & 7;
+      const uint32_t gr = r0 + row, gc = c0 + ch * 8;
+      uint4 v = make_uint4(0u, 0u, 0u, 0u);
+      if (gr < p.R && gc < p.C) v = ld_stream(p.x + (int64_t)gr * p.ld + gc);
+      *reinterpret_cast<uint4*>(&tile[row][(ch ^ (((row >> 3) & 1) << 2)) * 8]) = v;
+    }
+    __syncthreads();
+    const uint32_t rbase = r0 + 32u * seg;                   // the warp's 32 rows: one block per column
+    if (rbase >= p.R) continue;                               // warp-uniform (R is a multiple of 32)
+    const uint32_t cq = c0 + 32u * half + 4u * cgi;           // the lane's first column (a multiple of 4)
+    float x[8][4];
+    const int colt = 32 * half + 4 * cgi;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int row = 32 * seg + 8 * rgi + i;
+      const int phys = (((colt >> 3) ^ (((row >> 3) & 1) << 2)) << 3) + (colt & 7);
+      const uint2 w = *reinterpret_cast<const uint2*>(&tile[row][phys]);
+      x[i][0] = bf16_lo(w.x); x[i][1] = bf16_hi(w.x);
+      x[i][2] = bf16_lo(w.y); x[i][3] = bf16_hi(w.y);
+    }
+    float am[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      float m = 0.0f;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(x[i][k]));
+      m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+      m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
+      am[k] = m;
+    }
+    uint32_t byte[4];
+    float inv[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      byte[k] = mx_scale_byte_clip(am[k], p.mx_thr);
+      inv[k] = mx_inv_scale(byte[k]);
+    }
+    uint32_t words[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const unsigned long long row = rbase + 8u * rgi + i;
+      const unsigned long long j = p.jbase + ((row * p.C + cq) >> 2);
+      const u32x4 ph = philox4x32_10((uint32_t)j, (uint32_t)(j >> 32), p.keys);
+      const uint32_t r4[4] = {ph.x, ph.y, ph.z, ph.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) words[k] |= e2m1_sr(__fmul_rn(x[i][k], inv[k]), r4[k]) << (4 * i);   // exact scaling
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) words[k] = am[k] == 0.0f ? 0u : words[k];
+    uint32_t t4[4];
+    quad_transpose4(words, t4, lane);                         // t4[s]: column cq + rgi, rows 8s .. 8s + 7
+    const uint32_t c = cq + (uint32_t)rgi;
+    if (c >= p.C) continue;
+    *reinterpret_cast<uint4*>(p.codes + (size_t)c * (p.R / 2) + rbase / 2) = make_uint4(t4[0], t4[1], t4[2], t4[3]);
+    const uint32_t b = rgi == 0 ? byte[0] : rgi == 1 ? byte[1] : rgi == 2 ? byte[2] : byte[3];
+    const uint32_t g = rbase / 32u;
+    if (SFMMA) p.scales[sf_mma_offset(c, g, p.g4)] = (uint8_t)b;
+    else p.scales[(size_t)c * p.G + g] = (uint8_t)b;
+  }
+}
+
 // ===================================================== 2-D (square-tile) quantize ===
 // "Pretraining Large Language Models with NVFP4", Abstract: a two-dimensional
 // scheme gives weights one consistent representation forward and backward.
@@ -1721,11 +1805,14 @@ cudaError_t launch_quantize_nv_fused(const QuantizeParams& p, float* ts_out, con
 
 template <int FMT, int RND, bool SFMMA>
 static cudaError_t cols_launch(const QColParams& qp, int num_sms, cudaStream_t st) {
-  static int occ = resident_ctas(quantize_cols_kernel<FMT, RND, SFMMA>, 256);
+  // MXFP4 stochastic rounding: four columns a thread (quantize_cols_mx_sr_kernel)
+  constexpr bool kMxSr = FMT == FMT_MX && RND == RND_SR;
+  auto kernel = kMxSr ? quantize_cols_mx_sr_kernel<SFMMA> : quantize_cols_kernel<FMT, RND, SFMMA>;
+  static int occ = resident_ctas(kernel, 256);
   const uint32_t ntiles = ((qp.R + 127u) / 128u) * ((qp.C + 63u) / 64u);
   uint32_t grid = (uint32_t)num_sms * (uint32_t)occ;
   if (ntiles < grid) grid = ntiles > 0 ? ntiles : 1;
-  return launch_kernel(quantize_cols_kernel<FMT, RND, SFMMA>, dim3(grid), dim3(256), 0, st, false, 1u, qp);
+  return launch_kernel(kernel, dim3(grid), dim3(256), 0, st, false, 1u, qp);
 }
 
 template <int FMT, int RND>
