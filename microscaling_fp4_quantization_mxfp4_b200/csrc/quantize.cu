@@ -1060,7 +1060,7 @@ __global__ void __launch_bounds__(256, (RND == RND_SR && FMT != FMT_NV46) ? 3 : 
 // 128 x 64 bf16 tile's 16-byte chunks sit XOR-ed with bit 3 of the row moved to chunk bit 2, so
 // that the four 8-row slices of a warp's 8-byte reads fall in two bank halves.
 template <bool SFMMA>
-__global__ void __launch_bounds__(256, 3) quantize_cols_mx_sr_kernel(QColParams p) {
+__global__ void __launch_bounds__(256, 4) quantize_cols_mx_sr_kernel(QColParams p) {
   pdl_trigger();
   __shared__ __align__(16) uint16_t tile[128][64];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -1117,8 +1117,12 @@ __global__ void __launch_bounds__(256, 3) quantize_cols_mx_sr_kernel(QColParams 
       const unsigned long long j = p.jbase + ((row * p.C + cq) >> 2);
       const u32x4 ph = philox4x32_10((uint32_t)j, (uint32_t)(j >> 32), p.keys);
       const uint32_t r4[4] = {ph.x, ph.y, ph.z, ph.w};
-#pragma unroll
-      for (int k = 0; k < 4; ++k) words[k] |= e2m1_sr(__fmul_rn(x[i][k], inv[k]), r4[k]) << (4 * i);   // exact scaling
+      const float2 v01 = mul2(make_float2(x[i][0], x[i][1]), make_float2(inv[0], inv[1]));   // exact scaling
+      const float2 v23 = mul2(make_float2(x[i][2], x[i][3]), make_float2(inv[2], inv[3]));
+      words[0] |= e2m1_sr(v01.x, r4[0]) << (4 * i);
+      words[1] |= e2m1_sr(v01.y, r4[1]) << (4 * i);
+      words[2] |= e2m1_sr(v23.x, r4[2]) << (4 * i);
+      words[3] |= e2m1_sr(v23.y, r4[3]) << (4 * i);
     }
 #pragma unroll
     for (int k = 0; k < 4; ++k) words[k] = am[k] == 0.0f ? 0u : words[k];
