@@ -248,7 +248,9 @@ fp4_status fp4_dequantize(const uint8_t* codes, const uint8_t* scales, const flo
 /*
  * fp4_gemm -- block-scaled FP4 x FP4 GEMM with fp32 accumulation on the
  * tcgen05 tensor cores ("Bridging the Gap", Abstract: FP4 GEMM on B200;
- * "Oscillation-Reduced MXFP4 Training", Abstract: MX matmuls on Blackwell).
+ * "Oscillation-Reduced MXFP4 Training", Abstract: MX matmuls on Blackwell);
+ * M = 1 (one activation row, decoding) runs on the CUDA cores instead, with
+ * exact per-block sums and one fp32 rounding per block.
  *   Y[M,N] = alpha * sum_k a[m,k] * b[n,k],  alpha = 1 (MX) or *a_ts * *b_ts (NV)
  *   a     uint8 codes [M, K/2] (K-major), a_sf scales in FP4_SF_MMA layout
  *   b     uint8 codes [N, K/2] (K-major), b_sf scales in FP4_SF_MMA layout
