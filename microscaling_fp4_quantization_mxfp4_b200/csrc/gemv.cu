@@ -10,7 +10,8 @@
 // E2M1 values times E2M1 values are multiples of 1/4 below 36, so a sum of up
 // to eight of them (|sum| <= 288, 1152 quarters < 2^11) is exact in f16: each
 // half of an f16x2 fused multiply-add accumulator takes eight products of a
-// 16-element block, the two halves are added in fp32 (exact), and
+// 16-element block (an MXFP4 block fills two accumulators), the halves are
+// added in fp32 (exact), and
 // fp32(block sum) * (s_a * s_b) enters the fp32 accumulator with one rounding
 // per block (s_a * s_b is exact: two E4M3 values, or a power of two).
 //
@@ -37,6 +38,7 @@ using namespace fp4dev;
 
 constexpr int kGemvWarps = 16;                 // weight rows in flight per CTA
 constexpr int kGemvUnroll = 4;                 // 16-byte chunks a lane loads before using them
+
 struct GemvParams {
   const uint8_t* a;
   const uint8_t* a_sf;
