@@ -535,12 +535,16 @@ constexpr int kStreamSmem = kStreamStages * kStreamChunks * 16 + 2 * kStreamStag
 // 15 for MXFP4 stochastic
 // rounding, whose 32-element blocks with their eight Philox blocks want about
 // 124 registers; 15 for four-over-six NVFP4, whose second candidate scale and
-// fp64 error sums do not fit in 64 registers.  Units of a stage are dealt to
-// the warps round-robin, starting one place further on each stage, so that
+// fp64 error sums do not fit in 64 registers; 23 for NVFP4 stochastic rounding
+// without rotation or dequantized output, whose Philox words then get up to 80
+// registers (4096 x 4096: 31.9 -> 30.2 us; with the fused dequantize 23 warps
+// were slower, 35.4 -> 36.1 us, and 27 the same).  Units of a stage are dealt
+// to the warps round-robin, starting one place further on each stage, so that
 // counts that do not divide evenly still balance over a run.
-template <int FMT, int RND>
+template <int FMT, int RND, int HAD = 0, int DQ = 0>
 struct StreamWarps {
-  static constexpr int kWarps = FMT == FMT_NV ? 31 : (FMT == FMT_NV46 || RND == RND_SR ? 15 : 16);
+  static constexpr int kWarps =
+      FMT == FMT_NV ? (RND == RND_SR && HAD == 0 && DQ == 0 ? 23 : 31) : (FMT == FMT_NV46 || RND == RND_SR ? 15 : 16);
   static constexpr int kThreads = 32 * (kWarps + 1);
 };
 constexpr int kAmaxWarps = 31;
@@ -611,8 +615,8 @@ __device__ void stream_produce(const StreamRing& r, const uint16_t* x, uint32_t 
 }
 
 template <int FMT, int RND, int HAD, bool SFMMA, int DQ = 0>
-__global__ void __launch_bounds__(StreamWarps<FMT, RND>::kThreads, 1) quantize_stream_kernel(QRowParams p) {
-  constexpr int kStreamWarps = StreamWarps<FMT, RND>::kWarps;
+__global__ void __launch_bounds__(StreamWarps<FMT, RND, HAD, DQ>::kThreads, 1) quantize_stream_kernel(QRowParams p) {
+  constexpr int kStreamWarps = StreamWarps<FMT, RND, HAD, DQ>::kWarps;
   extern __shared__ __align__(1024) uint8_t smem[];
   __shared__ double tabd[128];
   pdl_trigger();
@@ -1671,7 +1675,7 @@ static cudaError_t rows_stream_launch(const QRowParams& qp, int num_sms, cudaStr
   const uint32_t ngran = (qp.nchunks + 511u) / 512u;         // stream_range's granules
   uint32_t grid = (uint32_t)num_sms;
   if (ngran < grid) grid = ngran > 0 ? ngran : 1;
-  return launch_kernel(kernel, dim3(grid), dim3(StreamWarps<FMT, RND>::kThreads), kStreamSmem, st, false, 1u, qp);
+  return launch_kernel(kernel, dim3(grid), dim3(StreamWarps<FMT, RND, HAD, DQ>::kThreads), kStreamSmem, st, false, 1u, qp);
 }
 
 template <int FMT, int RND, int HAD, bool SFMMA, int DQ = 0>

@@ -119,7 +119,9 @@ def test_gemm_cuda_core_rows(M, N, K, fmt):
     """One activation row runs on the CUDA cores (exact f16 block sums, fp32 across blocks): the
     Llama-7B decode shapes, a ragged N, the shortest K, a single output; a heavy-tailed activation
     row with a zero block; fp32 against the fp64 oracle (sampled columns for the large N), bf16
-    within one ulp, and a strided output."""
+    within one ulp, and a strided output.  N = 1000 x K = 11008 (weights for every SM, too few rows
+    to give each SM two CTAs of 16) stages each SM's rows whole in shared memory; the others stream
+    rows through the warps' registers."""
     g = np.random.default_rng(M * 7 + N + K)
     from workloads import bf16_bits
     a = mixed_input(M, K, M + K, fmt)
