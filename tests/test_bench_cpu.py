@@ -45,3 +45,21 @@ def test_single_pass_rule_matches_library_bound():
     assert bench._nv_single_pass(4096, 4096, 148)
     assert not bench._nv_single_pass(16384, 11008, 148)
     assert bench._nv_single_pass(1, 4096, 148)
+
+
+def test_reference_arm_two_ranks():
+    """Launched as the harness launches N > 1 (torchrun, two ranks on 127.0.0.1): rank 0 alone
+    prints the one JSON line, with n_gpus = 2; the other rank exits 0 without output."""
+    import socket
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+           "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.join(ROOT, "bench.py"),
+           "--impl", "reference", "--workload", "mx_linear_128x512", "--gpus", "2", "--steps", "1", "--warmup", "3"]
+    out = subprocess.run(cmd, capture_output=True, text=True, timeout=600, cwd=ROOT)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [l for l in out.stdout.splitlines() if l.strip().startswith("{")]
+    assert len(lines) == 1, out.stdout
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["value"] > 0
